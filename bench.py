@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of the Beam MoE block forward pass on B200 (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+                    [--impl ours|reference]
+
+A step is one forward pass of the whole block (router, dispatch, gate|up
+GEMM with SwiGLU, down GEMM, combine [+ post-norm and residual]) over one
+batch of T synthetic tokens, with weights and tokens already in HBM.  Each
+rank runs its own replica on its own batches (tokens are independent: weak
+scaling, no data-path collective); ``value`` is all ranks' tokens over the
+slowest rank's device time.
+
+``--impl reference`` times the plain CPU oracle on the host cores instead,
+one bounded sample of tokens per step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from group_limited_routing_sigmoid_b200 import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (Beam shape, bf16) and % of HBM / tensor-core roofline"
+KERNELS_PER_FORWARD = 8     # logits, select, count, scan, permute, gate|up, down, combine
+TOKEN_BATCHES = 8           # distinct token batches cycled through the steps
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, sampled every 20 ms)
+# ---------------------------------------------------------------------------
+REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
+           0x10: "sync_boost", 0x1: "gpu_idle"}
+
+
+class ClockSampler:
+    def __init__(self, cuda_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            phys = int(vis.split(",")[cuda_index]) if vis and vis.split(",")[0].isdigit() else cuda_index
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(phys)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._reason_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self._nv = None
+            self.error = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                bits = self._reason_fn(self._h)
+                for b, name in REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def report(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for fn in ("grouped_gemm.cu", "common.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "group_limited_routing_sigmoid_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch of the gate|up GEMM from the committed ncu summary,
+    scaled to this workload; None if absent or taken on other kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    entry = t.get(workload)
+    if not entry or entry.get("kernel_hash") != kernel_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def rank_workload(wl: W.Workload, rank: int) -> W.Workload:
+    return wl
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch.distributed as dist
+    from group_limited_routing_sigmoid_b200.build import build
+    from group_limited_routing_sigmoid_b200.binding import BeamMoE
+
+    ws, rank, local = dist_env()
+    if ws != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={ws}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    if rank == 0 or ws == 1:
+        build(quiet=True)
+    if ws > 1:
+        dist.barrier()
+
+    wl = W.WORKLOADS[args.workload]
+    T, H, I, E, k = wl.T, wl.hidden, wl.inter, wl.n_experts, wl.top_k
+    g = W.generator(wl, dev)
+    weights = W.make_weights(wl, dev, g)
+    # distinct token batches per rank (weights identical on every rank)
+    tg = torch.Generator(device=dev)
+    tg.manual_seed(wl.seed + 1000 * (rank + 1))
+    batches = [W.make_tokens(wl, dev, tg) for _ in range(TOKEN_BATCHES)]
+    if wl.post_norm:
+        weights["gamma"] = batches[0]["gamma"]
+    moe = BeamMoE.from_workload(wl, weights)
+    outs = [torch.empty(T, H, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    streams = [b["stream"] for b in batches]
+
+    # distinct experts each batch touches (for the algorithmic byte count)
+    distinct = []
+    for b in batches:
+        idx, _ = moe.route(b["x"])
+        distinct.append(int((torch.bincount(idx.reshape(-1).long(), minlength=E) > 0).sum()))
+    torch.cuda.synchronize(dev)
+
+    def step(i):
+        b = batches[i % TOKEN_BATCHES]
+        if wl.residual_k:
+            moe.forward(b["x"], out=outs[i & 1], residual=streams[i % TOKEN_BATCHES], k=wl.residual_k)
+        else:
+            moe.forward(b["x"], out=outs[i & 1])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert moe.get_status() == 0
+
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    moe.profile_begin(args.steps)
+    sampler = ClockSampler(local)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    if ws > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    calls, stage_ms = moe.profile_end()
+    if moe.get_status() != 0:
+        raise SystemExit("a device-side wait ran out during the timed region")
+    t_max = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    ms_max = float(t_max.item())
+
+    # end to end through the host-buffer entry point (pinned buffers)
+    x_host = [b["x"].cpu().pin_memory() for b in batches]
+    out_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    res_host = [s.cpu().pin_memory() for s in streams] if wl.residual_k else None
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step(i):
+        j = i % TOKEN_BATCHES
+        moe.forward_host(x_host[j], out_host=out_host,
+                         residual_host=res_host[j] if res_host else None, k=max(1, wl.residual_k))
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = torch.tensor([ev0.elapsed_time(ev1)], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    # roofline of the dominant kernel
+    pk = peaks()
+    steps_done = args.steps
+    d_mean = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(steps_done)) / steps_done
+    P = T * k
+    gate_up_ms = stage_ms["gate_up_gemm"] / max(calls, 1)
+    if args.workload in ("decode", "tiny"):
+        alg_bytes = d_mean * 2 * I * H * 2 + P * H * 2 + P * I * 2
+        achieved = alg_bytes / (gate_up_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "gate_up_gemm (grouped_gemm_kernel<BN,2>)",
+                "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
+                "algorithmic_bytes_per_launch": int(alg_bytes), "launch_ms": round(gate_up_ms, 4)}
+    else:
+        flops = 4.0 * H * I * P
+        achieved = flops / (gate_up_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "gate_up_gemm (grouped_gemm_kernel<BN,2>)",
+                "achieved": round(achieved, 1), "peak": pk["bf16_sus"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_sus"], 4), "peak_source": pk["source"] + " sustained",
+                "algorithmic_flops_per_launch": flops, "launch_ms": round(gate_up_ms, 4)}
+    roof["traffic"] = ncu_traffic(args.workload)
+    step_bytes = d_mean * 3 * H * I * 2 + E * H * 4 + T * H * 4 + (T * H * 8 if wl.residual_k else 0)
+    stage_avg = {kname: round(v / max(calls, 1), 4) for kname, v in stage_ms.items()}
+
+    line = {
+        "metric": METRIC,
+        "value": round(ws * steps_done * T / (ms_max * 1e-3), 1),
+        "unit": "tokens/s",
+        "n_gpus": ws,
+        "steps": steps_done,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / steps_done, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded random weights and tokens of the Beam block shape)",
+        "config": {"workload": f"beam_{args.workload}", "T": T, "hidden": H, "n_experts": E,
+                   "n_group": wl.n_group, "topk_group": wl.topk_group, "top_k": k, "inter": I,
+                   "routed_scaling": wl.routed_scaling, "residual_k": wl.residual_k,
+                   "post_norm": wl.post_norm, "token_batches": TOKEN_BATCHES,
+                   "distinct_experts_per_step": round(d_mean, 2),
+                   "l2": f"inputs larger than L2: each step streams {d_mean * 3 * H * I * 2 / 1e9:.1f} GB of expert weights",
+                   "parallelism": f"{ws} independent replicas (data parallel, no collective on the data path)"},
+        "hbm_fraction_whole_step": round(step_bytes / (ms_max / steps_done * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+        "stage_ms": stage_avg,
+        "clocks": sampler.report(),
+        "e2e": {"value": round(ws * e2e_steps * T / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0),
+                "d2h_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0)},
+        "gpu_launches": KERNELS_PER_FORWARD * steps_done,
+        "roofline": roof,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, weights, batches[0]["x"], args.cpu_tokens)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    moe.close()
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _oracle_on_tokens(wl, weights, x, n_tokens):
+    """Time the oracle on the first n_tokens of x (expert weights copied to
+    the host before the clock starts)."""
+    import oracle
+    oracle.build()
+    xs = W.bf16_bits(x[:n_tokens])
+    rw = weights["router_w"].cpu().numpy()
+    bias = weights["bias"].cpu().numpy()
+    r = oracle.route(xs, rw, bias, wl.n_group, wl.topk_group, wl.top_k)
+    cache = {}
+    for e in sorted(set(int(v) for v in r.idx.reshape(-1))):
+        cache[e] = (W.bf16_bits(weights["w_gate"][e]), W.bf16_bits(weights["w_up"][e]),
+                    W.bf16_bits(weights["w_down"][e]))
+    gamma = None if weights.get("gamma") is None else weights["gamma"].cpu().numpy()
+    stream = None
+    if wl.residual_k:
+        stream = torch.zeros(n_tokens, wl.hidden).numpy()
+    t0 = time.perf_counter()
+    oracle.moe_block(xs, rw, bias, cache.__getitem__, wl.n_group, wl.topk_group, wl.top_k,
+                     wl.routed_scaling, gamma=gamma, eps=wl.norm_eps, stream=stream, kstep=wl.residual_k)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, weights, x, n_tokens):
+    import oracle
+    sec = _oracle_on_tokens(wl, weights, x, n_tokens)
+    return {"value": round(n_tokens / sec, 3), "unit": "tokens/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"{n_tokens} tokens of one {wl.T}-token batch, all {wl.top_k} experts each, "
+                      f"fp64 oracle ({sec:.1f} s)"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    wl = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    g = W.generator(wl, dev)
+    weights = W.make_weights(wl, dev, g)
+    tg = torch.Generator(device=dev)
+    tg.manual_seed(wl.seed + 1000)
+    x = W.make_tokens(wl, dev, tg)["x"]
+    if wl.post_norm:
+        weights["gamma"] = 1.0 + 0.02 * torch.randn(wl.hidden, generator=tg, device=dev)
+    per_step = 1
+    times = []
+    for i in range(args.warmup + args.steps):
+        j = i % wl.T
+        sec = _oracle_on_tokens(wl, weights, x[j:j + 1].contiguous(), per_step)
+        if i >= args.warmup:
+            times.append(sec)
+    total = sum(times)
+    value = round(args.steps * per_step / total, 4)
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded random weights and tokens of the Beam block shape)",
+        "config": {"workload": f"beam_{args.workload}", "T": wl.T, "hidden": wl.hidden,
+                   "n_experts": wl.n_experts, "top_k": wl.top_k, "inter": wl.inter},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+                         "sample": f"{per_step} token per step (all {wl.top_k} experts), tokens "
+                                   f"cycled through one {wl.T}-token batch"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

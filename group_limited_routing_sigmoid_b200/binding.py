@@ -1,0 +1,218 @@
+"""ctypes binding of ``libbeam_moe.so`` (C ABI in ``include/beam_moe.h``).
+
+Argument marshalling only: every step of the block runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  If the
+library is missing the first call raises; there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import numpy as np
+import torch
+
+from .build import LIB
+
+BEAM_OK = 0
+BEAM_ERR_INVALID_ARG = -1
+BEAM_ERR_UNSUPPORTED = -2
+BEAM_ERR_CUDA = -3
+BEAM_ERR_OOM = -4
+BEAM_ERR_TIMEOUT = -5
+
+# every entry point declared in include/beam_moe.h
+SYMBOLS = (
+    "beam_moe_create", "beam_moe_route", "beam_moe_router_logits", "beam_moe_forward",
+    "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_get_status",
+    "beam_moe_set_wait_limit", "beam_moe_set_gemm_ctas", "beam_moe_profile_begin",
+    "beam_moe_profile_end", "beam_moe_check_wait_timeout", "beam_moe_last_error",
+    "beam_moe_create_error", "beam_moe_destroy",
+)
+
+_lib = None
+
+
+class BeamMoEError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"beam_moe error {code}: {msg}")
+        self.code = code
+
+
+def library() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise RuntimeError(f"{LIB} is missing: build it with "
+                               "`python -m group_limited_routing_sigmoid_b200.build`")
+        lib = ctypes.CDLL(LIB)
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        lib.beam_moe_create.argtypes = [ctypes.POINTER(P), I, I, I, I, I, I, F, P, P, P, P, P, P, F, I]
+        lib.beam_moe_route.argtypes = [P, P, P, I, P, P]
+        lib.beam_moe_router_logits.argtypes = [P, P, P, I, P]
+        lib.beam_moe_forward.argtypes = [P, P, P, I, P, P, I]
+        lib.beam_moe_forward_host.argtypes = [P, P, P, I, P, P, I]
+        lib.beam_moe_dispatch_info.argtypes = [P, P, I, P, P, P]
+        lib.beam_moe_get_status.argtypes = [P, P]
+        lib.beam_moe_set_wait_limit.argtypes = [P, ctypes.c_int64]
+        lib.beam_moe_set_gemm_ctas.argtypes = [P, I]
+        lib.beam_moe_check_wait_timeout.argtypes = [P, P]
+        lib.beam_moe_profile_begin.argtypes = [P, I]
+        lib.beam_moe_profile_end.argtypes = [P, P, P]
+        lib.beam_moe_last_error.argtypes = [P]
+        lib.beam_moe_last_error.restype = ctypes.c_char_p
+        lib.beam_moe_create_error.argtypes = []
+        lib.beam_moe_create_error.restype = ctypes.c_char_p
+        lib.beam_moe_destroy.argtypes = [P]
+        for name in SYMBOLS:
+            if name not in ("beam_moe_last_error", "beam_moe_create_error"):
+                getattr(lib, name).restype = I
+        _lib = lib
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dev(t: torch.Tensor, dtype, name: str):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise TypeError(f"{name}: expected a contiguous CUDA {dtype} tensor, got "
+                        f"{t.dtype} on {t.device} (contiguous={t.is_contiguous()})")
+    return t
+
+
+class BeamMoE:
+    """One MoE block on the current CUDA device (borrows the weight tensors)."""
+
+    def __init__(self, hidden: int, n_experts: int, inter: int, n_group: int, topk_group: int,
+                 top_k: int, routed_scaling: float, router_w: torch.Tensor, expert_bias: torch.Tensor,
+                 w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+                 post_norm_w: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
+                 max_tokens: int = 64):
+        lib = library()
+        _dev(router_w, torch.float32, "router_w")
+        _dev(expert_bias, torch.float32, "expert_bias")
+        for n, t in (("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down)):
+            _dev(t, torch.bfloat16, n)
+        if post_norm_w is not None:
+            _dev(post_norm_w, torch.float32, "post_norm_w")
+        self._keep = (router_w, expert_bias, w_gate, w_up, w_down, post_norm_w)
+        self.hidden, self.n_experts, self.inter = hidden, n_experts, inter
+        self.top_k = top_k
+        self.max_tokens = max_tokens
+        self.device = router_w.device
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            rc = lib.beam_moe_create(ctypes.byref(h), hidden, n_experts, inter, n_group, topk_group,
+                                     top_k, float(routed_scaling), _ptr(router_w), _ptr(expert_bias),
+                                     _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(post_norm_w),
+                                     float(norm_eps), max_tokens)
+        if rc != BEAM_OK:
+            raise BeamMoEError(rc, lib.beam_moe_create_error().decode())
+        self._h = h
+
+    @classmethod
+    def from_workload(cls, wl, weights, max_tokens: Optional[int] = None) -> "BeamMoE":
+        return cls(wl.hidden, wl.n_experts, wl.inter, wl.n_group, wl.topk_group, wl.top_k,
+                   wl.routed_scaling, weights["router_w"], weights["bias"], weights["w_gate"],
+                   weights["w_up"], weights["w_down"], weights.get("gamma"), wl.norm_eps,
+                   max_tokens or wl.T)
+
+    def _check(self, rc: int):
+        if rc != BEAM_OK:
+            raise BeamMoEError(rc, library().beam_moe_last_error(self._h).decode())
+
+    def route(self, x: torch.Tensor, idx: Optional[torch.Tensor] = None,
+              w: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+        _dev(x, torch.bfloat16, "x")
+        T = x.shape[0]
+        if idx is None:
+            idx = torch.empty(T, self.top_k, dtype=torch.int32, device=x.device)
+        if w is None:
+            w = torch.empty(T, self.top_k, dtype=torch.float32, device=x.device)
+        self._check(library().beam_moe_route(self._h, _stream(stream), _ptr(x), T, _ptr(idx), _ptr(w)))
+        return idx, w
+
+    def router_logits(self, x: torch.Tensor, logits: Optional[torch.Tensor] = None, stream=None):
+        _dev(x, torch.bfloat16, "x")
+        T = x.shape[0]
+        if logits is None:
+            logits = torch.empty(T, self.n_experts, dtype=torch.float32, device=x.device)
+        self._check(library().beam_moe_router_logits(self._h, _stream(stream), _ptr(x), T, _ptr(logits)))
+        return logits
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                residual: Optional[torch.Tensor] = None, k: int = 1, want_out: bool = True,
+                stream=None) -> Optional[torch.Tensor]:
+        _dev(x, torch.bfloat16, "x")
+        T = x.shape[0]
+        if out is None and want_out:
+            out = torch.empty(T, self.hidden, dtype=torch.bfloat16, device=x.device)
+        if residual is not None:
+            _dev(residual, torch.float32, "residual")
+        self._check(library().beam_moe_forward(self._h, _stream(stream), _ptr(x), T, _ptr(out),
+                                                _ptr(residual), int(k)))
+        return out
+
+    def forward_host(self, x_host: torch.Tensor, out_host: Optional[torch.Tensor] = None,
+                     residual_host: Optional[torch.Tensor] = None, k: int = 1, stream=None):
+        """Host buffers in, host buffers out (copies inside the call)."""
+        assert not x_host.is_cuda and x_host.dtype == torch.bfloat16 and x_host.is_contiguous()
+        T = x_host.shape[0]
+        self._check(library().beam_moe_forward_host(self._h, _stream(stream), _ptr(x_host), T,
+                                                     _ptr(out_host), _ptr(residual_host), int(k)))
+        return out_host
+
+    def dispatch_info(self, T: int, stream=None):
+        counts = np.empty(self.n_experts, np.int32)
+        offsets = np.empty(self.n_experts + 1, np.int32)
+        pair_row = np.empty(T * self.top_k, np.int32)
+        self._check(library().beam_moe_dispatch_info(
+            self._h, _stream(stream), T, counts.ctypes.data_as(ctypes.c_void_p),
+            offsets.ctypes.data_as(ctypes.c_void_p), pair_row.ctypes.data_as(ctypes.c_void_p)))
+        return counts, offsets, pair_row
+
+    def get_status(self, stream=None) -> int:
+        return library().beam_moe_get_status(self._h, _stream(stream))
+
+    def set_wait_limit(self, limit_ns: int):
+        self._check(library().beam_moe_set_wait_limit(self._h, int(limit_ns)))
+
+    def set_gemm_ctas(self, ctas: int):
+        self._check(library().beam_moe_set_gemm_ctas(self._h, int(ctas)))
+
+    STAGES = ("router", "dispatch", "gate_up_gemm", "down_gemm", "combine")
+
+    def profile_begin(self, max_calls: int):
+        self._check(library().beam_moe_profile_begin(self._h, int(max_calls)))
+
+    def profile_end(self):
+        """-> (calls, {stage: total ms}) over the forward passes since profile_begin."""
+        ms = (ctypes.c_float * 5)()
+        calls = ctypes.c_int()
+        self._check(library().beam_moe_profile_end(self._h, ctypes.cast(ms, ctypes.c_void_p),
+                                                    ctypes.cast(ctypes.pointer(calls), ctypes.c_void_p)))
+        return calls.value, dict(zip(self.STAGES, [float(v) for v in ms]))
+
+    def check_wait_timeout(self, stream=None) -> int:
+        return library().beam_moe_check_wait_timeout(self._h, _stream(stream))
+
+    def close(self):
+        if getattr(self, "_h", None):
+            library().beam_moe_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,605 @@
+// C ABI of the Beam MoE block (declared in include/beam_moe.h): argument
+// validation, workspace, TMA descriptors, and the stream-ordered launch
+// sequence router -> dispatch -> gate|up GEMM -> down GEMM -> combine.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "beam_moe.h"
+#include "kernels.cuh"
+
+using namespace beam;
+
+struct beam_moe {
+    int H, E, I, n_group, topk_group, top_k;
+    float scaling;
+    const float *router_w, *bias, *gamma;
+    const __nv_bfloat16 *w_gate, *w_up, *w_down;
+    float eps;
+    int max_tokens;
+    int device, num_sms;
+    int gemm_ctas;           // 0: num_sms
+    long long wait_limit_ns;
+
+    void *ws;
+    size_t ws_bytes;
+    float *partial;          // [nslice_max * T_max * E]
+    int32_t *idx;            // [P]
+    float *w;                // [P]
+    int32_t *block_cnt, *block_base, *rank, *counts, *offsets, *tile_off, *pair_row, *row_pair;
+    __nv_bfloat16 *xp;       // [P, H]
+    __nv_bfloat16 *hbuf;     // [P, I]
+    float *ybuf;             // [P, H]
+    int *status;             // device status word
+    __nv_bfloat16 *x_stage, *out_stage;
+    float *res_stage;
+
+    CUtensorMap tm_gate, tm_up, tm_down;
+    CUtensorMap tm_xp[4], tm_h[4];   // box rows 16, 32, 64, 128
+    int last_T;
+    std::vector<cudaEvent_t> prof_events;   // 6 per profiled forward pass
+    int prof_max, prof_calls;
+    char err[512];
+};
+
+namespace {
+
+char g_create_err[512] = "";
+
+int fail(beam_moe *h, int code, const char *fmt, ...)
+{
+    char *dst = h ? h->err : g_create_err;
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(dst, 512, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(beam_moe *h, cudaError_t e, const char *what)
+{
+    return fail(h, BEAM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] row-major, box {64 cols, box_rows}, 128B swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int tile_index(int BN) { return BN == 16 ? 0 : BN == 32 ? 1 : BN == 64 ? 2 : 3; }
+
+// Token rows per GEMM tile from the mean load per expert (the host never
+// reads the routing, so the choice depends on T only).
+int choose_tile_rows(int T, int top_k, int E)
+{
+    const double mean = (double)T * top_k / E;
+    if (mean <= 24) return 16;
+    if (mean <= 48) return 32;
+    if (mean <= 96) return 64;
+    return 128;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int check_device(beam_moe *h)
+{
+    int cur = -1;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaGetDevice");
+    if (cur != h->device)
+        return fail(h, BEAM_ERR_INVALID_ARG, "current device %d is not the handle's device %d", cur,
+                    h->device);
+    return BEAM_OK;
+}
+
+int run_router(beam_moe *h, cudaStream_t s, const void *x, int T, int32_t *idx, float *w,
+               float *logits)
+{
+    RouterArgs a;
+    a.x = static_cast<const __nv_bfloat16 *>(x);
+    a.router_w = h->router_w;
+    a.bias = h->bias;
+    a.T = T;
+    a.H = h->H;
+    a.E = h->E;
+    a.n_group = h->n_group;
+    a.topk_group = h->topk_group;
+    a.top_k = h->top_k;
+    a.nslice = router_slices(T, h->H, h->E, h->num_sms);
+    while (a.nslice > 1 && (size_t)a.nslice * T > (size_t)(h->max_tokens > 4096 ? h->max_tokens : 4096))
+        a.nslice /= 2;
+    a.partial = h->partial;
+    a.idx = idx;
+    a.w = w;
+    a.logits_out = logits;
+    cudaError_t e = launch_router(a, s);
+    return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "router launch");
+}
+
+void prof_mark(beam_moe *h, cudaStream_t s, int stage)
+{
+    if (h->prof_calls < h->prof_max)
+        cudaEventRecord(h->prof_events[(size_t)h->prof_calls * 6 + stage], s);
+}
+
+int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, float *residual,
+                int k)
+{
+    prof_mark(h, s, 0);
+    int rc = run_router(h, s, x, T, h->idx, h->w, nullptr);
+    if (rc != BEAM_OK) return rc;
+    prof_mark(h, s, 1);
+    const int BN = choose_tile_rows(T, h->top_k, h->E);
+    DispatchArgs d;
+    d.idx = h->idx;
+    d.x = static_cast<const __nv_bfloat16 *>(x);
+    d.T = T;
+    d.H = h->H;
+    d.E = h->E;
+    d.top_k = h->top_k;
+    d.tile_rows = BN;
+    d.block_cnt = h->block_cnt;
+    d.block_base = h->block_base;
+    d.rank = h->rank;
+    d.counts = h->counts;
+    d.offsets = h->offsets;
+    d.tile_off = h->tile_off;
+    d.pair_row = h->pair_row;
+    d.row_pair = h->row_pair;
+    d.xp = h->xp;
+    cudaError_t e = launch_dispatch(d, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "dispatch launch");
+    prof_mark(h, s, 2);
+
+    GemmArgs g;
+    g.E = h->E;
+    g.counts = h->counts;
+    g.offsets = h->offsets;
+    g.tile_off = h->tile_off;
+    g.ctl.status = h->status;
+    g.ctl.limit_ns = h->wait_limit_ns;
+    const int ti = tile_index(BN);
+    g.K = h->H;
+    g.R = h->I;
+    g.out = h->hbuf;
+    const int grid = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
+    e = launch_grouped_gemm(true, BN, h->tm_gate, h->tm_up, h->tm_xp[ti], g, grid, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "gate/up GEMM launch");
+    prof_mark(h, s, 3);
+    g.K = h->I;
+    g.R = h->H;
+    g.out = h->ybuf;
+    e = launch_grouped_gemm(false, BN, h->tm_down, h->tm_down, h->tm_h[ti], g, grid, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "down GEMM launch");
+    prof_mark(h, s, 4);
+
+    CombineArgs c;
+    c.y = h->ybuf;
+    c.pair_row = h->pair_row;
+    c.w = h->w;
+    c.T = T;
+    c.H = h->H;
+    c.top_k = h->top_k;
+    c.scaling = h->scaling;
+    c.out = static_cast<__nv_bfloat16 *>(out);
+    c.residual = residual;
+    c.gamma = residual ? h->gamma : nullptr;
+    c.eps = h->eps;
+    const int kk = k >= 1 ? k : 1;
+    c.keep = (float)std::sqrt((double)(kk - 1) / (double)kk);
+    c.add = (float)(1.0 / std::sqrt((double)kk));
+    e = launch_combine(c, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "combine launch");
+    prof_mark(h, s, 5);
+    if (h->prof_calls < h->prof_max) ++h->prof_calls;
+    h->last_T = T;
+    return BEAM_OK;
+}
+
+int check_tokens(beam_moe *h, const void *x, int T)
+{
+    if (T < 0 || T > h->max_tokens)
+        return fail(h, BEAM_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->max_tokens);
+    if (T > 0 && (!x || !aligned16(x)))
+        return fail(h, BEAM_ERR_INVALID_ARG, "x must be a non-NULL 16-byte aligned device pointer");
+    return BEAM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *beam_moe_create_error(void) { return g_create_err; }
+
+int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n_group,
+                    int topk_group, int top_k, float routed_scaling, const float *router_w,
+                    const float *expert_bias, const void *w_gate, const void *w_up,
+                    const void *w_down, const float *post_norm_w, float norm_eps, int max_tokens)
+{
+    g_create_err[0] = 0;
+    if (!out) return fail(nullptr, BEAM_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (hidden <= 0 || n_experts <= 0 || inter <= 0 || n_group <= 0 || max_tokens < 1)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "sizes must be positive");
+    if (n_experts % n_group != 0)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "n_experts %% n_group != 0");
+    const int gsize = n_experts / n_group;
+    if (gsize < 2) return fail(nullptr, BEAM_ERR_INVALID_ARG, "group size must be >= 2");
+    if (topk_group < 1 || topk_group > n_group)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "topk_group outside [1, n_group]");
+    if (top_k < 1 || top_k > topk_group * gsize)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "top_k outside [1, topk_group * group size]");
+    if (!(routed_scaling == routed_scaling) || !(norm_eps >= 0.f))
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "routed_scaling / norm_eps not valid");
+    if (!router_w || !expert_bias || !w_gate || !w_up || !w_down)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "weight pointer is NULL");
+    if (!aligned16(router_w) || !aligned16(expert_bias) || !aligned16(w_gate) || !aligned16(w_up) ||
+        !aligned16(w_down) || (post_norm_w && !aligned16(post_norm_w)))
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "weight pointers must be 16-byte aligned");
+    if (hidden % 128 != 0 || inter % 128 != 0)
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "hidden and inter must be multiples of 128");
+    if (hidden > 8192)
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "hidden > 8192");
+    if (n_experts % 32 != 0 || n_experts > 1024 || !is_pow2(n_experts / 32))
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED,
+                    "n_experts must be 32 x a power of two, at most 1024");
+    const int epl = n_experts / 32;
+    if (gsize % epl != 0 || !is_pow2(gsize / epl) || n_group > 32)
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "group size not supported by the router kernel");
+    if (top_k > 32) return fail(nullptr, BEAM_ERR_UNSUPPORTED, "top_k > 32");
+    if ((long long)max_tokens * top_k > (1LL << 30))
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "max_tokens * top_k too large");
+
+    beam_moe *h = new beam_moe();
+    memset(h, 0, sizeof(*h));
+    h->H = hidden;
+    h->E = n_experts;
+    h->I = inter;
+    h->n_group = n_group;
+    h->topk_group = topk_group;
+    h->top_k = top_k;
+    h->scaling = routed_scaling;
+    h->router_w = router_w;
+    h->bias = expert_bias;
+    h->gamma = post_norm_w;
+    h->w_gate = static_cast<const __nv_bfloat16 *>(w_gate);
+    h->w_up = static_cast<const __nv_bfloat16 *>(w_up);
+    h->w_down = static_cast<const __nv_bfloat16 *>(w_down);
+    h->eps = norm_eps;
+    h->max_tokens = max_tokens;
+    h->wait_limit_ns = 2000000000LL;
+
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+    if (e != cudaSuccess) {
+        int rc = cuda_fail(nullptr, e, "device query");
+        delete h;
+        return rc;
+    }
+
+    // Workspace
+    const size_t T = (size_t)max_tokens, E = (size_t)n_experts, P = T * top_k;
+    const size_t nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
+    // router partial sums: nslice(T) * T <= 4096 rows for every T (router_slices
+    // keeps the logits grid near two blocks per SM), and T rows for large T
+    const size_t partial_rows = T > 4096 ? T : 4096;
+    size_t off = 0;
+    auto carve = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    const size_t o_partial = carve(partial_rows * E * 4);
+    const size_t o_idx = carve(P * 4);
+    const size_t o_w = carve(P * 4);
+    const size_t o_bcnt = carve(nblk * E * 4);
+    const size_t o_bbase = carve(nblk * E * 4);
+    const size_t o_rank = carve(P * 4);
+    const size_t o_counts = carve(E * 4);
+    const size_t o_offsets = carve((E + 1) * 4);
+    const size_t o_tile = carve((E + 1) * 4);
+    const size_t o_prow = carve(P * 4);
+    const size_t o_rpair = carve(P * 4);
+    const size_t o_xp = carve(P * hidden * 2);
+    const size_t o_h = carve(P * inter * 2);
+    const size_t o_y = carve(P * hidden * 4);
+    const size_t o_status = carve(256);
+    const size_t o_xs = carve(T * hidden * 2);
+    const size_t o_os = carve(T * hidden * 2);
+    const size_t o_rs = carve(T * hidden * 4);
+    h->ws_bytes = off;
+    e = cudaMalloc(&h->ws, h->ws_bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        int rc = fail(nullptr, BEAM_ERR_OOM, "workspace of %zu bytes: %s", h->ws_bytes,
+                      cudaGetErrorString(e));
+        delete h;
+        return rc;
+    }
+    char *b = static_cast<char *>(h->ws);
+    h->partial = reinterpret_cast<float *>(b + o_partial);
+    h->idx = reinterpret_cast<int32_t *>(b + o_idx);
+    h->w = reinterpret_cast<float *>(b + o_w);
+    h->block_cnt = reinterpret_cast<int32_t *>(b + o_bcnt);
+    h->block_base = reinterpret_cast<int32_t *>(b + o_bbase);
+    h->rank = reinterpret_cast<int32_t *>(b + o_rank);
+    h->counts = reinterpret_cast<int32_t *>(b + o_counts);
+    h->offsets = reinterpret_cast<int32_t *>(b + o_offsets);
+    h->tile_off = reinterpret_cast<int32_t *>(b + o_tile);
+    h->pair_row = reinterpret_cast<int32_t *>(b + o_prow);
+    h->row_pair = reinterpret_cast<int32_t *>(b + o_rpair);
+    h->xp = reinterpret_cast<__nv_bfloat16 *>(b + o_xp);
+    h->hbuf = reinterpret_cast<__nv_bfloat16 *>(b + o_h);
+    h->ybuf = reinterpret_cast<float *>(b + o_y);
+    h->status = reinterpret_cast<int *>(b + o_status);
+    h->x_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_xs);
+    h->out_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_os);
+    h->res_stage = reinterpret_cast<float *>(b + o_rs);
+    e = cudaMemset(h->status, 0, sizeof(int));
+    if (e == cudaSuccess) e = prepare_grouped_gemm(n_experts);
+    if (e == cudaSuccess) e = prepare_dispatch(n_experts);
+    if (e != cudaSuccess) {
+        int rc = cuda_fail(nullptr, e, "workspace / kernel set-up");
+        cudaFree(h->ws);
+        delete h;
+        return rc;
+    }
+
+    bool ok = make_map(&h->tm_gate, w_gate, E * inter, hidden, 128) &&
+              make_map(&h->tm_up, w_up, E * inter, hidden, 128) &&
+              make_map(&h->tm_down, w_down, E * hidden, inter, 128);
+    const uint32_t boxes[4] = {16, 32, 64, 128};
+    for (int i = 0; i < 4 && ok; ++i)
+        ok = make_map(&h->tm_xp[i], h->xp, P, hidden, boxes[i]) &&
+             make_map(&h->tm_h[i], h->hbuf, P, inter, boxes[i]);
+    if (!ok) {
+        cudaFree(h->ws);
+        delete h;
+        return fail(nullptr, BEAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    }
+    *out = h;
+    return BEAM_OK;
+}
+
+int beam_moe_route(beam_moe_t h, void *stream, const void *x, int T, int32_t *topk_idx,
+                   float *topk_w)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    h->err[0] = 0;
+    int rc = check_tokens(h, x, T);
+    if (rc != BEAM_OK) return rc;
+    if (T == 0) return BEAM_OK;
+    if (!topk_idx || !topk_w) return fail(h, BEAM_ERR_INVALID_ARG, "output pointer is NULL");
+    if ((rc = check_device(h)) != BEAM_OK) return rc;
+    return run_router(h, static_cast<cudaStream_t>(stream), x, T, topk_idx, topk_w, nullptr);
+}
+
+int beam_moe_router_logits(beam_moe_t h, void *stream, const void *x, int T, float *logits)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    h->err[0] = 0;
+    int rc = check_tokens(h, x, T);
+    if (rc != BEAM_OK) return rc;
+    if (T == 0) return BEAM_OK;
+    if (!logits) return fail(h, BEAM_ERR_INVALID_ARG, "logits is NULL");
+    if ((rc = check_device(h)) != BEAM_OK) return rc;
+    return run_router(h, static_cast<cudaStream_t>(stream), x, T, h->idx, h->w, logits);
+}
+
+int beam_moe_forward(beam_moe_t h, void *stream, const void *x, int T, void *out,
+                     float *residual, int k)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    h->err[0] = 0;
+    int rc = check_tokens(h, x, T);
+    if (rc != BEAM_OK) return rc;
+    if (!out && !residual) return fail(h, BEAM_ERR_INVALID_ARG, "out and residual are both NULL");
+    if ((out && !aligned16(out)) || (residual && !aligned16(residual)))
+        return fail(h, BEAM_ERR_INVALID_ARG, "out / residual must be 16-byte aligned");
+    if (residual && k < 1) return fail(h, BEAM_ERR_INVALID_ARG, "residual step k must be >= 1");
+    if (T == 0) return BEAM_OK;
+    if ((rc = check_device(h)) != BEAM_OK) return rc;
+    return run_forward(h, static_cast<cudaStream_t>(stream), x, T, out, residual, k);
+}
+
+int beam_moe_forward_host(beam_moe_t h, void *stream, const void *x_host, int T, void *out_host,
+                          float *residual_host, int k)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    h->err[0] = 0;
+    if (T < 0 || T > h->max_tokens)
+        return fail(h, BEAM_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->max_tokens);
+    if (!out_host && !residual_host)
+        return fail(h, BEAM_ERR_INVALID_ARG, "out_host and residual_host are both NULL");
+    if (T > 0 && !x_host) return fail(h, BEAM_ERR_INVALID_ARG, "x_host is NULL");
+    if (residual_host && k < 1) return fail(h, BEAM_ERR_INVALID_ARG, "residual step k must be >= 1");
+    if (T == 0) return BEAM_OK;
+    int rc = check_device(h);
+    if (rc != BEAM_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = (size_t)T * h->H;
+    cudaError_t e = cudaMemcpyAsync(h->x_stage, x_host, n * 2, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && residual_host)
+        e = cudaMemcpyAsync(h->res_stage, residual_host, n * 4, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "host-to-device copy");
+    rc = run_forward(h, s, h->x_stage, T, out_host ? h->out_stage : nullptr,
+                     residual_host ? h->res_stage : nullptr, k);
+    if (rc != BEAM_OK) return rc;
+    if (out_host) e = cudaMemcpyAsync(out_host, h->out_stage, n * 2, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess && residual_host)
+        e = cudaMemcpyAsync(residual_host, h->res_stage, n * 4, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "device-to-host copy");
+}
+
+int beam_moe_dispatch_info(beam_moe_t h, void *stream, int T, int32_t *counts_host,
+                           int32_t *offsets_host, int32_t *pair_row_host)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    h->err[0] = 0;
+    if (T != h->last_T || T <= 0)
+        return fail(h, BEAM_ERR_INVALID_ARG, "T=%d is not the T of the last forward pass (%d)", T,
+                    h->last_T);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (counts_host)
+        e = cudaMemcpyAsync(counts_host, h->counts, sizeof(int32_t) * h->E, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess && offsets_host)
+        e = cudaMemcpyAsync(offsets_host, h->offsets, sizeof(int32_t) * (h->E + 1),
+                            cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess && pair_row_host)
+        e = cudaMemcpyAsync(pair_row_host, h->pair_row, sizeof(int32_t) * (size_t)T * h->top_k,
+                            cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "dispatch info copy");
+}
+
+int beam_moe_get_status(beam_moe_t h, void *stream)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && v != 0) e = cudaMemset(h->status, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(h, e, "status read");
+    if (v != 0) fail(h, v, "device-side wait ran out (status %d)", v);
+    return v;
+}
+
+int beam_moe_set_wait_limit(beam_moe_t h, int64_t limit_ns)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    if (limit_ns < 1000) return fail(h, BEAM_ERR_INVALID_ARG, "wait limit below 1000 ns");
+    h->wait_limit_ns = limit_ns;
+    return BEAM_OK;
+}
+
+static void prof_release(beam_moe *h)
+{
+    for (cudaEvent_t ev : h->prof_events) cudaEventDestroy(ev);
+    h->prof_events.clear();
+    h->prof_max = h->prof_calls = 0;
+}
+
+int beam_moe_profile_begin(beam_moe_t h, int max_calls)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    if (max_calls < 1 || max_calls > 100000)
+        return fail(h, BEAM_ERR_INVALID_ARG, "max_calls outside [1, 100000]");
+    int rc = check_device(h);
+    if (rc != BEAM_OK) return rc;
+    prof_release(h);
+    h->prof_events.resize((size_t)max_calls * 6);
+    for (auto &ev : h->prof_events) {
+        cudaError_t e = cudaEventCreate(&ev);
+        if (e != cudaSuccess) {
+            ev = nullptr;
+            prof_release(h);
+            return cuda_fail(h, e, "cudaEventCreate");
+        }
+    }
+    h->prof_max = max_calls;
+    h->prof_calls = 0;
+    return BEAM_OK;
+}
+
+int beam_moe_profile_end(beam_moe_t h, float *stage_ms, int *calls)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    if (!stage_ms || !calls) return fail(h, BEAM_ERR_INVALID_ARG, "output pointer is NULL");
+    for (int i = 0; i < 5; ++i) stage_ms[i] = 0.f;
+    *calls = h->prof_calls;
+    if (h->prof_calls > 0) {
+        cudaError_t e = cudaEventSynchronize(h->prof_events[(size_t)h->prof_calls * 6 - 1]);
+        for (int c = 0; c < h->prof_calls && e == cudaSuccess; ++c)
+            for (int i = 0; i < 5 && e == cudaSuccess; ++i) {
+                float ms = 0.f;
+                e = cudaEventElapsedTime(&ms, h->prof_events[(size_t)c * 6 + i],
+                                         h->prof_events[(size_t)c * 6 + i + 1]);
+                stage_ms[i] += ms;
+            }
+        if (e != cudaSuccess) {
+            prof_release(h);
+            return cuda_fail(h, e, "profile events");
+        }
+    }
+    prof_release(h);
+    return BEAM_OK;
+}
+
+int beam_moe_set_gemm_ctas(beam_moe_t h, int ctas)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    if (ctas < 0 || ctas > 65535) return fail(h, BEAM_ERR_INVALID_ARG, "ctas outside [0, 65535]");
+    h->gemm_ctas = ctas;
+    return BEAM_OK;
+}
+
+int beam_moe_check_wait_timeout(beam_moe_t h, void *stream)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    int rc = check_device(h);
+    if (rc != BEAM_OK) return rc;
+    WaitCtl ctl;
+    ctl.status = h->status;
+    ctl.limit_ns = h->wait_limit_ns;
+    cudaError_t e = launch_wait_timeout_check(ctl, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(h, e, "self-check launch");
+    return beam_moe_get_status(h, stream);
+}
+
+const char *beam_moe_last_error(beam_moe_t h) { return h ? h->err : g_create_err; }
+
+int beam_moe_destroy(beam_moe_t h)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != h->device) cudaSetDevice(h->device);
+    cudaError_t e = cudaDeviceSynchronize();
+    prof_release(h);
+    if (h->ws) cudaFree(h->ws);
+    if (prev >= 0 && prev != h->device) cudaSetDevice(prev);
+    delete h;
+    return e == cudaSuccess ? BEAM_OK : BEAM_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+// Launch interfaces of the Beam MoE kernels (host side).
+#pragma once
+
+#include "common.cuh"
+
+namespace beam {
+
+// ----------------------------------------------------------------- router
+struct RouterArgs {
+    const __nv_bfloat16 *x;   // [T, H]
+    const float *router_w;    // [E, H]
+    const float *bias;        // [E]
+    int T, H, E, n_group, topk_group, top_k;
+    int nslice;               // K slices of the logits (router_slices)
+    float *partial;           // [nslice, T, E] workspace
+    int32_t *idx;             // [T, top_k]
+    float *w;                 // [T, top_k]
+    float *logits_out;        // [T, E] or nullptr
+};
+int router_slices(int T, int H, int E, int num_sms);
+cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream);
+
+// --------------------------------------------------------------- dispatch
+constexpr int kDispatchBlock = 1024;   // pairs per counting block
+
+struct DispatchArgs {
+    const int32_t *idx;          // [P] expert of pair p = t*top_k + j
+    const __nv_bfloat16 *x;      // [T, H]
+    int T, H, E, top_k;
+    int tile_rows;               // token rows per GEMM tile (BN)
+    int32_t *block_cnt;          // [nblk, E]
+    int32_t *block_base;         // [nblk, E]
+    int32_t *rank;               // [P] rank of the pair among its block's pairs of that expert
+    int32_t *counts;             // [E]
+    int32_t *offsets;            // [E+1]
+    int32_t *tile_off;           // [E+1] prefix of ceil(counts/BN)
+    int32_t *pair_row;           // [P]
+    int32_t *row_pair;           // [P]
+    __nv_bfloat16 *xp;           // [P, H] expert-sorted activations
+};
+cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t stream);
+cudaError_t prepare_dispatch(int E);   // shared-memory limit of the counting kernel
+
+// ----------------------------------------------------------- grouped GEMM
+struct GemmArgs {
+    int K;                       // reduction length
+    int R;                       // weight rows per expert (multiple of 128)
+    int E;
+    const int32_t *counts;       // [E]
+    const int32_t *offsets;      // [E+1]
+    const int32_t *tile_off;     // [E+1]
+    void *out;                   // SwiGLU: bf16 [P, R]; plain: fp32 [P, R]
+    WaitCtl ctl;
+};
+// Gate|up GEMM with the SwiGLU epilogue (two A maps) or the down GEMM
+// (one A map, fp32 output), BN token rows per tile.
+cudaError_t launch_grouped_gemm(bool swiglu, int BN, const CUtensorMap &a0, const CUtensorMap &a1,
+                                const CUtensorMap &b, const GemmArgs &args, int grid,
+                                cudaStream_t stream);
+cudaError_t prepare_grouped_gemm(int E);   // sets shared-memory limits once per device
+bool gemm_tile_supported(int BN);
+
+// ---------------------------------------------------------------- combine
+struct CombineArgs {
+    const float *y;              // [P, H] expert outputs, fp32
+    const int32_t *pair_row;     // [P]
+    const float *w;              // [T, top_k]
+    int T, H, top_k;
+    float scaling;
+    __nv_bfloat16 *out;          // [T, H] or nullptr
+    float *residual;             // [T, H] or nullptr
+    const float *gamma;          // [H] or nullptr
+    float eps;
+    float keep, add;             // sqrt((k-1)/k), 1/sqrt(k)
+};
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream);
+
+// ------------------------------------------------------------- self-check
+cudaError_t launch_wait_timeout_check(WaitCtl ctl, cudaStream_t stream);
+
+}  // namespace beam

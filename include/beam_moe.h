@@ -1,0 +1,212 @@
+/*
+ * beam_moe.h -- C ABI of the Beam sparse mixture-of-experts block (forward
+ * pass) on NVIDIA B200 (sm_100a).
+ *
+ * The block, as the Beam pages define it:
+ *   - router: sigmoid scores over all experts, computed in FP32 from FP32
+ *     router weights; a learned per-expert bias is added for selection; the
+ *     experts form n_group groups, a group's score is the sum of its two best
+ *     biased scores, the topk_group best groups are kept and the top_k best
+ *     experts inside them are chosen (launch blog "Introducing Beam", section
+ *     "Mixture of Experts"; transformers page "Beam", section "Overview",
+ *     "Sparse MoE" bullet and the paragraph on FP32 router weights and bias);
+ *   - each chosen expert is a SwiGLU MLP, down(silu(gate x) * up x), with the
+ *     SwiGLU product in FP32 (launch blog, sections "Mixture of Experts" and
+ *     "Residual Stream");
+ *   - the expert outputs are combined with the normalised router weights and
+ *     scaled by routed_scaling (2.5 for Beam);
+ *   - optionally, the post-sub-layer RMSNorm ("sandwich" norm) and the
+ *     depth-scaled residual update of step k:
+ *         stream <- sqrt((k-1)/k) * stream + norm(out) / sqrt(k)
+ *     (launch blog, section "Residual Stream"; transformers page, "Overview",
+ *     depth-scaled residual bullet).
+ * Conventions the pages leave open, fixed here: the bias steers selection
+ * only; a group's score uses the biased scores; the combine weights are the
+ * unbiased sigmoid scores of the chosen experts divided by their sum; ties go
+ * to the lower group / expert index.
+ *
+ * Memory.  Every tensor argument is a DEVICE pointer unless its name ends in
+ * _host.  The caller owns all of them.  Weights are borrowed by the handle and
+ * must stay valid and unchanged until beam_moe_destroy.  The handle owns only
+ * its workspace (sized by max_tokens at create time) and its TMA descriptors.
+ * Device pointers must be 16-byte aligned.  Layouts are row-major, C order.
+ *
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL: the legacy
+ * default stream).  Calls are stream-ordered and asynchronous unless stated:
+ * the host does not wait.  A handle's workspace is shared by its calls, so a
+ * handle must not be used on two streams concurrently.
+ *
+ * Errors.  Every call validates its arguments on the host first and returns a
+ * negative beam_status without launching anything when they are invalid.
+ * Device-side failures (a bounded wait inside a kernel that ran out) set a
+ * sticky status word in the handle; beam_moe_get_status reads and clears it.
+ * beam_moe_last_error returns a text for the last host-side error.
+ */
+#ifndef BEAM_MOE_H
+#define BEAM_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct beam_moe *beam_moe_t;
+
+typedef enum {
+    BEAM_OK = 0,
+    BEAM_ERR_INVALID_ARG = -1, /* bad shape, pointer, size or alignment       */
+    BEAM_ERR_UNSUPPORTED = -2, /* valid for the method, not for these kernels */
+    BEAM_ERR_CUDA = -3,        /* a CUDA runtime / driver call failed          */
+    BEAM_ERR_OOM = -4,         /* workspace allocation failed                  */
+    BEAM_ERR_TIMEOUT = -5      /* a bounded device-side wait ran out           */
+} beam_status;
+
+/*
+ * Create a handle for one MoE block.
+ *
+ * hidden        H, hidden size (Beam: 5120).  Must be a multiple of 128.
+ * n_experts     E (Beam: 256).  Must be a multiple of 32 and at most 1024.
+ * inter         I, expert intermediate size (Beam: 2560).  Multiple of 128.
+ * n_group       number of expert groups (Beam: 8); E % n_group == 0, the
+ *               group size E/n_group must be >= 2.
+ * topk_group    groups kept per token (Beam: 4); 1 <= topk_group <= n_group.
+ * top_k         experts chosen per token (Beam: 8);
+ *               1 <= top_k <= min(32, topk_group * E / n_group).
+ * routed_scaling  scale applied to the combined output (Beam: 2.5).
+ * router_w      fp32 [E, H]: logit_e = x . router_w[e].
+ * expert_bias   fp32 [E]: added to the sigmoid scores for selection only.
+ * w_gate        bf16 [E, I, H]: gate projection of every expert.
+ * w_up          bf16 [E, I, H]: up projection.
+ * w_down        bf16 [E, H, I]: down projection.
+ * post_norm_w   fp32 [H] RMSNorm weight applied to the block output before
+ *               the residual update, or NULL for no norm.
+ * norm_eps      RMSNorm epsilon (Beam: 1e-6); ignored without post_norm_w.
+ * max_tokens    largest T any call on this handle will pass (>= 1); sizes
+ *               the workspace (about T*top_k*(4H + 2I) + T*(4H) bytes).
+ * Kernel-side shape limits (else BEAM_ERR_UNSUPPORTED): E/32 experts per
+ * lane in {1, 2, 4, 8, 16, 32}, group size a multiple of E/32 with
+ * (group size)/(E/32) a power of two, n_group <= 32.
+ * On success *out receives the handle.  Allocates device memory; launches no
+ * kernel.  The current CUDA device at create time is the handle's device.
+ */
+int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n_group,
+                    int topk_group, int top_k, float routed_scaling, const float *router_w,
+                    const float *expert_bias, const void *w_gate, const void *w_up,
+                    const void *w_down, const float *post_norm_w, float norm_eps,
+                    int max_tokens);
+
+/*
+ * Route T tokens: the router step alone.
+ * x         bf16 [T, H].
+ * topk_idx  int32 [T, top_k] (out): chosen experts, in descending biased
+ *           score, ties to the lower index.
+ * topk_w    fp32 [T, top_k] (out): the chosen experts' unbiased sigmoid
+ *           scores divided by their sum (sum to 1; routed_scaling not
+ *           applied).
+ * 0 <= T <= max_tokens; T == 0 returns BEAM_OK and launches nothing.
+ */
+int beam_moe_route(beam_moe_t h, void *stream, const void *x, int T, int32_t *topk_idx,
+                   float *topk_w);
+
+/*
+ * Router logits for T tokens, x . router_w^T in FP32 (the quantity the
+ * transformers page returns with output_router_logits=True).
+ * logits    fp32 [T, E] (out).
+ */
+int beam_moe_router_logits(beam_moe_t h, void *stream, const void *x, int T, float *logits);
+
+/*
+ * Forward pass of the block for T tokens.
+ * x         bf16 [T, H].
+ * out       bf16 [T, H] (out): routed_scaling * sum_j w_j * expert_j(x),
+ *           rounded to nearest even; may be NULL when residual is given.
+ * residual  fp32 [T, H] (in/out) or NULL.  When given, the block output o
+ *           (fp32, before rounding) is normalised with post_norm_w if the
+ *           handle has one, n = o / sqrt(mean(o^2) + eps) * post_norm_w,
+ *           else n = o; then residual <- sqrt((k-1)/k) * residual + n/sqrt(k).
+ * k         residual step (>= 1); ignored without residual.
+ * out and residual must not both be NULL.  0 <= T <= max_tokens.
+ */
+int beam_moe_forward(beam_moe_t h, void *stream, const void *x, int T, void *out,
+                     float *residual, int k);
+
+/*
+ * beam_moe_forward with HOST buffers: copies x_host (and residual_host) to
+ * the handle's device staging buffers, runs the forward pass and copies the
+ * results back, all on `stream`, then waits for the stream.  Pinned host
+ * memory gives asynchronous copies; pageable memory works too.
+ * x_host bf16 [T, H]; out_host bf16 [T, H] or NULL; residual_host fp32
+ * [T, H] (in/out) or NULL.  Synchronous: returns after the results landed.
+ */
+int beam_moe_forward_host(beam_moe_t h, void *stream, const void *x_host, int T,
+                          void *out_host, float *residual_host, int k);
+
+/*
+ * Dispatch bookkeeping of the last forward pass on this handle (for checks):
+ * copies to HOST buffers, after synchronising `stream`.
+ * counts_host   int32 [E]: tokens routed to each expert.
+ * offsets_host  int32 [E+1]: exclusive prefix sum of counts.
+ * pair_row_host int32 [T*top_k]: row of (token t, slot j) = pair t*top_k+j in
+ *               the expert-sorted activation buffer; rows of one expert are
+ *               contiguous and ordered by pair index.
+ * T must equal the T of that forward pass.  Any pointer may be NULL.
+ */
+int beam_moe_dispatch_info(beam_moe_t h, void *stream, int T, int32_t *counts_host,
+                           int32_t *offsets_host, int32_t *pair_row_host);
+
+/*
+ * Synchronise `stream`, then return and clear the device status word:
+ * BEAM_OK, or BEAM_ERR_TIMEOUT when a bounded in-kernel wait ran out since
+ * the last call.  While the word is set, kernels of this handle stop at
+ * their next wait, so results of calls made meanwhile are not valid.
+ */
+int beam_moe_get_status(beam_moe_t h, void *stream);
+
+/*
+ * Set the limit of every in-kernel wait of this handle, in nanoseconds
+ * (default 2e9).  Values < 1000 are rejected.
+ */
+int beam_moe_set_wait_limit(beam_moe_t h, int64_t limit_ns);
+
+/*
+ * Number of CTAs of the persistent grouped-GEMM kernels (0 = one per SM, the
+ * default).  Fewer CTAs put more work items on each CTA; results do not
+ * depend on it.  0 <= ctas <= 65535.
+ */
+int beam_moe_set_gemm_ctas(beam_moe_t h, int ctas);
+
+/*
+ * Per-stage timing of forward passes, for measurement.  After
+ * beam_moe_profile_begin(h, max_calls), each of the next max_calls forward
+ * passes records CUDA events on its stream around its five stages: router,
+ * dispatch, gate|up GEMM, down GEMM, combine.  beam_moe_profile_end waits for
+ * the last recorded event, writes the summed milliseconds of each stage to
+ * stage_ms (fp32 [5], host) and the number of timed passes to *calls (host),
+ * and stops recording.  Synchronous; allocates no device memory.
+ */
+int beam_moe_profile_begin(beam_moe_t h, int max_calls);
+int beam_moe_profile_end(beam_moe_t h, float *stage_ms, int *calls);
+
+/*
+ * Failure-detection check: launch one kernel that waits, with the handle's
+ * wait limit, on a barrier that nothing completes; it must give up, record
+ * BEAM_ERR_TIMEOUT in the status word and return.  Returns the status word
+ * as beam_moe_get_status does.  Synchronous.
+ */
+int beam_moe_check_wait_timeout(beam_moe_t h, void *stream);
+
+/* Text of the last host-side error on this handle ("" if none). */
+const char *beam_moe_last_error(beam_moe_t h);
+
+/* Text of the last error of a beam_moe_create call that returned no handle. */
+const char *beam_moe_create_error(void);
+
+/* Free the workspace and the handle.  Synchronises the handle's device. */
+int beam_moe_destroy(beam_moe_t h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BEAM_MOE_H */

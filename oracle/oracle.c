@@ -230,10 +230,12 @@ void oracle_expert_swiglu(int n, int H, int I, const uint16_t *x,
                           const uint16_t *w_gate, const uint16_t *w_up,
                           const uint16_t *w_down, double *y, uint16_t *h_out)
 {
-#pragma omp parallel for schedule(dynamic, 1)
+    double *hv = (double *)malloc(sizeof(double) * (size_t)I);
     for (int r = 0; r < n; ++r) {
         const uint16_t *xr = x + (size_t)r * H;
-        double *hv = (double *)malloc(sizeof(double) * (size_t)I);
+        /* every output element is one sequential sum; the threads split the
+         * independent outputs, never a sum */
+#pragma omp parallel for schedule(static)
         for (int i = 0; i < I; ++i) {
             const uint16_t *wg = w_gate + (size_t)i * H;
             const uint16_t *wu = w_up + (size_t)i * H;
@@ -248,14 +250,15 @@ void oracle_expert_swiglu(int n, int H, int I, const uint16_t *x,
             hv[i] = oracle_bf16_to_double(hb);
             if (h_out) h_out[(size_t)r * I + i] = hb;
         }
+#pragma omp parallel for schedule(static)
         for (int h = 0; h < H; ++h) {
             const uint16_t *wd = w_down + (size_t)h * I;
             double acc = 0.0;
             for (int i = 0; i < I; ++i) acc += hv[i] * oracle_bf16_to_double(wd[i]);
             y[(size_t)r * H + h] = acc;
         }
-        free(hv);
     }
+    free(hv);
 }
 
 /* ------------------------------------------------------------------ */

@@ -1,0 +1,154 @@
+"""Parity harness: the CUDA path (through the C ABI binding) against the CPU
+oracle on the same seeded inputs.
+
+Tolerances (the block's stated bar):
+  * expert indices bit-exact, except tokens whose oracle biased-score gap
+    between the k-th and (k+1)-th candidate, or between the 4th and 5th group
+    score, is below 1e-6 (exempt, counted);
+  * outputs: relative Frobenius error <= 5e-3 and max abs error <= 2e-2 x
+    the RMS of the oracle output.  Both sides round to bf16; where the two
+    bf16 values are neighbours (at most one bf16 ulp of the oracle value
+    apart) the pair is a rounding-boundary case -- two valid roundings of
+    values that differ by far less than the tolerance -- and it is counted
+    (``ulp_neighbours``) rather than held to the max-abs bound.  At 5 sigma one
+    bf16 ulp is already ~2e-2 x RMS, so without this any large sample would
+    fail on correct roundings.  The Frobenius bound covers every element;
+  * combine weights (before x routed_scaling): max abs error <= 1e-5.
+With a residual stream, the update's contribution
+    stream_out - sqrt((k-1)/k) * stream_in
+is compared with the oracle's n / sqrt(k) under the output tolerances.
+"""
+from __future__ import annotations
+
+import math
+import time
+from dataclasses import dataclass, field
+from typing import Optional
+
+import numpy as np
+import torch
+
+import oracle
+from group_limited_routing_sigmoid_b200 import workloads as W
+
+NEAR_TIE = 1e-6
+REL_FRO = 5e-3
+MAX_ABS_RMS = 2e-2
+W_ABS = 1e-5
+
+
+@dataclass
+class Report:
+    tokens: int = 0
+    exempt: int = 0
+    idx_mismatch: int = 0
+    set_mismatch: int = 0
+    w_max_err: float = 0.0
+    rel_fro: float = 0.0
+    max_abs_over_rms: float = 0.0
+    max_abs_over_rms_raw: float = 0.0
+    ulp_neighbours: int = 0
+    res_rel_fro: Optional[float] = None
+    res_max_abs_over_rms: Optional[float] = None
+    oracle_seconds: float = 0.0
+    notes: list = field(default_factory=list)
+
+    def ok(self) -> bool:
+        good = (self.idx_mismatch == 0 and self.w_max_err <= W_ABS and self.rel_fro <= REL_FRO
+                and self.max_abs_over_rms <= MAX_ABS_RMS)
+        if self.res_rel_fro is not None:
+            good = good and self.res_rel_fro <= REL_FRO and self.res_max_abs_over_rms <= MAX_ABS_RMS
+        return good
+
+
+def errors(got: np.ndarray, ref: np.ndarray):
+    d = got.astype(np.float64) - ref.astype(np.float64)
+    rms = math.sqrt(float((ref.astype(np.float64) ** 2).mean()))
+    rel = float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-300))
+    mx = float(np.abs(d).max() / max(rms, 1e-300)) if d.size else 0.0
+    return rel, mx
+
+
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values at |v| (8-bit significand, binary32 exponents)."""
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def bf16_errors(got: np.ndarray, ref: np.ndarray):
+    """(rel_fro, max_abs/rms over non-neighbour pairs, raw max_abs/rms, neighbours)."""
+    rel, raw = errors(got, ref)
+    d = np.abs(got - ref)
+    neighbour = (d > 0) & (d <= bf16_ulp(ref) * (1 + 1e-12))
+    rms = math.sqrt(float((ref ** 2).mean()))
+    rest = d[~neighbour]
+    mx = float(rest.max() / max(rms, 1e-300)) if rest.size else 0.0
+    return rel, mx, raw, int(neighbour.sum())
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return oracle.bf16_to_f64(W.bf16_bits(t))
+
+
+def check_block(wl: W.Workload, d: dict, moe, sample: Optional[torch.Tensor] = None,
+                T: Optional[int] = None) -> Report:
+    """Run the CUDA forward (and route) on d['x'][:T] and compare the sampled
+    tokens with the oracle."""
+    x = d["x"] if T is None else d["x"][:T]
+    T = x.shape[0]
+    dev = x.device
+    rep = Report()
+    stream_in = None
+    out = None
+    if wl.residual_k:
+        stream_in = d["stream"][:T].clone()
+        stream_dev = stream_in.clone()
+        out = moe.forward(x, residual=stream_dev, k=wl.residual_k)
+    else:
+        out = moe.forward(x)
+    idx_g, w_g = moe.route(x)
+    torch.cuda.synchronize(dev)
+    assert moe.get_status() == 0, "device-side wait ran out"
+
+    if sample is None:
+        sample = torch.arange(T)
+    sample = sample[sample < T]
+    s_dev = sample.to(dev)
+    xs_bits = W.bf16_bits(x.index_select(0, s_dev))
+    router_w = d["router_w"].cpu().numpy()
+    bias = d["bias"].cpu().numpy()
+    gamma = None if d.get("gamma") is None else d["gamma"].cpu().numpy()
+
+    def fetch(e):
+        return (W.bf16_bits(d["w_gate"][e]), W.bf16_bits(d["w_up"][e]), W.bf16_bits(d["w_down"][e]))
+
+    t0 = time.time()
+    res = oracle.moe_block(xs_bits, router_w, bias, fetch, wl.n_group, wl.topk_group, wl.top_k,
+                           wl.routed_scaling, gamma=gamma, eps=wl.norm_eps,
+                           stream=None if stream_in is None else stream_in.index_select(0, s_dev).cpu().numpy(),
+                           kstep=wl.residual_k)
+    rep.oracle_seconds = time.time() - t0
+
+    r = res.routing
+    exempt = (r.gap_expert < NEAR_TIE) | (r.gap_group < NEAR_TIE)
+    keep = ~exempt
+    rep.tokens = len(sample)
+    rep.exempt = int(exempt.sum())
+    ig = idx_g.index_select(0, s_dev).cpu().numpy()
+    wg = w_g.index_select(0, s_dev).cpu().numpy()
+    rep.idx_mismatch = int((ig[keep] != r.idx[keep]).any(axis=1).sum())
+    rep.set_mismatch = int(sum(set(a.tolist()) != set(b.tolist()) for a, b in zip(ig[keep], r.idx[keep])))
+    if keep.any():
+        rep.w_max_err = float(np.abs(wg[keep] - r.w[keep]).max())
+        if out is not None:
+            got = bf16_to_f64(out.index_select(0, s_dev))[keep]
+            ref = oracle.bf16_to_f64(res.out)[keep]
+            (rep.rel_fro, rep.max_abs_over_rms, rep.max_abs_over_rms_raw,
+             rep.ulp_neighbours) = bf16_errors(got, ref)
+        if stream_in is not None:
+            keep_f = math.sqrt((wl.residual_k - 1) / wl.residual_k)
+            s_out = stream_dev.index_select(0, s_dev).cpu().double().numpy()
+            s_in = stream_in.index_select(0, s_dev).cpu().double().numpy()
+            delta = (s_out - keep_f * s_in)[keep]
+            rep.res_rel_fro, rep.res_max_abs_over_rms = errors(delta, res.contrib[keep])
+    return rep

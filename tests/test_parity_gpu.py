@@ -1,0 +1,146 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on the seeded workloads.
+
+Small block (H=256, 32 experts): every token, at several T (ragged tails,
+T=1, tiles of 16..128 token rows) and GEMM grid sizes (many work items per
+CTA).  Beam shape (H=5120, 256 experts, I=2560): the decode batch in full;
+the 8192- and 32768-token workloads on a seeded sample of tokens (512 by
+default; BEAM_PARITY_SAMPLE overrides).
+"""
+import dataclasses
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_limited_routing_sigmoid_b200 import workloads as W
+from group_limited_routing_sigmoid_b200.binding import BeamMoE, BEAM_ERR_TIMEOUT
+from group_limited_routing_sigmoid_b200.build import build
+
+from parity import check_block
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build(quiet=True)
+    oracle.build()
+
+
+def _log(name, rep):
+    path = os.environ.get("BEAM_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": name, **dataclasses.asdict(rep)}) + "\n")
+
+
+def _inputs(wl, T=None):
+    g = W.generator(wl, "cuda")
+    d = W.make_weights(wl, "cuda", g)
+    d.update(W.make_tokens(wl, "cuda", g, T=T))
+    return d
+
+
+@pytest.mark.parametrize("T,ctas", [(64, 0), (64, 1), (1, 0), (3, 0), (37, 5), (100, 0),
+                                    (200, 3), (1000, 0), (1000, 2), (4096, 0)])
+def test_tiny_block(T, ctas):
+    wl = W.WORKLOADS["tiny"]
+    d = _inputs(wl, T)
+    moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    if ctas:
+        moe.set_gemm_ctas(ctas)
+    rep = check_block(wl, d, moe)
+    _log(f"tiny_T{T}_ctas{ctas}", rep)
+    assert rep.ok(), rep
+    moe.close()
+
+
+@pytest.mark.parametrize("norm", [True, False])
+def test_tiny_residual(norm):
+    wl = dataclasses.replace(W.WORKLOADS["tiny"], post_norm=norm, residual_k=20)
+    d = _inputs(wl, 300)
+    if not norm:
+        d["gamma"] = None
+    moe = BeamMoE.from_workload(wl, d, max_tokens=300)
+    rep = check_block(wl, d, moe)
+    _log(f"tiny_residual_norm{norm}", rep)
+    assert rep.ok(), rep
+    assert rep.res_rel_fro is not None
+    moe.close()
+
+
+def test_tiny_dispatch_is_a_stable_counting_sort():
+    wl = W.WORKLOADS["tiny"]
+    T = 1000
+    d = _inputs(wl, T)
+    moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    moe.forward(d["x"])
+    idx, _ = moe.route(d["x"])
+    counts, offsets, pair_row = moe.dispatch_info(T)
+    flat = idx.cpu().numpy().reshape(-1)
+    np.testing.assert_array_equal(counts, np.bincount(flat, minlength=wl.n_experts))
+    np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+    order = np.argsort(flat, kind="stable")          # rows: pairs sorted by (expert, pair index)
+    expect = np.empty_like(order)
+    expect[order] = np.arange(order.size)
+    np.testing.assert_array_equal(pair_row, expect)
+    moe.close()
+
+
+def test_tiny_router_logits():
+    wl = W.WORKLOADS["tiny"]
+    d = _inputs(wl)
+    moe = BeamMoE.from_workload(wl, d)
+    got = moe.router_logits(d["x"]).cpu().double().numpy()
+    ref = oracle.bf16_to_f64(W.bf16_bits(d["x"])) @ d["router_w"].cpu().double().numpy().T
+    assert np.abs(got - ref).max() < 1e-5 * max(1.0, np.abs(ref).max())
+    moe.close()
+
+
+def test_empty_batch_is_a_no_op():
+    wl = W.WORKLOADS["tiny"]
+    d = _inputs(wl)
+    moe = BeamMoE.from_workload(wl, d)
+    x0 = d["x"][:0]
+    out = torch.full((0, wl.hidden), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.forward(x0, out=out)
+    moe.route(x0)
+    assert moe.get_status() == 0
+    moe.close()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait on a barrier that nothing completes gives up after the limit,
+    records BEAM_ERR_TIMEOUT and returns; the context stays usable."""
+    wl = W.WORKLOADS["tiny"]
+    d = _inputs(wl)
+    moe = BeamMoE.from_workload(wl, d)
+    moe.set_wait_limit(1_000_000)   # 1 ms
+    assert moe.check_wait_timeout() == BEAM_ERR_TIMEOUT
+    assert moe.get_status() == 0     # read-and-clear
+    moe.set_wait_limit(2_000_000_000)
+    rep = check_block(wl, d, moe)
+    assert rep.ok(), rep
+    moe.close()
+
+
+def _sample(wl):
+    s = W.sample_tokens(wl)
+    n = int(os.environ.get("BEAM_PARITY_SAMPLE", "0") or 0)
+    return s[:n] if n else s
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill", "skewed", "long"])
+def test_beam_shape(name):
+    wl = W.WORKLOADS[name]
+    d = W.make_inputs(wl, "cuda")
+    moe = BeamMoE.from_workload(wl, d)
+    rep = check_block(wl, d, moe, sample=_sample(wl))
+    _log(f"beam_{name}", rep)
+    assert rep.ok(), rep
+    moe.close()
+    del d, moe
+    torch.cuda.empty_cache()
