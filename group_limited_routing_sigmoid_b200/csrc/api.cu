@@ -430,6 +430,7 @@ int beam_moe_forward(beam_moe_t h, void *stream, const void *x, int T, void *out
     h->err[0] = 0;
     int rc = check_tokens(h, x, T);
     if (rc != BEAM_OK) return rc;
+    if (T == 0) return BEAM_OK;
     if (!out && !residual) return fail(h, BEAM_ERR_INVALID_ARG, "out and residual are both NULL");
     if ((out && !aligned16(out)) || (residual && !aligned16(residual)))
         return fail(h, BEAM_ERR_INVALID_ARG, "out / residual must be 16-byte aligned");
@@ -446,6 +447,7 @@ int beam_moe_forward_host(beam_moe_t h, void *stream, const void *x_host, int T,
     h->err[0] = 0;
     if (T < 0 || T > h->max_tokens)
         return fail(h, BEAM_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->max_tokens);
+    if (T == 0) return BEAM_OK;
     if (!out_host && !residual_host)
         return fail(h, BEAM_ERR_INVALID_ARG, "out_host and residual_host are both NULL");
     if (T > 0 && !x_host) return fail(h, BEAM_ERR_INVALID_ARG, "x_host is NULL");
