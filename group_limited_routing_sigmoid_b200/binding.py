@@ -24,7 +24,7 @@ BEAM_ERR_TIMEOUT = -5
 
 # every entry point declared in include/beam_moe.h
 SYMBOLS = (
-    "beam_moe_create", "beam_moe_route", "beam_moe_router_logits", "beam_moe_forward",
+    "beam_moe_create", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_forward",
     "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_get_status",
     "beam_moe_set_wait_limit", "beam_moe_set_gemm_ctas", "beam_moe_profile_begin",
     "beam_moe_profile_end", "beam_moe_check_wait_timeout", "beam_moe_last_error",
@@ -52,6 +52,7 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_create.argtypes = [ctypes.POINTER(P), I, I, I, I, I, I, F, P, P, P, P, P, P, F, I]
         lib.beam_moe_route.argtypes = [P, P, P, I, P, P]
         lib.beam_moe_router_logits.argtypes = [P, P, P, I, P]
+        lib.beam_moe_route_static.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P]
         lib.beam_moe_forward.argtypes = [P, P, P, I, P, P, I]
         lib.beam_moe_forward_host.argtypes = [P, P, P, I, P, P, I]
         lib.beam_moe_dispatch_info.argtypes = [P, P, I, P, P, P]
@@ -88,6 +89,27 @@ def _dev(t: torch.Tensor, dtype, name: str):
         raise TypeError(f"{name}: expected a contiguous CUDA {dtype} tensor, got "
                         f"{t.dtype} on {t.device} (contiguous={t.is_contiguous()})")
     return t
+
+
+def route_static(x: torch.Tensor, router_w: torch.Tensor, expert_bias: torch.Tensor, n_group: int,
+                 topk_group: int, top_k: int, idx: Optional[torch.Tensor] = None,
+                 w: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Routing through beam_moe_route_static: no handle, no device allocation
+    inside the library (its scratch is a fixed device array)."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(router_w, torch.float32, "router_w")
+    _dev(expert_bias, torch.float32, "expert_bias")
+    T, H = x.shape
+    E = router_w.shape[0]
+    if idx is None:
+        idx = torch.empty(T, top_k, dtype=torch.int32, device=x.device)
+    if w is None:
+        w = torch.empty(T, top_k, dtype=torch.float32, device=x.device)
+    rc = library().beam_moe_route_static(_stream(stream), _ptr(x), T, H, E, n_group, topk_group,
+                                         top_k, _ptr(router_w), _ptr(expert_bias), _ptr(idx), _ptr(w))
+    if rc != BEAM_OK:
+        raise BeamMoEError(rc, "beam_moe_route_static rejected the call")
+    return idx, w
 
 
 class BeamMoE:

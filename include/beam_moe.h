@@ -110,6 +110,36 @@ int beam_moe_route(beam_moe_t h, void *stream, const void *x, int T, int32_t *to
                    float *topk_w);
 
 /*
+ * Routing without any device allocation (the Beam pages have no counterpart:
+ * this entry point exists for callers, not for the method).  Callers that
+ * cannot call cudaMalloc -- an inference engine that reserves nearly all GPU
+ * memory for its own pools at start-up, or a latency-critical path that must
+ * not enter the CUDA allocator, whose cudaMalloc / cudaFree can synchronise
+ * the device -- and so cannot create a handle, get the same routing as
+ * beam_moe_route here, with no handle.
+ * Scratch: a fixed 8 MiB device array inside the library (2,097,152 fp32
+ * partial logits), held by every GPU that loads the library until the
+ * process exits.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  All calls on a device share the array, so
+ * calls that overlap on the GPU (different streams, no ordering between them)
+ * race and give undefined results; calls ordered on one stream are safe.
+ * Nothing in the array needs clearing: each call writes every element it
+ * reads.  No cudaMalloc, cudaFree or allocating library call is made.
+ * Arguments as beam_moe_create / beam_moe_route: x bf16 [T, H], router_w fp32
+ * [E, H], expert_bias fp32 [E] (16-byte aligned device pointers), topk_idx
+ * int32 [T, top_k] and topk_w fp32 [T, top_k] (device, out).  hidden must be
+ * a multiple of 32; n_experts, n_group, topk_group, top_k follow the rules of
+ * beam_moe_create.  Returns BEAM_ERR_INVALID_ARG for bad arguments and when
+ * T * n_experts > 2,097,152 (the scratch capacity), BEAM_ERR_UNSUPPORTED for
+ * shapes the kernels do not cover, BEAM_ERR_CUDA if the set-up or the launch
+ * fails.  T == 0 returns BEAM_OK.  Asynchronous on `stream`.
+ */
+int beam_moe_route_static(void *stream, const void *x, int T, int hidden, int n_experts,
+                          int n_group, int topk_group, int top_k, const float *router_w,
+                          const float *expert_bias, int32_t *topk_idx, float *topk_w);
+
+/*
  * Router logits for T tokens, x . router_w^T in FP32 (the quantity the
  * transformers page returns with output_router_logits=True).
  * logits    fp32 [T, E] (out).
