@@ -139,8 +139,23 @@ def dist_env():
     return ws, rank, local
 
 
-def rank_workload(wl: W.Workload, rank: int) -> W.Workload:
-    return wl
+def token_seed(wl: W.Workload, rank: int) -> int:
+    """Seed of a rank's token batches: every rank shares the weights (seed
+    wl.seed) and draws its own tokens."""
+    return wl.seed + 1000 * (rank + 1)
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time (all ranks take this collective step)."""
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, steps: int, T: int, ms_max: float) -> float:
+    """All ranks' tokens over the slowest rank's device time."""
+    return world * steps * T / (ms_max * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -171,7 +186,7 @@ def run_ours(args):
     weights = W.make_weights(wl, dev, g)
     # distinct token batches per rank (weights identical on every rank)
     tg = torch.Generator(device=dev)
-    tg.manual_seed(wl.seed + 1000 * (rank + 1))
+    tg.manual_seed(token_seed(wl, rank))
     batches = [W.make_tokens(wl, dev, tg) for _ in range(TOKEN_BATCHES)]
     if wl.post_norm:
         weights["gamma"] = batches[0]["gamma"]
@@ -217,10 +232,7 @@ def run_ours(args):
     calls, stage_ms = moe.profile_end()
     if moe.get_status() != 0:
         raise SystemExit("a device-side wait ran out during the timed region")
-    t_max = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    ms_max = float(t_max.item())
+    ms_max = max_over_ranks(ms, dist, dev)
 
     # end to end through the host-buffer entry point (pinned buffers)
     x_host = [b["x"].cpu().pin_memory() for b in batches]
@@ -243,10 +255,7 @@ def run_ours(args):
         e2e_step(i)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = torch.tensor([ev0.elapsed_time(ev1)], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
 
     # roofline of the dominant kernel
     pk = peaks()
@@ -254,7 +263,7 @@ def run_ours(args):
     d_mean = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(steps_done)) / steps_done
     P = T * k
     gate_up_ms = stage_ms["gate_up_gemm"] / max(calls, 1)
-    if args.workload in ("decode", "tiny"):
+    if args.workload in ("decode", "tiny", "decode_small"):
         alg_bytes = d_mean * 2 * I * H * 2 + P * H * 2 + P * I * 2
         achieved = alg_bytes / (gate_up_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": "gate_up_gemm (grouped_gemm_kernel<BN,2>)",
@@ -274,7 +283,7 @@ def run_ours(args):
 
     line = {
         "metric": METRIC,
-        "value": round(ws * steps_done * T / (ms_max * 1e-3), 1),
+        "value": round(whole_job_tokens_per_s(ws, steps_done, T, ms_max), 1),
         "unit": "tokens/s",
         "n_gpus": ws,
         "steps": steps_done,
@@ -295,7 +304,7 @@ def run_ours(args):
         "hbm_fraction_whole_step": round(step_bytes / (ms_max / steps_done * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
         "stage_ms": stage_avg,
         "clocks": sampler.report(),
-        "e2e": {"value": round(ws * e2e_steps * T / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(whole_job_tokens_per_s(ws, e2e_steps, T, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0),
                 "d2h_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0)},
         "gpu_launches": KERNELS_PER_FORWARD * steps_done,
@@ -357,7 +366,7 @@ def run_reference(args):
     g = W.generator(wl, dev)
     weights = W.make_weights(wl, dev, g)
     tg = torch.Generator(device=dev)
-    tg.manual_seed(wl.seed + 1000)
+    tg.manual_seed(token_seed(wl, 0))
     x = W.make_tokens(wl, dev, tg)["x"]
     if wl.post_norm:
         weights["gamma"] = 1.0 + 0.02 * torch.randn(wl.hidden, generator=tg, device=dev)

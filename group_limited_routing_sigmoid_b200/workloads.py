@@ -72,6 +72,10 @@ WORKLOADS: Dict[str, Workload] = {
     "skewed": Workload("skewed", T=8192, hot_experts=16, hot_bias=3.0, sample=512, **_BEAM),
     # Beam shape, 32768 tokens, post-MoE RMSNorm + depth-scaled residual at step 20
     "long": Workload("long", T=32768, post_norm=True, residual_k=20, sample=512, **_BEAM),
+    # profiling case: Beam-shaped experts (H=5120, I=2560), only 32 of them
+    # (2.5 GB of weights), 8 tokens: the decode kernels on a few GB of memory
+    "decode_small": Workload("decode_small", T=8, hidden=5120, n_experts=32, n_group=8,
+                             topk_group=4, top_k=8, inter=2560),
 }
 
 
