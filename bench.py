@@ -191,6 +191,7 @@ def run_ours(args):
     if wl.post_norm:
         weights["gamma"] = batches[0]["gamma"]
     moe = BeamMoE.from_workload(wl, weights)
+    moe.set_gemm_tuning(0, args.gemm_tile, args.down_pair)
     outs = [torch.empty(T, H, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     streams = [b["stream"] for b in batches]
 
@@ -404,6 +405,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm-tile", type=int, default=0, help="largest GEMM token tile (0 = auto)")
+    ap.add_argument("--down-pair", type=int, default=-1, help="paired down tiles: -1 auto, 0, 1")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

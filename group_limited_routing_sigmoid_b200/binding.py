@@ -26,7 +26,7 @@ BEAM_ERR_TIMEOUT = -5
 SYMBOLS = (
     "beam_moe_create", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_forward",
     "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_get_status",
-    "beam_moe_set_wait_limit", "beam_moe_set_gemm_ctas", "beam_moe_profile_begin",
+    "beam_moe_set_wait_limit", "beam_moe_set_gemm_tuning", "beam_moe_profile_begin",
     "beam_moe_profile_end", "beam_moe_check_wait_timeout", "beam_moe_last_error",
     "beam_moe_create_error", "beam_moe_destroy",
 )
@@ -58,7 +58,7 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_dispatch_info.argtypes = [P, P, I, P, P, P]
         lib.beam_moe_get_status.argtypes = [P, P]
         lib.beam_moe_set_wait_limit.argtypes = [P, ctypes.c_int64]
-        lib.beam_moe_set_gemm_ctas.argtypes = [P, I]
+        lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I]
         lib.beam_moe_check_wait_timeout.argtypes = [P, P]
         lib.beam_moe_profile_begin.argtypes = [P, I]
         lib.beam_moe_profile_end.argtypes = [P, P, P]
@@ -209,8 +209,9 @@ class BeamMoE:
     def set_wait_limit(self, limit_ns: int):
         self._check(library().beam_moe_set_wait_limit(self._h, int(limit_ns)))
 
-    def set_gemm_ctas(self, ctas: int):
-        self._check(library().beam_moe_set_gemm_ctas(self._h, int(ctas)))
+    def set_gemm_tuning(self, ctas: int = 0, tile_rows: int = 0, down_pair: int = -1):
+        self._check(library().beam_moe_set_gemm_tuning(self._h, int(ctas), int(tile_rows),
+                                                        int(down_pair)))
 
     STAGES = ("router", "dispatch", "gate_up_gemm", "down_gemm", "combine")
 

@@ -38,7 +38,9 @@ struct beam_moe {
     float *res_stage;
 
     CUtensorMap tm_gate, tm_up, tm_down;
-    CUtensorMap tm_xp[4], tm_h[4];   // box rows 16, 32, 64, 128
+    BoxMaps tm_xp, tm_h;             // box rows 16, 32, 64, 128, 256
+    int tile_rows;                   // 0: chosen from T
+    int down_pair;                   // -1: auto, 0: single tiles, 1: paired tiles
     int last_T;
     std::vector<cudaEvent_t> prof_events;   // 6 per profiled forward pass
     int prof_max, prof_calls;
@@ -102,17 +104,16 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uin
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int tile_index(int BN) { return BN == 16 ? 0 : BN == 32 ? 1 : BN == 64 ? 2 : 3; }
-
-// Token rows per GEMM tile from the mean load per expert (the host never
-// reads the routing, so the choice depends on T only).
+// Largest token tile of the GEMMs from the mean load per expert (the host
+// never reads the routing, so the choice depends on T only).
 int choose_tile_rows(int T, int top_k, int E)
 {
     const double mean = (double)T * top_k / E;
     if (mean <= 24) return 16;
     if (mean <= 48) return 32;
     if (mean <= 96) return 64;
-    return 128;
+    if (mean <= 160) return 128;
+    return 256;
 }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -165,7 +166,7 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     int rc = run_router(h, s, x, T, h->idx, h->w, nullptr);
     if (rc != BEAM_OK) return rc;
     prof_mark(h, s, 1);
-    const int BN = choose_tile_rows(T, h->top_k, h->E);
+    const int BN = h->tile_rows ? h->tile_rows : choose_tile_rows(T, h->top_k, h->E);
     DispatchArgs d;
     d.idx = h->idx;
     d.x = static_cast<const __nv_bfloat16 *>(x);
@@ -194,18 +195,23 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.tile_off = h->tile_off;
     g.ctl.status = h->status;
     g.ctl.limit_ns = h->wait_limit_ns;
-    const int ti = tile_index(BN);
     g.K = h->H;
     g.R = h->I;
     g.out = h->hbuf;
+
     const int grid = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
-    e = launch_grouped_gemm(true, BN, h->tm_gate, h->tm_up, h->tm_xp[ti], g, grid, s);
+    e = launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_xp, g, grid, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "gate/up GEMM launch");
     prof_mark(h, s, 3);
     g.K = h->I;
     g.R = h->H;
     g.out = h->ybuf;
-    e = launch_grouped_gemm(false, BN, h->tm_down, h->tm_down, h->tm_h[ti], g, grid, s);
+
+    // pair the down projection's weight tiles when H allows; a lone 128-row
+    // tile per item for decode-sized token tiles keeps more items in flight
+    const bool pair = h->H % 256 == 0 && (h->down_pair == 1 || (h->down_pair < 0 && BN >= 64));
+    e = launch_grouped_gemm(pair ? GemmKind::kDownPaired : GemmKind::kDown, BN, h->tm_down,
+                            h->tm_down, h->tm_h, g, grid, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "down GEMM launch");
     prof_mark(h, s, 4);
 
@@ -304,6 +310,7 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     h->eps = norm_eps;
     h->max_tokens = max_tokens;
     h->wait_limit_ns = 2000000000LL;
+    h->down_pair = -1;
 
     cudaError_t e = cudaGetDevice(&h->device);
     if (e == cudaSuccess)
@@ -385,10 +392,9 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     bool ok = make_map(&h->tm_gate, w_gate, E * inter, hidden, 128) &&
               make_map(&h->tm_up, w_up, E * inter, hidden, 128) &&
               make_map(&h->tm_down, w_down, E * hidden, inter, 128);
-    const uint32_t boxes[4] = {16, 32, 64, 128};
-    for (int i = 0; i < 4 && ok; ++i)
-        ok = make_map(&h->tm_xp[i], h->xp, P, hidden, boxes[i]) &&
-             make_map(&h->tm_h[i], h->hbuf, P, inter, boxes[i]);
+    for (int i = 0; i < 5 && ok; ++i)
+        ok = make_map(&h->tm_xp.m[i], h->xp, P, hidden, 16u << i) &&
+             make_map(&h->tm_h.m[i], h->hbuf, P, inter, 16u << i);
     if (!ok) {
         cudaFree(h->ws);
         delete h;
@@ -567,11 +573,17 @@ int beam_moe_profile_end(beam_moe_t h, float *stage_ms, int *calls)
     return BEAM_OK;
 }
 
-int beam_moe_set_gemm_ctas(beam_moe_t h, int ctas)
+int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
     if (ctas < 0 || ctas > 65535) return fail(h, BEAM_ERR_INVALID_ARG, "ctas outside [0, 65535]");
+    if (tile_rows != 0 && !gemm_tile_supported(tile_rows))
+        return fail(h, BEAM_ERR_INVALID_ARG, "tile_rows must be 0, 16, 32, 64, 128 or 256");
+    if (down_pair < -1 || down_pair > 1)
+        return fail(h, BEAM_ERR_INVALID_ARG, "down_pair outside [-1, 1]");
     h->gemm_ctas = ctas;
+    h->tile_rows = tile_rows;
+    h->down_pair = down_pair;
     return BEAM_OK;
 }
 

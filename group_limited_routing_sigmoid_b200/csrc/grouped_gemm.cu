@@ -10,32 +10,45 @@
 // for every row of the expert-sorted activation buffer, e = the row's expert.
 //
 // Tiling (weights as the MMA's M operand).  A work item is (expert e, a
-// 128-row tile of that expert's weight matrix, a tile of BN token rows of
-// e).  The weight tile is the UMMA A operand (M = 128) and the token tile is
-// B (N = BN), so a decode batch with a handful of tokens per expert still
-// uses full 128-row MMAs while streaming every weight byte exactly once.
-// Gate and up go to two accumulators in TMEM (columns [0,BN) and [BN,2BN)),
-// so TMEM lane r holds gate and up of the same intermediate row and the
-// SwiGLU needs no data exchange between threads.
+// weight tile of e, a token tile of e).  Weight rows are the UMMA A operand
+// (M = 128) and the token rows are B, so a decode batch with a handful of
+// tokens per expert still issues full 128-row MMAs and streams every weight
+// byte once.  An expert's tokens are split into ceil(count / BN) tiles of
+// equal size, and each item's MMA N is its tile size rounded up to 16 (a
+// runtime field of the instruction descriptor), so ragged experts waste at
+// most 15 rows per tile.  The TMA loads of a token tile fetch exactly those
+// rows, as a sum of power-of-two boxes.
+//   gate|up: two A tiles (gate and up rows i0..i0+127) into two TMEM
+//            accumulators, so TMEM lane r holds gate and up of one
+//            intermediate row and the SwiGLU needs no exchange;
+//   down:    one or two A tiles (rows c0..c0+127 and c0+128..c0+255) that
+//            share the token tile, halving the token bytes per MMA.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over the item list):
-//   warp 0      TMA producer: K-slices of 64 into a ring of smem stages;
+//   warp 0      TMA producer: K slices of 64 into a ring of smem stages;
 //   warp 1      TMEM allocator and UMMA issuer (one thread);
-//   warps 2..5  epilogue: tcgen05.ld from TMEM, SwiGLU or fp32 store.
-// Accumulators are double-buffered in TMEM so the epilogue of one item
-// overlaps the mainloop of the next.  Every wait is bounded (WaitCtl).
+//   warps 2..5  epilogue: tcgen05.ld, SwiGLU or plain fp32, a 32x32
+//               transpose through shared memory, 16-byte stores.
+// Accumulators are double-buffered in TMEM when two fit in its 512 columns,
+// so the epilogue of one item overlaps the mainloop of the next.  Every wait
+// is bounded (WaitCtl).
 #include "kernels.cuh"
 
 namespace beam {
 
 namespace {
 
-constexpr int kBM = 128;          // weight rows per tile (UMMA M)
+constexpr int kBM = 128;          // weight rows per A tile (UMMA M)
 constexpr int kBK = 64;           // K per stage: one 128-byte swizzle row of bf16
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;      // two per TMEM lane quadrant, alternating column chunks
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxDynSmem = 232448;
 constexpr int kTableBytes = 3 * (1024 + 1) * 4 + 4;   // counts, offsets, tile_off (E <= 1024)
 constexpr int kBarrierBytes = 256;
+constexpr int kStagingWarpBytes = 2048;                // one 32-row x CH-column block per epilogue warp
+constexpr int kStagingBytes = kEpiWarps * kStagingWarpBytes;
+
+enum Epi { kSwiGLU = 0, kStoreF32 = 1 };
 
 constexpr int pow2_at_least(int v, int lo)
 {
@@ -44,22 +57,29 @@ constexpr int pow2_at_least(int v, int lo)
     return p;
 }
 
-template <int BN, int NUM_A>
+template <int BN, int NUM_A, int EPI>
 struct Cfg {
     static constexpr int A_BYTES = kBM * kBK * 2;
     static constexpr int B_BYTES = BN * kBK * 2;
     static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
-    static constexpr int STAGE_BUDGET = kMaxDynSmem - 1024 - kBarrierBytes - kTableBytes;
+    static constexpr int STAGE_BUDGET =
+        kMaxDynSmem - 1024 - kBarrierBytes - kTableBytes - kStagingBytes;
     static constexpr int STAGES_FIT = STAGE_BUDGET / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-    static constexpr int ACC_COLS = NUM_A * BN;            // one accumulator buffer
-    static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_COLS, 32);
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + kBarrierBytes + kTableBytes;
+    static constexpr int ACC_COLS = NUM_A * BN;             // one accumulator buffer
+    static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
+    static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS, 32);
+    // epilogue columns per chunk: a 32 x CH block of outputs fits the warp's staging
+    static constexpr int CH = (EPI == kSwiGLU && BN >= 32) ? 32 : 16;
+    static constexpr int ROWS_PER_ITEM = EPI == kSwiGLU ? kBM : NUM_A * kBM;
+    static constexpr int SMEM_BYTES =
+        1024 + STAGES * STAGE_BYTES + kStagingBytes + kBarrierBytes + kTableBytes;
     static_assert(STAGES >= 2, "pipeline needs two stages");
     static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
     static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of the next tile");
     static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory");
+    static_assert(EPI == kStoreF32 || NUM_A == 2, "SwiGLU needs the gate and up tiles");
 };
 
 struct Item {
@@ -67,8 +87,10 @@ struct Item {
 };
 
 // Item i of the list ordered (expert, weight tile, token tile): the expert is
-// the largest e with WT * tile_off[e] <= i.
-__device__ __forceinline__ Item decode_item(int i, int WT, int E, int BN, const int *s_counts,
+// the largest e with WT * tile_off[e] <= i; its count c is split into
+// nt = tile_off[e+1] - tile_off[e] tiles of ceil(c / nt) rows (the last may
+// be shorter).
+__device__ __forceinline__ Item decode_item(int i, int WT, int E, const int *s_counts,
                                             const int *s_offsets, const int *s_tile)
 {
     int lo = 0, hi = E - 1;
@@ -83,27 +105,40 @@ __device__ __forceinline__ Item decode_item(int i, int WT, int E, int BN, const 
     const int nt = s_tile[lo + 1] - s_tile[lo];
     it.wt = local / nt;
     const int tt = local - it.wt * nt;
-    it.row0 = s_offsets[lo] + tt * BN;
-    it.nrows = min(BN, s_counts[lo] - tt * BN);
+    const int c = s_counts[lo];
+    const int bal = (c + nt - 1) / nt;
+    it.row0 = s_offsets[lo] + tt * bal;
+    it.nrows = min(bal, c - tt * bal);
     return it;
 }
 
-__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + expf(-g)); }
+// silu(g) = g / (1 + e^-g) in FP32 with the fast exponential and divide; the
+// product with u is rounded to bf16 right after, which the approximations
+// (a few FP32 ulps) do not reach but in rare rounding-boundary cases.
+__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&v)[N])
+{
+    if constexpr (N == 32) tmem_ld32(taddr, v);
+    else tmem_ld16(taddr, v);
+}
 
 }  // namespace
 
-template <int BN, int NUM_A>
+template <int BN, int NUM_A, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                         const __grid_constant__ CUtensorMap tmA1,
-                        const __grid_constant__ CUtensorMap tmB, GemmArgs p)
+                        const __grid_constant__ BoxMaps tmB, GemmArgs p)
 {
-    using C = Cfg<BN, NUM_A>;
+    using C = Cfg<BN, NUM_A, EPI>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t *base_ptr = smem_raw + (base - raw_addr);
-    uint8_t *bar_ptr = base_ptr + C::STAGES * C::STAGE_BYTES;
+    uint8_t *staging = base_ptr + C::STAGES * C::STAGE_BYTES;   // 16 KB, 1024-aligned
+    uint8_t *bar_ptr = staging + kStagingBytes;
     uint64_t *full = reinterpret_cast<uint64_t *>(bar_ptr);
     uint64_t *empty = full + C::STAGES;
     uint64_t *tfull = empty + C::STAGES;
@@ -129,13 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
-            mbar_init(smem_u32(&tempty[a]), 128);
+            mbar_init(smem_u32(&tempty[a]), 32 * kEpiWarps);
         }
         mbar_init(smem_u32(drain), 1);
         fence_barrier_init();
         tma_prefetch_desc(&tmA0);
         if (NUM_A == 2) tma_prefetch_desc(&tmA1);
-        tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
         __syncwarp();
@@ -147,12 +181,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int WT = p.R / kBM;
+    const int WT = p.R / C::ROWS_PER_ITEM;
     const int total = WT * s_tile[p.E];
     const int KB = p.K / kBK;
 
-    if (warp == 0 && lane == 0) {
-        // ------------------------------------------------ TMA producer
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (lane 0)
         const uint64_t pol_w = l2_policy_evict_first();   // weights: streamed
         const uint64_t pol_x = l2_policy_evict_last();    // activations: reused across tiles
         int stage = 0;
@@ -160,19 +194,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         long long issued = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const Item it = decode_item(item, WT, p.E, BN, s_counts, s_offsets, s_tile);
-            const int a_row = it.e * p.R + it.wt * kBM;
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const int a_row = it.e * p.R + it.wt * C::ROWS_PER_ITEM;
+            const int n_load = (it.nrows + 15) & ~15;
+            const uint32_t bytes = NUM_A * C::A_BYTES + n_load * (kBK * 2);
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl)) {
-                    ok = false;
-                    break;
+                bool got = true;
+                if (lane == 0) {
+                    got = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl);
+                    if (got) {
+                        const uint32_t sa = base + stage * C::STAGE_BYTES;
+                        const uint32_t fb = smem_u32(&full[stage]);
+                        mbar_arrive_expect_tx(fb, bytes);
+                        tma_load_2d(sa, &tmA0, kb * kBK, a_row, fb, pol_w);
+                        if (NUM_A == 2) {
+                            // gate|up: the up matrix at the same rows; down: the next 128 rows
+                            const int a_row1 = EPI == kSwiGLU ? a_row : a_row + kBM;
+                            tma_load_2d(sa + C::A_BYTES, &tmA1, kb * kBK, a_row1, fb, pol_w);
+                        }
+                        const uint32_t sb = sa + NUM_A * C::A_BYTES;
+                        int off = 0;
+#pragma unroll
+                        for (int bi = 4; bi >= 0; --bi) {   // boxes of 256, 128, 64, 32, 16 rows
+                            const int hgt = 16 << bi;
+                            if (hgt <= BN && n_load - off >= hgt) {
+                                tma_load_2d(sb + off * (kBK * 2), &tmB.m[bi], kb * kBK,
+                                            it.row0 + off, fb, pol_x);
+                                off += hgt;
+                            }
+                        }
+                    }
                 }
-                const uint32_t sa = base + stage * C::STAGE_BYTES;
-                const uint32_t fb = smem_u32(&full[stage]);
-                mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-                tma_load_2d(sa, &tmA0, kb * kBK, a_row, fb, pol_w);
-                if (NUM_A == 2) tma_load_2d(sa + C::A_BYTES, &tmA1, kb * kBK, a_row, fb, pol_w);
-                tma_load_2d(sa + NUM_A * C::A_BYTES, &tmB, kb * kBK, it.row0, fb, pol_x);
+                ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                if (!ok) break;
                 ++issued;
                 if (++stage == C::STAGES) {
                     stage = 0;
@@ -180,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        if (!ok) {
+        if (!ok && lane == 0) {
             // Give the copies already in flight time to land before the CTA
             // exits: wait (time-bounded, status ignored) on the last ones.
             long long n = issued < C::STAGES ? issued : C::STAGES;
@@ -198,15 +252,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ UMMA issuer
-        constexpr uint32_t idesc = umma_idesc_bf16_f32(kBM, BN);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         bool issued_any = false;
         int iter = 0;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++iter) {
-            const int acc = iter & 1;
-            const uint32_t acc_phase = (uint32_t)(iter >> 1) & 1u;
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const int n_mma = (it.nrows + 15) & ~15;
+            const uint32_t idesc = umma_idesc_bf16_f32(kBM, n_mma);
+            const int acc = iter % C::NBUF;
+            const uint32_t acc_phase = (uint32_t)(iter / C::NBUF) & 1u;
             if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.ctl)) {
                 ok = false;
                 break;
@@ -226,10 +282,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bdesc = umma_desc_sw128(sb + k * 32);
                     const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
                     umma_bf16(d0, umma_desc_sw128(sa + k * 32), bdesc, idesc, accum);
-                    issued_any = true;
                     if (NUM_A == 2)
                         umma_bf16(d0 + BN, umma_desc_sw128(sa + C::A_BYTES + k * 32), bdesc, idesc,
                                   accum);
+                    issued_any = true;
                 }
                 umma_commit(smem_u32(&empty[stage]));
                 if (++stage == C::STAGES) {
@@ -247,42 +303,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue
-        const int quad = warp & 3;            // TMEM lanes this warp may access
-        const int r_in_tile = quad * 32 + lane;
+        constexpr int CH = C::CH;
+        constexpr int ESZ = EPI == kSwiGLU ? 2 : 4;        // output element bytes
+        constexpr int VPR = 32 * ESZ / 16;                 // 16-byte vectors per 32-row slice
+        static_assert(32 * CH * ESZ <= kStagingWarpBytes, "staging block");
+        const int quad = warp & 3;                         // TMEM lanes this warp may access
+        const int half = (warp - 2) >> 2;                  // which alternate column chunks
+        uint8_t *stg = staging + (warp - 2) * kStagingWarpBytes;
         int iter = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x, ++iter) {
-            const int acc = iter & 1;
-            const uint32_t acc_phase = (uint32_t)(iter >> 1) & 1u;
+            const int acc = iter % C::NBUF;
+            const uint32_t acc_phase = (uint32_t)(iter / C::NBUF) & 1u;
             const bool ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.ctl);
             if (!__all_sync(0xffffffffu, ok)) break;   // warp-uniform from here on
             tc_fence_after();
-            const Item it = decode_item(item, WT, p.E, BN, s_counts, s_offsets, s_tile);
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
-            const int r = it.wt * kBM + r_in_tile;   // row of this expert's weight matrix
-            for (int c = 0; c < it.nrows; c += 16) {
-                uint32_t g[16];
-                tmem_ld16(taddr + c, g);
-                if (NUM_A == 2) {
-                    uint32_t u[16];
-                    tmem_ld16(taddr + BN + c, u);
-                    tmem_ld_wait();
-                    __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(p.out);
+            constexpr int NOUT = EPI == kSwiGLU ? 1 : NUM_A;
+#pragma unroll 1
+            for (int a = 0; a < NOUT; ++a) {
+                // first output column (weight row) of this warp's 32-row slice
+                const int col0 = it.wt * C::ROWS_PER_ITEM + a * kBM + quad * 32;
+                uint8_t *out = static_cast<uint8_t *>(p.out) + (size_t)col0 * ESZ;
+#pragma unroll 1
+                for (int c0 = half * CH; c0 < it.nrows; c0 += 2 * CH) {
+                    uint32_t g[CH];
+                    tmem_ld<CH>(taddr + a * BN + c0, g);
+                    if constexpr (EPI == kSwiGLU) {
+                        uint32_t u[CH];
+                        tmem_ld<CH>(taddr + BN + c0, u);
+                        tmem_ld_wait();
+                        __nv_bfloat16 *sh = reinterpret_cast<__nv_bfloat16 *>(stg);
 #pragma unroll
-                    for (int n = 0; n < 16; ++n) {
-                        if (c + n < it.nrows) {
-                            const float gv = __uint_as_float(g[n]);
-                            const float uv = __uint_as_float(u[n]);
-                            h[(size_t)(it.row0 + c + n) * p.R + r] = __float2bfloat16_rn(silu_f32(gv) * uv);
+                        for (int j = 0; j < CH; ++j)
+                            sh[j * 32 + lane] = __float2bfloat16_rn(
+                                silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]));
+                    } else {
+                        tmem_ld_wait();
+                        float *sf = reinterpret_cast<float *>(stg);
+#pragma unroll
+                        for (int j = 0; j < CH; ++j) sf[j * 32 + lane] = __uint_as_float(g[j]);
+                    }
+                    __syncwarp();
+                    // token row c0+j of the slice: VPR vectors of 16 bytes
+#pragma unroll
+                    for (int v = lane; v < CH * VPR; v += 32) {
+                        const int j = v / VPR, part = v - j * VPR;
+                        if (c0 + j < it.nrows) {
+                            const uint4 val = *reinterpret_cast<const uint4 *>(stg + v * 16);
+                            *reinterpret_cast<uint4 *>(
+                                out + (size_t)(it.row0 + c0 + j) * p.R * ESZ + part * 16) = val;
                         }
                     }
-                } else {
-                    tmem_ld_wait();
-                    float *y = reinterpret_cast<float *>(p.out);
-#pragma unroll
-                    for (int n = 0; n < 16; ++n)
-                        if (c + n < it.nrows)
-                            y[(size_t)(it.row0 + c + n) * p.R + r] = __uint_as_float(g[n]);
+                    __syncwarp();
                 }
             }
             tc_fence_before();
@@ -304,57 +378,75 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 
 namespace {
-template <int BN, int NUM_A>
+template <int BN, int NUM_A, int EPI>
 cudaError_t set_smem()
 {
-    return cudaFuncSetAttribute(grouped_gemm_kernel<BN, NUM_A>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN, NUM_A>::SMEM_BYTES);
+    return cudaFuncSetAttribute(grouped_gemm_kernel<BN, NUM_A, EPI>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg<BN, NUM_A, EPI>::SMEM_BYTES);
 }
 
-template <int BN, int NUM_A>
-cudaError_t launch(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
+template <int BN, int NUM_A, int EPI>
+cudaError_t launch(const CUtensorMap &a0, const CUtensorMap &a1, const BoxMaps &b,
                    const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    grouped_gemm_kernel<BN, NUM_A>
-        <<<grid, kThreads, Cfg<BN, NUM_A>::SMEM_BYTES, stream>>>(a0, a1, b, args);
+    grouped_gemm_kernel<BN, NUM_A, EPI>
+        <<<grid, kThreads, Cfg<BN, NUM_A, EPI>::SMEM_BYTES, stream>>>(a0, a1, b, args);
     return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_kind(GemmKind kind, const CUtensorMap &a0, const CUtensorMap &a1,
+                        const BoxMaps &b, const GemmArgs &args, int grid, cudaStream_t stream)
+{
+    switch (kind) {
+        case GemmKind::kGateUp:
+            return launch<BN, 2, kSwiGLU>(a0, a1, b, args, grid, stream);
+        case GemmKind::kDown:
+            return launch<BN, 1, kStoreF32>(a0, a1, b, args, grid, stream);
+        case GemmKind::kDownPaired:
+            return launch<BN, 2, kStoreF32>(a0, a1, b, args, grid, stream);
+    }
+    return cudaErrorInvalidValue;
 }
 }  // namespace
 
-bool gemm_tile_supported(int BN) { return BN == 16 || BN == 32 || BN == 64 || BN == 128; }
+bool gemm_tile_supported(int BN)
+{
+    return BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256;
+}
+
+int gemm_rows_per_item(GemmKind kind) { return kind == GemmKind::kDownPaired ? 2 * kBM : kBM; }
 
 cudaError_t prepare_grouped_gemm(int E)
 {
     if (E > 1024) return cudaErrorInvalidValue;
     cudaError_t err;
-#define BEAM_PREP(BN)                                  \
-    if ((err = set_smem<BN, 1>()) != cudaSuccess) return err; \
-    if ((err = set_smem<BN, 2>()) != cudaSuccess) return err;
+#define BEAM_PREP(BN)                                                        \
+    if ((err = set_smem<BN, 2, kSwiGLU>()) != cudaSuccess) return err;       \
+    if ((err = set_smem<BN, 1, kStoreF32>()) != cudaSuccess) return err;     \
+    if ((err = set_smem<BN, 2, kStoreF32>()) != cudaSuccess) return err;
     BEAM_PREP(16)
     BEAM_PREP(32)
     BEAM_PREP(64)
     BEAM_PREP(128)
+    BEAM_PREP(256)
 #undef BEAM_PREP
     return cudaSuccess;
 }
 
-cudaError_t launch_grouped_gemm(bool swiglu, int BN, const CUtensorMap &a0, const CUtensorMap &a1,
-                                const CUtensorMap &b, const GemmArgs &args, int grid,
+cudaError_t launch_grouped_gemm(GemmKind kind, int BN, const CUtensorMap &a0, const CUtensorMap &a1,
+                                const BoxMaps &b, const GemmArgs &args, int grid,
                                 cudaStream_t stream)
 {
-#define BEAM_CASE(BNV)                                                          \
-    case BNV:                                                                   \
-        return swiglu ? launch<BNV, 2>(a0, a1, b, args, grid, stream)           \
-                      : launch<BNV, 1>(a0, a1, b, args, grid, stream);
     switch (BN) {
-        BEAM_CASE(16)
-        BEAM_CASE(32)
-        BEAM_CASE(64)
-        BEAM_CASE(128)
-        default:
-            return cudaErrorInvalidValue;
+        case 16: return launch_kind<16>(kind, a0, a1, b, args, grid, stream);
+        case 32: return launch_kind<32>(kind, a0, a1, b, args, grid, stream);
+        case 64: return launch_kind<64>(kind, a0, a1, b, args, grid, stream);
+        case 128: return launch_kind<128>(kind, a0, a1, b, args, grid, stream);
+        case 256: return launch_kind<256>(kind, a0, a1, b, args, grid, stream);
+        default: return cudaErrorInvalidValue;
     }
-#undef BEAM_CASE
 }
 
 }  // namespace beam

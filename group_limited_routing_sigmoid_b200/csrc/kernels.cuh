@@ -44,21 +44,33 @@ cudaError_t prepare_dispatch(int E);   // shared-memory limit of the counting ke
 // ----------------------------------------------------------- grouped GEMM
 struct GemmArgs {
     int K;                       // reduction length
-    int R;                       // weight rows per expert (multiple of 128)
+    int R;                       // weight rows per expert (= output row stride)
     int E;
     const int32_t *counts;       // [E]
     const int32_t *offsets;      // [E+1]
     const int32_t *tile_off;     // [E+1]
-    void *out;                   // SwiGLU: bf16 [P, R]; plain: fp32 [P, R]
+    void *out;                   // gate|up: bf16 [P, R]; down: fp32 [P, R]
     WaitCtl ctl;
 };
-// Gate|up GEMM with the SwiGLU epilogue (two A maps) or the down GEMM
-// (one A map, fp32 output), BN token rows per tile.
-cudaError_t launch_grouped_gemm(bool swiglu, int BN, const CUtensorMap &a0, const CUtensorMap &a1,
-                                const CUtensorMap &b, const GemmArgs &args, int grid,
-                                cudaStream_t stream);
+
+// Tensor maps of one activation buffer with boxes of 16, 32, 64, 128 and 256
+// rows (64 columns each): a token tile is loaded as a sum of these.
+struct BoxMaps {
+    CUtensorMap m[5];
+};
+
+enum class GemmKind {
+    kGateUp,       // gate and up tiles, SwiGLU epilogue, bf16 out
+    kDown,         // one 128-row tile, fp32 out
+    kDownPaired    // two consecutive 128-row tiles sharing the token tile, fp32 out
+};
+// BN: largest token tile (16..256, power of two).
+cudaError_t launch_grouped_gemm(GemmKind kind, int BN, const CUtensorMap &a0,
+                                const CUtensorMap &a1, const BoxMaps &b, const GemmArgs &args,
+                                int grid, cudaStream_t stream);
 cudaError_t prepare_grouped_gemm(int E);   // sets shared-memory limits once per device
 bool gemm_tile_supported(int BN);
+int gemm_rows_per_item(GemmKind kind);
 
 // ---------------------------------------------------------------- combine
 struct CombineArgs {

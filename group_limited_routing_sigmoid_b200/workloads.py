@@ -76,6 +76,10 @@ WORKLOADS: Dict[str, Workload] = {
     # (2.5 GB of weights), 8 tokens: the decode kernels on a few GB of memory
     "decode_small": Workload("decode_small", T=8, hidden=5120, n_experts=32, n_group=8,
                              topk_group=4, top_k=8, inter=2560),
+    # profiling case: the same 32 Beam-shaped experts with 1024 tokens, i.e.
+    # ~256 tokens per expert as in the 8192-token prefill
+    "prefill_small": Workload("prefill_small", T=1024, hidden=5120, n_experts=32, n_group=8,
+                              topk_group=4, top_k=8, inter=2560, bias_lo=-0.01, bias_hi=0.01),
 }
 
 

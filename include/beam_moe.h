@@ -200,11 +200,17 @@ int beam_moe_get_status(beam_moe_t h, void *stream);
 int beam_moe_set_wait_limit(beam_moe_t h, int64_t limit_ns);
 
 /*
- * Number of CTAs of the persistent grouped-GEMM kernels (0 = one per SM, the
- * default).  Fewer CTAs put more work items on each CTA; results do not
- * depend on it.  0 <= ctas <= 65535.
+ * Tuning of the grouped GEMMs; results do not depend on any of it.
+ * ctas            CTAs of the persistent kernels, 0 = one per SM (default);
+ *                 fewer CTAs put more work items on each.  0..65535.
+ * tile_rows       largest token tile: 16, 32, 64, 128 or 256 rows, or 0 to
+ *                 choose from the mean number of tokens per expert (default).
+ * down_pair       -1: choose (default); 0: the down projection takes one
+ *                 128-row weight tile per work item; 1: two consecutive tiles
+ *                 that share the token tile (needs hidden % 256 == 0, else
+ *                 ignored).
  */
-int beam_moe_set_gemm_ctas(beam_moe_t h, int ctas);
+int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair);
 
 /*
  * Per-stage timing of forward passes, for measurement.  After

@@ -44,16 +44,22 @@ def _inputs(wl, T=None):
     return d
 
 
-@pytest.mark.parametrize("T,ctas", [(64, 0), (64, 1), (1, 0), (3, 0), (37, 5), (100, 0),
-                                    (200, 3), (1000, 0), (1000, 2), (4096, 0)])
-def test_tiny_block(T, ctas):
+# (T, GEMM CTAs (0 = one per SM), largest token tile (0 = auto), paired down tiles (-1 = auto))
+TINY_CASES = [(64, 0, 0, -1), (64, 1, 0, -1), (1, 0, 0, -1), (3, 0, 0, -1), (37, 5, 0, -1),
+              (100, 0, 0, -1), (200, 3, 0, -1), (1000, 0, 0, -1), (1000, 2, 0, -1),
+              (4096, 0, 0, -1), (1000, 0, 16, 0), (1000, 0, 32, 1), (1000, 0, 64, 0),
+              (1000, 3, 128, 1), (1000, 0, 256, 0), (1000, 2, 256, 1), (300, 0, 256, 1),
+              (4096, 7, 256, 1)]
+
+
+@pytest.mark.parametrize("T,ctas,tile,pair", TINY_CASES)
+def test_tiny_block(T, ctas, tile, pair):
     wl = W.WORKLOADS["tiny"]
     d = _inputs(wl, T)
     moe = BeamMoE.from_workload(wl, d, max_tokens=T)
-    if ctas:
-        moe.set_gemm_ctas(ctas)
+    moe.set_gemm_tuning(ctas, tile, pair)
     rep = check_block(wl, d, moe)
-    _log(f"tiny_T{T}_ctas{ctas}", rep)
+    _log(f"tiny_T{T}_ctas{ctas}_tile{tile}_pair{pair}", rep)
     assert rep.ok(), rep
     moe.close()
 
