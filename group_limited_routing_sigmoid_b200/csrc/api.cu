@@ -32,7 +32,7 @@ struct beam_moe {
     int32_t *block_cnt, *block_base, *rank, *counts, *offsets, *tile_off, *pair_row, *row_pair;
     __nv_bfloat16 *xp;       // [P, H]
     __nv_bfloat16 *hbuf;     // [P, I]
-    float *ybuf;             // [P, H]
+    __nv_bfloat16 *ybuf;     // [P, H]
     int *status;             // device status word
     __nv_bfloat16 *x_stage, *out_stage;
     float *res_stage;
@@ -142,9 +142,7 @@ int run_router(beam_moe *h, cudaStream_t s, const void *x, int T, int32_t *idx, 
     a.n_group = h->n_group;
     a.topk_group = h->topk_group;
     a.top_k = h->top_k;
-    a.nslice = router_slices(T, h->H, h->E, h->num_sms);
-    while (a.nslice > 1 && (size_t)a.nslice * T > (size_t)(h->max_tokens > 4096 ? h->max_tokens : 4096))
-        a.nslice /= 2;
+    a.nslice = router_slices(T, h->H, h->E, h->num_sms);   // the workspace holds nslice * T rows
     a.partial = h->partial;
     a.idx = idx;
     a.w = w;
@@ -324,9 +322,12 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     // Workspace
     const size_t T = (size_t)max_tokens, E = (size_t)n_experts, P = T * top_k;
     const size_t nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
-    // router partial sums: nslice(T) * T <= 4096 rows for every T (router_slices
-    // keeps the logits grid near two blocks per SM), and T rows for large T
-    const size_t partial_rows = T > 4096 ? T : 4096;
+    // router partial sums: the largest nslice(t) * t over t <= max_tokens
+    size_t partial_rows = 0;
+    for (int t = 1; t <= max_tokens; ++t) {
+        const size_t r = (size_t)router_slices(t, hidden, n_experts, h->num_sms) * t;
+        if (r > partial_rows) partial_rows = r;
+    }
     size_t off = 0;
     auto carve = [&](size_t bytes) {
         size_t o = off;
@@ -346,7 +347,7 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     const size_t o_rpair = carve(P * 4);
     const size_t o_xp = carve(P * hidden * 2);
     const size_t o_h = carve(P * inter * 2);
-    const size_t o_y = carve(P * hidden * 4);
+    const size_t o_y = carve(P * hidden * 2);
     const size_t o_status = carve(256);
     const size_t o_xs = carve(T * hidden * 2);
     const size_t o_os = carve(T * hidden * 2);
@@ -374,7 +375,7 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     h->row_pair = reinterpret_cast<int32_t *>(b + o_rpair);
     h->xp = reinterpret_cast<__nv_bfloat16 *>(b + o_xp);
     h->hbuf = reinterpret_cast<__nv_bfloat16 *>(b + o_h);
-    h->ybuf = reinterpret_cast<float *>(b + o_y);
+    h->ybuf = reinterpret_cast<__nv_bfloat16 *>(b + o_y);
     h->status = reinterpret_cast<int *>(b + o_status);
     h->x_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_xs);
     h->out_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_os);

@@ -1,7 +1,7 @@
 // Combine of the Beam MoE block, with the optional post-norm and
 // depth-scaled residual update fused in.
 //
-//   o[t]   = routed_scaling * sum_j w[t,j] * y[row(t,j)]     (fp32, slot order)
+//   o[t]   = routed_scaling * sum_j w[t,j] * y[row(t,j)]     (bf16 y, fp32 sum, slot order)
 //   out[t] = bf16_rn(o[t])
 //   n[t]   = o[t] / sqrt(mean(o[t]^2) + eps) * gamma          (if gamma)
 //   stream[t] <- sqrt((k-1)/k) * stream[t] + n[t] / sqrt(k)
@@ -36,7 +36,10 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a)
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (i < nvec) {
             for (int j = 0; j < a.top_k; ++j) {
-                const float4 y = reinterpret_cast<const float4 *>(a.y + (size_t)rows[j] * a.H)[i];
+                const uint2 raw = reinterpret_cast<const uint2 *>(a.y + (size_t)rows[j] * a.H)[i];
+                const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                const float4 y = make_float4(lo.x, lo.y, hi.x, hi.y);
                 acc.x = fmaf(wts[j], y.x, acc.x);
                 acc.y = fmaf(wts[j], y.y, acc.y);
                 acc.z = fmaf(wts[j], y.z, acc.z);

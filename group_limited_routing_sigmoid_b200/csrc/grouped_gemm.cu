@@ -6,7 +6,7 @@
 // product is taken in FP32 (section "Residual Stream", FP32 sites).  Two
 // kernels per forward pass:
 //   gate|up:  h[row, i] = bf16( silu(W_g[e,i,:] . xp[row,:]) * (W_u[e,i,:] . xp[row,:]) )
-//   down:     y[row, c] = W_d[e,c,:] . h[row,:]                      (fp32 out)
+//   down:     y[row, c] = bf16( W_d[e,c,:] . h[row,:] )
 // for every row of the expert-sorted activation buffer, e = the row's expert.
 //
 // Tiling (weights as the MMA's M operand).  A work item is (expert e, a
@@ -27,8 +27,9 @@
 // Warp roles (192 threads, one CTA per SM, persistent over the item list):
 //   warp 0      TMA producer: K slices of 64 into a ring of smem stages;
 //   warp 1      TMEM allocator and UMMA issuer (one thread);
-//   warps 2..5  epilogue: tcgen05.ld, SwiGLU or plain fp32, a 32x32
-//               transpose through shared memory, 16-byte stores.
+//   warps 2..9  epilogue (two per TMEM lane quadrant): tcgen05.ld, SwiGLU or
+//               the plain accumulator, rounded to bf16, a 32x32 transpose
+//               through shared memory, 16-byte stores.
 // Accumulators are double-buffered in TMEM when two fit in its 512 columns,
 // so the epilogue of one item overlaps the mainloop of the next.  Every wait
 // is bounded (WaitCtl).
@@ -48,7 +49,7 @@ constexpr int kBarrierBytes = 256;
 constexpr int kStagingWarpBytes = 2048;                // one 32-row x CH-column block per epilogue warp
 constexpr int kStagingBytes = kEpiWarps * kStagingWarpBytes;
 
-enum Epi { kSwiGLU = 0, kStoreF32 = 1 };
+enum Epi { kSwiGLU = 0, kStoreBF16 = 1 };   // gate|up with SwiGLU; plain (down)
 
 constexpr int pow2_at_least(int v, int lo)
 {
@@ -69,8 +70,8 @@ struct Cfg {
     static constexpr int ACC_COLS = NUM_A * BN;             // one accumulator buffer
     static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
     static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS, 32);
-    // epilogue columns per chunk: a 32 x CH block of outputs fits the warp's staging
-    static constexpr int CH = (EPI == kSwiGLU && BN >= 32) ? 32 : 16;
+    // epilogue columns per chunk: a 32 x CH block of bf16 outputs in the warp's staging
+    static constexpr int CH = BN >= 32 ? 32 : 16;
     static constexpr int ROWS_PER_ITEM = EPI == kSwiGLU ? kBM : NUM_A * kBM;
     static constexpr int SMEM_BYTES =
         1024 + STAGES * STAGE_BYTES + kStagingBytes + kBarrierBytes + kTableBytes;
@@ -79,7 +80,7 @@ struct Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
     static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of the next tile");
     static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory");
-    static_assert(EPI == kStoreF32 || NUM_A == 2, "SwiGLU needs the gate and up tiles");
+    static_assert(EPI == kStoreBF16 || NUM_A == 2, "SwiGLU needs the gate and up tiles");
 };
 
 struct Item {
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue
         constexpr int CH = C::CH;
-        constexpr int ESZ = EPI == kSwiGLU ? 2 : 4;        // output element bytes
+        constexpr int ESZ = 2;                             // bf16 outputs
         constexpr int VPR = 32 * ESZ / 16;                 // 16-byte vectors per 32-row slice
         static_assert(32 * CH * ESZ <= kStagingWarpBytes, "staging block");
         const int quad = warp & 3;                         // TMEM lanes this warp may access
@@ -325,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int a = 0; a < NOUT; ++a) {
                 // first output column (weight row) of this warp's 32-row slice
                 const int col0 = it.wt * C::ROWS_PER_ITEM + a * kBM + quad * 32;
-                uint8_t *out = static_cast<uint8_t *>(p.out) + (size_t)col0 * ESZ;
+                uint8_t *out = reinterpret_cast<uint8_t *>(p.out) + (size_t)col0 * ESZ;
 #pragma unroll 1
                 for (int c0 = half * CH; c0 < it.nrows; c0 += 2 * CH) {
                     uint32_t g[CH];
@@ -341,9 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]));
                     } else {
                         tmem_ld_wait();
-                        float *sf = reinterpret_cast<float *>(stg);
+                        __nv_bfloat16 *sh = reinterpret_cast<__nv_bfloat16 *>(stg);
 #pragma unroll
-                        for (int j = 0; j < CH; ++j) sf[j * 32 + lane] = __uint_as_float(g[j]);
+                        for (int j = 0; j < CH; ++j)
+                            sh[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(g[j]));
                     }
                     __syncwarp();
                     // token row c0+j of the slice: VPR vectors of 16 bytes
@@ -403,9 +405,9 @@ cudaError_t launch_kind(GemmKind kind, const CUtensorMap &a0, const CUtensorMap 
         case GemmKind::kGateUp:
             return launch<BN, 2, kSwiGLU>(a0, a1, b, args, grid, stream);
         case GemmKind::kDown:
-            return launch<BN, 1, kStoreF32>(a0, a1, b, args, grid, stream);
+            return launch<BN, 1, kStoreBF16>(a0, a1, b, args, grid, stream);
         case GemmKind::kDownPaired:
-            return launch<BN, 2, kStoreF32>(a0, a1, b, args, grid, stream);
+            return launch<BN, 2, kStoreBF16>(a0, a1, b, args, grid, stream);
     }
     return cudaErrorInvalidValue;
 }
@@ -424,8 +426,8 @@ cudaError_t prepare_grouped_gemm(int E)
     cudaError_t err;
 #define BEAM_PREP(BN)                                                        \
     if ((err = set_smem<BN, 2, kSwiGLU>()) != cudaSuccess) return err;       \
-    if ((err = set_smem<BN, 1, kStoreF32>()) != cudaSuccess) return err;     \
-    if ((err = set_smem<BN, 2, kStoreF32>()) != cudaSuccess) return err;
+    if ((err = set_smem<BN, 1, kStoreBF16>()) != cudaSuccess) return err;     \
+    if ((err = set_smem<BN, 2, kStoreBF16>()) != cudaSuccess) return err;
     BEAM_PREP(16)
     BEAM_PREP(32)
     BEAM_PREP(64)

@@ -49,7 +49,7 @@ struct GemmArgs {
     const int32_t *counts;       // [E]
     const int32_t *offsets;      // [E+1]
     const int32_t *tile_off;     // [E+1]
-    void *out;                   // gate|up: bf16 [P, R]; down: fp32 [P, R]
+    __nv_bfloat16 *out;          // bf16 [P, R]: h (gate|up) or y (down)
     WaitCtl ctl;
 };
 
@@ -61,8 +61,8 @@ struct BoxMaps {
 
 enum class GemmKind {
     kGateUp,       // gate and up tiles, SwiGLU epilogue, bf16 out
-    kDown,         // one 128-row tile, fp32 out
-    kDownPaired    // two consecutive 128-row tiles sharing the token tile, fp32 out
+    kDown,         // one 128-row tile, bf16 out
+    kDownPaired    // two consecutive 128-row tiles sharing the token tile, bf16 out
 };
 // BN: largest token tile (16..256, power of two).
 cudaError_t launch_grouped_gemm(GemmKind kind, int BN, const CUtensorMap &a0,
@@ -74,7 +74,7 @@ int gemm_rows_per_item(GemmKind kind);
 
 // ---------------------------------------------------------------- combine
 struct CombineArgs {
-    const float *y;              // [P, H] expert outputs, fp32
+    const __nv_bfloat16 *y;      // [P, H] expert outputs
     const int32_t *pair_row;     // [P]
     const float *w;              // [T, top_k]
     int T, H, top_k;

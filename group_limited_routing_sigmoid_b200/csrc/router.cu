@@ -14,13 +14,14 @@ namespace beam {
 
 // ---------------------------------------------------------------------------
 // Logits: partial[s][t][e] = sum over the s-th K slice of x[t,h] * W[e,h].
-// 64 tokens x 64 experts per block, 256 threads, 4 x 4 outputs per thread,
-// K staged through shared memory 32 at a time.  Each thread folds its
-// running sums into a second accumulator every 256 K so that no FP32 chain
-// is longer than 256 terms.
+// 128 tokens x 64 experts per block, 256 threads, 8 x 4 outputs per thread.
+// K goes through shared memory 32 at a time; the next 32 are loaded into
+// registers while the current ones are used.  Each thread folds its running
+// FP32 sums into a second accumulator every 256 K, so no FP32 chain is
+// longer than 256 terms.
 // ---------------------------------------------------------------------------
 namespace {
-constexpr int kLT = 64;   // tokens per block
+constexpr int kLT = 128;  // tokens per block
 constexpr int kLE = 64;   // experts per block
 constexpr int kLK = 32;   // K per shared-memory stage
 }  // namespace
@@ -37,62 +38,76 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16 
     const int e0 = blockIdx.y * kLE;
     const int kbeg = blockIdx.z * kslice;
     const int kend = min(H, kbeg + kslice);
-    const int tx = tid & 15;   // expert quad
-    const int ty = tid >> 4;   // token quad
+    const int tx = tid & 15;   // 4 experts: e0 + 4*tx ..
+    const int ty = tid >> 4;   // 8 tokens:  t0 + 8*ty ..
 
-    float acc[4][4], tot[4][4];
+    float acc[8][4], tot[8][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = tot[i][j] = 0.f;
 
-    const int lrow = tid >> 2;         // 0..63: token (x) or expert (w) row loaded
-    const int lk = (tid & 3) * 8;      // 8 consecutive K per thread
+    // loaders: x -- 128 tokens x 32 K bf16 = 4096 values: 16 per thread
+    //          (token tid/2, K half (tid&1)*16);
+    //          W -- 64 experts x 32 K fp32 = 2048 values: 8 per thread
+    //          (expert tid/4, K quarter (tid&3)*8).
+    const int xr = tid >> 1, xk = (tid & 1) * 16;
+    const int wr = tid >> 2, wk = (tid & 3) * 8;
+    const bool xvalid = t0 + xr < T;
+    const bool wvalid = e0 + wr < E;
+    const __nv_bfloat16 *xp = x + (size_t)(t0 + xr) * H + xk;
+    const float *wp = w + (size_t)(e0 + wr) * H + wk;
+    uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+    float4 wa = make_float4(0.f, 0.f, 0.f, 0.f), wb = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto fetch = [&](int k0) {
+        if (xvalid) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(xp + k0);
+            xa = src[0];
+            xb = src[1];
+        }
+        if (wvalid) {
+            const float4 *src = reinterpret_cast<const float4 *>(wp + k0);
+            wa = src[0];
+            wb = src[1];
+        }
+    };
+    auto stash = [&]() {
+        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&xa);
+        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&xb);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(p2[i]);
+            const float2 g = __bfloat1622float2(q2[i]);
+            xs[xk + 2 * i][xr] = f.x;
+            xs[xk + 2 * i + 1][xr] = f.y;
+            xs[xk + 8 + 2 * i][xr] = g.x;
+            xs[xk + 8 + 2 * i + 1][xr] = g.y;
+        }
+        ws[wk + 0][wr] = wa.x;
+        ws[wk + 1][wr] = wa.y;
+        ws[wk + 2][wr] = wa.z;
+        ws[wk + 3][wr] = wa.w;
+        ws[wk + 4][wr] = wb.x;
+        ws[wk + 5][wr] = wb.y;
+        ws[wk + 6][wr] = wb.z;
+        ws[wk + 7][wr] = wb.w;
+    };
+
     int folded = 0;
+    if (kbeg < kend) fetch(kbeg);
     for (int k0 = kbeg; k0 < kend; k0 += kLK) {
-        {
-            float v[8];
-            const int t = t0 + lrow;
-            if (t < T) {
-                uint4 raw = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + k0 + lk);
-                const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float2 f = __bfloat1622float2(p2[i]);
-                    v[2 * i] = f.x;
-                    v[2 * i + 1] = f.y;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) xs[lk + i][lrow] = v[i];
-        }
-        {
-            float v[8];
-            const int e = e0 + lrow;
-            if (e < E) {
-                const float4 *src = reinterpret_cast<const float4 *>(w + (size_t)e * H + k0 + lk);
-                float4 a = src[0], b = src[1];
-                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-                v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ws[lk + i][lrow] = v[i];
-        }
+        stash();
         __syncthreads();
+        if (k0 + kLK < kend) fetch(k0 + kLK);   // in flight while the tile below is used
 #pragma unroll 8
         for (int kk = 0; kk < kLK; ++kk) {
-            const float4 a = *reinterpret_cast<const float4 *>(&xs[kk][ty * 4]);
+            const float4 a0 = *reinterpret_cast<const float4 *>(&xs[kk][ty * 8]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&xs[kk][ty * 8 + 4]);
             const float4 b = *reinterpret_cast<const float4 *>(&ws[kk][tx * 4]);
-            const float av[4] = {a.x, a.y, a.z, a.w};
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
@@ -101,7 +116,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16 
         if (folded == 256) {
             folded = 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     tot[i][j] += acc[i][j];
@@ -111,13 +126,18 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16 
     }
     float *dst = partial + (size_t)blockIdx.z * T * E;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = t0 + ty * 4 + i;
+    for (int i = 0; i < 8; ++i) {
+        const int t = t0 + ty * 8 + i;
         if (t >= T) continue;
+        const int e = e0 + tx * 4;
+        if (e + 3 < E) {
+            *reinterpret_cast<float4 *>(dst + (size_t)t * E + e) =
+                make_float4(tot[i][0] + acc[i][0], tot[i][1] + acc[i][1], tot[i][2] + acc[i][2],
+                            tot[i][3] + acc[i][3]);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int e = e0 + tx * 4 + j;
-            if (e < E) dst[(size_t)t * E + e] = tot[i][j] + acc[i][j];
+            for (int j = 0; j < 4; ++j)
+                if (e + j < E) dst[(size_t)t * E + e + j] = tot[i][j] + acc[i][j];
         }
     }
 }
@@ -226,11 +246,16 @@ __global__ void __launch_bounds__(256) router_select_kernel(
 // Host launchers
 // ---------------------------------------------------------------------------
 
+// K slices of the logits: enough blocks for several per SM (the selection
+// sums the slices in a fixed order).  Slices stay a multiple of 32 wide and
+// at least 1024 wide, or 256 when the grid would not fill the GPU anyway.
 int router_slices(int T, int H, int E, int num_sms)
 {
     const int base = ((T + kLT - 1) / kLT) * ((E + kLE - 1) / kLE);
+    const int min_width = base < num_sms ? 256 : 1024;
     int ns = 1;
-    while (ns * 2 * base <= 2 * num_sms && (H / (ns * 2)) >= 256 && H % (ns * 2 * kLK) == 0) ns *= 2;
+    while (ns * base < 6 * num_sms && (H / (ns * 2)) >= min_width && H % (ns * 2 * kLK) == 0)
+        ns *= 2;
     return ns;
 }
 

@@ -11,12 +11,13 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from group_limited_routing_sigmoid_b200 import workloads as W
 from group_limited_routing_sigmoid_b200.binding import (BEAM_ERR_INVALID_ARG, BeamMoE,
                                                         BeamMoEError, route_static)
 from group_limited_routing_sigmoid_b200.build import build
 
-from parity import W_ABS
+from parity import NEAR_TIE, W_ABS
 
 pytestmark = pytest.mark.gpu
 
@@ -32,11 +33,19 @@ def test_route_static_matches_route(name, T):
     d.update(W.make_tokens(wl, "cuda", g, T=T))
     moe = BeamMoE.from_workload(wl, d, max_tokens=T)
     idx_ref, w_ref = moe.route(d["x"])
+    # the two entry points may split the router's K range differently (the
+    # static scratch caps the slices), so logits can differ by rounding:
+    # near-ties (the oracle's expert or group gap below the parity tests'
+    # threshold) are exempt from the index comparison, as in those tests
+    r = oracle.route(W.bf16_bits(d["x"]), d["router_w"].cpu().numpy(), d["bias"].cpu().numpy(),
+                     wl.n_group, wl.topk_group, wl.top_k)
+    keep = (r.gap_expert >= NEAR_TIE) & (r.gap_group >= NEAR_TIE)
     for _ in range(2):
         idx, w = route_static(d["x"], d["router_w"], d["bias"], wl.n_group, wl.topk_group, wl.top_k)
         torch.cuda.synchronize()
-        np.testing.assert_array_equal(idx.cpu().numpy(), idx_ref.cpu().numpy())
+        np.testing.assert_array_equal(idx.cpu().numpy()[keep], idx_ref.cpu().numpy()[keep])
         assert float((w - w_ref).abs().max()) <= W_ABS
+    assert keep.mean() > 0.99
     moe.close()
 
 
