@@ -191,7 +191,7 @@ def run_ours(args):
     if wl.post_norm:
         weights["gamma"] = batches[0]["gamma"]
     moe = BeamMoE.from_workload(wl, weights)
-    moe.set_gemm_tuning(0, args.gemm_tile, args.down_pair)
+    moe.set_gemm_tuning(0, args.gemm_tile, args.down_pair, args.cta_pairs)
     outs = [torch.empty(T, H, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     streams = [b["stream"] for b in batches]
 
@@ -407,6 +407,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm-tile", type=int, default=0, help="largest GEMM token tile (0 = auto)")
     ap.add_argument("--down-pair", type=int, default=-1, help="paired down tiles: -1 auto, 0, 1")
+    ap.add_argument("--cta-pairs", type=int, default=1, help="SM-pair GEMMs for large tiles: 1 or 0")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -58,7 +58,7 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_dispatch_info.argtypes = [P, P, I, P, P, P]
         lib.beam_moe_get_status.argtypes = [P, P]
         lib.beam_moe_set_wait_limit.argtypes = [P, ctypes.c_int64]
-        lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I]
+        lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I, I]
         lib.beam_moe_check_wait_timeout.argtypes = [P, P]
         lib.beam_moe_profile_begin.argtypes = [P, I]
         lib.beam_moe_profile_end.argtypes = [P, P, P]
@@ -209,9 +209,10 @@ class BeamMoE:
     def set_wait_limit(self, limit_ns: int):
         self._check(library().beam_moe_set_wait_limit(self._h, int(limit_ns)))
 
-    def set_gemm_tuning(self, ctas: int = 0, tile_rows: int = 0, down_pair: int = -1):
+    def set_gemm_tuning(self, ctas: int = 0, tile_rows: int = 0, down_pair: int = -1,
+                        cta_pairs: int = 1):
         self._check(library().beam_moe_set_gemm_tuning(self._h, int(ctas), int(tile_rows),
-                                                        int(down_pair)))
+                                                        int(down_pair), int(cta_pairs)))
 
     STAGES = ("router", "dispatch", "gate_up_gemm", "down_gemm", "combine")
 

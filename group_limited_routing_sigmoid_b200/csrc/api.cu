@@ -41,6 +41,7 @@ struct beam_moe {
     BoxMaps tm_xp, tm_h;             // box rows 16, 32, 64, 128, 256
     int tile_rows;                   // 0: chosen from T
     int down_pair;                   // -1: auto, 0: single tiles, 1: paired tiles
+    int use_pair;                    // 1: CTA-pair kernels for large token tiles (default)
     int last_T;
     std::vector<cudaEvent_t> prof_events;   // 6 per profiled forward pass
     int prof_max, prof_calls;
@@ -193,23 +194,38 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.tile_off = h->tile_off;
     g.ctl.status = h->status;
     g.ctl.limit_ns = h->wait_limit_ns;
+    // CTA pairs (cta_group::2) for large token tiles when the weight rows
+    // split into 256-row blocks; single CTAs otherwise
+    const bool use_pair = h->use_pair != 0 && gemm_pair_supported(BN) && h->I % 256 == 0 &&
+                          h->H % 256 == 0 && gemm_pair_max_ctas() >= 2;
+    int grid = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
+    if (use_pair) {
+        const int cap = gemm_pair_max_ctas();
+        grid = grid > cap ? cap : grid;
+        grid &= ~1;
+        if (grid < 2) grid = 2;
+    }
     g.K = h->H;
     g.R = h->I;
     g.out = h->hbuf;
-
-    const int grid = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
-    e = launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_xp, g, grid, s);
+    e = use_pair ? launch_grouped_gemm_pair(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_xp, g,
+                                            grid, s)
+                 : launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_xp, g,
+                                       grid, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "gate/up GEMM launch");
     prof_mark(h, s, 3);
     g.K = h->I;
     g.R = h->H;
     g.out = h->ybuf;
-
-    // pair the down projection's weight tiles when H allows; a lone 128-row
-    // tile per item for decode-sized token tiles keeps more items in flight
-    const bool pair = h->H % 256 == 0 && (h->down_pair == 1 || (h->down_pair < 0 && BN >= 64));
-    e = launch_grouped_gemm(pair ? GemmKind::kDownPaired : GemmKind::kDown, BN, h->tm_down,
-                            h->tm_down, h->tm_h, g, grid, s);
+    // pair the down projection's weight blocks (two blocks share a token
+    // tile) when H allows; lone blocks for decode-sized token tiles keep more
+    // items in flight
+    const int block_rows = use_pair ? 512 : 256;
+    const bool pair_down =
+        h->H % block_rows == 0 && (h->down_pair == 1 || (h->down_pair < 0 && BN >= 64));
+    const GemmKind dk = pair_down ? GemmKind::kDownPaired : GemmKind::kDown;
+    e = use_pair ? launch_grouped_gemm_pair(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s)
+                 : launch_grouped_gemm(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "down GEMM launch");
     prof_mark(h, s, 4);
 
@@ -309,6 +325,7 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     h->max_tokens = max_tokens;
     h->wait_limit_ns = 2000000000LL;
     h->down_pair = -1;
+    h->use_pair = 1;
 
     cudaError_t e = cudaGetDevice(&h->device);
     if (e == cudaSuccess)
@@ -393,9 +410,9 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     bool ok = make_map(&h->tm_gate, w_gate, E * inter, hidden, 128) &&
               make_map(&h->tm_up, w_up, E * inter, hidden, 128) &&
               make_map(&h->tm_down, w_down, E * hidden, inter, 128);
-    for (int i = 0; i < 5 && ok; ++i)
-        ok = make_map(&h->tm_xp.m[i], h->xp, P, hidden, 16u << i) &&
-             make_map(&h->tm_h.m[i], h->hbuf, P, inter, 16u << i);
+    for (int i = 0; i < 6 && ok; ++i)
+        ok = make_map(&h->tm_xp.m[i], h->xp, P, hidden, 8u << i) &&
+             make_map(&h->tm_h.m[i], h->hbuf, P, inter, 8u << i);
     if (!ok) {
         cudaFree(h->ws);
         delete h;
@@ -574,7 +591,7 @@ int beam_moe_profile_end(beam_moe_t h, float *stage_ms, int *calls)
     return BEAM_OK;
 }
 
-int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair)
+int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair, int cta_pairs)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
     if (ctas < 0 || ctas > 65535) return fail(h, BEAM_ERR_INVALID_ARG, "ctas outside [0, 65535]");
@@ -582,9 +599,11 @@ int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pai
         return fail(h, BEAM_ERR_INVALID_ARG, "tile_rows must be 0, 16, 32, 64, 128 or 256");
     if (down_pair < -1 || down_pair > 1)
         return fail(h, BEAM_ERR_INVALID_ARG, "down_pair outside [-1, 1]");
+    if (cta_pairs < 0 || cta_pairs > 1) return fail(h, BEAM_ERR_INVALID_ARG, "cta_pairs must be 0 or 1");
     h->gemm_ctas = ctas;
     h->tile_rows = tile_rows;
     h->down_pair = down_pair;
+    h->use_pair = cta_pairs;
     return BEAM_OK;
 }
 

@@ -1,5 +1,7 @@
 // Grouped expert GEMMs of the Beam MoE block on the 5th-generation tensor
-// cores (tcgen05 / TMEM), fed by TMA.
+// cores (tcgen05 / TMEM), fed by TMA: the single-CTA kernel, used for small
+// token tiles (decode).  The CTA-pair kernel for large tiles is in
+// grouped_gemm_pair.cu.
 //
 // Each Beam expert is a SwiGLU MLP with hidden 5120 and intermediate 2560
 // (launch blog "Introducing Beam", section "Mixture of Experts"); the SwiGLU
@@ -24,8 +26,8 @@
 //   down:    one or two A tiles (rows c0..c0+127 and c0+128..c0+255) that
 //            share the token tile, halving the token bytes per MMA.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over the item list):
-//   warp 0      TMA producer: K slices of 64 into a ring of smem stages;
+// Warp roles (320 threads, one CTA per SM, persistent over the item list):
+//   warp 0      TMA producer (lane 0);
 //   warp 1      TMEM allocator and UMMA issuer (one thread);
 //   warps 2..9  epilogue (two per TMEM lane quadrant): tcgen05.ld, SwiGLU or
 //               the plain accumulator, rounded to bf16, a 32x32 transpose
@@ -33,45 +35,25 @@
 // Accumulators are double-buffered in TMEM when two fit in its 512 columns,
 // so the epilogue of one item overlaps the mainloop of the next.  Every wait
 // is bounded (WaitCtl).
-#include "kernels.cuh"
+#include "gemm_common.cuh"
 
 namespace beam {
 
+using namespace gemm;
+
 namespace {
-
-constexpr int kBM = 128;          // weight rows per A tile (UMMA M)
-constexpr int kBK = 64;           // K per stage: one 128-byte swizzle row of bf16
-constexpr int kEpiWarps = 8;      // two per TMEM lane quadrant, alternating column chunks
-constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kMaxDynSmem = 232448;
-constexpr int kTableBytes = 3 * (1024 + 1) * 4 + 4;   // counts, offsets, tile_off (E <= 1024)
-constexpr int kBarrierBytes = 256;
-constexpr int kStagingWarpBytes = 2048;                // one 32-row x CH-column block per epilogue warp
-constexpr int kStagingBytes = kEpiWarps * kStagingWarpBytes;
-
-enum Epi { kSwiGLU = 0, kStoreBF16 = 1 };   // gate|up with SwiGLU; plain (down)
-
-constexpr int pow2_at_least(int v, int lo)
-{
-    int p = lo;
-    while (p < v) p <<= 1;
-    return p;
-}
 
 template <int BN, int NUM_A, int EPI>
 struct Cfg {
     static constexpr int A_BYTES = kBM * kBK * 2;
     static constexpr int B_BYTES = BN * kBK * 2;
     static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
-    static constexpr int STAGE_BUDGET =
-        kMaxDynSmem - 1024 - kBarrierBytes - kTableBytes - kStagingBytes;
-    static constexpr int STAGES_FIT = STAGE_BUDGET / STAGE_BYTES;
+    static constexpr int STAGES_FIT = kStageBudget / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
     static constexpr int ACC_COLS = NUM_A * BN;             // one accumulator buffer
     static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
     static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS, 32);
-    // epilogue columns per chunk: a 32 x CH block of bf16 outputs in the warp's staging
-    static constexpr int CH = BN >= 32 ? 32 : 16;
+    static constexpr int CH = BN >= 32 ? 32 : 16;           // epilogue columns per chunk
     static constexpr int ROWS_PER_ITEM = EPI == kSwiGLU ? kBM : NUM_A * kBM;
     static constexpr int SMEM_BYTES =
         1024 + STAGES * STAGE_BYTES + kStagingBytes + kBarrierBytes + kTableBytes;
@@ -81,49 +63,8 @@ struct Cfg {
     static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of the next tile");
     static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory");
     static_assert(EPI == kStoreBF16 || NUM_A == 2, "SwiGLU needs the gate and up tiles");
+    static_assert(32 * CH * 2 <= kStagingWarpBytes, "staging block");
 };
-
-struct Item {
-    int e, wt, row0, nrows;
-};
-
-// Item i of the list ordered (expert, weight tile, token tile): the expert is
-// the largest e with WT * tile_off[e] <= i; its count c is split into
-// nt = tile_off[e+1] - tile_off[e] tiles of ceil(c / nt) rows (the last may
-// be shorter).
-__device__ __forceinline__ Item decode_item(int i, int WT, int E, const int *s_counts,
-                                            const int *s_offsets, const int *s_tile)
-{
-    int lo = 0, hi = E - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (WT * s_tile[mid] <= i) lo = mid;
-        else hi = mid - 1;
-    }
-    Item it;
-    it.e = lo;
-    const int local = i - WT * s_tile[lo];
-    const int nt = s_tile[lo + 1] - s_tile[lo];
-    it.wt = local / nt;
-    const int tt = local - it.wt * nt;
-    const int c = s_counts[lo];
-    const int bal = (c + nt - 1) / nt;
-    it.row0 = s_offsets[lo] + tt * bal;
-    it.nrows = min(bal, c - tt * bal);
-    return it;
-}
-
-// silu(g) = g / (1 + e^-g) in FP32 with the fast exponential and divide; the
-// product with u is rounded to bf16 right after, which the approximations
-// (a few FP32 ulps) do not reach but in rare rounding-boundary cases.
-__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
-
-template <int N>
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&v)[N])
-{
-    if constexpr (N == 32) tmem_ld32(taddr, v);
-    else tmem_ld16(taddr, v);
-}
 
 }  // namespace
 
@@ -138,7 +79,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t *base_ptr = smem_raw + (base - raw_addr);
-    uint8_t *staging = base_ptr + C::STAGES * C::STAGE_BYTES;   // 16 KB, 1024-aligned
+    uint8_t *staging = base_ptr + C::STAGES * C::STAGE_BYTES;   // 1024-aligned
     uint8_t *bar_ptr = staging + kStagingBytes;
     uint64_t *full = reinterpret_cast<uint64_t *>(bar_ptr);
     uint64_t *empty = full + C::STAGES;
@@ -153,11 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    for (int i = threadIdx.x; i < p.E; i += kThreads) s_counts[i] = p.counts[i];
-    for (int i = threadIdx.x; i <= p.E; i += kThreads) {
-        s_offsets[i] = p.offsets[i];
-        s_tile[i] = p.tile_off[i];
-    }
+    load_tables(p, s_counts, s_offsets, s_tile);
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
@@ -216,8 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t sb = sa + NUM_A * C::A_BYTES;
                         int off = 0;
 #pragma unroll
-                        for (int bi = 4; bi >= 0; --bi) {   // boxes of 256, 128, 64, 32, 16 rows
-                            const int hgt = 16 << bi;
+                        for (int bi = 5; bi >= 1; --bi) {   // boxes of 256, 128, 64, 32, 16 rows
+                            const int hgt = 8 << bi;
                             if (hgt <= BN && n_load - off >= hgt) {
                                 tma_load_2d(sb + off * (kBK * 2), &tmB.m[bi], kb * kBK,
                                             it.row0 + off, fb, pol_x);
@@ -304,10 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue
-        constexpr int CH = C::CH;
-        constexpr int ESZ = 2;                             // bf16 outputs
-        constexpr int VPR = 32 * ESZ / 16;                 // 16-byte vectors per 32-row slice
-        static_assert(32 * CH * ESZ <= kStagingWarpBytes, "staging block");
         const int quad = warp & 3;                         // TMEM lanes this warp may access
         const int half = (warp - 2) >> 2;                  // which alternate column chunks
         uint8_t *stg = staging + (warp - 2) * kStagingWarpBytes;
@@ -321,44 +254,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
-            constexpr int NOUT = EPI == kSwiGLU ? 1 : NUM_A;
+            if constexpr (EPI == kSwiGLU) {
+                const int col0 = it.wt * C::ROWS_PER_ITEM + quad * 32;
+                epilogue_block<EPI, C::CH, BN>(taddr, it.nrows, it.row0, half, lane, stg,
+                                               p.out + col0, p.R);
+            } else {
 #pragma unroll 1
-            for (int a = 0; a < NOUT; ++a) {
-                // first output column (weight row) of this warp's 32-row slice
-                const int col0 = it.wt * C::ROWS_PER_ITEM + a * kBM + quad * 32;
-                uint8_t *out = reinterpret_cast<uint8_t *>(p.out) + (size_t)col0 * ESZ;
-#pragma unroll 1
-                for (int c0 = half * CH; c0 < it.nrows; c0 += 2 * CH) {
-                    uint32_t g[CH];
-                    tmem_ld<CH>(taddr + a * BN + c0, g);
-                    if constexpr (EPI == kSwiGLU) {
-                        uint32_t u[CH];
-                        tmem_ld<CH>(taddr + BN + c0, u);
-                        tmem_ld_wait();
-                        __nv_bfloat16 *sh = reinterpret_cast<__nv_bfloat16 *>(stg);
-#pragma unroll
-                        for (int j = 0; j < CH; ++j)
-                            sh[j * 32 + lane] = __float2bfloat16_rn(
-                                silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]));
-                    } else {
-                        tmem_ld_wait();
-                        __nv_bfloat16 *sh = reinterpret_cast<__nv_bfloat16 *>(stg);
-#pragma unroll
-                        for (int j = 0; j < CH; ++j)
-                            sh[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(g[j]));
-                    }
-                    __syncwarp();
-                    // token row c0+j of the slice: VPR vectors of 16 bytes
-#pragma unroll
-                    for (int v = lane; v < CH * VPR; v += 32) {
-                        const int j = v / VPR, part = v - j * VPR;
-                        if (c0 + j < it.nrows) {
-                            const uint4 val = *reinterpret_cast<const uint4 *>(stg + v * 16);
-                            *reinterpret_cast<uint4 *>(
-                                out + (size_t)(it.row0 + c0 + j) * p.R * ESZ + part * 16) = val;
-                        }
-                    }
-                    __syncwarp();
+                for (int a = 0; a < NUM_A; ++a) {
+                    const int col0 = it.wt * C::ROWS_PER_ITEM + a * kBM + quad * 32;
+                    epilogue_block<EPI, C::CH, 0>(taddr + a * BN, it.nrows, it.row0, half, lane,
+                                                  stg, p.out + col0, p.R);
                 }
             }
             tc_fence_before();
@@ -418,15 +323,13 @@ bool gemm_tile_supported(int BN)
     return BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256;
 }
 
-int gemm_rows_per_item(GemmKind kind) { return kind == GemmKind::kDownPaired ? 2 * kBM : kBM; }
-
 cudaError_t prepare_grouped_gemm(int E)
 {
     if (E > 1024) return cudaErrorInvalidValue;
     cudaError_t err;
 #define BEAM_PREP(BN)                                                        \
     if ((err = set_smem<BN, 2, kSwiGLU>()) != cudaSuccess) return err;       \
-    if ((err = set_smem<BN, 1, kStoreBF16>()) != cudaSuccess) return err;     \
+    if ((err = set_smem<BN, 1, kStoreBF16>()) != cudaSuccess) return err;    \
     if ((err = set_smem<BN, 2, kStoreBF16>()) != cudaSuccess) return err;
     BEAM_PREP(16)
     BEAM_PREP(32)
@@ -434,7 +337,7 @@ cudaError_t prepare_grouped_gemm(int E)
     BEAM_PREP(128)
     BEAM_PREP(256)
 #undef BEAM_PREP
-    return cudaSuccess;
+    return prepare_grouped_gemm_pair();
 }
 
 cudaError_t launch_grouped_gemm(GemmKind kind, int BN, const CUtensorMap &a0, const CUtensorMap &a1,

@@ -1,0 +1,364 @@
+// Grouped expert GEMMs of the Beam MoE block on CTA pairs: clusters of two
+// CTAs on two SMs share each tcgen05 MMA (cta_group::2).  Used for large
+// token tiles (prefill).  Same computation and item order as
+// grouped_gemm.cu; see there for the block's definition.
+//
+// A pair item covers 256 weight rows per A matrix and up to BN tokens.  CTA r
+// of the pair holds weight rows r*128 .. r*128+127 (its half of the MMA's
+// M = 256) and token rows r*N/2 .. r*N/2+N/2-1 (its half of N); the MMA,
+// issued by CTA 0, reads both CTAs' shared memory and writes each CTA's TMEM
+// (128 lanes, its weight rows, all N token columns).  Per SM this halves the
+// token bytes of every stage, so more stages fit in shared memory and more
+// weight bytes are in flight for the same MMA work.
+//
+// Synchronisation (every wait bounded):
+//   full[s]    in CTA 0: CTA 0's producer expects the bytes of both CTAs;
+//              both CTAs' TMA loads complete on it;
+//   empty[s]   in each CTA: the MMA's completion, multicast to both;
+//   tfull[a]   in each CTA: accumulator ready, multicast to both;
+//   tempty[a]  in CTA 0: both CTAs' epilogue threads arrive;
+//   drain      in each CTA: all MMAs complete, before TMEM is released.
+// Only local TMA loads (no multicast).
+#include "gemm_common.cuh"
+
+namespace beam {
+
+using namespace gemm;
+
+namespace {
+
+template <int BN, int NUM_A, int EPI>
+struct PairCfg {
+    static constexpr int HALF = BN / 2;                    // token rows per CTA, at most
+    static constexpr int A_BYTES = kBM * kBK * 2;
+    static constexpr int B_BYTES = HALF * kBK * 2;
+    static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
+    static constexpr int STAGES_FIT = kStageBudget / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
+    static constexpr int ACC_COLS = NUM_A * BN;            // per CTA: 128 lanes x N per matrix
+    static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
+    static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS, 32);
+    static constexpr int CH = 32;
+    static constexpr int ROWS_PER_ITEM = 2 * kBM * (EPI == kSwiGLU ? 1 : NUM_A);
+    static constexpr int SMEM_BYTES =
+        1024 + STAGES * STAGE_BYTES + kStagingBytes + kBarrierBytes + kTableBytes;
+    static_assert(STAGES >= 2, "pipeline needs two stages");
+    static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
+    static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair UMMA N");
+    static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of the next tile");
+    static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory");
+    static_assert(EPI == kStoreBF16 || NUM_A == 2, "SwiGLU needs the gate and up tiles");
+};
+
+constexpr uint16_t kPairMask = 0x3;
+
+}  // namespace
+
+template <int BN, int NUM_A, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
+                             const __grid_constant__ CUtensorMap tmA1,
+                             const __grid_constant__ BoxMaps tmB, GemmArgs p)
+{
+    using C = PairCfg<BN, NUM_A, EPI>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *base_ptr = smem_raw + (base - raw_addr);
+    uint8_t *staging = base_ptr + C::STAGES * C::STAGE_BYTES;
+    uint8_t *bar_ptr = staging + kStagingBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(bar_ptr);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *tfull = empty + C::STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    int *s_counts = reinterpret_cast<int *>(bar_ptr + kBarrierBytes);
+    int *s_offsets = s_counts + p.E;
+    int *s_tile = s_offsets + (p.E + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();     // 0: issues the MMAs
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    load_tables(p, s_counts, s_offsets, s_tile);
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 2 * 32 * kEpiWarps);
+        }
+        mbar_init(smem_u32(drain), 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tmA0);
+        if (NUM_A == 2) tma_prefetch_desc(&tmA1);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    cluster_sync();   // both CTAs' barriers exist before either signals the other
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int WT = p.R / C::ROWS_PER_ITEM;
+    const int total = WT * s_tile[p.E];
+    const int KB = p.K / kBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (lane 0)
+        const uint64_t pol_w = l2_policy_evict_first();
+        const uint64_t pol_x = l2_policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        long long issued = 0;
+        bool ok = true;
+        for (int item = pair; item < total && ok; item += npairs) {
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const int n_mma = (it.nrows + 15) & ~15;
+            const int half = n_mma >> 1;                    // this CTA's token rows
+            const int b_row = it.row0 + (int)rank * half;
+            // A rows of this CTA: its 128-row half of each 256-row block
+            const int a_base = it.e * p.R + it.wt * C::ROWS_PER_ITEM + (int)rank * kBM;
+            const uint32_t pair_bytes = 2u * (NUM_A * C::A_BYTES + half * (kBK * 2));
+            for (int kb = 0; kb < KB; ++kb) {
+                bool got = true;
+                if (lane == 0) {
+                    got = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl);
+                    if (got) {
+                        const uint32_t sa = base + stage * C::STAGE_BYTES;
+                        const uint32_t fb_local = smem_u32(&full[stage]);
+                        const uint32_t fb = mapa_shared(fb_local, 0);   // CTA 0's barrier
+                        if (rank == 0) mbar_arrive_expect_tx(fb_local, pair_bytes);
+                        tma_load_2d_pair(sa, &tmA0, kb * kBK, a_base, fb, pol_w);
+                        if (NUM_A == 2) {
+                            // gate|up: the up matrix at the same rows; down: the next 256-row block
+                            const int a_row1 = EPI == kSwiGLU ? a_base : a_base + 2 * kBM;
+                            tma_load_2d_pair(sa + C::A_BYTES, &tmA1, kb * kBK, a_row1, fb, pol_w);
+                        }
+                        const uint32_t sb = sa + NUM_A * C::A_BYTES;
+                        int off = 0;
+#pragma unroll
+                        for (int bi = 4; bi >= 0; --bi) {   // boxes of 128, 64, 32, 16, 8 rows
+                            const int hgt = 8 << bi;
+                            if (hgt <= C::HALF && half - off >= hgt) {
+                                tma_load_2d_pair(sb + off * (kBK * 2), &tmB.m[bi], kb * kBK,
+                                                 b_row + off, fb, pol_x);
+                                off += hgt;
+                            }
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                ++issued;
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0 && rank == 0) {
+            // Let both CTAs' copies in flight land (CTA 0's barrier counts
+            // both) before the pair leaves; time-bounded, status ignored.
+            long long n = issued < C::STAGES ? issued : C::STAGES;
+            int s = stage;
+            uint32_t ph = phase;
+            for (long long j = 0; j < n; ++j) {
+                if (s == 0) {
+                    s = C::STAGES - 1;
+                    ph ^= 1u;
+                } else {
+                    --s;
+                }
+                mbar_wait_drain(smem_u32(&full[s]), ph, p.ctl.limit_ns);
+            }
+        }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ------------------------------------------------ UMMA issuer (CTA 0)
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        bool issued_any = false;
+        int iter = 0;
+        for (int item = pair; item < total && ok; item += npairs, ++iter) {
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const int n_mma = (it.nrows + 15) & ~15;
+            const uint32_t idesc = umma_idesc_bf16_f32(2 * kBM, n_mma);
+            const int acc = iter % C::NBUF;
+            const uint32_t acc_phase = (uint32_t)(iter / C::NBUF) & 1u;
+            if (!mbar_wait_cluster(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.ctl)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait(smem_u32(&full[stage]), phase, p.ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = base + stage * C::STAGE_BYTES;
+                const uint32_t sb = sa + NUM_A * C::A_BYTES;
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k) {
+                    const uint64_t bdesc = umma_desc_sw128(sb + k * 32);
+                    const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+                    umma_bf16_pair(d0, umma_desc_sw128(sa + k * 32), bdesc, idesc, accum);
+                    if (NUM_A == 2)
+                        umma_bf16_pair(d0 + BN, umma_desc_sw128(sa + C::A_BYTES + k * 32), bdesc,
+                                       idesc, accum);
+                    issued_any = true;
+                }
+                umma_commit_pair(smem_u32(&empty[stage]), kPairMask);
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            umma_commit_pair(smem_u32(&tfull[acc]), kPairMask);
+        }
+        if (issued_any) umma_commit_pair(smem_u32(drain), kPairMask);
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int quad = warp & 3;
+        const int half_sel = (warp - 2) >> 2;
+        uint8_t *stg = staging + (warp - 2) * kStagingWarpBytes;
+        const uint32_t tempty_remote0 = mapa_shared(smem_u32(&tempty[0]), 0);
+        const uint32_t tempty_remote1 = mapa_shared(smem_u32(&tempty[1]), 0);
+        int iter = 0;
+        for (int item = pair; item < total; item += npairs, ++iter) {
+            const int acc = iter % C::NBUF;
+            const uint32_t acc_phase = (uint32_t)(iter / C::NBUF) & 1u;
+            const bool ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.ctl);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const uint32_t taddr =
+                tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
+            if constexpr (EPI == kSwiGLU) {
+                const int col0 = it.wt * C::ROWS_PER_ITEM + (int)rank * kBM + quad * 32;
+                epilogue_block<EPI, C::CH, BN>(taddr, it.nrows, it.row0, half_sel, lane, stg,
+                                               p.out + col0, p.R);
+            } else {
+#pragma unroll 1
+                for (int a = 0; a < NUM_A; ++a) {
+                    const int col0 =
+                        it.wt * C::ROWS_PER_ITEM + a * 2 * kBM + (int)rank * kBM + quad * 32;
+                    epilogue_block<EPI, C::CH, 0>(taddr + a * BN, it.nrows, it.row0, half_sel,
+                                                  lane, stg, p.out + col0, p.R);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_cluster(acc == 0 ? tempty_remote0 : tempty_remote1);
+        }
+    }
+
+    // Both CTAs: no TMEM release until CTA 0's MMAs are complete.
+    if (warp == 1 && lane == 0 && pair < total)
+        mbar_wait_drain(smem_u32(drain), 0, p.ctl.limit_ns);
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    cluster_sync();   // no CTA leaves while the other may still signal it
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+namespace {
+int g_pair_max_ctas = 0;
+
+template <int BN, int NUM_A, int EPI>
+cudaError_t set_smem_pair()
+{
+    return cudaFuncSetAttribute(grouped_gemm_pair_kernel<BN, NUM_A, EPI>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                PairCfg<BN, NUM_A, EPI>::SMEM_BYTES);
+}
+
+template <int BN, int NUM_A, int EPI>
+cudaError_t launch_pair(const CUtensorMap &a0, const CUtensorMap &a1, const BoxMaps &b,
+                        const GemmArgs &args, int grid, cudaStream_t stream)
+{
+    grouped_gemm_pair_kernel<BN, NUM_A, EPI>
+        <<<grid, kThreads, PairCfg<BN, NUM_A, EPI>::SMEM_BYTES, stream>>>(a0, a1, b, args);
+    return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_pair_kind(GemmKind kind, const CUtensorMap &a0, const CUtensorMap &a1,
+                             const BoxMaps &b, const GemmArgs &args, int grid, cudaStream_t stream)
+{
+    switch (kind) {
+        case GemmKind::kGateUp:
+            return launch_pair<BN, 2, kSwiGLU>(a0, a1, b, args, grid, stream);
+        case GemmKind::kDown:
+            return launch_pair<BN, 1, kStoreBF16>(a0, a1, b, args, grid, stream);
+        case GemmKind::kDownPaired:
+            return launch_pair<BN, 2, kStoreBF16>(a0, a1, b, args, grid, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+}  // namespace
+
+bool gemm_pair_supported(int BN) { return BN == 64 || BN == 128 || BN == 256; }
+
+int gemm_pair_max_ctas() { return g_pair_max_ctas; }
+
+cudaError_t prepare_grouped_gemm_pair()
+{
+    cudaError_t err;
+#define BEAM_PREP_PAIR(BN)                                                        \
+    if ((err = set_smem_pair<BN, 2, kSwiGLU>()) != cudaSuccess) return err;       \
+    if ((err = set_smem_pair<BN, 1, kStoreBF16>()) != cudaSuccess) return err;    \
+    if ((err = set_smem_pair<BN, 2, kStoreBF16>()) != cudaSuccess) return err;
+    BEAM_PREP_PAIR(64)
+    BEAM_PREP_PAIR(128)
+    BEAM_PREP_PAIR(256)
+#undef BEAM_PREP_PAIR
+    // How many pairs fit at once (one CTA per SM; pairs must sit on SM pairs
+    // of one GPC), so that the persistent grid is fully resident.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = PairCfg<256, 2, kSwiGLU>::SMEM_BYTES;
+    cfg.numAttrs = 0;   // the cluster shape comes from the kernel's __cluster_dims__
+    int clusters = 0;
+    err = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<256, 2, kSwiGLU>, &cfg);
+    if (err != cudaSuccess) return err;
+    g_pair_max_ctas = 2 * clusters;
+    return cudaSuccess;
+}
+
+cudaError_t launch_grouped_gemm_pair(GemmKind kind, int BN, const CUtensorMap &a0,
+                                     const CUtensorMap &a1, const BoxMaps &b,
+                                     const GemmArgs &args, int grid, cudaStream_t stream)
+{
+    if (grid < 2 || grid % 2 != 0) return cudaErrorInvalidValue;
+    switch (BN) {
+        case 64: return launch_pair_kind<64>(kind, a0, a1, b, args, grid, stream);
+        case 128: return launch_pair_kind<128>(kind, a0, a1, b, args, grid, stream);
+        case 256: return launch_pair_kind<256>(kind, a0, a1, b, args, grid, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace beam

@@ -53,10 +53,10 @@ struct GemmArgs {
     WaitCtl ctl;
 };
 
-// Tensor maps of one activation buffer with boxes of 16, 32, 64, 128 and 256
-// rows (64 columns each): a token tile is loaded as a sum of these.
+// Tensor maps of one activation buffer with boxes of 8, 16, 32, 64, 128 and
+// 256 rows (64 columns each): a token tile is loaded as a sum of these.
 struct BoxMaps {
-    CUtensorMap m[5];
+    CUtensorMap m[6];
 };
 
 enum class GemmKind {
@@ -70,7 +70,16 @@ cudaError_t launch_grouped_gemm(GemmKind kind, int BN, const CUtensorMap &a0,
                                 int grid, cudaStream_t stream);
 cudaError_t prepare_grouped_gemm(int E);   // sets shared-memory limits once per device
 bool gemm_tile_supported(int BN);
-int gemm_rows_per_item(GemmKind kind);
+
+// CTA-pair version (cta_group::2, clusters of two CTAs) for token tiles of
+// 64..256 rows: the pair shares each MMA, each CTA holding half the token
+// tile.  `grid` must be even.
+cudaError_t launch_grouped_gemm_pair(GemmKind kind, int BN, const CUtensorMap &a0,
+                                     const CUtensorMap &a1, const BoxMaps &b,
+                                     const GemmArgs &args, int grid, cudaStream_t stream);
+cudaError_t prepare_grouped_gemm_pair();
+bool gemm_pair_supported(int BN);
+int gemm_pair_max_ctas();   // CTAs of the pair kernels that can be resident at once (even)
 
 // ---------------------------------------------------------------- combine
 struct CombineArgs {

@@ -64,6 +64,10 @@ WORKLOADS: Dict[str, Workload] = {
     # small block: H=256, 32 experts in 8 groups of 4, I=128
     "tiny": Workload("tiny", T=64, hidden=256, n_experts=32, n_group=8, topk_group=4, top_k=8,
                      inter=128),
+    # small block whose weight rows split into 256-row blocks (H=512, I=256):
+    # covers the CTA-pair GEMM path at sizes the oracle checks in full
+    "small": Workload("small", T=1024, hidden=512, n_experts=32, n_group=8, topk_group=4, top_k=8,
+                      inter=256),
     # Beam shape, decode batch of 64 tokens
     "decode": Workload("decode", T=64, **_BEAM),
     # Beam shape, prefill of 8192 tokens, near-uniform routing

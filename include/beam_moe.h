@@ -206,11 +206,15 @@ int beam_moe_set_wait_limit(beam_moe_t h, int64_t limit_ns);
  * tile_rows       largest token tile: 16, 32, 64, 128 or 256 rows, or 0 to
  *                 choose from the mean number of tokens per expert (default).
  * down_pair       -1: choose (default); 0: the down projection takes one
- *                 128-row weight tile per work item; 1: two consecutive tiles
- *                 that share the token tile (needs hidden % 256 == 0, else
- *                 ignored).
+ *                 weight block per work item; 1: two consecutive blocks that
+ *                 share the token tile (needs hidden to be a multiple of two
+ *                 blocks, else ignored).
+ * cta_pairs       1 (default): token tiles of 64 rows or more run on pairs of
+ *                 SMs that share each MMA (needs inter and hidden to be
+ *                 multiples of 256); 0: one CTA per SM always.
  */
-int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair);
+int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair,
+                             int cta_pairs);
 
 /*
  * Per-stage timing of forward passes, for measurement.  After

@@ -64,6 +64,24 @@ def test_tiny_block(T, ctas, tile, pair):
     moe.close()
 
 
+# (T, GEMM CTAs, largest token tile, paired down tiles, CTA pairs): H=512, I=256
+SMALL_CASES = [(1024, 0, 0, -1, 1), (1024, 0, 0, -1, 0), (1024, 0, 64, 0, 1), (1024, 4, 128, 1, 1),
+               (1024, 0, 256, 0, 1), (3000, 0, 256, 1, 1), (3000, 6, 256, 1, 1), (777, 0, 128, -1, 1),
+               (2048, 2, 64, 1, 1), (64, 0, 64, -1, 1)]
+
+
+@pytest.mark.parametrize("T,ctas,tile,pair,pairs", SMALL_CASES)
+def test_small_block(T, ctas, tile, pair, pairs):
+    wl = W.WORKLOADS["small"]
+    d = _inputs(wl, T)
+    moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    moe.set_gemm_tuning(ctas, tile, pair, pairs)
+    rep = check_block(wl, d, moe)
+    _log(f"small_T{T}_ctas{ctas}_tile{tile}_pair{pair}_pairs{pairs}", rep)
+    assert rep.ok(), rep
+    moe.close()
+
+
 @pytest.mark.parametrize("norm", [True, False])
 def test_tiny_residual(norm):
     wl = dataclasses.replace(W.WORKLOADS["tiny"], post_norm=norm, residual_k=20)
