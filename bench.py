@@ -191,7 +191,7 @@ def run_ours(args):
     if wl.post_norm:
         weights["gamma"] = batches[0]["gamma"]
     moe = BeamMoE.from_workload(wl, weights)
-    moe.set_gemm_tuning(0, args.gemm_tile, args.down_pair, args.cta_pairs)
+    moe.set_gemm_tuning(0, args.gemm_tile, args.down_pair, args.cta_pairs, args.router)
     outs = [torch.empty(T, H, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     streams = [b["stream"] for b in batches]
 
@@ -231,6 +231,7 @@ def run_ours(args):
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
     calls, stage_ms = moe.profile_end()
+    rederived = moe.router_stats()
     if moe.get_status() != 0:
         raise SystemExit("a device-side wait ran out during the timed region")
     ms_max = max_over_ranks(ms, dist, dev)
@@ -304,6 +305,7 @@ def run_ours(args):
                    "parallelism": f"{ws} independent replicas (data parallel, no collective on the data path)"},
         "hbm_fraction_whole_step": round(step_bytes / (ms_max / steps_done * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
         "stage_ms": stage_avg,
+        "router_tokens_rederived_last_step": rederived,
         "clocks": sampler.report(),
         "e2e": {"value": round(whole_job_tokens_per_s(ws, e2e_steps, T, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0),
@@ -408,6 +410,7 @@ def main():
     ap.add_argument("--gemm-tile", type=int, default=0, help="largest GEMM token tile (0 = auto)")
     ap.add_argument("--down-pair", type=int, default=-1, help="paired down tiles: -1 auto, 0, 1")
     ap.add_argument("--cta-pairs", type=int, default=1, help="SM-pair GEMMs for large tiles: 1 or 0")
+    ap.add_argument("--router", type=int, default=-1, help="router logits: -1 auto, 0 CUDA cores, 1 tensor cores")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -25,7 +25,7 @@ BEAM_ERR_TIMEOUT = -5
 # every entry point declared in include/beam_moe.h
 SYMBOLS = (
     "beam_moe_create", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_forward",
-    "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_get_status",
+    "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_get_status",
     "beam_moe_set_wait_limit", "beam_moe_set_gemm_tuning", "beam_moe_profile_begin",
     "beam_moe_profile_end", "beam_moe_check_wait_timeout", "beam_moe_last_error",
     "beam_moe_create_error", "beam_moe_destroy",
@@ -57,8 +57,9 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_forward_host.argtypes = [P, P, P, I, P, P, I]
         lib.beam_moe_dispatch_info.argtypes = [P, P, I, P, P, P]
         lib.beam_moe_get_status.argtypes = [P, P]
+        lib.beam_moe_router_stats.argtypes = [P, P, P]
         lib.beam_moe_set_wait_limit.argtypes = [P, ctypes.c_int64]
-        lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I, I]
+        lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I, I, I]
         lib.beam_moe_check_wait_timeout.argtypes = [P, P]
         lib.beam_moe_profile_begin.argtypes = [P, I]
         lib.beam_moe_profile_end.argtypes = [P, P, P]
@@ -203,6 +204,13 @@ class BeamMoE:
             offsets.ctypes.data_as(ctypes.c_void_p), pair_row.ctypes.data_as(ctypes.c_void_p)))
         return counts, offsets, pair_row
 
+    def router_stats(self, stream=None) -> int:
+        """Tokens of the last call whose routing was re-derived on the exact path."""
+        n = ctypes.c_int32()
+        self._check(library().beam_moe_router_stats(self._h, _stream(stream),
+                                                     ctypes.cast(ctypes.pointer(n), ctypes.c_void_p)))
+        return n.value
+
     def get_status(self, stream=None) -> int:
         return library().beam_moe_get_status(self._h, _stream(stream))
 
@@ -210,9 +218,10 @@ class BeamMoE:
         self._check(library().beam_moe_set_wait_limit(self._h, int(limit_ns)))
 
     def set_gemm_tuning(self, ctas: int = 0, tile_rows: int = 0, down_pair: int = -1,
-                        cta_pairs: int = 1):
+                        cta_pairs: int = 1, router_mode: int = -1):
         self._check(library().beam_moe_set_gemm_tuning(self._h, int(ctas), int(tile_rows),
-                                                        int(down_pair), int(cta_pairs)))
+                                                        int(down_pair), int(cta_pairs),
+                                                        int(router_mode)))
 
     STAGES = ("router", "dispatch", "gate_up_gemm", "down_gemm", "combine")
 

@@ -38,6 +38,11 @@ struct beam_moe {
     float *res_stage;
 
     CUtensorMap tm_gate, tm_up, tm_down;
+    CUtensorMap tm_wcat;             // router weight as three bf16 pieces [E, 3H]
+    __nv_bfloat16 *wcat;
+    int router_mode;                 // -1: auto, 0: FP32 SIMT, 1: tensor cores, 2: 1 + every token re-derived
+    int *fix_list;                   // [max_tokens] tokens re-derived on the exact path
+    int *fix_count;
     BoxMaps tm_xp, tm_h;             // box rows 16, 32, 64, 128, 256
     int tile_rows;                   // 0: chosen from T
     int down_pair;                   // -1: auto, 0: single tiles, 1: paired tiles
@@ -130,6 +135,34 @@ int check_device(beam_moe *h)
     return BEAM_OK;
 }
 
+// Tensor-core router slices: the fewest K slices (dividing the 3H/64 steps,
+// each at least 16 steps) that give two work items per SM.
+int router_mma_slices(int T, int H, int E, int num_sms)
+{
+    const int items = ((E + router_mma_experts_per_tile() - 1) / router_mma_experts_per_tile()) *
+                      ((T + router_mma_tokens_per_tile() - 1) / router_mma_tokens_per_tile());
+    const int kb = 3 * H / 64;
+    int best = 1;
+    for (int d = 1; d <= kb / 16; ++d) {
+        if (kb % d) continue;
+        best = d;
+        if (items * d >= 2 * num_sms) break;
+    }
+    return best;
+}
+
+bool router_on_tensor_cores(const beam_moe *h, int T)
+{
+    if (h->router_mode >= 0) return h->router_mode >= 1;
+    return T >= 512;
+}
+
+// Decision margin below which a token's routing is re-derived from FP32
+// CUDA-core logits: the tensor-core logits' accumulation error stays below
+// 4e-5 (logit units, measured against exact sums at 320-step chains), i.e.
+// below 1e-5 in sigmoid-score units; 4e-5 leaves a factor of four.
+constexpr float kRouterMargin = 4e-5f;
+
 int run_router(beam_moe *h, cudaStream_t s, const void *x, int T, int32_t *idx, float *w,
                float *logits)
 {
@@ -143,12 +176,55 @@ int run_router(beam_moe *h, cudaStream_t s, const void *x, int T, int32_t *idx, 
     a.n_group = h->n_group;
     a.topk_group = h->topk_group;
     a.top_k = h->top_k;
-    a.nslice = router_slices(T, h->H, h->E, h->num_sms);   // the workspace holds nslice * T rows
     a.partial = h->partial;
     a.idx = idx;
     a.w = w;
     a.logits_out = logits;
-    cudaError_t e = launch_router(a, s);
+    cudaError_t e;
+    if (!logits && router_on_tensor_cores(h, T)) {
+        CUtensorMap tmx;
+        if (!make_map(&tmx, x, (uint64_t)T, (uint64_t)h->H, (uint32_t)router_mma_tokens_per_tile()))
+            return fail(h, BEAM_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+        RouterMmaArgs m;
+        m.T = T;
+        m.E = h->E;
+        m.nslice = router_mma_slices(T, h->H, h->E, h->num_sms);
+        m.kb_per_slice = 3 * h->H / 64 / m.nslice;
+        m.kb_per_h = h->H / 64;
+        m.partial = h->partial;
+        m.ctl.status = h->status;
+        m.ctl.limit_ns = h->wait_limit_ns;
+        const int items = ((h->E + router_mma_experts_per_tile() - 1) / router_mma_experts_per_tile()) *
+                          ((T + router_mma_tokens_per_tile() - 1) / router_mma_tokens_per_tile()) *
+                          m.nslice;
+        e = cudaMemsetAsync(h->fix_count, 0, sizeof(int), s);
+        if (e == cudaSuccess)
+            e = launch_router_mma(h->tm_wcat, tmx, m, items < h->num_sms ? items : h->num_sms, s);
+        if (e == cudaSuccess) {
+            // select on the tensor-core logits, listing tokens whose margins
+            // are too thin for their accumulation error ...
+            a.nslice = m.nslice;
+            SelectExtra ex;
+            ex.margin = h->router_mode == 2 ? INFINITY : kRouterMargin;
+            ex.fix_list = h->fix_list;
+            ex.fix_count = h->fix_count;
+            e = launch_router_select(a, ex, 0, s);
+        }
+        if (e == cudaSuccess)   // ... recompute theirs in FP32 on CUDA cores ...
+            e = launch_router_fix(a.x, h->router_w, h->H, h->E, T, h->fix_list, h->fix_count,
+                                  h->partial, 4 * h->num_sms, s);
+        if (e == cudaSuccess) {   // ... and select them again
+            RouterArgs b = a;
+            b.nslice = 1;
+            SelectExtra ex;
+            ex.token_list = h->fix_list;
+            ex.list_count = h->fix_count;
+            e = launch_router_select(b, ex, 4 * h->num_sms, s);
+        }
+    } else {
+        a.nslice = router_slices(T, h->H, h->E, h->num_sms);   // the workspace holds nslice * T rows
+        e = launch_router(a, s);
+    }
     return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "router launch");
 }
 
@@ -326,6 +402,7 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     h->wait_limit_ns = 2000000000LL;
     h->down_pair = -1;
     h->use_pair = 1;
+    h->router_mode = -1;
 
     cudaError_t e = cudaGetDevice(&h->device);
     if (e == cudaSuccess)
@@ -339,11 +416,14 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     // Workspace
     const size_t T = (size_t)max_tokens, E = (size_t)n_experts, P = T * top_k;
     const size_t nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
-    // router partial sums: the largest nslice(t) * t over t <= max_tokens
+    // router partial sums: the largest nslice(t) * t over t <= max_tokens, for
+    // either router path
     size_t partial_rows = 0;
     for (int t = 1; t <= max_tokens; ++t) {
-        const size_t r = (size_t)router_slices(t, hidden, n_experts, h->num_sms) * t;
-        if (r > partial_rows) partial_rows = r;
+        const size_t r1 = (size_t)router_slices(t, hidden, n_experts, h->num_sms) * t;
+        const size_t r2 = (size_t)router_mma_slices(t, hidden, n_experts, h->num_sms) * t;
+        if (r1 > partial_rows) partial_rows = r1;
+        if (r2 > partial_rows) partial_rows = r2;
     }
     size_t off = 0;
     auto carve = [&](size_t bytes) {
@@ -369,6 +449,8 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     const size_t o_xs = carve(T * hidden * 2);
     const size_t o_os = carve(T * hidden * 2);
     const size_t o_rs = carve(T * hidden * 4);
+    const size_t o_wcat = carve(E * 3 * (size_t)hidden * 2);
+    const size_t o_fix = carve((T + 1) * 4);
     h->ws_bytes = off;
     e = cudaMalloc(&h->ws, h->ws_bytes);
     if (e != cudaSuccess) {
@@ -397,9 +479,19 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     h->x_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_xs);
     h->out_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_os);
     h->res_stage = reinterpret_cast<float *>(b + o_rs);
+    h->wcat = reinterpret_cast<__nv_bfloat16 *>(b + o_wcat);
+    h->fix_count = reinterpret_cast<int *>(b + o_fix);
+    h->fix_list = h->fix_count + 1;
+    e = cudaMemset(h->fix_count, 0, sizeof(int));
     e = cudaMemset(h->status, 0, sizeof(int));
     if (e == cudaSuccess) e = prepare_grouped_gemm(n_experts);
     if (e == cudaSuccess) e = prepare_dispatch(n_experts);
+    if (e == cudaSuccess) e = prepare_router_mma();
+    if (e == cudaSuccess) e = prepare_router_fix(hidden);
+    // the router weight's bf16 pieces for the tensor-core router (the weight
+    // is borrowed and must not change while the handle lives)
+    if (e == cudaSuccess) e = launch_router_split(router_w, n_experts, hidden, h->wcat, 0);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(0);
     if (e != cudaSuccess) {
         int rc = cuda_fail(nullptr, e, "workspace / kernel set-up");
         cudaFree(h->ws);
@@ -407,7 +499,8 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
         return rc;
     }
 
-    bool ok = make_map(&h->tm_gate, w_gate, E * inter, hidden, 128) &&
+    bool ok = make_map(&h->tm_wcat, h->wcat, E, 3 * (uint64_t)hidden, 128) &&
+              make_map(&h->tm_gate, w_gate, E * inter, hidden, 128) &&
               make_map(&h->tm_up, w_up, E * inter, hidden, 128) &&
               make_map(&h->tm_down, w_down, E * hidden, inter, 128);
     for (int i = 0; i < 6 && ok; ++i)
@@ -517,6 +610,17 @@ int beam_moe_dispatch_info(beam_moe_t h, void *stream, int T, int32_t *counts_ho
     return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "dispatch info copy");
 }
 
+int beam_moe_router_stats(beam_moe_t h, void *stream, int32_t *rederived_host)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    if (!rederived_host) return fail(h, BEAM_ERR_INVALID_ARG, "rederived_host is NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(rederived_host, h->fix_count, sizeof(int32_t),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "router stats copy");
+}
+
 int beam_moe_get_status(beam_moe_t h, void *stream)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
@@ -591,7 +695,8 @@ int beam_moe_profile_end(beam_moe_t h, float *stage_ms, int *calls)
     return BEAM_OK;
 }
 
-int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair, int cta_pairs)
+int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair, int cta_pairs,
+                             int router_mode)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
     if (ctas < 0 || ctas > 65535) return fail(h, BEAM_ERR_INVALID_ARG, "ctas outside [0, 65535]");
@@ -600,6 +705,9 @@ int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pai
     if (down_pair < -1 || down_pair > 1)
         return fail(h, BEAM_ERR_INVALID_ARG, "down_pair outside [-1, 1]");
     if (cta_pairs < 0 || cta_pairs > 1) return fail(h, BEAM_ERR_INVALID_ARG, "cta_pairs must be 0 or 1");
+    if (router_mode < -1 || router_mode > 2)
+        return fail(h, BEAM_ERR_INVALID_ARG, "router_mode outside [-1, 2]");
+    h->router_mode = router_mode;
     h->gemm_ctas = ctas;
     h->tile_rows = tile_rows;
     h->down_pair = down_pair;

@@ -18,7 +18,40 @@ struct RouterArgs {
     float *logits_out;        // [T, E] or nullptr
 };
 int router_slices(int T, int H, int E, int num_sms);
-cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream);
+cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream);          // SIMT logits + selection
+
+// Selection extras: a decision-margin check that lists tokens for the exact
+// path, or selection of listed tokens only (logits in compact rows).
+struct SelectExtra {
+    float margin = 0.f;
+    int *fix_list = nullptr;
+    int *fix_count = nullptr;
+    const int *token_list = nullptr;
+    const int *list_count = nullptr;
+};
+cudaError_t launch_router_select(const RouterArgs &a, const SelectExtra &ex, int max_blocks,
+                                 cudaStream_t stream);
+cudaError_t prepare_router_fix(int H);
+// FP32 CUDA-core logits of the listed tokens into compact rows of `logits`.
+cudaError_t launch_router_fix(const __nv_bfloat16 *x, const float *w, int H, int E, int T,
+                              const int *list, const int *count, float *logits, int grid,
+                              cudaStream_t stream);
+
+// Tensor-core logits: W split into bf16 pieces (Wcat [E, 3H]) x tokens.
+struct RouterMmaArgs {
+    int T, E;
+    int nslice;          // K slices of the concatenated 3H
+    int kb_per_slice;    // 64-wide K steps per slice
+    int kb_per_h;        // H / 64 (the token operand wraps around every H)
+    float *partial;      // [nslice, T, E]
+    WaitCtl ctl;
+};
+cudaError_t launch_router_split(const float *w, int E, int H, __nv_bfloat16 *wcat, cudaStream_t s);
+cudaError_t prepare_router_mma();
+cudaError_t launch_router_mma(const CUtensorMap &tmW, const CUtensorMap &tmX,
+                              const RouterMmaArgs &a, int grid, cudaStream_t stream);
+int router_mma_tokens_per_tile();
+int router_mma_experts_per_tile();
 
 // --------------------------------------------------------------- dispatch
 constexpr int kDispatchBlock = 1024;   // pairs per counting block

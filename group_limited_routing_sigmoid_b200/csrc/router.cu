@@ -144,101 +144,209 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16 
 
 // ---------------------------------------------------------------------------
 // Selection: one warp per token; lane l owns experts l*EPL .. l*EPL+EPL-1,
-// so a group of g experts spans g/EPL consecutive lanes.
+// so a group of g experts spans g/EPL consecutive lanes.  Grid-stride over
+// the tokens.  Optional extras (SelectExtra):
+//   margin > 0: tokens whose decision margin -- the smallest gap between
+//     neighbours in the ranking of the top k+1 candidates of the kept groups
+//     (it decides the chosen set and its order), or the weakest kept group's
+//     score minus the strongest dropped one's -- is below `margin` are
+//     appended to fix_list (their logits are recomputed on CUDA cores);
+//   token_list: select only the listed tokens, whose logits are the compact
+//     rows 0..*list_count-1 of `partial` (one slice).
 // ---------------------------------------------------------------------------
 template <int EPL>
 __global__ void __launch_bounds__(256) router_select_kernel(
     const float *__restrict__ partial, int nslice, int T, int E, int n_group, int topk_group,
     int top_k, const float *__restrict__ bias, int32_t *__restrict__ idx_out,
-    float *__restrict__ w_out, float *__restrict__ logits_out)
+    float *__restrict__ w_out, float *__restrict__ logits_out, SelectExtra ex)
 {
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= T) return;
     const int lpg = (E / n_group) / EPL;   // lanes per group (power of two)
     const int my_group = lane / lpg;
     const int e_base = lane * EPL;
+    const int limit = ex.token_list ? min(*ex.list_count, T) : T;
+    const int stride = gridDim.x * (blockDim.x >> 5);
+    for (int wi = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wi < limit; wi += stride) {
+        const int t = ex.token_list ? ex.token_list[wi] : wi;   // output row
+        const int r = wi;                                         // logits row
 
-    float s[EPL], b[EPL];
-#pragma unroll
-    for (int m = 0; m < EPL; ++m) {
-        const int e = e_base + m;
-        float l = 0.f;
-        for (int q = 0; q < nslice; ++q) l += partial[((size_t)q * T + t) * E + e];
-        if (logits_out) logits_out[(size_t)t * E + e] = l;
-        s[m] = 1.0f / (1.0f + expf(-l));
-        b[m] = s[m] + bias[e];
-    }
-
-    // group score: sum of the group's two largest biased scores
-    float t1 = -INFINITY, t2 = -INFINITY;
-#pragma unroll
-    for (int m = 0; m < EPL; ++m) {
-        if (b[m] > t1) {
-            t2 = t1;
-            t1 = b[m];
-        } else if (b[m] > t2) {
-            t2 = b[m];
-        }
-    }
-    for (int off = 1; off < lpg; off <<= 1) {
-        const float o1 = __shfl_xor_sync(0xffffffffu, t1, off);
-        const float o2 = __shfl_xor_sync(0xffffffffu, t2, off);
-        const float hi = fmaxf(t1, o1);
-        const float lo = fmaxf(fminf(t1, o1), fmaxf(t2, o2));
-        t1 = hi;
-        t2 = lo;
-    }
-    const float gs = t1 + t2;
-
-    // keep the topk_group best groups (ties to the lower group index)
-    int rank = 0;
-    for (int j = 0; j < n_group; ++j) {
-        const float v = __shfl_sync(0xffffffffu, gs, j * lpg);
-        rank += (v > gs || (v == gs && j < my_group)) ? 1 : 0;
-    }
-    const bool kept = rank < topk_group;
-
-    float cand[EPL];
-#pragma unroll
-    for (int m = 0; m < EPL; ++m) cand[m] = kept ? b[m] : -INFINITY;
-    uint32_t taken = 0;
-    int my_idx = 0;
-    float my_s = 0.f, ssum = 0.f;
-    for (int r = 0; r < top_k; ++r) {
-        float bv = -INFINITY, bs = 0.f;
-        int bi = 0x7fffffff;
+        float s[EPL], b[EPL];
 #pragma unroll
         for (int m = 0; m < EPL; ++m) {
-            if (taken & (1u << m)) continue;
             const int e = e_base + m;
-            if (cand[m] > bv || (cand[m] == bv && e < bi)) {
-                bv = cand[m];
-                bi = e;
-                bs = s[m];
-            }
+            float l = 0.f;
+            for (int q = 0; q < nslice; ++q) l += partial[((size_t)q * T + r) * E + e];
+            if (logits_out) logits_out[(size_t)t * E + e] = l;
+            s[m] = 1.0f / (1.0f + expf(-l));
+            b[m] = s[m] + bias[e];
         }
+
+        // group score: sum of the group's two largest biased scores
+        float t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-            if (ov > bv || (ov == bv && oi < bi)) {
-                bv = ov;
-                bi = oi;
-                bs = os;
+        for (int m = 0; m < EPL; ++m) {
+            if (b[m] > t1) {
+                t2 = t1;
+                t1 = b[m];
+            } else if (b[m] > t2) {
+                t2 = b[m];
             }
         }
-        if (bi / EPL == lane) taken |= 1u << (bi - e_base);
-        if (lane == r) {
-            my_idx = bi;
-            my_s = bs;
+        for (int off = 1; off < lpg; off <<= 1) {
+            const float o1 = __shfl_xor_sync(0xffffffffu, t1, off);
+            const float o2 = __shfl_xor_sync(0xffffffffu, t2, off);
+            const float hi = fmaxf(t1, o1);
+            const float lo = fmaxf(fminf(t1, o1), fmaxf(t2, o2));
+            t1 = hi;
+            t2 = lo;
         }
-        ssum += bs;
+        const float gs = t1 + t2;
+
+        // keep the topk_group best groups (ties to the lower group index)
+        int rank = 0;
+        for (int j = 0; j < n_group; ++j) {
+            const float v = __shfl_sync(0xffffffffu, gs, j * lpg);
+            rank += (v > gs || (v == gs && j < my_group)) ? 1 : 0;
+        }
+        const bool kept = rank < topk_group;
+
+        float cand[EPL];
+#pragma unroll
+        for (int m = 0; m < EPL; ++m) cand[m] = kept ? b[m] : -INFINITY;
+        uint32_t taken = 0;
+        int my_idx = 0;
+        float my_s = 0.f, ssum = 0.f, prev = INFINITY, min_gap = INFINITY;
+        const int rounds = ex.margin > 0.f ? top_k + 1 : top_k;   // one more for the margin
+        for (int rr = 0; rr < rounds; ++rr) {
+            float bv = -INFINITY, bs = 0.f;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int m = 0; m < EPL; ++m) {
+                if (taken & (1u << m)) continue;
+                const int e = e_base + m;
+                if (cand[m] > bv || (cand[m] == bv && e < bi)) {
+                    bv = cand[m];
+                    bi = e;
+                    bs = s[m];
+                }
+            }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+                if (ov > bv || (ov == bv && oi < bi)) {
+                    bv = ov;
+                    bi = oi;
+                    bs = os;
+                }
+            }
+            // adjacent gap in the ranking: decides both the order of the
+            // chosen experts and (at rr == top_k) which of them are chosen
+            if (rr > 0) min_gap = fminf(min_gap, prev - bv);
+            if (rr == top_k) break;   // the (k+1)-th candidate only feeds the margin
+            if (bi / EPL == lane) taken |= 1u << (bi - e_base);
+            if (lane == rr) {
+                my_idx = bi;
+                my_s = bs;
+            }
+            ssum += bs;
+            prev = bv;
+        }
+        if (lane < top_k) {
+            idx_out[(size_t)t * top_k + lane] = my_idx;
+            w_out[(size_t)t * top_k + lane] = my_s / ssum;
+        }
+        if (ex.margin > 0.f) {
+            // weakest kept group vs strongest dropped group
+            float kmin = kept ? gs : INFINITY, dmax = kept ? -INFINITY : gs;
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+                kmin = fminf(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+                dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
+            }
+            const float gap_group = kmin - dmax;      // +inf when every group is kept
+            if (lane == 0 && !(fminf(gap_group, min_gap) >= ex.margin)) {
+                const int slot = atomicAdd(ex.fix_count, 1);
+                if (slot < T) ex.fix_list[slot] = t;
+            }
+        }
     }
-    if (lane < top_k) {
-        idx_out[(size_t)t * top_k + lane] = my_idx;
-        w_out[(size_t)t * top_k + lane] = my_s / ssum;
+}
+
+// ---------------------------------------------------------------------------
+// Exact-path logits for listed tokens: FP32 dot products on CUDA cores.
+// A work unit is (8 listed tokens, 32 experts): the tokens' rows are staged
+// in shared memory as bf16, each warp takes 4 experts, the lanes split K
+// (lane l reads the 16-byte chunks l, l+32, ... of the weight row, so every
+// load is 512 contiguous bytes), and the 8 per-lane sums (chains of at most
+// 256 terms, folded) are combined by a shuffle tree: logits[slot][e] for
+// list slots 0..*count-1.
+// ---------------------------------------------------------------------------
+constexpr int kFixTokens = 8;
+constexpr int kFixExperts = 32;
+
+__global__ void __launch_bounds__(256) router_fix_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                         const float *__restrict__ w, int H, int E,
+                                                         int T, const int *__restrict__ list,
+                                                         const int *__restrict__ count,
+                                                         float *__restrict__ logits)
+{
+    extern __shared__ __align__(16) __nv_bfloat16 xs[];   // [kFixTokens][H]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = min(*count, T);
+    const int nchunk = (E + kFixExperts - 1) / kFixExperts;
+    const int units = ((n + kFixTokens - 1) / kFixTokens) * nchunk;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        const int b0 = (u / nchunk) * kFixTokens, c = u % nchunk;
+        const int nb = min(kFixTokens, n - b0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < kFixTokens * H / 8; i += blockDim.x) {
+            const int j = i / (H / 8), q = i - j * (H / 8);
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (j < nb) v = reinterpret_cast<const uint4 *>(x + (size_t)list[b0 + j] * H)[q];
+            reinterpret_cast<uint4 *>(xs + (size_t)j * H)[q] = v;
+        }
+        __syncthreads();
+        for (int m = 0; m < kFixExperts / 8; ++m) {
+            const int e = c * kFixExperts + warp * (kFixExperts / 8) + m;
+            if (e >= E) break;
+            const float4 *wr = reinterpret_cast<const float4 *>(w + (size_t)e * H);
+            float acc[kFixTokens], tot[kFixTokens];
+#pragma unroll
+            for (int j = 0; j < kFixTokens; ++j) acc[j] = tot[j] = 0.f;
+            int terms = 0;
+            for (int q = lane; q < H / 4; q += 32) {
+                const float4 wv = wr[q];
+#pragma unroll
+                for (int j = 0; j < kFixTokens; ++j) {
+                    const __nv_bfloat162 *p2 =
+                        reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)j * H + 4 * q);
+                    const float2 a = __bfloat1622float2(p2[0]);
+                    const float2 b = __bfloat1622float2(p2[1]);
+                    acc[j] = fmaf(wv.x, a.x, acc[j]);
+                    acc[j] = fmaf(wv.y, a.y, acc[j]);
+                    acc[j] = fmaf(wv.z, b.x, acc[j]);
+                    acc[j] = fmaf(wv.w, b.y, acc[j]);
+                }
+                terms += 4;
+                if (terms == 256) {
+                    terms = 0;
+#pragma unroll
+                    for (int j = 0; j < kFixTokens; ++j) {
+                        tot[j] += acc[j];
+                        acc[j] = 0.f;
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kFixTokens; ++j) {
+                float v = tot[j] + acc[j];
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == 0 && j < nb) logits[(size_t)(b0 + j) * E + e] = v;
+            }
+        }
     }
 }
 
@@ -275,7 +383,7 @@ cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream)
     case EPLV:                                                                                   \
         router_select_kernel<EPLV><<<sgrid, warps * 32, 0, stream>>>(                            \
             a.partial, ns, a.T, a.E, a.n_group, a.topk_group, a.top_k, a.bias, a.idx, a.w,       \
-            a.logits_out);                                                                       \
+            a.logits_out, SelectExtra{});                                                        \
         break;
     switch (epl) {
         BEAM_SELECT(1)
@@ -288,6 +396,282 @@ cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream)
             return cudaErrorInvalidValue;
     }
 #undef BEAM_SELECT
+    return cudaGetLastError();
+}
+
+}  // namespace beam
+
+namespace beam {
+
+// ---------------------------------------------------------------------------
+// Tensor-core logits for large T.  The FP32 router weight is split once into
+// three bf16 pieces, W = w0 + w1 + w2 (each the nearest bf16 to what the
+// previous pieces leave; the remainder is below 2^-27 |W|), stored side by
+// side as Wcat [E, 3H].  A product of a bf16 token value and a bf16 piece is
+// exact in FP32, so x . W = sum over k < 3H of Wcat[e,k] * x[t, k mod H] is
+// an FP32 sum of exact products: the tensor core accumulates it in TMEM.
+// Work items: (128-expert tile, BN-token tile, K slice); the MMA has the
+// experts as M (A = Wcat rows) and the tokens as N (B = x rows), and writes
+// partial[slice][t][e] like the SIMT kernel, so the selection is shared.
+// ---------------------------------------------------------------------------
+
+__global__ void router_split_kernel(const float *__restrict__ w, int n, __nv_bfloat16 *__restrict__ wcat,
+                                    int H)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const int e = i / H, h = i - e * H;
+    const float v = w[i];
+    const __nv_bfloat16 p0 = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(p0);        // exact in FP32
+    const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(p1);       // exact in FP32
+    const __nv_bfloat16 p2 = __float2bfloat16_rn(r2);
+    __nv_bfloat16 *row = wcat + (size_t)e * 3 * H;
+    row[h] = p0;
+    row[H + h] = p1;
+    row[2 * H + h] = p2;
+}
+
+cudaError_t launch_router_split(const float *w, int E, int H, __nv_bfloat16 *wcat, cudaStream_t s)
+{
+    const int n = E * H;
+    router_split_kernel<<<(n + 255) / 256, 256, 0, s>>>(w, n, wcat, H);
+    return cudaGetLastError();
+}
+
+namespace {
+constexpr int kRBM = 128;   // experts per tile (UMMA M)
+constexpr int kRBN = 128;   // tokens per tile (UMMA N)
+constexpr int kRBK = 64;
+constexpr int kRStageBytes = kRBM * kRBK * 2 + kRBN * kRBK * 2;
+constexpr int kRStages = 6;
+constexpr int kRAccCols = kRBN;
+constexpr int kRSmem = 1024 + kRStages * kRStageBytes + 256;
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    router_mma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                      RouterMmaArgs p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *bar_ptr = smem_raw + (base - raw_addr) + kRStages * kRStageBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(bar_ptr);
+    uint64_t *empty = full + kRStages;
+    uint64_t *tfull = empty + kRStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < kRStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 128);
+        }
+        mbar_init(smem_u32(drain), 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmX);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tmem_alloc(smem_u32(tmem_slot), 2 * kRAccCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int n_mt = (p.E + kRBM - 1) / kRBM;
+    const int n_tt = (p.T + kRBN - 1) / kRBN;
+    const int total = n_mt * n_tt * p.nslice;
+    // item = ((tt * nslice) + s) * n_mt + mt: neighbours share the token tile
+
+    if (warp == 0 && lane == 0) {
+        const uint64_t pol = l2_policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        long long issued = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            const int mt = item % n_mt, rest = item / n_mt;
+            const int s = rest % p.nslice, tt = rest / p.nslice;
+            for (int j = 0; j < p.kb_per_slice; ++j) {
+                const int kb = s * p.kb_per_slice + j;   // over the concatenated 3H
+                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = base + stage * kRStageBytes;
+                const uint32_t fb = smem_u32(&full[stage]);
+                mbar_arrive_expect_tx(fb, kRStageBytes);
+                tma_load_2d(sa, &tmW, kb * kRBK, mt * kRBM, fb, pol);
+                tma_load_2d(sa + kRBM * kRBK * 2, &tmX, (kb % p.kb_per_h) * kRBK, tt * kRBN, fb, pol);
+                ++issued;
+                if (++stage == kRStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok) {
+            long long n = issued < kRStages ? issued : kRStages;
+            int st = stage;
+            uint32_t ph = phase;
+            for (long long j = 0; j < n; ++j) {
+                if (st == 0) {
+                    st = kRStages - 1;
+                    ph ^= 1u;
+                } else {
+                    --st;
+                }
+                mbar_wait_drain(smem_u32(&full[st]), ph, p.ctl.limit_ns);
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        constexpr uint32_t idesc = umma_idesc_bf16_f32(kRBM, kRBN);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true, issued_any = false;
+        int iter = 0;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++iter) {
+            const int acc = iter & 1;
+            const uint32_t acc_phase = (uint32_t)(iter >> 1) & 1u;
+            if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.ctl)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem_base + (uint32_t)(acc * kRAccCols);
+            for (int j = 0; j < p.kb_per_slice; ++j) {
+                if (!mbar_wait(smem_u32(&full[stage]), phase, p.ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = base + stage * kRStageBytes;
+                const uint32_t sb = sa + kRBM * kRBK * 2;
+#pragma unroll
+                for (int k = 0; k < kRBK / 16; ++k) {
+                    umma_bf16(d, umma_desc_sw128(sa + k * 32), umma_desc_sw128(sb + k * 32), idesc,
+                              (j > 0 || k > 0) ? 1u : 0u);
+                    issued_any = true;
+                }
+                umma_commit(smem_u32(&empty[stage]));
+                if (++stage == kRStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            umma_commit(smem_u32(&tfull[acc]));
+        }
+        if (issued_any) {
+            umma_commit(smem_u32(drain));
+            mbar_wait_drain(smem_u32(drain), 0, p.ctl.limit_ns);
+        }
+    } else if (warp >= 2) {
+        const int quad = warp & 3;
+        int iter = 0;
+        for (int item = blockIdx.x; item < total; item += gridDim.x, ++iter) {
+            const int acc = iter & 1;
+            const uint32_t acc_phase = (uint32_t)(iter >> 1) & 1u;
+            const bool ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.ctl);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int mt = item % n_mt, rest = item / n_mt;
+            const int s = rest % p.nslice, tt = rest / p.nslice;
+            const int e = mt * kRBM + quad * 32 + lane;
+            const int t0 = tt * kRBN;
+            float *dst = p.partial + (size_t)s * p.T * p.E;
+            const uint32_t taddr =
+                tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kRAccCols);
+#pragma unroll 1
+            for (int c0 = 0; c0 < kRBN && t0 + c0 < p.T; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(taddr + c0, v);
+                tmem_ld_wait();
+                if (e < p.E) {
+#pragma unroll
+                    for (int n = 0; n < 32; ++n)
+                        if (t0 + c0 + n < p.T) dst[(size_t)(t0 + c0 + n) * p.E + e] = __uint_as_float(v[n]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty[acc]));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 2 * kRAccCols);
+    }
+}
+
+cudaError_t prepare_router_mma()
+{
+    return cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem);
+}
+
+cudaError_t launch_router_mma(const CUtensorMap &tmW, const CUtensorMap &tmX, const RouterMmaArgs &a,
+                              int grid, cudaStream_t stream)
+{
+    router_mma_kernel<<<grid, 192, kRSmem, stream>>>(tmW, tmX, a);
+    return cudaGetLastError();
+}
+
+int router_mma_tokens_per_tile() { return kRBN; }
+int router_mma_experts_per_tile() { return kRBM; }
+
+cudaError_t launch_router_select(const RouterArgs &a, const SelectExtra &ex, int max_blocks,
+                                 cudaStream_t stream)
+{
+    const int warps = 8;
+    int blocks = (a.T + warps - 1) / warps;
+    if (max_blocks > 0 && blocks > max_blocks) blocks = max_blocks;
+    const int epl = a.E / 32;
+#define BEAM_SELECT2(EPLV)                                                                       \
+    case EPLV:                                                                                   \
+        router_select_kernel<EPLV><<<blocks, warps * 32, 0, stream>>>(                           \
+            a.partial, a.nslice, a.T, a.E, a.n_group, a.topk_group, a.top_k, a.bias, a.idx, a.w, \
+            a.logits_out, ex);                                                                   \
+        break;
+    switch (epl) {
+        BEAM_SELECT2(1)
+        BEAM_SELECT2(2)
+        BEAM_SELECT2(4)
+        BEAM_SELECT2(8)
+        BEAM_SELECT2(16)
+        BEAM_SELECT2(32)
+        default:
+            return cudaErrorInvalidValue;
+    }
+#undef BEAM_SELECT2
+    return cudaGetLastError();
+}
+
+cudaError_t prepare_router_fix(int H)
+{
+    return cudaFuncSetAttribute(router_fix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(kFixTokens * (size_t)H * 2));
+}
+
+cudaError_t launch_router_fix(const __nv_bfloat16 *x, const float *w, int H, int E, int T,
+                              const int *list, const int *count, float *logits, int grid,
+                              cudaStream_t stream)
+{
+    router_fix_kernel<<<grid, 256, kFixTokens * (size_t)H * 2, stream>>>(x, w, H, E, T, list, count,
+                                                                       logits);
     return cudaGetLastError();
 }
 

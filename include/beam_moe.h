@@ -87,8 +87,10 @@ typedef enum {
  * Kernel-side shape limits (else BEAM_ERR_UNSUPPORTED): E/32 experts per
  * lane in {1, 2, 4, 8, 16, 32}, group size a multiple of E/32 with
  * (group size)/(E/32) a power of two, n_group <= 32.
- * On success *out receives the handle.  Allocates device memory; launches no
- * kernel.  The current CUDA device at create time is the handle's device.
+ * On success *out receives the handle.  Allocates device memory and launches
+ * one kernel on the legacy default stream (splitting router_w into the bf16
+ * pieces the tensor-core router uses), waiting for it.  The current CUDA
+ * device at create time is the handle's device.
  */
 int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n_group,
                     int topk_group, int top_k, float routed_scaling, const float *router_w,
@@ -186,6 +188,15 @@ int beam_moe_dispatch_info(beam_moe_t h, void *stream, int T, int32_t *counts_ho
                            int32_t *offsets_host, int32_t *pair_row_host);
 
 /*
+ * Routing statistics of the last route / forward call on this handle:
+ * *rederived_host (host) receives how many tokens had their decision
+ * re-derived from FP32 CUDA-core logits because their margin on the
+ * tensor-core logits was too thin (0 when the CUDA-core path ran).
+ * Synchronises `stream`.
+ */
+int beam_moe_router_stats(beam_moe_t h, void *stream, int32_t *rederived_host);
+
+/*
  * Synchronise `stream`, then return and clear the device status word:
  * BEAM_OK, or BEAM_ERR_TIMEOUT when a bounded in-kernel wait ran out since
  * the last call.  While the word is set, kernels of this handle stop at
@@ -212,9 +223,24 @@ int beam_moe_set_wait_limit(beam_moe_t h, int64_t limit_ns);
  * cta_pairs       1 (default): token tiles of 64 rows or more run on pairs of
  *                 SMs that share each MMA (needs inter and hidden to be
  *                 multiples of 256); 0: one CTA per SM always.
+ * router_mode     -1 (default): FP32 CUDA-core logits below 512 tokens,
+ *                 tensor-core logits from 512 on; 0: always CUDA cores;
+ *                 1: always tensor cores; 2: tensor cores with every token's
+ *                 routing re-derived on the CUDA-core path (a check of that
+ *                 path).  The tensor-core logits use the router weight split
+ *                 into three bf16 pieces (every product with a bf16 token
+ *                 value is exact in FP32, the sum is accumulated in FP32 by
+ *                 the tensor cores); a token whose decision margin -- the
+ *                 smallest gap between neighbours in the ranking of its top
+ *                 k+1 candidates (it fixes the chosen set and their order),
+ *                 or weakest kept vs strongest dropped group score -- is
+ *                 below 4e-5 has
+ *                 its logits recomputed with FP32 CUDA-core dot products and
+ *                 is selected again, so decisions keep CUDA-core accuracy.
+ *                 beam_moe_router_logits always uses the CUDA-core path.
  */
 int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair,
-                             int cta_pairs);
+                             int cta_pairs, int router_mode);
 
 /*
  * Per-stage timing of forward passes, for measurement.  After

@@ -56,7 +56,7 @@ def _load():
         P = ctypes.c_void_p
         I = ctypes.c_int
         D = ctypes.c_double
-        lib.oracle_route.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P]
+        lib.oracle_route.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_route.restype = I
         lib.oracle_expert_swiglu.argtypes = [I, I, I, P, P, P, P, P, P]
         lib.oracle_expert_swiglu.restype = None
@@ -125,6 +125,7 @@ class Routing:
     gap_expert: np.ndarray   # float64 [T]
     gap_group: np.ndarray    # float64 [T]
     kept_mask: np.ndarray    # int32 [T], bit j = group j kept
+    gap_order: np.ndarray    # float64 [T] smallest neighbour gap within the chosen sequence
 
 
 def route(x_bits: np.ndarray, router_w: np.ndarray, bias: np.ndarray,
@@ -144,11 +145,13 @@ def route(x_bits: np.ndarray, router_w: np.ndarray, bias: np.ndarray,
     ge = np.empty((T,), np.float64)
     gg = np.empty((T,), np.float64)
     km = np.empty((T,), np.int32)
+    go = np.empty((T,), np.float64)
     rc = lib.oracle_route(T, H, E, n_group, topk_group, top_k, _ptr(x), _ptr(wr), _ptr(b),
-                          _ptr(idx), _ptr(w), _ptr(scores), _ptr(biased), _ptr(ge), _ptr(gg), _ptr(km))
+                          _ptr(idx), _ptr(w), _ptr(scores), _ptr(biased), _ptr(ge), _ptr(gg), _ptr(km),
+                          _ptr(go))
     if rc != 0:
         raise ValueError("oracle_route: routing configuration not defined by the method")
-    return Routing(idx, w, scores, biased, ge, gg, km)
+    return Routing(idx, w, scores, biased, ge, gg, km, go)
 
 
 def expert_swiglu(x_bits: np.ndarray, w_gate_bits: np.ndarray, w_up_bits: np.ndarray,

@@ -110,13 +110,18 @@ static double silu(double z) { return z / (1.0 + exp(-z)); }
  *   gap_group double [T]        min double group score over kept groups minus
  *                               max over dropped groups (+inf if none)
  *                               (may be NULL)
+ *   gap_order double [T]        smallest difference of double biased scores
+ *                               between neighbours of the chosen sequence
+ *                               (the order the method returns them in; +inf
+ *                               for top_k == 1) (may be NULL)
  *   kept_mask int32 [T]         bit j set iff group j was kept (may be NULL)
  * Returns 0, or -1 on an argument the method does not define.
  */
 int oracle_route(int T, int H, int E, int n_group, int topk_group, int top_k,
                  const uint16_t *x, const float *router_w, const float *bias,
                  int32_t *idx, double *w, double *scores, double *biased,
-                 double *gap_expert, double *gap_group, int32_t *kept_mask)
+                 double *gap_expert, double *gap_group, int32_t *kept_mask,
+                 double *gap_order)
 {
     if (T < 0 || H <= 0 || E <= 0 || n_group <= 0 || E % n_group != 0) return -1;
     const int gsize = E / n_group;
@@ -203,6 +208,14 @@ int oracle_route(int T, int H, int E, int n_group, int topk_group, int top_k,
                 else if (gsd[j] > max_d) max_d = gsd[j];
             }
             gap_group[t] = (max_d == -INFINITY) ? INFINITY : min_k - max_d;
+        }
+        if (gap_order) {
+            double g = INFINITY;
+            for (int r = 0; r + 1 < top_k; ++r) {
+                const double d = bd[idx[(size_t)t * top_k + r]] - bd[idx[(size_t)t * top_k + r + 1]];
+                if (d < g) g = d;
+            }
+            gap_order[t] = g;
         }
         if (kept_mask) kept_mask[t] = mask;
         if (scores) memcpy(scores + (size_t)t * E, s, sizeof(double) * (size_t)E);

@@ -169,6 +169,10 @@ def test_route_invariants_beam_shape(oracle_lib):
         assert b32[idx].min() >= b32[others].max()
         assert np.all(r.w[t] > 0)
         assert abs(r.w[t].sum() - 1.0) < 1e-12
+        # the near-tie diagnostics: gaps at the set boundary and within the order
+        bd = r.biased[t]
+        assert r.gap_expert[t] == bd[idx].min() - bd[others].max()
+        assert r.gap_order[t] == np.min(bd[idx][:-1] - bd[idx][1:])
 
 
 def test_single_group_reduces_to_topk(oracle_lib):

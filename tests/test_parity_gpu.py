@@ -64,20 +64,22 @@ def test_tiny_block(T, ctas, tile, pair):
     moe.close()
 
 
-# (T, GEMM CTAs, largest token tile, paired down tiles, CTA pairs): H=512, I=256
-SMALL_CASES = [(1024, 0, 0, -1, 1), (1024, 0, 0, -1, 0), (1024, 0, 64, 0, 1), (1024, 4, 128, 1, 1),
-               (1024, 0, 256, 0, 1), (3000, 0, 256, 1, 1), (3000, 6, 256, 1, 1), (777, 0, 128, -1, 1),
-               (2048, 2, 64, 1, 1), (64, 0, 64, -1, 1)]
+# (T, GEMM CTAs, largest token tile, paired down tiles, CTA pairs, router mode): H=512, I=256
+SMALL_CASES = [(1024, 0, 0, -1, 1, -1), (1024, 0, 0, -1, 0, 0), (1024, 0, 64, 0, 1, 1),
+               (1024, 4, 128, 1, 1, 1), (1024, 0, 256, 0, 1, 0), (3000, 0, 256, 1, 1, 1),
+               (3000, 6, 256, 1, 1, -1), (777, 0, 128, -1, 1, 1), (2048, 2, 64, 1, 1, 0),
+               (64, 0, 64, -1, 1, 1), (1, 0, 0, -1, 1, 1), (130, 0, 0, -1, 1, 1),
+               (1024, 0, 0, -1, 1, 2), (3000, 0, 0, -1, 1, 2)]
 
 
-@pytest.mark.parametrize("T,ctas,tile,pair,pairs", SMALL_CASES)
-def test_small_block(T, ctas, tile, pair, pairs):
+@pytest.mark.parametrize("T,ctas,tile,pair,pairs,router", SMALL_CASES)
+def test_small_block(T, ctas, tile, pair, pairs, router):
     wl = W.WORKLOADS["small"]
     d = _inputs(wl, T)
     moe = BeamMoE.from_workload(wl, d, max_tokens=T)
-    moe.set_gemm_tuning(ctas, tile, pair, pairs)
+    moe.set_gemm_tuning(ctas, tile, pair, pairs, router)
     rep = check_block(wl, d, moe)
-    _log(f"small_T{T}_ctas{ctas}_tile{tile}_pair{pair}_pairs{pairs}", rep)
+    _log(f"small_T{T}_ctas{ctas}_tile{tile}_pair{pair}_pairs{pairs}_router{router}", rep)
     assert rep.ok(), rep
     moe.close()
 
@@ -121,6 +123,56 @@ def test_tiny_router_logits():
     got = moe.router_logits(d["x"]).cpu().double().numpy()
     ref = oracle.bf16_to_f64(W.bf16_bits(d["x"])) @ d["router_w"].cpu().double().numpy().T
     assert np.abs(got - ref).max() < 1e-5 * max(1.0, np.abs(ref).max())
+    moe.close()
+
+
+@pytest.mark.parametrize("mode,T", [(0, 1024), (1, 1024), (1, 8192), (1, 100)])
+def test_router_logits_precision(mode, T):
+    """FP32 logits of the Beam-shaped router (H=5120, 256 experts) against
+    the exact value.  beam_moe_router_logits always takes the CUDA-core path
+    (whatever the routing mode), whose error is far below the 1e-6 near-tie
+    threshold of the routing comparison."""
+    wl = dataclasses.replace(W.WORKLOADS["decode"], inter=128)
+    d = _inputs(wl, T)
+    moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    moe.set_gemm_tuning(0, 0, -1, 1, mode)
+    got = moe.router_logits(d["x"]).cpu().double().numpy()
+    ref = oracle.bf16_to_f64(W.bf16_bits(d["x"])) @ d["router_w"].cpu().double().numpy().T
+    err = float(np.abs(got - ref).max())
+    path = os.environ.get("BEAM_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": f"router_logits_mode{mode}_T{T}", "max_abs_err": err}) + "\n")
+    assert err < 2e-6, err
+    moe.close()
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_tensor_core_routing_matches_oracle(mode):
+    """Routing of 8192 tokens at the Beam router shape through the
+    tensor-core path (mode 1: thin-margin tokens re-derived on CUDA cores;
+    mode 2: every token re-derived) against the oracle on every token."""
+    from parity import NEAR_TIE, W_ABS
+    wl = dataclasses.replace(W.WORKLOADS["prefill"], inter=128)
+    T = 8192
+    d = _inputs(wl, T)
+    moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    moe.set_gemm_tuning(0, 0, -1, 1, mode)
+    idx, w = moe.route(d["x"])
+    rederived = moe.router_stats()
+    if mode == 2:
+        assert rederived == T
+    r = oracle.route(W.bf16_bits(d["x"]), d["router_w"].cpu().numpy(), d["bias"].cpu().numpy(),
+                     wl.n_group, wl.topk_group, wl.top_k)
+    keep = (r.gap_expert >= NEAR_TIE) & (r.gap_group >= NEAR_TIE) & (r.gap_order >= NEAR_TIE)
+    mism = int((idx.cpu().numpy()[keep] != r.idx[keep]).any(axis=1).sum())
+    werr = float(np.abs(w.cpu().numpy()[keep] - r.w[keep]).max())
+    path = os.environ.get("BEAM_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": f"tc_routing_mode{mode}", "tokens": T, "exempt": int((~keep).sum()),
+                                "idx_mismatch": mism, "w_max_err": werr, "rederived": rederived}) + "\n")
+    assert mism == 0 and werr <= W_ABS, (mism, werr)
     moe.close()
 
 

@@ -39,7 +39,7 @@ def test_route_static_matches_route(name, T):
     # threshold) are exempt from the index comparison, as in those tests
     r = oracle.route(W.bf16_bits(d["x"]), d["router_w"].cpu().numpy(), d["bias"].cpu().numpy(),
                      wl.n_group, wl.topk_group, wl.top_k)
-    keep = (r.gap_expert >= NEAR_TIE) & (r.gap_group >= NEAR_TIE)
+    keep = (r.gap_expert >= NEAR_TIE) & (r.gap_group >= NEAR_TIE) & (r.gap_order >= NEAR_TIE)
     for _ in range(2):
         idx, w = route_static(d["x"], d["router_w"], d["bias"], wl.n_group, wl.topk_group, wl.top_k)
         torch.cuda.synchronize()
