@@ -112,7 +112,7 @@ class ClockSampler:
 
 def kernel_hash() -> str:
     h = hashlib.sha256()
-    for fn in ("grouped_gemm.cu", "common.cuh", "kernels.cuh"):
+    for fn in ("grouped_gemm.cu", "grouped_gemm_pair.cu", "gemm_common.cuh", "common.cuh", "kernels.cuh"):
         with open(os.path.join(ROOT, "group_limited_routing_sigmoid_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -268,17 +268,21 @@ def run_ours(args):
     if args.workload in ("decode", "tiny", "decode_small"):
         alg_bytes = d_mean * 2 * I * H * 2 + P * H * 2 + P * I * 2
         achieved = alg_bytes / (gate_up_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "kernel": "gate_up_gemm (grouped_gemm_kernel<BN,2>)",
+        roof = {"bound": "hbm",
                 "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk["source"],
                 "algorithmic_bytes_per_launch": int(alg_bytes), "launch_ms": round(gate_up_ms, 4)}
     else:
         flops = 4.0 * H * I * P
         achieved = flops / (gate_up_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "kernel": "gate_up_gemm (grouped_gemm_kernel<BN,2>)",
+        roof = {"bound": "tensor",
                 "achieved": round(achieved, 1), "peak": pk["bf16_sus"], "unit": "TFLOP/s",
                 "frac": round(achieved / pk["bf16_sus"], 4), "peak_source": pk["source"] + " sustained",
                 "algorithmic_flops_per_launch": flops, "launch_ms": round(gate_up_ms, 4)}
+    plan = moe.launch_plan(T)
+    roof["kernel"] = ("gate_up_gemm (grouped_gemm_pair_kernel<%d,2,0>, CTA pairs, grid %d)"
+                      if plan["cta_pairs"] else
+                      "gate_up_gemm (grouped_gemm_kernel<%d,2,0>, grid %d)") % (plan["tile_rows"], plan["grid"])
     roof["traffic"] = ncu_traffic(args.workload)
     step_bytes = d_mean * 3 * H * I * 2 + E * H * 4 + T * H * 4 + (T * H * 8 if wl.residual_k else 0)
     stage_avg = {kname: round(v / max(calls, 1), 4) for kname, v in stage_ms.items()}
@@ -312,9 +316,11 @@ def run_ours(args):
                 "d2h_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0)},
         "gpu_launches": KERNELS_PER_FORWARD * steps_done,
         "roofline": roof,
+        "launch_plan": plan,
     }
     if ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, weights, batches[0]["x"], args.cpu_tokens)
+        pool = torch.cat([b["x"] for b in batches])
+        line["cpu_baseline"] = cpu_baseline(wl, weights, pool, min(args.cpu_tokens, pool.shape[0]))
     if rank == 0:
         print(json.dumps(line), flush=True)
     moe.close()
@@ -351,8 +357,8 @@ def cpu_baseline(wl, weights, x, n_tokens):
     sec = _oracle_on_tokens(wl, weights, x, n_tokens)
     return {"value": round(n_tokens / sec, 3), "unit": "tokens/s", "cores": oracle.threads(),
             "kind": "oracle",
-            "sample": f"{n_tokens} tokens of one {wl.T}-token batch, all {wl.top_k} experts each, "
-                      f"fp64 oracle ({sec:.1f} s)"}
+            "sample": f"the first {n_tokens} tokens of the bench's token batches, all {wl.top_k} "
+                      f"experts each, fp64 oracle ({sec:.1f} s)"}
 
 
 # ---------------------------------------------------------------------------
@@ -405,7 +411,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the CPU-baseline sample")
+    ap.add_argument("--cpu-tokens", type=int, default=128,
+                    help="tokens in the CPU-baseline sample (about 10 s of oracle work at the decode shape)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm-tile", type=int, default=0, help="largest GEMM token tile (0 = auto)")
     ap.add_argument("--down-pair", type=int, default=-1, help="paired down tiles: -1 auto, 0, 1")

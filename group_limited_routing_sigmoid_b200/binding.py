@@ -25,7 +25,8 @@ BEAM_ERR_TIMEOUT = -5
 # every entry point declared in include/beam_moe.h
 SYMBOLS = (
     "beam_moe_create", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_forward",
-    "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_get_status",
+    "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_launch_plan",
+    "beam_moe_get_status",
     "beam_moe_set_wait_limit", "beam_moe_set_gemm_tuning", "beam_moe_profile_begin",
     "beam_moe_profile_end", "beam_moe_check_wait_timeout", "beam_moe_last_error",
     "beam_moe_create_error", "beam_moe_destroy",
@@ -58,6 +59,7 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_dispatch_info.argtypes = [P, P, I, P, P, P]
         lib.beam_moe_get_status.argtypes = [P, P]
         lib.beam_moe_router_stats.argtypes = [P, P, P]
+        lib.beam_moe_launch_plan.argtypes = [P, I, P]
         lib.beam_moe_set_wait_limit.argtypes = [P, ctypes.c_int64]
         lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I, I, I]
         lib.beam_moe_check_wait_timeout.argtypes = [P, P]
@@ -210,6 +212,13 @@ class BeamMoE:
         self._check(library().beam_moe_router_stats(self._h, _stream(stream),
                                                      ctypes.cast(ctypes.pointer(n), ctypes.c_void_p)))
         return n.value
+
+    def launch_plan(self, T: int) -> dict:
+        """The kernels and launch shapes a forward pass of T tokens uses."""
+        p = (ctypes.c_int32 * 6)()
+        self._check(library().beam_moe_launch_plan(self._h, int(T), ctypes.cast(p, ctypes.c_void_p)))
+        keys = ("tile_rows", "cta_pairs", "grid", "down_paired", "router_tensor_cores", "router_slices")
+        return dict(zip(keys, (int(v) for v in p)))
 
     def get_status(self, stream=None) -> int:
         return library().beam_moe_get_status(self._h, _stream(stream))

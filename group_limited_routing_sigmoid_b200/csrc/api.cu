@@ -234,6 +234,45 @@ void prof_mark(beam_moe *h, cudaStream_t s, int stage)
         cudaEventRecord(h->prof_events[(size_t)h->prof_calls * 6 + stage], s);
 }
 
+// The kernels and launch shapes a forward pass of T tokens uses.  A function
+// of the handle's tuning and of T only, so that the host never waits on the
+// routing to launch the GEMMs.
+struct ForwardPlan {
+    int tile_rows;     // largest token tile of the grouped GEMMs
+    int cta_pairs;     // 1: cta_group::2 kernels
+    int grid;          // CTAs of each grouped GEMM
+    int down_paired;   // 1: two weight blocks per down work item
+    int router_tc;     // 1: tensor-core logits with exact re-derivation
+    int router_slices; // K slices of the router logits
+};
+
+ForwardPlan plan_forward(const beam_moe *h, int T)
+{
+    ForwardPlan p;
+    p.tile_rows = h->tile_rows ? h->tile_rows : choose_tile_rows(T, h->top_k, h->E);
+    // CTA pairs (cta_group::2) for large token tiles when the weight rows
+    // split into 256-row blocks; single CTAs otherwise
+    p.cta_pairs = h->use_pair != 0 && gemm_pair_supported(p.tile_rows) && h->I % 256 == 0 &&
+                  h->H % 256 == 0 && gemm_pair_max_ctas() >= 2;
+    p.grid = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
+    if (p.cta_pairs) {
+        const int cap = gemm_pair_max_ctas();
+        p.grid = p.grid > cap ? cap : p.grid;
+        p.grid &= ~1;
+        if (p.grid < 2) p.grid = 2;
+    }
+    // pair the down projection's weight blocks (two blocks share a token
+    // tile) when H allows; lone blocks for decode-sized token tiles keep more
+    // items in flight
+    const int block_rows = p.cta_pairs ? 512 : 256;
+    p.down_paired = h->H % block_rows == 0 &&
+                    (h->down_pair == 1 || (h->down_pair < 0 && p.tile_rows >= 64));
+    p.router_tc = router_on_tensor_cores(h, T);
+    p.router_slices = p.router_tc ? router_mma_slices(T, h->H, h->E, h->num_sms)
+                                  : router_slices(T, h->H, h->E, h->num_sms);
+    return p;
+}
+
 int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, float *residual,
                 int k)
 {
@@ -241,7 +280,8 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     int rc = run_router(h, s, x, T, h->idx, h->w, nullptr);
     if (rc != BEAM_OK) return rc;
     prof_mark(h, s, 1);
-    const int BN = h->tile_rows ? h->tile_rows : choose_tile_rows(T, h->top_k, h->E);
+    const ForwardPlan plan = plan_forward(h, T);
+    const int BN = plan.tile_rows;
     DispatchArgs d;
     d.idx = h->idx;
     d.x = static_cast<const __nv_bfloat16 *>(x);
@@ -270,17 +310,8 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.tile_off = h->tile_off;
     g.ctl.status = h->status;
     g.ctl.limit_ns = h->wait_limit_ns;
-    // CTA pairs (cta_group::2) for large token tiles when the weight rows
-    // split into 256-row blocks; single CTAs otherwise
-    const bool use_pair = h->use_pair != 0 && gemm_pair_supported(BN) && h->I % 256 == 0 &&
-                          h->H % 256 == 0 && gemm_pair_max_ctas() >= 2;
-    int grid = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
-    if (use_pair) {
-        const int cap = gemm_pair_max_ctas();
-        grid = grid > cap ? cap : grid;
-        grid &= ~1;
-        if (grid < 2) grid = 2;
-    }
+    const bool use_pair = plan.cta_pairs != 0;
+    const int grid = plan.grid;
     g.K = h->H;
     g.R = h->I;
     g.out = h->hbuf;
@@ -293,13 +324,7 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.K = h->I;
     g.R = h->H;
     g.out = h->ybuf;
-    // pair the down projection's weight blocks (two blocks share a token
-    // tile) when H allows; lone blocks for decode-sized token tiles keep more
-    // items in flight
-    const int block_rows = use_pair ? 512 : 256;
-    const bool pair_down =
-        h->H % block_rows == 0 && (h->down_pair == 1 || (h->down_pair < 0 && BN >= 64));
-    const GemmKind dk = pair_down ? GemmKind::kDownPaired : GemmKind::kDown;
+    const GemmKind dk = plan.down_paired ? GemmKind::kDownPaired : GemmKind::kDown;
     e = use_pair ? launch_grouped_gemm_pair(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s)
                  : launch_grouped_gemm(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "down GEMM launch");
@@ -619,6 +644,22 @@ int beam_moe_router_stats(beam_moe_t h, void *stream, int32_t *rederived_host)
                                     cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "router stats copy");
+}
+
+int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    if (!plan_host) return fail(h, BEAM_ERR_INVALID_ARG, "plan_host is NULL");
+    if (T < 0 || T > h->max_tokens)
+        return fail(h, BEAM_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->max_tokens);
+    const ForwardPlan p = plan_forward(h, T);
+    plan_host[0] = p.tile_rows;
+    plan_host[1] = p.cta_pairs;
+    plan_host[2] = p.grid;
+    plan_host[3] = p.down_paired;
+    plan_host[4] = p.router_tc;
+    plan_host[5] = p.router_slices;
+    return BEAM_OK;
 }
 
 int beam_moe_get_status(beam_moe_t h, void *stream)

@@ -170,14 +170,34 @@ __global__ void __launch_bounds__(256) router_select_kernel(
         const int t = ex.token_list ? ex.token_list[wi] : wi;   // output row
         const int r = wi;                                         // logits row
 
+        // the lane's logits: slices summed in order; the loads of one slice
+        // are independent of each other (vectors when EPL allows)
+        float l[EPL];
+#pragma unroll
+        for (int m = 0; m < EPL; ++m) l[m] = 0.f;
+#pragma unroll 4
+        for (int q = 0; q < nslice; ++q) {
+            const float *src = partial + ((size_t)q * T + r) * E + e_base;
+            if constexpr (EPL % 4 == 0) {
+#pragma unroll
+                for (int m = 0; m < EPL; m += 4) {
+                    const float4 v = *reinterpret_cast<const float4 *>(src + m);
+                    l[m] += v.x;
+                    l[m + 1] += v.y;
+                    l[m + 2] += v.z;
+                    l[m + 3] += v.w;
+                }
+            } else {
+#pragma unroll
+                for (int m = 0; m < EPL; ++m) l[m] += src[m];
+            }
+        }
         float s[EPL], b[EPL];
 #pragma unroll
         for (int m = 0; m < EPL; ++m) {
             const int e = e_base + m;
-            float l = 0.f;
-            for (int q = 0; q < nslice; ++q) l += partial[((size_t)q * T + r) * E + e];
-            if (logits_out) logits_out[(size_t)t * E + e] = l;
-            s[m] = 1.0f / (1.0f + expf(-l));
+            if (logits_out) logits_out[(size_t)t * E + e] = l[m];
+            s[m] = 1.0f / (1.0f + expf(-l[m]));
             b[m] = s[m] + bias[e];
         }
 
@@ -356,11 +376,11 @@ __global__ void __launch_bounds__(256) router_fix_kernel(const __nv_bfloat16 *__
 
 // K slices of the logits: enough blocks for several per SM (the selection
 // sums the slices in a fixed order).  Slices stay a multiple of 32 wide and
-// at least 1024 wide, or 256 when the grid would not fill the GPU anyway.
+// at least 1024 wide, or 128 when the grid would not fill the GPU anyway.
 int router_slices(int T, int H, int E, int num_sms)
 {
     const int base = ((T + kLT - 1) / kLT) * ((E + kLE - 1) / kLE);
-    const int min_width = base < num_sms ? 256 : 1024;
+    const int min_width = base < num_sms ? 128 : 1024;
     int ns = 1;
     while (ns * base < 6 * num_sms && (H / (ns * 2)) >= min_width && H % (ns * 2 * kLK) == 0)
         ns *= 2;

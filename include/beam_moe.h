@@ -197,6 +197,18 @@ int beam_moe_dispatch_info(beam_moe_t h, void *stream, int T, int32_t *counts_ho
 int beam_moe_router_stats(beam_moe_t h, void *stream, int32_t *rederived_host);
 
 /*
+ * The launch configuration a forward pass of T tokens (0 <= T <= max_tokens)
+ * uses under the handle's current tuning, written to plan_host (int32 [6],
+ * host): {largest token tile of the grouped GEMMs (rows), 1 if they run on
+ * CTA pairs (cta_group::2), CTAs per grouped GEMM, 1 if the down projection
+ * takes two weight blocks per work item, 1 if the router logits run on the
+ * tensor cores (with exact re-derivation of thin-margin tokens), K slices of
+ * the router logits}.  A function of T and the tuning only; launches nothing.
+ * Returns BEAM_ERR_INVALID_ARG for a NULL pointer or T out of range.
+ */
+int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host);
+
+/*
  * Synchronise `stream`, then return and clear the device status word:
  * BEAM_OK, or BEAM_ERR_TIMEOUT when a bounded in-kernel wait ran out since
  * the last call.  While the word is set, kernels of this handle stop at

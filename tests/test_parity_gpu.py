@@ -16,7 +16,7 @@ import torch
 
 import oracle
 from group_limited_routing_sigmoid_b200 import workloads as W
-from group_limited_routing_sigmoid_b200.binding import BeamMoE, BEAM_ERR_TIMEOUT
+from group_limited_routing_sigmoid_b200.binding import BeamMoE, BeamMoEError, BEAM_ERR_TIMEOUT
 from group_limited_routing_sigmoid_b200.build import build
 
 from parity import check_block
@@ -185,6 +185,29 @@ def test_empty_batch_is_a_no_op():
     moe.forward(x0, out=out)
     moe.route(x0)
     assert moe.get_status() == 0
+    moe.close()
+
+
+def test_launch_plan_follows_tokens_per_expert_and_tuning():
+    """The plan a forward pass follows: 16-row tiles on single CTAs and
+    CUDA-core router logits for a few tokens per expert; 256-row tiles on CTA
+    pairs with paired down blocks and tensor-core logits for many; tuning
+    overrides apply; T outside [0, max_tokens] is rejected."""
+    wl = W.WORKLOADS["small"]
+    d = _inputs(wl)
+    moe = BeamMoE.from_workload(wl, d)
+    p = moe.launch_plan(8)
+    assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"]) == (16, 0, 0, 0)
+    assert p["grid"] == torch.cuda.get_device_properties(0).multi_processor_count
+    p = moe.launch_plan(wl.T)
+    assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"]) == (256, 1, 1, 1)
+    assert p["grid"] % 2 == 0 and p["router_slices"] >= 1
+    moe.set_gemm_tuning(6, 64, 0, 0, 0)
+    p = moe.launch_plan(wl.T)
+    assert (p["tile_rows"], p["cta_pairs"], p["grid"], p["down_paired"], p["router_tensor_cores"]) == \
+        (64, 0, 6, 0, 0)
+    with pytest.raises(BeamMoEError):
+        moe.launch_plan(wl.T + 1)
     moe.close()
 
 
