@@ -47,6 +47,7 @@ struct beam_moe {
     int tile_rows;                   // 0: chosen from T
     int down_pair;                   // -1: auto, 0: single tiles, 1: paired tiles
     int use_pair;                    // 1: CTA-pair kernels for large token tiles (default)
+    int gather_rows;                 // -1: auto (default), 0: never, 1: always
     int last_T;
     std::vector<cudaEvent_t> prof_events;   // 6 per profiled forward pass
     int prof_max, prof_calls;
@@ -244,6 +245,7 @@ struct ForwardPlan {
     int down_paired;   // 1: two weight blocks per down work item
     int router_tc;     // 1: tensor-core logits with exact re-derivation
     int router_slices; // K slices of the router logits
+    int gather;        // 1: gate|up gathers token rows from x; no sorted copy
 };
 
 ForwardPlan plan_forward(const beam_moe *h, int T)
@@ -267,6 +269,11 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
     const int block_rows = p.cta_pairs ? 512 : 256;
     p.down_paired = h->H % block_rows == 0 &&
                     (h->down_pair == 1 || (h->down_pair < 0 && p.tile_rows >= 64));
+    // Gathered token rows spare dispatch the sorted copy of x, but each
+    // gather4 copy costs the TMA unit about as much as a whole box: with
+    // large token tiles the gathers of a stage outlast its MMAs.  Automatic
+    // only for tiles of up to 32 rows, where the weight stream sets the pace.
+    p.gather = h->gather_rows < 0 ? (p.tile_rows <= 32 ? 1 : 0) : h->gather_rows;
     p.router_tc = router_on_tensor_cores(h, T);
     p.router_slices = p.router_tc ? router_mma_slices(T, h->H, h->E, h->num_sms)
                                   : router_slices(T, h->H, h->E, h->num_sms);
@@ -299,6 +306,7 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     d.pair_row = h->pair_row;
     d.row_pair = h->row_pair;
     d.xp = h->xp;
+    d.copy_rows = !plan.gather;
     cudaError_t e = launch_dispatch(d, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "dispatch launch");
     prof_mark(h, s, 2);
@@ -310,20 +318,34 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.tile_off = h->tile_off;
     g.ctl.status = h->status;
     g.ctl.limit_ns = h->wait_limit_ns;
+    g.row_pair = h->row_pair;
+    g.top_k = h->top_k;
+    g.gather = plan.gather;
+    // token rows of the gate|up GEMM: x itself, four rows per gather4 copy,
+    // or boxes of the sorted copy
+    BoxMaps bx_local;
+    const BoxMaps *bx = &h->tm_xp;
+    if (plan.gather) {
+        bx_local = h->tm_xp;
+        if (!make_map(&bx_local.gather, x, (uint64_t)T, (uint64_t)h->H, 1u))
+            return fail(h, BEAM_ERR_CUDA, "tensor map of x");
+        bx = &bx_local;
+    }
     const bool use_pair = plan.cta_pairs != 0;
     const int grid = plan.grid;
     g.K = h->H;
     g.R = h->I;
     g.out = h->hbuf;
-    e = use_pair ? launch_grouped_gemm_pair(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_xp, g,
+    e = use_pair ? launch_grouped_gemm_pair(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx, g,
                                             grid, s)
-                 : launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_xp, g,
+                 : launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx, g,
                                        grid, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "gate/up GEMM launch");
     prof_mark(h, s, 3);
     g.K = h->I;
     g.R = h->H;
     g.out = h->ybuf;
+    g.gather = 0;
     const GemmKind dk = plan.down_paired ? GemmKind::kDownPaired : GemmKind::kDown;
     e = use_pair ? launch_grouped_gemm_pair(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s)
                  : launch_grouped_gemm(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s);
@@ -407,8 +429,7 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     if ((long long)max_tokens * top_k > (1LL << 30))
         return fail(nullptr, BEAM_ERR_UNSUPPORTED, "max_tokens * top_k too large");
 
-    beam_moe *h = new beam_moe();
-    memset(h, 0, sizeof(*h));
+    beam_moe *h = new beam_moe();   // value-initialised: every plain field starts at zero
     h->H = hidden;
     h->E = n_experts;
     h->I = inter;
@@ -427,6 +448,7 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     h->wait_limit_ns = 2000000000LL;
     h->down_pair = -1;
     h->use_pair = 1;
+    h->gather_rows = -1;
     h->router_mode = -1;
 
     cudaError_t e = cudaGetDevice(&h->device);
@@ -659,6 +681,7 @@ int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host)
     plan_host[3] = p.down_paired;
     plan_host[4] = p.router_tc;
     plan_host[5] = p.router_slices;
+    plan_host[6] = p.gather;
     return BEAM_OK;
 }
 
@@ -737,7 +760,7 @@ int beam_moe_profile_end(beam_moe_t h, float *stage_ms, int *calls)
 }
 
 int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair, int cta_pairs,
-                             int router_mode)
+                             int router_mode, int gather_rows)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
     if (ctas < 0 || ctas > 65535) return fail(h, BEAM_ERR_INVALID_ARG, "ctas outside [0, 65535]");
@@ -748,7 +771,10 @@ int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pai
     if (cta_pairs < 0 || cta_pairs > 1) return fail(h, BEAM_ERR_INVALID_ARG, "cta_pairs must be 0 or 1");
     if (router_mode < -1 || router_mode > 2)
         return fail(h, BEAM_ERR_INVALID_ARG, "router_mode outside [-1, 2]");
+    if (gather_rows < -1 || gather_rows > 1)
+        return fail(h, BEAM_ERR_INVALID_ARG, "gather_rows outside [-1, 1]");
     h->router_mode = router_mode;
+    h->gather_rows = gather_rows;
     h->gemm_ctas = ctas;
     h->tile_rows = tile_rows;
     h->down_pair = down_pair;

@@ -127,6 +127,21 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
     for (int i = lane; i < H / 8; i += 32) dst[i] = src[i];
 }
 
+// The maps only, a thread per pair: used when the gate|up GEMM gathers its
+// token rows from x, so no sorted copy of x is made.
+__global__ void __launch_bounds__(256) dispatch_rows_kernel(
+    const int32_t *__restrict__ idx, const int32_t *__restrict__ rank,
+    const int32_t *__restrict__ block_base, const int32_t *__restrict__ offsets, int P, int E,
+    int32_t *__restrict__ pair_row, int32_t *__restrict__ row_pair)
+{
+    const int p = blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= P) return;
+    const int e = idx[p];
+    const int row = offsets[e] + block_base[(size_t)(p / kDispatchBlock) * E + e] + rank[p];
+    pair_row[p] = row;
+    row_pair[row] = p;
+}
+
 cudaError_t prepare_dispatch(int E)
 {
     return cudaFuncSetAttribute(dispatch_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -147,9 +162,13 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t stream)
                                                     a.block_base, a.counts, a.offsets, a.tile_off);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    dispatch_permute_kernel<<<(P + 7) / 8, 256, 0, stream>>>(a.idx, a.rank, a.block_base,
-                                                             a.offsets, a.x, P, a.H, a.E, a.top_k,
-                                                             a.pair_row, a.row_pair, a.xp);
+    if (a.copy_rows)
+        dispatch_permute_kernel<<<(P + 7) / 8, 256, 0, stream>>>(
+            a.idx, a.rank, a.block_base, a.offsets, a.x, P, a.H, a.E, a.top_k, a.pair_row,
+            a.row_pair, a.xp);
+    else
+        dispatch_rows_kernel<<<(P + 255) / 256, 256, 0, stream>>>(
+            a.idx, a.rank, a.block_base, a.offsets, P, a.E, a.pair_row, a.row_pair);
     return cudaGetLastError();
 }
 

@@ -56,6 +56,28 @@ __device__ __forceinline__ Item decode_item(int i, int WT, int E, const int *s_c
     return it;
 }
 
+// Rows of x for this CTA's gather4 copies of a token tile: copy j (this lane
+// takes j = lane, lane + 32, ...) fills tile rows first + 4j .. first + 4j + 3.
+// Row r of the expert-sorted order is pair row_pair[r] = t * top_k + slot, so
+// its token is row_pair[r] / top_k.  Rows past the tile's valid rows (the MMA
+// N is rounded up to 16) repeat the tile's first row; their results are
+// never stored.
+template <int G>
+__device__ __forceinline__ void gather_tokens(const GemmArgs &p, const Item &it, int first,
+                                              int n_ops, int lane, int (&tok)[G][4])
+{
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const int op = lane + 32 * g;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = first + 4 * op + q;
+            const int row = (op < n_ops && r < it.nrows) ? it.row0 + r : it.row0;
+            tok[g][q] = p.row_pair[row] / p.top_k;
+        }
+    }
+}
+
 // silu(g) = g / (1 + e^-g) in FP32 with the fast exponential and divide; the
 // product with u is rounded to bf16 right after, which the approximations
 // (a few FP32 ulps) do not reach but in rare rounding-boundary cases.

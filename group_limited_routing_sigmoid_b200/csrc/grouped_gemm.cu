@@ -19,7 +19,9 @@
 // equal size, and each item's MMA N is its tile size rounded up to 16 (a
 // runtime field of the instruction descriptor), so ragged experts waste at
 // most 15 rows per tile.  The TMA loads of a token tile fetch exactly those
-// rows, as a sum of power-of-two boxes.
+// rows, as a sum of power-of-two boxes of the sorted buffer, or (gate|up,
+// by default) four rows at a time straight from x, which spares the sorted
+// copy of x altogether.
 //   gate|up: two A tiles (gate and up rows i0..i0+127) into two TMEM
 //            accumulators, so TMEM lane r holds gate and up of one
 //            intermediate row and the SwiGLU needs no exchange;
@@ -27,7 +29,8 @@
 //            share the token tile, halving the token bytes per MMA.
 //
 // Warp roles (320 threads, one CTA per SM, persistent over the item list):
-//   warp 0      TMA producer (lane 0);
+//   warp 0      TMA producer (lane 0; all lanes when gate|up gathers token
+//               rows from x with tile::gather4);
 //   warp 1      TMEM allocator and UMMA issuer (one thread);
 //   warps 2..9  epilogue (two per TMEM lane quadrant): tcgen05.ld, SwiGLU or
 //               the plain accumulator, rounded to bf16, a 32x32 transpose
@@ -124,9 +127,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int KB = p.K / kBK;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer (lane 0)
+        // ------------------------------------------------ TMA producer
+        // Lane 0 loads the weight tiles (and the token tile from the sorted
+        // buffer); with gathering, every lane also issues its gather4 copies
+        // of token rows straight from x.
         const uint64_t pol_w = l2_policy_evict_first();   // weights: streamed
         const uint64_t pol_x = l2_policy_evict_last();    // activations: reused across tiles
+        constexpr int G = (BN / 4 + 31) / 32;             // gather4 copies per lane, at most
+        const bool gather = EPI == kSwiGLU && p.gather != 0;
         int stage = 0;
         uint32_t phase = 0;
         long long issued = 0;
@@ -136,21 +144,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int a_row = it.e * p.R + it.wt * C::ROWS_PER_ITEM;
             const int n_load = (it.nrows + 15) & ~15;
             const uint32_t bytes = NUM_A * C::A_BYTES + n_load * (kBK * 2);
+            int tok[G][4];
+            if (gather) gather_tokens<G>(p, it, 0, n_load >> 2, lane, tok);
             for (int kb = 0; kb < KB; ++kb) {
                 bool got = true;
+                if (lane == 0 || gather) got = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl);
+                ok = __all_sync(0xffffffffu, got);
+                if (!ok) break;
+                const uint32_t sa = base + stage * C::STAGE_BYTES;
+                const uint32_t sb = sa + NUM_A * C::A_BYTES;
+                const uint32_t fb = smem_u32(&full[stage]);
                 if (lane == 0) {
-                    got = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl);
-                    if (got) {
-                        const uint32_t sa = base + stage * C::STAGE_BYTES;
-                        const uint32_t fb = smem_u32(&full[stage]);
-                        mbar_arrive_expect_tx(fb, bytes);
-                        tma_load_2d(sa, &tmA0, kb * kBK, a_row, fb, pol_w);
-                        if (NUM_A == 2) {
-                            // gate|up: the up matrix at the same rows; down: the next 128 rows
-                            const int a_row1 = EPI == kSwiGLU ? a_row : a_row + kBM;
-                            tma_load_2d(sa + C::A_BYTES, &tmA1, kb * kBK, a_row1, fb, pol_w);
-                        }
-                        const uint32_t sb = sa + NUM_A * C::A_BYTES;
+                    mbar_arrive_expect_tx(fb, bytes);
+                    tma_load_2d(sa, &tmA0, kb * kBK, a_row, fb, pol_w);
+                    if (NUM_A == 2) {
+                        // gate|up: the up matrix at the same rows; down: the next 128 rows
+                        const int a_row1 = EPI == kSwiGLU ? a_row : a_row + kBM;
+                        tma_load_2d(sa + C::A_BYTES, &tmA1, kb * kBK, a_row1, fb, pol_w);
+                    }
+                    if (!gather) {
                         int off = 0;
 #pragma unroll
                         for (int bi = 5; bi >= 1; --bi) {   // boxes of 256, 128, 64, 32, 16 rows
@@ -163,8 +175,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
-                if (!ok) break;
+                if (gather) {
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const int op = lane + 32 * g;
+                        if (op < (n_load >> 2))
+                            tma_gather4(sb + op * (4 * kBK * 2), &tmB.gather, kb * kBK, tok[g][0],
+                                        tok[g][1], tok[g][2], tok[g][3], fb, pol_x);
+                    }
+                }
                 ++issued;
                 if (++stage == C::STAGES) {
                     stage = 0;

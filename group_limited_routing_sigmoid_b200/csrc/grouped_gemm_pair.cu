@@ -115,9 +115,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int KB = p.K / kBK;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer (lane 0)
+        // ------------------------------------------------ TMA producer
+        // Lane 0 loads the weight tiles (and the token rows from the sorted
+        // buffer); with gathering, every lane also issues its gather4 copies
+        // of token rows straight from x.
         const uint64_t pol_w = l2_policy_evict_first();
         const uint64_t pol_x = l2_policy_evict_last();
+        constexpr int G = (C::HALF / 4 + 31) / 32;          // gather4 copies per lane, at most
+        const bool gather = EPI == kSwiGLU && p.gather != 0;
         int stage = 0;
         uint32_t phase = 0;
         long long issued = 0;
@@ -130,22 +135,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // A rows of this CTA: its 128-row half of each 256-row block
             const int a_base = it.e * p.R + it.wt * C::ROWS_PER_ITEM + (int)rank * kBM;
             const uint32_t pair_bytes = 2u * (NUM_A * C::A_BYTES + half * (kBK * 2));
+            int tok[G][4];
+            if (gather) gather_tokens<G>(p, it, (int)rank * half, half >> 2, lane, tok);
             for (int kb = 0; kb < KB; ++kb) {
                 bool got = true;
+                if (lane == 0 || gather) got = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl);
+                ok = __all_sync(0xffffffffu, got);
+                if (!ok) break;
+                const uint32_t sa = base + stage * C::STAGE_BYTES;
+                const uint32_t sb = sa + NUM_A * C::A_BYTES;
+                const uint32_t fb_local = smem_u32(&full[stage]);
+                const uint32_t fb = mapa_shared(fb_local, 0);   // CTA 0's barrier
                 if (lane == 0) {
-                    got = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl);
-                    if (got) {
-                        const uint32_t sa = base + stage * C::STAGE_BYTES;
-                        const uint32_t fb_local = smem_u32(&full[stage]);
-                        const uint32_t fb = mapa_shared(fb_local, 0);   // CTA 0's barrier
-                        if (rank == 0) mbar_arrive_expect_tx(fb_local, pair_bytes);
-                        tma_load_2d_pair(sa, &tmA0, kb * kBK, a_base, fb, pol_w);
-                        if (NUM_A == 2) {
-                            // gate|up: the up matrix at the same rows; down: the next 256-row block
-                            const int a_row1 = EPI == kSwiGLU ? a_base : a_base + 2 * kBM;
-                            tma_load_2d_pair(sa + C::A_BYTES, &tmA1, kb * kBK, a_row1, fb, pol_w);
-                        }
-                        const uint32_t sb = sa + NUM_A * C::A_BYTES;
+                    if (rank == 0) mbar_arrive_expect_tx(fb_local, pair_bytes);
+                    tma_load_2d_pair(sa, &tmA0, kb * kBK, a_base, fb, pol_w);
+                    if (NUM_A == 2) {
+                        // gate|up: the up matrix at the same rows; down: the next 256-row block
+                        const int a_row1 = EPI == kSwiGLU ? a_base : a_base + 2 * kBM;
+                        tma_load_2d_pair(sa + C::A_BYTES, &tmA1, kb * kBK, a_row1, fb, pol_w);
+                    }
+                    if (!gather) {
                         int off = 0;
 #pragma unroll
                         for (int bi = 4; bi >= 0; --bi) {   // boxes of 128, 64, 32, 16, 8 rows
@@ -158,8 +167,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
-                if (!ok) break;
+                if (gather) {
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const int op = lane + 32 * g;
+                        if (op < (half >> 2))
+                            tma_gather4_pair(sb + op * (4 * kBK * 2), &tmB.gather, kb * kBK,
+                                             tok[g][0], tok[g][1], tok[g][2], tok[g][3], fb, pol_x);
+                    }
+                }
                 ++issued;
                 if (++stage == C::STAGES) {
                     stage = 0;

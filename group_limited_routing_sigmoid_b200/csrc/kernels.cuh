@@ -70,6 +70,7 @@ struct DispatchArgs {
     int32_t *pair_row;           // [P]
     int32_t *row_pair;           // [P]
     __nv_bfloat16 *xp;           // [P, H] expert-sorted activations
+    int copy_rows;               // 0: maps only (the gate|up GEMM gathers from x)
 };
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t stream);
 cudaError_t prepare_dispatch(int E);   // shared-memory limit of the counting kernel
@@ -83,13 +84,20 @@ struct GemmArgs {
     const int32_t *offsets;      // [E+1]
     const int32_t *tile_off;     // [E+1]
     __nv_bfloat16 *out;          // bf16 [P, R]: h (gate|up) or y (down)
+    // gate|up only: when `gather` is set, token rows come straight from x
+    // (BoxMaps::gather), row r of the sorted order being token row_pair[r] / top_k
+    const int32_t *row_pair;     // [P]
+    int top_k;
+    int gather;
     WaitCtl ctl;
 };
 
 // Tensor maps of one activation buffer with boxes of 8, 16, 32, 64, 128 and
-// 256 rows (64 columns each): a token tile is loaded as a sum of these.
+// 256 rows (64 columns each): a token tile is loaded as a sum of these; or,
+// for the gate|up GEMM with gathering on, four token rows at a time from x.
 struct BoxMaps {
     CUtensorMap m[6];
+    CUtensorMap gather;          // x [T, H] with a 64-column, one-row box (tile::gather4)
 };
 
 enum class GemmKind {

@@ -198,12 +198,13 @@ int beam_moe_router_stats(beam_moe_t h, void *stream, int32_t *rederived_host);
 
 /*
  * The launch configuration a forward pass of T tokens (0 <= T <= max_tokens)
- * uses under the handle's current tuning, written to plan_host (int32 [6],
- * host): {largest token tile of the grouped GEMMs (rows), 1 if they run on
- * CTA pairs (cta_group::2), CTAs per grouped GEMM, 1 if the down projection
- * takes two weight blocks per work item, 1 if the router logits run on the
- * tensor cores (with exact re-derivation of thin-margin tokens), K slices of
- * the router logits}.  A function of T and the tuning only; launches nothing.
+ * uses under the handle's current tuning, written to plan_host (int32 [7],
+ * host): {largest token tile of the grouped GEMMs (rows), 1 if
+ * they run on CTA pairs (cta_group::2), CTAs per grouped GEMM, 1 if the down
+ * projection takes two weight blocks per work item, 1 if the router logits
+ * run on the tensor cores (with exact re-derivation of thin-margin tokens),
+ * K slices of the router logits, 1 if the gate|up GEMM gathers token rows
+ * from x}.  A function of T and the tuning only; launches nothing.
  * Returns BEAM_ERR_INVALID_ARG for a NULL pointer or T out of range.
  */
 int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host);
@@ -246,13 +247,19 @@ int beam_moe_set_wait_limit(beam_moe_t h, int64_t limit_ns);
  *                 smallest gap between neighbours in the ranking of its top
  *                 k+1 candidates (it fixes the chosen set and their order),
  *                 or weakest kept vs strongest dropped group score -- is
- *                 below 4e-5 has
- *                 its logits recomputed with FP32 CUDA-core dot products and
- *                 is selected again, so decisions keep CUDA-core accuracy.
- *                 beam_moe_router_logits always uses the CUDA-core path.
+ *                 below 4e-5 has its logits recomputed with FP32 CUDA-core
+ *                 dot products and is selected again, so decisions keep
+ *                 CUDA-core accuracy.  beam_moe_router_logits always uses
+ *                 the CUDA-core path.
+ * gather_rows     1: the gate|up GEMM loads its token rows straight from x,
+ *                 four rows per TMA gather4 copy, so dispatch makes no
+ *                 expert-sorted copy of x; 0: dispatch copies x into the
+ *                 sorted buffer and the GEMM loads boxes of it; -1
+ *                 (default): gather when token tiles are at most 32 rows
+ *                 (the gathers of a large tile outlast its MMAs).
  */
 int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair,
-                             int cta_pairs, int router_mode);
+                             int cta_pairs, int router_mode, int gather_rows);
 
 /*
  * Per-stage timing of forward passes, for measurement.  After

@@ -44,42 +44,47 @@ def _inputs(wl, T=None):
     return d
 
 
-# (T, GEMM CTAs (0 = one per SM), largest token tile (0 = auto), paired down tiles (-1 = auto))
-TINY_CASES = [(64, 0, 0, -1), (64, 1, 0, -1), (1, 0, 0, -1), (3, 0, 0, -1), (37, 5, 0, -1),
-              (100, 0, 0, -1), (200, 3, 0, -1), (1000, 0, 0, -1), (1000, 2, 0, -1),
-              (4096, 0, 0, -1), (1000, 0, 16, 0), (1000, 0, 32, 1), (1000, 0, 64, 0),
-              (1000, 3, 128, 1), (1000, 0, 256, 0), (1000, 2, 256, 1), (300, 0, 256, 1),
-              (4096, 7, 256, 1)]
+# (T, GEMM CTAs (0 = one per SM), largest token tile (0 = auto), paired down tiles (-1 = auto),
+#  gate|up token rows gathered from x: -1 auto, 1 always, 0 never (sorted copy))
+TINY_CASES = [(64, 0, 0, -1, -1), (64, 1, 0, -1, -1), (1, 0, 0, -1, -1), (3, 0, 0, -1, -1),
+              (37, 5, 0, -1, -1), (100, 0, 0, -1, -1), (200, 3, 0, -1, -1), (1000, 0, 0, -1, -1),
+              (1000, 2, 0, -1, -1), (4096, 0, 0, -1, -1), (1000, 0, 16, 0, 1), (1000, 0, 32, 1, 1),
+              (1000, 0, 64, 0, 1), (1000, 3, 128, 1, 1), (1000, 0, 256, 0, 1), (1000, 2, 256, 1, 1),
+              (300, 0, 256, 1, 1), (4096, 7, 256, 1, 1),
+              (37, 5, 0, -1, 0), (1000, 0, 0, -1, 0), (1000, 0, 32, 1, 0), (4096, 7, 256, 1, 0)]
 
 
-@pytest.mark.parametrize("T,ctas,tile,pair", TINY_CASES)
-def test_tiny_block(T, ctas, tile, pair):
+@pytest.mark.parametrize("T,ctas,tile,pair,gather", TINY_CASES)
+def test_tiny_block(T, ctas, tile, pair, gather):
     wl = W.WORKLOADS["tiny"]
     d = _inputs(wl, T)
     moe = BeamMoE.from_workload(wl, d, max_tokens=T)
-    moe.set_gemm_tuning(ctas, tile, pair)
+    moe.set_gemm_tuning(ctas, tile, pair, gather_rows=gather)
     rep = check_block(wl, d, moe)
-    _log(f"tiny_T{T}_ctas{ctas}_tile{tile}_pair{pair}", rep)
+    _log(f"tiny_T{T}_ctas{ctas}_tile{tile}_pair{pair}_gather{gather}", rep)
     assert rep.ok(), rep
     moe.close()
 
 
-# (T, GEMM CTAs, largest token tile, paired down tiles, CTA pairs, router mode): H=512, I=256
-SMALL_CASES = [(1024, 0, 0, -1, 1, -1), (1024, 0, 0, -1, 0, 0), (1024, 0, 64, 0, 1, 1),
-               (1024, 4, 128, 1, 1, 1), (1024, 0, 256, 0, 1, 0), (3000, 0, 256, 1, 1, 1),
-               (3000, 6, 256, 1, 1, -1), (777, 0, 128, -1, 1, 1), (2048, 2, 64, 1, 1, 0),
-               (64, 0, 64, -1, 1, 1), (1, 0, 0, -1, 1, 1), (130, 0, 0, -1, 1, 1),
-               (1024, 0, 0, -1, 1, 2), (3000, 0, 0, -1, 1, 2)]
+# (T, GEMM CTAs, largest token tile, paired down tiles, CTA pairs, router mode, gathered
+#  token rows): H=512, I=256
+SMALL_CASES = [(1024, 0, 0, -1, 1, -1, -1), (1024, 0, 0, -1, 0, 0, 1), (1024, 0, 64, 0, 1, 1, 1),
+               (1024, 4, 128, 1, 1, 1, 1), (1024, 0, 256, 0, 1, 0, 1), (3000, 0, 256, 1, 1, 1, 1),
+               (3000, 6, 256, 1, 1, -1, -1), (777, 0, 128, -1, 1, 1, 1), (2048, 2, 64, 1, 1, 0, 1),
+               (64, 0, 64, -1, 1, 1, 1), (1, 0, 0, -1, 1, 1, -1), (130, 0, 0, -1, 1, 1, -1),
+               (1024, 0, 0, -1, 1, 2, 1), (3000, 0, 0, -1, 1, 2, 1),
+               (1024, 0, 0, -1, 1, -1, 0), (1024, 0, 0, -1, 0, 0, 0), (777, 0, 128, -1, 1, 1, 0),
+               (3000, 6, 256, 1, 1, -1, 0)]
 
 
-@pytest.mark.parametrize("T,ctas,tile,pair,pairs,router", SMALL_CASES)
-def test_small_block(T, ctas, tile, pair, pairs, router):
+@pytest.mark.parametrize("T,ctas,tile,pair,pairs,router,gather", SMALL_CASES)
+def test_small_block(T, ctas, tile, pair, pairs, router, gather):
     wl = W.WORKLOADS["small"]
     d = _inputs(wl, T)
     moe = BeamMoE.from_workload(wl, d, max_tokens=T)
-    moe.set_gemm_tuning(ctas, tile, pair, pairs, router)
+    moe.set_gemm_tuning(ctas, tile, pair, pairs, router, gather)
     rep = check_block(wl, d, moe)
-    _log(f"small_T{T}_ctas{ctas}_tile{tile}_pair{pair}_pairs{pairs}_router{router}", rep)
+    _log(f"small_T{T}_ctas{ctas}_tile{tile}_pair{pair}_pairs{pairs}_router{router}_gather{gather}", rep)
     assert rep.ok(), rep
     moe.close()
 
@@ -98,11 +103,13 @@ def test_tiny_residual(norm):
     moe.close()
 
 
-def test_tiny_dispatch_is_a_stable_counting_sort():
+@pytest.mark.parametrize("gather", [-1, 1, 0])
+def test_tiny_dispatch_is_a_stable_counting_sort(gather):
     wl = W.WORKLOADS["tiny"]
     T = 1000
     d = _inputs(wl, T)
     moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    moe.set_gemm_tuning(gather_rows=gather)
     moe.forward(d["x"])
     idx, _ = moe.route(d["x"])
     counts, offsets, pair_row = moe.dispatch_info(T)
@@ -197,15 +204,17 @@ def test_launch_plan_follows_tokens_per_expert_and_tuning():
     d = _inputs(wl)
     moe = BeamMoE.from_workload(wl, d)
     p = moe.launch_plan(8)
-    assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"]) == (16, 0, 0, 0)
+    assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"],
+            p["gather_rows"]) == (16, 0, 0, 0, 1)
     assert p["grid"] == torch.cuda.get_device_properties(0).multi_processor_count
     p = moe.launch_plan(wl.T)
     assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"]) == (256, 1, 1, 1)
     assert p["grid"] % 2 == 0 and p["router_slices"] >= 1
-    moe.set_gemm_tuning(6, 64, 0, 0, 0)
+    assert p["gather_rows"] == 0
+    moe.set_gemm_tuning(6, 64, 0, 0, 0, 1)
     p = moe.launch_plan(wl.T)
-    assert (p["tile_rows"], p["cta_pairs"], p["grid"], p["down_paired"], p["router_tensor_cores"]) == \
-        (64, 0, 6, 0, 0)
+    assert (p["tile_rows"], p["cta_pairs"], p["grid"], p["down_paired"], p["router_tensor_cores"],
+            p["gather_rows"]) == (64, 0, 6, 0, 0, 1)
     with pytest.raises(BeamMoEError):
         moe.launch_plan(wl.T + 1)
     moe.close()
