@@ -58,6 +58,8 @@ def _load():
         D = ctypes.c_double
         lib.oracle_route.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_route.restype = I
+        lib.oracle_route_logits.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P]
+        lib.oracle_route_logits.restype = I
         lib.oracle_expert_swiglu.argtypes = [I, I, I, P, P, P, P, P, P]
         lib.oracle_expert_swiglu.restype = None
         lib.oracle_combine.argtypes = [I, I, I, P, P, D, P, P]
@@ -152,6 +154,30 @@ def route(x_bits: np.ndarray, router_w: np.ndarray, bias: np.ndarray,
     if rc != 0:
         raise ValueError("oracle_route: routing configuration not defined by the method")
     return Routing(idx, w, scores, biased, ge, gg, km, go)
+
+
+def route_logits(logits: np.ndarray, bias: np.ndarray, n_group: int, topk_group: int,
+                 top_k: int) -> Routing:
+    """The same routing from given FP32 logits [T, E] (selection only): what a
+    re-route under another expert bias computes.  scores/biased are left
+    empty."""
+    lib = _load()
+    lg = _f32(logits)
+    b = _f32(bias)
+    T, E = lg.shape
+    assert b.shape == (E,)
+    idx = np.empty((T, top_k), np.int32)
+    w = np.empty((T, top_k), np.float64)
+    ge = np.empty((T,), np.float64)
+    gg = np.empty((T,), np.float64)
+    km = np.empty((T,), np.int32)
+    go = np.empty((T,), np.float64)
+    rc = lib.oracle_route_logits(T, E, n_group, topk_group, top_k, _ptr(lg), _ptr(b), _ptr(idx),
+                                 _ptr(w), _ptr(ge), _ptr(gg), _ptr(km), _ptr(go))
+    if rc != 0:
+        raise ValueError("oracle_route_logits: routing configuration not defined by the method")
+    empty = np.empty((T, 0), np.float64)
+    return Routing(idx, w, empty, empty, ge, gg, km, go)
 
 
 def expert_swiglu(x_bits: np.ndarray, w_gate_bits: np.ndarray, w_up_bits: np.ndarray,

@@ -91,6 +91,116 @@ static double silu(double z) { return z / (1.0 + exp(-z)); }
 /* ------------------------------------------------------------------ */
 
 /*
+ * Selection for one token from its E logits (double): sigmoid scores, FP32
+ * biased scores, group scores, kept groups, top_k experts and their
+ * normalised unbiased weights, plus the near-tie gaps; the outputs are the
+ * token's rows of oracle_route's outputs.
+ */
+static void route_one(int E, int n_group, int topk_group, int top_k, const double *logit,
+                      const float *bias, int32_t *idx, double *w, double *scores,
+                      double *biased, double *gap_expert, double *gap_group,
+                      int32_t *kept_mask, double *gap_order)
+{
+    const int gsize = E / n_group;
+    double *s = (double *)malloc(sizeof(double) * (size_t)E);
+    double *bd = (double *)malloc(sizeof(double) * (size_t)E);
+    float *b32 = (float *)malloc(sizeof(float) * (size_t)E);
+    float *gs = (float *)malloc(sizeof(float) * (size_t)n_group);
+    double *gsd = (double *)malloc(sizeof(double) * (size_t)n_group);
+    char *kept = (char *)calloc((size_t)n_group, 1);
+    char *chosen = (char *)calloc((size_t)E, 1);
+
+    /* sigmoid scores, biased scores */
+    for (int e = 0; e < E; ++e) {
+        s[e] = sigmoid(logit[e]);
+        bd[e] = s[e] + (double)bias[e];
+        b32[e] = (float)bd[e];
+    }
+
+    /* group score: sum of the two largest biased scores of the group */
+    for (int j = 0; j < n_group; ++j) {
+        float t1 = -INFINITY, t2 = -INFINITY;
+        double d1 = -INFINITY, d2 = -INFINITY;
+        for (int e = j * gsize; e < (j + 1) * gsize; ++e) {
+            if (b32[e] > t1) { t2 = t1; t1 = b32[e]; }
+            else if (b32[e] > t2) { t2 = b32[e]; }
+            if (bd[e] > d1) { d2 = d1; d1 = bd[e]; }
+            else if (bd[e] > d2) { d2 = bd[e]; }
+        }
+        gs[j] = t1 + t2; /* FP32 addition */
+        gsd[j] = d1 + d2;
+    }
+
+    /* keep topk_group groups: greater score first, ties to lower index */
+    int32_t mask = 0;
+    for (int r = 0; r < topk_group; ++r) {
+        int best = -1;
+        for (int j = 0; j < n_group; ++j) {
+            if (kept[j]) continue;
+            if (best < 0 || gs[j] > gs[best]) best = j;
+        }
+        kept[best] = 1;
+        mask |= (int32_t)1 << best;
+    }
+
+    /* top_k experts among the kept groups' experts */
+    double ssum = 0.0;
+    for (int r = 0; r < top_k; ++r) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+            if (!kept[e / gsize] || chosen[e]) continue;
+            if (best < 0 || b32[e] > b32[best]) best = e;
+        }
+        chosen[best] = 1;
+        idx[r] = best;
+        ssum += s[best];
+    }
+    for (int r = 0; r < top_k; ++r) w[r] = s[idx[r]] / ssum;
+
+    if (gap_expert) {
+        double min_sel = INFINITY, max_uns = -INFINITY;
+        for (int e = 0; e < E; ++e) {
+            if (!kept[e / gsize]) continue;
+            if (chosen[e]) { if (bd[e] < min_sel) min_sel = bd[e]; }
+            else if (bd[e] > max_uns) max_uns = bd[e];
+        }
+        *gap_expert = (max_uns == -INFINITY) ? INFINITY : min_sel - max_uns;
+    }
+    if (gap_group) {
+        double min_k = INFINITY, max_d = -INFINITY;
+        for (int j = 0; j < n_group; ++j) {
+            if (kept[j]) { if (gsd[j] < min_k) min_k = gsd[j]; }
+            else if (gsd[j] > max_d) max_d = gsd[j];
+        }
+        *gap_group = (max_d == -INFINITY) ? INFINITY : min_k - max_d;
+    }
+    if (gap_order) {
+        double g = INFINITY;
+        for (int r = 0; r + 1 < top_k; ++r) {
+            const double d = bd[idx[r]] - bd[idx[r + 1]];
+            if (d < g) g = d;
+        }
+        *gap_order = g;
+    }
+    if (kept_mask) *kept_mask = mask;
+    if (scores) memcpy(scores, s, sizeof(double) * (size_t)E);
+    if (biased) memcpy(biased, bd, sizeof(double) * (size_t)E);
+    free(s); free(bd); free(b32); free(gs); free(gsd); free(kept); free(chosen);
+}
+
+/* The routing configurations the method defines. */
+static int route_args_ok(int E, int n_group, int topk_group, int top_k)
+{
+    if (E <= 0 || n_group <= 0 || E % n_group != 0) return 0;
+    const int gsize = E / n_group;
+    if (gsize < 2 || topk_group < 1 || topk_group > n_group || n_group > 31) return 0;
+    if (top_k < 1 || top_k > topk_group * gsize) return 0;
+    return 1;
+}
+
+#define ROW(p, t, n) ((p) ? (p) + (size_t)(t) * (n) : NULL)
+
+/*
  * Group-limited sigmoid routing for T tokens.
  *
  * x        bf16 [T, H] row-major
@@ -123,104 +233,47 @@ int oracle_route(int T, int H, int E, int n_group, int topk_group, int top_k,
                  double *gap_expert, double *gap_group, int32_t *kept_mask,
                  double *gap_order)
 {
-    if (T < 0 || H <= 0 || E <= 0 || n_group <= 0 || E % n_group != 0) return -1;
-    const int gsize = E / n_group;
-    if (gsize < 2 || topk_group < 1 || topk_group > n_group || n_group > 31) return -1;
-    if (top_k < 1 || top_k > topk_group * gsize) return -1;
+    if (T < 0 || H <= 0 || !route_args_ok(E, n_group, topk_group, top_k)) return -1;
 
 #pragma omp parallel for schedule(dynamic, 1)
     for (int t = 0; t < T; ++t) {
-        double *s = (double *)malloc(sizeof(double) * (size_t)E);
-        double *bd = (double *)malloc(sizeof(double) * (size_t)E);
-        float *b32 = (float *)malloc(sizeof(float) * (size_t)E);
-        float *gs = (float *)malloc(sizeof(float) * (size_t)n_group);
-        double *gsd = (double *)malloc(sizeof(double) * (size_t)n_group);
-        char *kept = (char *)calloc((size_t)n_group, 1);
-        char *chosen = (char *)calloc((size_t)E, 1);
+        double *logit = (double *)malloc(sizeof(double) * (size_t)E);
         const uint16_t *xt = x + (size_t)t * H;
-
-        /* logits, sigmoid scores, biased scores */
+        /* logits: x . router_w[e], exact products summed in double */
         for (int e = 0; e < E; ++e) {
             const float *wr = router_w + (size_t)e * H;
             double acc = 0.0;
             for (int h = 0; h < H; ++h) acc += oracle_bf16_to_double(xt[h]) * (double)wr[h];
-            s[e] = sigmoid(acc);
-            bd[e] = s[e] + (double)bias[e];
-            b32[e] = (float)bd[e];
+            logit[e] = acc;
         }
+        route_one(E, n_group, topk_group, top_k, logit, bias, idx + (size_t)t * top_k,
+                  w + (size_t)t * top_k, ROW(scores, t, E), ROW(biased, t, E), ROW(gap_expert, t, 1),
+                  ROW(gap_group, t, 1), ROW(kept_mask, t, 1), ROW(gap_order, t, 1));
+        free(logit);
+    }
+    return 0;
+}
 
-        /* group score: sum of the two largest biased scores of the group */
-        for (int j = 0; j < n_group; ++j) {
-            float t1 = -INFINITY, t2 = -INFINITY;
-            double d1 = -INFINITY, d2 = -INFINITY;
-            for (int e = j * gsize; e < (j + 1) * gsize; ++e) {
-                if (b32[e] > t1) { t2 = t1; t1 = b32[e]; }
-                else if (b32[e] > t2) { t2 = b32[e]; }
-                if (bd[e] > d1) { d2 = d1; d1 = bd[e]; }
-                else if (bd[e] > d2) { d2 = bd[e]; }
-            }
-            gs[j] = t1 + t2; /* FP32 addition */
-            gsd[j] = d1 + d2;
-        }
+/*
+ * The same routing from given FP32 logits [T, E] (row-major) instead of x and
+ * the router matrix: selection under another expert bias reuses the logits
+ * (the bias steers selection only).  Outputs as oracle_route.
+ */
+int oracle_route_logits(int T, int E, int n_group, int topk_group, int top_k,
+                        const float *logits, const float *bias, int32_t *idx, double *w,
+                        double *gap_expert, double *gap_group, int32_t *kept_mask,
+                        double *gap_order)
+{
+    if (T < 0 || !route_args_ok(E, n_group, topk_group, top_k)) return -1;
 
-        /* keep topk_group groups: greater score first, ties to lower index */
-        int32_t mask = 0;
-        for (int r = 0; r < topk_group; ++r) {
-            int best = -1;
-            for (int j = 0; j < n_group; ++j) {
-                if (kept[j]) continue;
-                if (best < 0 || gs[j] > gs[best]) best = j;
-            }
-            kept[best] = 1;
-            mask |= (int32_t)1 << best;
-        }
-
-        /* top_k experts among the kept groups' experts */
-        double ssum = 0.0;
-        for (int r = 0; r < top_k; ++r) {
-            int best = -1;
-            for (int e = 0; e < E; ++e) {
-                if (!kept[e / gsize] || chosen[e]) continue;
-                if (best < 0 || b32[e] > b32[best]) best = e;
-            }
-            chosen[best] = 1;
-            idx[(size_t)t * top_k + r] = best;
-            ssum += s[best];
-        }
-        for (int r = 0; r < top_k; ++r) {
-            int e = idx[(size_t)t * top_k + r];
-            w[(size_t)t * top_k + r] = s[e] / ssum;
-        }
-
-        if (gap_expert) {
-            double min_sel = INFINITY, max_uns = -INFINITY;
-            for (int e = 0; e < E; ++e) {
-                if (!kept[e / gsize]) continue;
-                if (chosen[e]) { if (bd[e] < min_sel) min_sel = bd[e]; }
-                else if (bd[e] > max_uns) max_uns = bd[e];
-            }
-            gap_expert[t] = (max_uns == -INFINITY) ? INFINITY : min_sel - max_uns;
-        }
-        if (gap_group) {
-            double min_k = INFINITY, max_d = -INFINITY;
-            for (int j = 0; j < n_group; ++j) {
-                if (kept[j]) { if (gsd[j] < min_k) min_k = gsd[j]; }
-                else if (gsd[j] > max_d) max_d = gsd[j];
-            }
-            gap_group[t] = (max_d == -INFINITY) ? INFINITY : min_k - max_d;
-        }
-        if (gap_order) {
-            double g = INFINITY;
-            for (int r = 0; r + 1 < top_k; ++r) {
-                const double d = bd[idx[(size_t)t * top_k + r]] - bd[idx[(size_t)t * top_k + r + 1]];
-                if (d < g) g = d;
-            }
-            gap_order[t] = g;
-        }
-        if (kept_mask) kept_mask[t] = mask;
-        if (scores) memcpy(scores + (size_t)t * E, s, sizeof(double) * (size_t)E);
-        if (biased) memcpy(biased + (size_t)t * E, bd, sizeof(double) * (size_t)E);
-        free(s); free(bd); free(b32); free(gs); free(gsd); free(kept); free(chosen);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int t = 0; t < T; ++t) {
+        double *logit = (double *)malloc(sizeof(double) * (size_t)E);
+        for (int e = 0; e < E; ++e) logit[e] = (double)logits[(size_t)t * E + e];
+        route_one(E, n_group, topk_group, top_k, logit, bias, idx + (size_t)t * top_k,
+                  w + (size_t)t * top_k, NULL, NULL, ROW(gap_expert, t, 1), ROW(gap_group, t, 1),
+                  ROW(kept_mask, t, 1), ROW(gap_order, t, 1));
+        free(logit);
     }
     return 0;
 }

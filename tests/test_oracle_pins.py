@@ -10,6 +10,8 @@ Each pin is chosen so that a plausible slip in the oracle fails it:
   * bias left out of selection, or put into the weights
     -> test_bias_selects_but_does_not_weigh;
   * group limiting not applied -> test_single_group_reduces_to_topk;
+  * selection from given logits (re-route under another bias)
+    -> test_route_from_logits_*;
   * weights not normalised, x2.5 missing, slot/expert mix-up
     -> test_identical_experts_closed_form / test_permutation_experts_closed_form;
   * a transposed expert matrix -> test_permutation_experts_closed_form;
@@ -216,6 +218,55 @@ def test_bias_selects_but_does_not_weigh(oracle_lib):
         np.testing.assert_allclose(r.w[t], sel / sel.sum(), rtol=1e-14)
         biased_w = (sel + 10.0) / (sel + 10.0).sum()
         assert np.abs(r.w[t] - biased_w).max() > 1e-3
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_route_from_logits_bruteforce(oracle_lib, seed):
+    """Selection from given FP32 logits (the re-route under another bias):
+    exhaustive search over group subsets and expert subsets on the tiny
+    layout, with logits and a bias drawn directly."""
+    rng = np.random.default_rng(100 + seed)
+    logits = rng.standard_normal((20, 32)).astype(np.float32)
+    bias = rng.uniform(-0.1, 0.1, 32).astype(np.float32)
+    r = oracle_lib.route_logits(logits, bias, 8, 4, 8)
+    s = expit(logits.astype(np.float64))
+    for t in range(20):
+        b32 = (s[t] + bias.astype(np.float64)).astype(np.float32)
+        groups, experts = _brute_force(b32, 8, 4, 8)
+        assert {j for j in range(8) if (r.kept_mask[t] >> j) & 1} == groups
+        assert set(r.idx[t].tolist()) == experts
+        assert r.idx[t].tolist() == sorted(experts, key=lambda e: (-float(b32[e]), e))
+        sel = s[t, r.idx[t]]
+        np.testing.assert_allclose(r.w[t], sel / sel.sum(), rtol=1e-14)
+
+
+def test_route_from_logits_single_group_is_topk(oracle_lib):
+    """One group kept of one: a plain top-k of FP32(sigmoid(logit) + bias)."""
+    rng = np.random.default_rng(7)
+    logits = rng.standard_normal((50, 256)).astype(np.float32)
+    bias = rng.uniform(-0.1, 0.1, 256).astype(np.float32)
+    r = oracle_lib.route_logits(logits, bias, 1, 1, 8)
+    biased32 = (torch.sigmoid(torch.from_numpy(logits).double()) + torch.from_numpy(bias).double()).float()
+    vals, ref = torch.topk(biased32, 8, dim=1)
+    np.testing.assert_array_equal(biased32.gather(1, torch.from_numpy(r.idx).long()).numpy(), vals.numpy())
+
+
+def test_route_from_logits_bias_steers_selection_only(oracle_lib):
+    """Re-routing the same logits with a +10 bias on eight experts in four
+    groups forces exactly those experts; the weights stay the unbiased
+    sigmoid scores of the chosen experts, normalised."""
+    rng = np.random.default_rng(8)
+    logits = rng.standard_normal((30, 256)).astype(np.float32)
+    bias = np.zeros(256, np.float32)
+    forced = [3, 40, 41, 100, 101, 102, 250, 255]      # groups 0, 1, 3, 7 of 32 experts
+    bias[forced] = 10.0
+    r = oracle_lib.route_logits(logits, bias, 8, 4, 8)
+    s = expit(logits.astype(np.float64))
+    for t in range(30):
+        assert set(r.idx[t].tolist()) == set(forced)
+        assert r.kept_mask[t] == (1 << 0) | (1 << 1) | (1 << 3) | (1 << 7)
+        sel = s[t, r.idx[t]]
+        np.testing.assert_allclose(r.w[t], sel / sel.sum(), rtol=1e-14)
 
 
 # --------------------------------------------------------------------------
