@@ -24,7 +24,8 @@ BEAM_ERR_TIMEOUT = -5
 
 # every entry point declared in include/beam_moe.h
 SYMBOLS = (
-    "beam_moe_create", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_forward",
+    "beam_moe_create", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_route_logits",
+    "beam_moe_forward",
     "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_launch_plan",
     "beam_moe_get_status",
     "beam_moe_set_wait_limit", "beam_moe_set_gemm_tuning", "beam_moe_profile_begin",
@@ -54,6 +55,7 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_route.argtypes = [P, P, P, I, P, P]
         lib.beam_moe_router_logits.argtypes = [P, P, P, I, P]
         lib.beam_moe_route_static.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P]
+        lib.beam_moe_route_logits.argtypes = [P, P, P, I, P, P, P]
         lib.beam_moe_forward.argtypes = [P, P, P, I, P, P, I]
         lib.beam_moe_forward_host.argtypes = [P, P, P, I, P, P, I]
         lib.beam_moe_dispatch_info.argtypes = [P, P, I, P, P, P]
@@ -174,6 +176,24 @@ class BeamMoE:
             logits = torch.empty(T, self.n_experts, dtype=torch.float32, device=x.device)
         self._check(library().beam_moe_router_logits(self._h, _stream(stream), _ptr(x), T, _ptr(logits)))
         return logits
+
+    def route_logits(self, logits: torch.Tensor, expert_bias: Optional[torch.Tensor] = None,
+                     idx: Optional[torch.Tensor] = None, w: Optional[torch.Tensor] = None,
+                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+        """Routing from given FP32 logits [T, E], under `expert_bias` (fp32 [E])
+        or the handle's bias."""
+        _dev(logits, torch.float32, "logits")
+        if expert_bias is not None:
+            _dev(expert_bias, torch.float32, "expert_bias")
+        T = logits.shape[0]
+        if idx is None:
+            idx = torch.empty(T, self.top_k, dtype=torch.int32, device=logits.device)
+        if w is None:
+            w = torch.empty(T, self.top_k, dtype=torch.float32, device=logits.device)
+        self._check(library().beam_moe_route_logits(
+            self._h, _stream(stream), _ptr(logits), T,
+            None if expert_bias is None else _ptr(expert_bias), _ptr(idx), _ptr(w)))
+        return idx, w
 
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
                 residual: Optional[torch.Tensor] = None, k: int = 1, want_out: bool = True,

@@ -587,6 +587,40 @@ int beam_moe_router_logits(beam_moe_t h, void *stream, const void *x, int T, flo
     return run_router(h, static_cast<cudaStream_t>(stream), x, T, h->idx, h->w, logits);
 }
 
+int beam_moe_route_logits(beam_moe_t h, void *stream, const float *logits, int T,
+                          const float *expert_bias, int32_t *topk_idx, float *topk_w)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    h->err[0] = 0;
+    if (T < 0 || T > h->max_tokens)
+        return fail(h, BEAM_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->max_tokens);
+    if (T == 0) return BEAM_OK;
+    if (!logits || !topk_idx || !topk_w)
+        return fail(h, BEAM_ERR_INVALID_ARG, "logits, topk_idx and topk_w must be non-NULL");
+    if (!aligned16(logits) || (expert_bias && !aligned16(expert_bias)))
+        return fail(h, BEAM_ERR_INVALID_ARG, "logits / expert_bias must be 16-byte aligned");
+    int rc = check_device(h);
+    if (rc != BEAM_OK) return rc;
+    // the selection kernel over one K slice that already holds the logits
+    RouterArgs a;
+    a.x = nullptr;
+    a.router_w = nullptr;
+    a.bias = expert_bias ? expert_bias : h->bias;
+    a.T = T;
+    a.H = h->H;
+    a.E = h->E;
+    a.n_group = h->n_group;
+    a.topk_group = h->topk_group;
+    a.top_k = h->top_k;
+    a.nslice = 1;
+    a.partial = const_cast<float *>(logits);   // read only by the selection
+    a.idx = topk_idx;
+    a.w = topk_w;
+    a.logits_out = nullptr;
+    cudaError_t e = launch_router_select(a, SelectExtra(), 0, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "selection launch");
+}
+
 int beam_moe_forward(beam_moe_t h, void *stream, const void *x, int T, void *out,
                      float *residual, int k)
 {
@@ -599,7 +633,6 @@ int beam_moe_forward(beam_moe_t h, void *stream, const void *x, int T, void *out
     if ((out && !aligned16(out)) || (residual && !aligned16(residual)))
         return fail(h, BEAM_ERR_INVALID_ARG, "out / residual must be 16-byte aligned");
     if (residual && k < 1) return fail(h, BEAM_ERR_INVALID_ARG, "residual step k must be >= 1");
-    if (T == 0) return BEAM_OK;
     if ((rc = check_device(h)) != BEAM_OK) return rc;
     return run_forward(h, static_cast<cudaStream_t>(stream), x, T, out, residual, k);
 }

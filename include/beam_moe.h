@@ -149,6 +149,20 @@ int beam_moe_route_static(void *stream, const void *x, int T, int hidden, int n_
 int beam_moe_router_logits(beam_moe_t h, void *stream, const void *x, int T, float *logits);
 
 /*
+ * Routing of T tokens from given FP32 logits [T, E] (device, 16-byte
+ * aligned; e.g. from beam_moe_router_logits), with `expert_bias` (fp32 [E],
+ * device, 16-byte aligned) in place of the handle's bias, or the handle's
+ * bias when NULL.  The expert bias steers selection only (launch blog
+ * "Introducing Beam", section "Mixture of Experts"; transformers page
+ * "Beam", "Sparse MoE" bullet), so the effect of a new bias on the routing
+ * and the expert loads needs no new logits.  Outputs as beam_moe_route.
+ * Reads nothing of x or the router matrix; T <= max_tokens; T == 0 returns
+ * BEAM_OK.  Asynchronous on `stream`.
+ */
+int beam_moe_route_logits(beam_moe_t h, void *stream, const float *logits, int T,
+                          const float *expert_bias, int32_t *topk_idx, float *topk_w);
+
+/*
  * Forward pass of the block for T tokens.
  * x         bf16 [T, H].
  * out       bf16 [T, H] (out): routed_scaling * sum_j w_j * expert_j(x),

@@ -19,7 +19,7 @@ from group_limited_routing_sigmoid_b200 import workloads as W
 from group_limited_routing_sigmoid_b200.binding import BeamMoE, BeamMoEError, BEAM_ERR_TIMEOUT
 from group_limited_routing_sigmoid_b200.build import build
 
-from parity import check_block
+from parity import NEAR_TIE, W_ABS, check_block
 
 pytestmark = pytest.mark.gpu
 
@@ -180,6 +180,34 @@ def test_tensor_core_routing_matches_oracle(mode):
             f.write(json.dumps({"case": f"tc_routing_mode{mode}", "tokens": T, "exempt": int((~keep).sum()),
                                 "idx_mismatch": mism, "w_max_err": werr, "rederived": rederived}) + "\n")
     assert mism == 0 and werr <= W_ABS, (mism, werr)
+    moe.close()
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 1000), ("decode", 512)])
+def test_reroute_from_logits_under_a_new_bias(name, T):
+    """Routing from the router's FP32 logits: with the handle's bias it
+    matches beam_moe_route; under another bias it matches the oracle's
+    selection from the same logits, index for index (near-ties exempt)."""
+    wl = W.WORKLOADS[name]
+    if name == "decode":
+        wl = dataclasses.replace(wl, inter=128)   # routing does not depend on the experts' size
+    d = _inputs(wl, T)
+    moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    moe.set_gemm_tuning(router_mode=0)             # CUDA-core logits for both calls
+    logits = moe.router_logits(d["x"])
+    idx0, w0 = moe.route(d["x"])
+    idx1, w1 = moe.route_logits(logits)
+    np.testing.assert_array_equal(idx1.cpu().numpy(), idx0.cpu().numpy())
+    torch.testing.assert_close(w1, w0, rtol=0, atol=0)
+    g = torch.Generator().manual_seed(11)
+    bias2 = (torch.rand(wl.n_experts, generator=g) * 0.4 - 0.2).float()
+    idx2, w2 = moe.route_logits(logits, bias2.cuda())
+    r = oracle.route_logits(logits.cpu().numpy(), bias2.numpy(), wl.n_group, wl.topk_group, wl.top_k)
+    keep = (r.gap_expert >= NEAR_TIE) & (r.gap_group >= NEAR_TIE) & (r.gap_order >= NEAR_TIE)
+    np.testing.assert_array_equal(idx2.cpu().numpy()[keep], r.idx[keep])
+    assert np.abs(w2.cpu().numpy()[keep] - r.w[keep]).max() <= W_ABS
+    assert keep.mean() > 0.99
+    assert (idx2.cpu().numpy() != idx0.cpu().numpy()).any()   # the new bias moved some tokens
     moe.close()
 
 
