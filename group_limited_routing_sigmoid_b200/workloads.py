@@ -84,6 +84,18 @@ WORKLOADS: Dict[str, Workload] = {
     # ~256 tokens per expert as in the 8192-token prefill
     "prefill_small": Workload("prefill_small", T=1024, hidden=5120, n_experts=32, n_group=8,
                               topk_group=4, top_k=8, inter=2560, bias_lo=-0.01, bias_hi=0.01),
+    # dense SwiGLU MLP layers (the first three layers): one expert that every
+    # token takes with weight 1, no routing and no routed scaling.  The pages
+    # do not give the layers' intermediate size; 20480 (= 8 x 2560, the
+    # routed width a token sees in a MoE layer) fits the pages' parameter
+    # counts.  The router weight and bias are drawn (draw order) but unused.
+    # (dense_tiny: K long enough for split-K slices of at least 8 steps)
+    "dense_tiny": Workload("dense_tiny", T=64, hidden=1024, n_experts=1, n_group=1, topk_group=1,
+                           top_k=1, inter=2048, routed_scaling=1.0),
+    "dense_decode": Workload("dense_decode", T=64, hidden=5120, n_experts=1, n_group=1,
+                             topk_group=1, top_k=1, inter=20480, routed_scaling=1.0),
+    "dense_prefill": Workload("dense_prefill", T=8192, hidden=5120, n_experts=1, n_group=1,
+                              topk_group=1, top_k=1, inter=20480, routed_scaling=1.0, sample=256),
 }
 
 

@@ -278,6 +278,27 @@ def moe_block(x_bits: np.ndarray, router_w: np.ndarray, bias: np.ndarray,
     return res
 
 
+def dense_block(x_bits: np.ndarray, w_gate_bits: np.ndarray, w_up_bits: np.ndarray,
+                w_down_bits: np.ndarray, gamma: Optional[np.ndarray] = None, eps: float = 1e-6,
+                stream: Optional[np.ndarray] = None, kstep: int = 0) -> BlockResult:
+    """A dense SwiGLU MLP layer (the blog's first three layers) on the tokens
+    in ``x_bits``: the one-expert SwiGLU, its output rounded to bf16, and the
+    same optional post-norm and residual update as the sparse block.  It
+    composes the steps above with one slot of weight 1 and no scaling; no
+    routing."""
+    x = _u16(x_bits)
+    T = x.shape[0]
+    y = expert_swiglu(x, w_gate_bits, w_up_bits, w_down_bits)
+    o, out = combine(y.reshape(T, 1, -1), np.ones((T, 1)), 1.0)
+    empty = np.empty((T, 0))
+    routing = Routing(np.zeros((T, 1), np.int32), np.ones((T, 1)), empty, empty,
+                      np.full(T, np.inf), np.full(T, np.inf), np.ones(T, np.int32), np.full(T, np.inf))
+    res = BlockResult(routing, y.reshape(T, 1, -1), o, out)
+    if stream is not None:
+        res.contrib, res.stream_out = post_norm_residual(o, gamma, eps, kstep, stream)
+    return res
+
+
 def dense_fetch(w_gate_bits: np.ndarray, w_up_bits: np.ndarray, w_down_bits: np.ndarray) -> ExpertFetch:
     """fetch_expert over in-memory [E, ...] weight arrays."""
     return lambda e: (np.ascontiguousarray(w_gate_bits[e]), np.ascontiguousarray(w_up_bits[e]),

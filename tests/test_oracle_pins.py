@@ -299,6 +299,29 @@ def test_identical_experts_closed_form(oracle_lib):
     assert len(set(res.routing.idx.reshape(-1).tolist())) > 8  # the routing really varies
 
 
+def test_dense_layer_vs_torch(oracle_lib):
+    """The dense SwiGLU layer (one expert, weight 1, no scaling) against the
+    textbook formula written with numpy matmuls, the SwiGLU product rounded
+    to FP32 then bf16; and its residual update against the closed form with
+    the post-norm."""
+    wl = W.WORKLOADS["dense_tiny"]
+    d = W.make_inputs(wl, "cpu")
+    x = W.bf16_bits(d["x"][:16])
+    wg, wu, wd = (W.bf16_bits(d[k][0]) for k in ("w_gate", "w_up", "w_down"))
+    xf = oracle_lib.bf16_to_f64(x)
+    g = xf @ oracle_lib.bf16_to_f64(wg).T
+    u = xf @ oracle_lib.bf16_to_f64(wu).T
+    h = W.bf16_bits(torch.from_numpy((_silu(g) * u).astype(np.float32)).to(torch.bfloat16))
+    y = oracle_lib.bf16_to_f64(h) @ oracle_lib.bf16_to_f64(wd).T
+    gamma = (1.0 + 0.02 * np.random.default_rng(3).standard_normal(wl.hidden)).astype(np.float32)
+    stream = np.random.default_rng(4).standard_normal((16, wl.hidden)).astype(np.float32)
+    res = oracle_lib.dense_block(x, wg, wu, wd, gamma=gamma, eps=1e-6, stream=stream, kstep=20)
+    np.testing.assert_allclose(res.o, y, rtol=1e-10, atol=1e-14)
+    n = y / np.sqrt((y * y).mean(axis=1, keepdims=True) + 1e-6) * gamma.astype(np.float64)
+    np.testing.assert_allclose(res.stream_out, math.sqrt(19 / 20) * stream.astype(np.float64) + n / math.sqrt(20),
+                               rtol=1e-10, atol=1e-12)
+
+
 def test_permutation_experts_closed_form(oracle_lib):
     """Expert e = (a_e P_e, b_e Q_e, c_e R_e) with permutation matrices and
     power-of-two scales.  Then g_i = a_e x[p_e(i)], u_i = b_e x[q_e(i)],
