@@ -34,7 +34,8 @@ sys.path.insert(0, ROOT)
 from group_limited_routing_sigmoid_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (Beam shape, bf16) and % of HBM / tensor-core roofline"
-KERNELS_PER_FORWARD = 8     # logits, select, count, scan, permute, gate|up, down, combine
+# workloads whose dominant kernel streams weights (roofline against HBM)
+HBM_BOUND = ("decode", "tiny", "decode_small", "dense_decode", "dense_tiny")
 TOKEN_BATCHES = 8           # distinct token batches cycled through the steps
 
 
@@ -153,6 +154,19 @@ def max_over_ranks(value: float, dist, device) -> float:
     return float(t.item())
 
 
+def kernels_per_forward(plan: dict, dense: bool, residual: bool) -> int:
+    """Kernels of this library one forward pass launches, from its launch plan."""
+    if dense:
+        # table set-up, gate|up (+ SwiGLU over split-K partials), down, combine
+        # (needed for split-K partials or the residual update)
+        return (1 + 1 + (plan["ksplit_gate_up"] > 1) + 1
+                + (plan["ksplit_down"] > 1 or residual))
+    # router: logits + selection (CUDA cores) or tensor-core logits, selection,
+    # exact re-derivation, selection of the re-derived tokens; dispatch:
+    # count, scan, permute or row maps; the two GEMMs; combine
+    return (4 if plan["router_tensor_cores"] else 2) + 3 + 2 + 1
+
+
 def whole_job_tokens_per_s(world: int, steps: int, T: int, ms_max: float) -> float:
     """All ranks' tokens over the slowest rank's device time."""
     return world * steps * T / (ms_max * 1e-3)
@@ -195,9 +209,14 @@ def run_ours(args):
     outs = [torch.empty(T, H, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     streams = [b["stream"] for b in batches]
 
-    # distinct experts each batch touches (for the algorithmic byte count)
+    # distinct experts each batch touches (for the algorithmic byte count);
+    # a dense layer is one expert that every token takes
+    dense = E == 1
     distinct = []
     for b in batches:
+        if dense:
+            distinct.append(1)
+            continue
         idx, _ = moe.route(b["x"])
         distinct.append(int((torch.bincount(idx.reshape(-1).long(), minlength=E) > 0).sum()))
     torch.cuda.synchronize(dev)
@@ -265,7 +284,7 @@ def run_ours(args):
     d_mean = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(steps_done)) / steps_done
     P = T * k
     gate_up_ms = stage_ms["gate_up_gemm"] / max(calls, 1)
-    if args.workload in ("decode", "tiny", "decode_small"):
+    if args.workload in HBM_BOUND:
         alg_bytes = d_mean * 2 * I * H * 2 + P * H * 2 + P * I * 2
         achieved = alg_bytes / (gate_up_ms * 1e-3) / 1e9
         roof = {"bound": "hbm",
@@ -280,11 +299,16 @@ def run_ours(args):
                 "frac": round(achieved / pk["bf16_sus"], 4), "peak_source": pk["source"] + " sustained",
                 "algorithmic_flops_per_launch": flops, "launch_ms": round(gate_up_ms, 4)}
     plan = moe.launch_plan(T)
-    roof["kernel"] = ("gate_up_gemm (grouped_gemm_pair_kernel<%d,2,0>, CTA pairs, grid %d)"
-                      if plan["cta_pairs"] else
-                      "gate_up_gemm (grouped_gemm_kernel<%d,2,0>, grid %d)") % (plan["tile_rows"], plan["grid"])
+    if plan["ksplit_gate_up"] > 1:
+        roof["kernel"] = ("gate_up_gemm (grouped_gemm_kernel<%d,2,2>, split-K %d, + dense_swiglu_kernel)"
+                          % (plan["tile_rows"], plan["ksplit_gate_up"]))
+    else:
+        roof["kernel"] = ("gate_up_gemm (grouped_gemm_pair_kernel<%d,2,0>, CTA pairs, grid %d)"
+                          if plan["cta_pairs"] else
+                          "gate_up_gemm (grouped_gemm_kernel<%d,2,0>, grid %d)") % (plan["tile_rows"], plan["grid"])
     roof["traffic"] = ncu_traffic(args.workload)
-    step_bytes = d_mean * 3 * H * I * 2 + E * H * 4 + T * H * 4 + (T * H * 8 if wl.residual_k else 0)
+    step_bytes = (d_mean * 3 * H * I * 2 + (0 if dense else E * H * 4) + T * H * 4
+                  + (T * H * 8 if wl.residual_k else 0))
     stage_avg = {kname: round(v / max(calls, 1), 4) for kname, v in stage_ms.items()}
 
     line = {
@@ -314,7 +338,7 @@ def run_ours(args):
         "e2e": {"value": round(whole_job_tokens_per_s(ws, e2e_steps, T, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0),
                 "d2h_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0)},
-        "gpu_launches": KERNELS_PER_FORWARD * steps_done,
+        "gpu_launches": kernels_per_forward(plan, dense, bool(wl.residual_k)) * steps_done,
         "roofline": roof,
         "launch_plan": plan,
     }
@@ -335,6 +359,14 @@ def _oracle_on_tokens(wl, weights, x, n_tokens):
     import oracle
     oracle.build()
     xs = W.bf16_bits(x[:n_tokens])
+    gamma = None if weights.get("gamma") is None else weights["gamma"].cpu().numpy()
+    stream = torch.zeros(n_tokens, wl.hidden).numpy() if wl.residual_k else None
+    if wl.n_experts == 1:   # a dense layer: no routing
+        wg, wu, wd = (W.bf16_bits(weights[k][0]) for k in ("w_gate", "w_up", "w_down"))
+        t0 = time.perf_counter()
+        oracle.dense_block(xs, wg, wu, wd, gamma=gamma, eps=wl.norm_eps, stream=stream,
+                           kstep=wl.residual_k)
+        return time.perf_counter() - t0
     rw = weights["router_w"].cpu().numpy()
     bias = weights["bias"].cpu().numpy()
     r = oracle.route(xs, rw, bias, wl.n_group, wl.topk_group, wl.top_k)
@@ -342,10 +374,6 @@ def _oracle_on_tokens(wl, weights, x, n_tokens):
     for e in sorted(set(int(v) for v in r.idx.reshape(-1))):
         cache[e] = (W.bf16_bits(weights["w_gate"][e]), W.bf16_bits(weights["w_up"][e]),
                     W.bf16_bits(weights["w_down"][e]))
-    gamma = None if weights.get("gamma") is None else weights["gamma"].cpu().numpy()
-    stream = None
-    if wl.residual_k:
-        stream = torch.zeros(n_tokens, wl.hidden).numpy()
     t0 = time.perf_counter()
     oracle.moe_block(xs, rw, bias, cache.__getitem__, wl.n_group, wl.topk_group, wl.top_k,
                      wl.routed_scaling, gamma=gamma, eps=wl.norm_eps, stream=stream, kstep=wl.residual_k)

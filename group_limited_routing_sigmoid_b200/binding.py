@@ -24,7 +24,7 @@ BEAM_ERR_TIMEOUT = -5
 
 # every entry point declared in include/beam_moe.h
 SYMBOLS = (
-    "beam_moe_create", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_route_logits",
+    "beam_moe_create", "beam_moe_create_dense", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_route_logits",
     "beam_moe_forward",
     "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_launch_plan",
     "beam_moe_get_status",
@@ -55,6 +55,7 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_route.argtypes = [P, P, P, I, P, P]
         lib.beam_moe_router_logits.argtypes = [P, P, P, I, P]
         lib.beam_moe_route_static.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P]
+        lib.beam_moe_create_dense.argtypes = [P, I, I, P, P, P, P, ctypes.c_float, I]
         lib.beam_moe_route_logits.argtypes = [P, P, P, I, P, P, P]
         lib.beam_moe_forward.argtypes = [P, P, P, I, P, P, I]
         lib.beam_moe_forward_host.argtypes = [P, P, P, I, P, P, I]
@@ -148,7 +149,35 @@ class BeamMoE:
         self._h = h
 
     @classmethod
+    def dense(cls, hidden: int, inter: int, w_gate: torch.Tensor, w_up: torch.Tensor,
+              w_down: torch.Tensor, post_norm_w: Optional[torch.Tensor] = None,
+              norm_eps: float = 1e-6, max_tokens: int = 64) -> "BeamMoE":
+        """A dense SwiGLU MLP layer (beam_moe_create_dense): forward only."""
+        lib = library()
+        for n, t in (("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down)):
+            _dev(t, torch.bfloat16, n)
+        if post_norm_w is not None:
+            _dev(post_norm_w, torch.float32, "post_norm_w")
+        self = cls.__new__(cls)
+        self._keep = (w_gate, w_up, w_down, post_norm_w)
+        self.hidden, self.n_experts, self.inter, self.top_k = hidden, 1, inter, 1
+        self.max_tokens = max_tokens
+        self.device = w_gate.device
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            rc = lib.beam_moe_create_dense(ctypes.byref(h), hidden, inter, _ptr(w_gate), _ptr(w_up),
+                                           _ptr(w_down), _ptr(post_norm_w), float(norm_eps), max_tokens)
+        if rc != BEAM_OK:
+            raise BeamMoEError(rc, lib.beam_moe_create_error().decode())
+        self._h = h
+        return self
+
+    @classmethod
     def from_workload(cls, wl, weights, max_tokens: Optional[int] = None) -> "BeamMoE":
+        if wl.n_experts == 1:
+            return cls.dense(wl.hidden, wl.inter, weights["w_gate"][0], weights["w_up"][0],
+                             weights["w_down"][0], weights.get("gamma"), wl.norm_eps,
+                             max_tokens or wl.T)
         return cls(wl.hidden, wl.n_experts, wl.inter, wl.n_group, wl.topk_group, wl.top_k,
                    wl.routed_scaling, weights["router_w"], weights["bias"], weights["w_gate"],
                    weights["w_up"], weights["w_down"], weights.get("gamma"), wl.norm_eps,
@@ -235,10 +264,10 @@ class BeamMoE:
 
     def launch_plan(self, T: int) -> dict:
         """The kernels and launch shapes a forward pass of T tokens uses."""
-        p = (ctypes.c_int32 * 7)()
+        p = (ctypes.c_int32 * 9)()
         self._check(library().beam_moe_launch_plan(self._h, int(T), ctypes.cast(p, ctypes.c_void_p)))
         keys = ("tile_rows", "cta_pairs", "grid", "down_paired", "router_tensor_cores", "router_slices",
-                "gather_rows")
+                "gather_rows", "ksplit_gate_up", "ksplit_down")
         return dict(zip(keys, (int(v) for v in p)))
 
     def get_status(self, stream=None) -> int:

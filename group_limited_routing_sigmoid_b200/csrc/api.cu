@@ -26,7 +26,9 @@ struct beam_moe {
 
     void *ws;
     size_t ws_bytes;
+    int dense;               // 1: dense SwiGLU MLP (one expert, no router)
     float *partial;          // [nslice_max * T_max * E]
+    float *split;            // dense layers: FP32 split-K partial sums
     int32_t *idx;            // [P]
     float *w;                // [P]
     int32_t *block_cnt, *block_base, *rank, *counts, *offsets, *tile_off, *pair_row, *row_pair;
@@ -43,7 +45,10 @@ struct beam_moe {
     int router_mode;                 // -1: auto, 0: FP32 SIMT, 1: tensor cores, 2: 1 + every token re-derived
     int *fix_list;                   // [max_tokens] tokens re-derived on the exact path
     int *fix_count;
-    BoxMaps tm_xp, tm_h;             // box rows 16, 32, 64, 128, 256
+    BoxMaps tm_xp, tm_h;             // box rows 8, 16, 32, 64, 128, 256
+    BoxMaps tm_x;                    // dense layers: boxes of the caller's x ...
+    const void *tm_x_ptr;            // ... for this pointer and token count
+    int tm_x_T;
     int tile_rows;                   // 0: chosen from T
     int down_pair;                   // -1: auto, 0: single tiles, 1: paired tiles
     int use_pair;                    // 1: CTA-pair kernels for large token tiles (default)
@@ -246,12 +251,59 @@ struct ForwardPlan {
     int router_tc;     // 1: tensor-core logits with exact re-derivation
     int router_slices; // K slices of the router logits
     int gather;        // 1: gate|up gathers token rows from x; no sorted copy
+    int ksplit_gate_up;   // dense layers: K slices of the gate|up GEMM (1: fused SwiGLU)
+    int ksplit_down;      // dense layers: K slices of the down GEMM
 };
+
+// Split-K slices for a GEMM of `items` work items and KB K steps: the fewest
+// slices (dividing KB, at least 8 steps each) that give three work items per
+// SM, or the most such slices when none does; 1 when the items suffice.
+int split_for(long long items, int KB, int num_sms)
+{
+    int best = 1;
+    for (int d = 1; d <= KB / 8; ++d) {
+        if (KB % d) continue;
+        best = d;
+        if (items * d >= 3LL * num_sms) break;
+    }
+    return best;
+}
+
+// Dense layers: K slices of the gate|up and down GEMMs for T tokens in tiles
+// of BN rows (none above 64 rows: there the token tiles give work enough).
+void dense_splits(const beam_moe *h, int T, int BN, int *s_gate_up, int *s_down)
+{
+    *s_gate_up = *s_down = 1;
+    if (BN > 64) return;
+    const long long tiles = (T + BN - 1) / BN;
+    *s_gate_up = split_for(tiles * (h->I / 128), h->H / 64, h->num_sms);
+    *s_down = split_for(tiles * (h->H / 128), h->I / 64, h->num_sms);
+}
+
+// FP32 partial sums the split GEMMs of T tokens in BN-row tiles write.
+size_t dense_split_floats(const beam_moe *h, int T, int BN)
+{
+    int a, b;
+    dense_splits(h, T, BN, &a, &b);
+    size_t n = 0;
+    if (a > 1) n = (size_t)a * T * 2 * h->I;
+    if (b > 1 && (size_t)b * T * h->H > n) n = (size_t)b * T * h->H;
+    return n;
+}
+
+// Dense layers: the smallest power-of-two token tile (16..256) that holds T.
+int dense_tile_rows(int T)
+{
+    int bn = 16;
+    while (bn < T && bn < 256) bn <<= 1;
+    return bn;
+}
 
 ForwardPlan plan_forward(const beam_moe *h, int T)
 {
     ForwardPlan p;
-    p.tile_rows = h->tile_rows ? h->tile_rows : choose_tile_rows(T, h->top_k, h->E);
+    p.tile_rows = h->tile_rows ? h->tile_rows
+                               : (h->dense ? dense_tile_rows(T) : choose_tile_rows(T, h->top_k, h->E));
     // CTA pairs (cta_group::2) for large token tiles when the weight rows
     // split into 256-row blocks; single CTAs otherwise
     p.cta_pairs = h->use_pair != 0 && gemm_pair_supported(p.tile_rows) && h->I % 256 == 0 &&
@@ -274,15 +326,145 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
     // large token tiles the gathers of a stage outlast its MMAs.  Automatic
     // only for tiles of up to 32 rows, where the weight stream sets the pace.
     p.gather = h->gather_rows < 0 ? (p.tile_rows <= 32 ? 1 : 0) : h->gather_rows;
+    p.ksplit_gate_up = 1;
+    p.ksplit_down = 1;
+    if (h->dense) {
+        // one expert: with decode-sized T the weight tiles alone give too few
+        // work items, so K is split and FP32 partial sums are reduced after
+        p.gather = 0;
+        p.router_tc = 0;
+        p.router_slices = 0;
+        dense_splits(h, T, p.tile_rows, &p.ksplit_gate_up, &p.ksplit_down);
+        return p;
+    }
     p.router_tc = router_on_tensor_cores(h, T);
     p.router_slices = p.router_tc ? router_mma_slices(T, h->H, h->E, h->num_sms)
                                   : router_slices(T, h->H, h->E, h->num_sms);
     return p;
 }
 
+void finish_profile(beam_moe *h, cudaStream_t s, int T)
+{
+    prof_mark(h, s, 5);
+    if (h->prof_calls < h->prof_max) ++h->prof_calls;
+    h->last_T = T;
+}
+
+// The dense SwiGLU MLP: the grouped GEMMs over one expert of T rows that
+// reads x directly; split-K partial sums when the plan asks for them; the
+// combine only where something is left to do (split partials to sum, or
+// the post-norm and residual update).  Stage marks as the sparse block's,
+// with empty router and a table set-up in place of the dispatch.
+int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *out,
+                      float *residual, int k)
+{
+    prof_mark(h, s, 0);
+    prof_mark(h, s, 1);
+    const ForwardPlan plan = plan_forward(h, T);
+    const int BN = plan.tile_rows;
+    const int tiles = (T + BN - 1) / BN;
+    cudaError_t e = launch_dense_setup(T, tiles, h->counts, h->offsets, h->tile_off, h->pair_row,
+                                       h->row_pair, h->w, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "dense set-up launch");
+    prof_mark(h, s, 2);
+    if (h->tm_x_ptr != x || h->tm_x_T != T) {
+        for (int i = 0; i < 6; ++i)
+            if (!make_map(&h->tm_x.m[i], x, (uint64_t)T, (uint64_t)h->H, 8u << i)) {
+                h->tm_x_ptr = nullptr;
+                return fail(h, BEAM_ERR_CUDA, "tensor map of x");
+            }
+        h->tm_x_ptr = x;
+        h->tm_x_T = T;
+    }
+    GemmArgs g;
+    g.E = 1;
+    g.counts = h->counts;
+    g.offsets = h->offsets;
+    g.tile_off = h->tile_off;
+    g.row_pair = h->row_pair;
+    g.top_k = 1;
+    g.gather = 0;
+    g.ctl.status = h->status;
+    g.ctl.limit_ns = h->wait_limit_ns;
+    const int grid1 = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
+
+    g.K = h->H;
+    g.R = h->I;
+    if (plan.ksplit_gate_up > 1) {
+        g.ksplit = plan.ksplit_gate_up;
+        g.out = nullptr;
+        g.out_f32 = h->split;
+        g.slice_stride = (long long)T * 2 * h->I;
+        e = launch_grouped_gemm(GemmKind::kGateUpF32, BN, h->tm_gate, h->tm_up, h->tm_x, g, grid1, s);
+        if (e == cudaSuccess)
+            e = launch_dense_swiglu(h->split, g.ksplit, g.slice_stride, T, h->I, h->hbuf, s);
+    } else {
+        g.ksplit = 1;
+        g.out = h->hbuf;
+        g.out_f32 = nullptr;
+        g.slice_stride = 0;
+        e = plan.cta_pairs
+                ? launch_grouped_gemm_pair(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_x, g,
+                                           plan.grid, s)
+                : launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_x, g,
+                                      plan.grid, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(h, e, "gate/up GEMM launch");
+    prof_mark(h, s, 3);
+
+    g.K = h->I;
+    g.R = h->H;
+    if (plan.ksplit_down > 1) {
+        g.ksplit = plan.ksplit_down;
+        g.out = nullptr;
+        g.out_f32 = h->split;
+        g.slice_stride = (long long)T * h->H;
+        e = launch_grouped_gemm(GemmKind::kDownF32, BN, h->tm_down, h->tm_down, h->tm_h, g, grid1, s);
+    } else {
+        // without a residual the down projection's bf16 rows are the output
+        g.ksplit = 1;
+        g.out = residual ? h->ybuf : static_cast<__nv_bfloat16 *>(out);
+        g.out_f32 = nullptr;
+        g.slice_stride = 0;
+        const GemmKind dk = plan.down_paired ? GemmKind::kDownPaired : GemmKind::kDown;
+        e = plan.cta_pairs ? launch_grouped_gemm_pair(dk, BN, h->tm_down, h->tm_down, h->tm_h, g,
+                                                      plan.grid, s)
+                           : launch_grouped_gemm(dk, BN, h->tm_down, h->tm_down, h->tm_h, g,
+                                                 plan.grid, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(h, e, "down GEMM launch");
+    prof_mark(h, s, 4);
+
+    if (plan.ksplit_down > 1 || residual) {
+        CombineArgs c;
+        c.y = h->ybuf;
+        c.y_f32 = plan.ksplit_down > 1 ? h->split : nullptr;
+        c.nslice = plan.ksplit_down;
+        c.slice_stride = (long long)T * h->H;
+        c.pair_row = h->pair_row;
+        c.w = h->w;
+        c.T = T;
+        c.H = h->H;
+        c.top_k = 1;
+        c.scaling = 1.0f;
+        c.out = static_cast<__nv_bfloat16 *>(out);
+        c.residual = residual;
+        c.gamma = residual ? h->gamma : nullptr;
+        c.eps = h->eps;
+        const int kk = k >= 1 ? k : 1;
+        c.keep = (float)std::sqrt((double)(kk - 1) / (double)kk);
+        c.add = (float)(1.0 / std::sqrt((double)kk));
+        e = launch_combine(c, s);
+        if (e != cudaSuccess) return cuda_fail(h, e, "combine launch");
+    }
+    finish_profile(h, s, T);
+    return BEAM_OK;
+}
+
 int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, float *residual,
                 int k)
 {
+    if (h->dense) return run_forward_dense(h, s, x, T, out, residual, k);
     prof_mark(h, s, 0);
     int rc = run_router(h, s, x, T, h->idx, h->w, nullptr);
     if (rc != BEAM_OK) return rc;
@@ -321,6 +503,9 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.row_pair = h->row_pair;
     g.top_k = h->top_k;
     g.gather = plan.gather;
+    g.ksplit = 1;
+    g.out_f32 = nullptr;
+    g.slice_stride = 0;
     // token rows of the gate|up GEMM: x itself, four rows per gather4 copy,
     // or boxes of the sorted copy
     BoxMaps bx_local;
@@ -354,6 +539,9 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
 
     CombineArgs c;
     c.y = h->ybuf;
+    c.y_f32 = nullptr;
+    c.nslice = 0;
+    c.slice_stride = 0;
     c.pair_row = h->pair_row;
     c.w = h->w;
     c.T = T;
@@ -369,9 +557,7 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     c.add = (float)(1.0 / std::sqrt((double)kk));
     e = launch_combine(c, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "combine launch");
-    prof_mark(h, s, 5);
-    if (h->prof_calls < h->prof_max) ++h->prof_calls;
-    h->last_T = T;
+    finish_profile(h, s, T);
     return BEAM_OK;
 }
 
@@ -381,6 +567,141 @@ int check_tokens(beam_moe *h, const void *x, int T)
         return fail(h, BEAM_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->max_tokens);
     if (T > 0 && (!x || !aligned16(x)))
         return fail(h, BEAM_ERR_INVALID_ARG, "x must be a non-NULL 16-byte aligned device pointer");
+    return BEAM_OK;
+}
+
+// Device set-up common to both handle kinds: workspace, kernel attributes,
+// the router weight's bf16 pieces (sparse blocks) and the tensor maps.
+int finish_create(beam_moe *h, beam_moe_t *out)
+{
+    const int hidden = h->H, inter = h->I, n_experts = h->E, top_k = h->top_k;
+    const int max_tokens = h->max_tokens;
+    h->wait_limit_ns = 2000000000LL;
+    h->down_pair = -1;
+    h->use_pair = 1;
+    h->gather_rows = -1;
+    h->router_mode = -1;
+
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+    if (e != cudaSuccess) {
+        int rc = cuda_fail(nullptr, e, "device query");
+        delete h;
+        return rc;
+    }
+
+    // Workspace
+    const size_t T = (size_t)max_tokens, E = (size_t)n_experts, P = T * top_k;
+    const size_t nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
+    // router partial sums: the largest nslice(t) * t over t <= max_tokens, for
+    // either router path; dense layers: the largest split-K partial sums
+    size_t partial_rows = 0, split_floats = 0;
+    for (int t = 1; t <= max_tokens; ++t) {
+        if (h->dense) {   // every token tile a tuning may ask for
+            for (int bn = 16; bn <= 64; bn <<= 1) {
+                const size_t n = dense_split_floats(h, t, bn);
+                if (n > split_floats) split_floats = n;
+            }
+            continue;
+        }
+        const size_t r1 = (size_t)router_slices(t, hidden, n_experts, h->num_sms) * t;
+        const size_t r2 = (size_t)router_mma_slices(t, hidden, n_experts, h->num_sms) * t;
+        if (r1 > partial_rows) partial_rows = r1;
+        if (r2 > partial_rows) partial_rows = r2;
+    }
+    size_t off = 0;
+    auto carve = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    const size_t o_partial = carve(partial_rows * E * 4);
+    const size_t o_split = carve(split_floats * 4);
+    const size_t o_idx = carve(P * 4);
+    const size_t o_w = carve(P * 4);
+    const size_t o_bcnt = carve(nblk * E * 4);
+    const size_t o_bbase = carve(nblk * E * 4);
+    const size_t o_rank = carve(P * 4);
+    const size_t o_counts = carve(E * 4);
+    const size_t o_offsets = carve((E + 1) * 4);
+    const size_t o_tile = carve((E + 1) * 4);
+    const size_t o_prow = carve(P * 4);
+    const size_t o_rpair = carve(P * 4);
+    const size_t o_xp = carve(h->dense ? 0 : P * hidden * 2);   // dense: the GEMM reads x
+    const size_t o_h = carve(P * inter * 2);
+    const size_t o_y = carve(P * hidden * 2);
+    const size_t o_status = carve(256);
+    const size_t o_xs = carve(T * hidden * 2);
+    const size_t o_os = carve(T * hidden * 2);
+    const size_t o_rs = carve(T * hidden * 4);
+    const size_t o_wcat = carve(h->dense ? 0 : E * 3 * (size_t)hidden * 2);
+    const size_t o_fix = carve((T + 1) * 4);
+    h->ws_bytes = off;
+    e = cudaMalloc(&h->ws, h->ws_bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        int rc = fail(nullptr, BEAM_ERR_OOM, "workspace of %zu bytes: %s", h->ws_bytes,
+                      cudaGetErrorString(e));
+        delete h;
+        return rc;
+    }
+    char *b = static_cast<char *>(h->ws);
+    h->partial = reinterpret_cast<float *>(b + o_partial);
+    h->split = reinterpret_cast<float *>(b + o_split);
+    h->idx = reinterpret_cast<int32_t *>(b + o_idx);
+    h->w = reinterpret_cast<float *>(b + o_w);
+    h->block_cnt = reinterpret_cast<int32_t *>(b + o_bcnt);
+    h->block_base = reinterpret_cast<int32_t *>(b + o_bbase);
+    h->rank = reinterpret_cast<int32_t *>(b + o_rank);
+    h->counts = reinterpret_cast<int32_t *>(b + o_counts);
+    h->offsets = reinterpret_cast<int32_t *>(b + o_offsets);
+    h->tile_off = reinterpret_cast<int32_t *>(b + o_tile);
+    h->pair_row = reinterpret_cast<int32_t *>(b + o_prow);
+    h->row_pair = reinterpret_cast<int32_t *>(b + o_rpair);
+    h->xp = reinterpret_cast<__nv_bfloat16 *>(b + o_xp);
+    h->hbuf = reinterpret_cast<__nv_bfloat16 *>(b + o_h);
+    h->ybuf = reinterpret_cast<__nv_bfloat16 *>(b + o_y);
+    h->status = reinterpret_cast<int *>(b + o_status);
+    h->x_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_xs);
+    h->out_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_os);
+    h->res_stage = reinterpret_cast<float *>(b + o_rs);
+    h->wcat = reinterpret_cast<__nv_bfloat16 *>(b + o_wcat);
+    h->fix_count = reinterpret_cast<int *>(b + o_fix);
+    h->fix_list = h->fix_count + 1;
+    e = cudaMemset(h->fix_count, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
+    if (e == cudaSuccess) e = prepare_grouped_gemm(n_experts);
+    if (e == cudaSuccess) e = prepare_dispatch(n_experts);
+    if (!h->dense) {
+        if (e == cudaSuccess) e = prepare_router_mma();
+        if (e == cudaSuccess) e = prepare_router_fix(hidden);
+        // the router weight's bf16 pieces for the tensor-core router (the
+        // weight is borrowed and must not change while the handle lives)
+        if (e == cudaSuccess) e = launch_router_split(h->router_w, n_experts, hidden, h->wcat, 0);
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(0);
+    if (e != cudaSuccess) {
+        int rc = cuda_fail(nullptr, e, "workspace / kernel set-up");
+        cudaFree(h->ws);
+        delete h;
+        return rc;
+    }
+
+    bool ok = make_map(&h->tm_gate, h->w_gate, E * inter, hidden, 128) &&
+              make_map(&h->tm_up, h->w_up, E * inter, hidden, 128) &&
+              make_map(&h->tm_down, h->w_down, E * hidden, inter, 128);
+    if (!h->dense) ok = ok && make_map(&h->tm_wcat, h->wcat, E, 3 * (uint64_t)hidden, 128);
+    for (int i = 0; i < 6 && ok; ++i) {
+        ok = make_map(&h->tm_h.m[i], h->hbuf, P, inter, 8u << i);
+        if (ok && !h->dense) ok = make_map(&h->tm_xp.m[i], h->xp, P, hidden, 8u << i);
+    }
+    if (!ok) {
+        cudaFree(h->ws);
+        delete h;
+        return fail(nullptr, BEAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    }
+    *out = h;
     return BEAM_OK;
 }
 
@@ -445,127 +766,53 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     h->w_down = static_cast<const __nv_bfloat16 *>(w_down);
     h->eps = norm_eps;
     h->max_tokens = max_tokens;
-    h->wait_limit_ns = 2000000000LL;
-    h->down_pair = -1;
-    h->use_pair = 1;
-    h->gather_rows = -1;
-    h->router_mode = -1;
+    return finish_create(h, out);
+}
 
-    cudaError_t e = cudaGetDevice(&h->device);
-    if (e == cudaSuccess)
-        e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
-    if (e != cudaSuccess) {
-        int rc = cuda_fail(nullptr, e, "device query");
-        delete h;
-        return rc;
-    }
+int beam_moe_create_dense(beam_moe_t *out, int hidden, int inter, const void *w_gate,
+                          const void *w_up, const void *w_down, const float *post_norm_w,
+                          float norm_eps, int max_tokens)
+{
+    g_create_err[0] = 0;
+    if (!out) return fail(nullptr, BEAM_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (hidden <= 0 || inter <= 0 || max_tokens < 1)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "sizes must be positive");
+    if (!(norm_eps >= 0.f)) return fail(nullptr, BEAM_ERR_INVALID_ARG, "norm_eps not valid");
+    if (!w_gate || !w_up || !w_down)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "weight pointer is NULL");
+    if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+        (post_norm_w && !aligned16(post_norm_w)))
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "weight pointers must be 16-byte aligned");
+    if (hidden % 128 != 0 || inter % 128 != 0)
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "hidden and inter must be multiples of 128");
+    if (hidden > 8192) return fail(nullptr, BEAM_ERR_UNSUPPORTED, "hidden > 8192");
+    if ((long long)max_tokens > (1LL << 30))
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "max_tokens too large");
 
-    // Workspace
-    const size_t T = (size_t)max_tokens, E = (size_t)n_experts, P = T * top_k;
-    const size_t nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
-    // router partial sums: the largest nslice(t) * t over t <= max_tokens, for
-    // either router path
-    size_t partial_rows = 0;
-    for (int t = 1; t <= max_tokens; ++t) {
-        const size_t r1 = (size_t)router_slices(t, hidden, n_experts, h->num_sms) * t;
-        const size_t r2 = (size_t)router_mma_slices(t, hidden, n_experts, h->num_sms) * t;
-        if (r1 > partial_rows) partial_rows = r1;
-        if (r2 > partial_rows) partial_rows = r2;
-    }
-    size_t off = 0;
-    auto carve = [&](size_t bytes) {
-        size_t o = off;
-        off = align_up(off + bytes, 256);
-        return o;
-    };
-    const size_t o_partial = carve(partial_rows * E * 4);
-    const size_t o_idx = carve(P * 4);
-    const size_t o_w = carve(P * 4);
-    const size_t o_bcnt = carve(nblk * E * 4);
-    const size_t o_bbase = carve(nblk * E * 4);
-    const size_t o_rank = carve(P * 4);
-    const size_t o_counts = carve(E * 4);
-    const size_t o_offsets = carve((E + 1) * 4);
-    const size_t o_tile = carve((E + 1) * 4);
-    const size_t o_prow = carve(P * 4);
-    const size_t o_rpair = carve(P * 4);
-    const size_t o_xp = carve(P * hidden * 2);
-    const size_t o_h = carve(P * inter * 2);
-    const size_t o_y = carve(P * hidden * 2);
-    const size_t o_status = carve(256);
-    const size_t o_xs = carve(T * hidden * 2);
-    const size_t o_os = carve(T * hidden * 2);
-    const size_t o_rs = carve(T * hidden * 4);
-    const size_t o_wcat = carve(E * 3 * (size_t)hidden * 2);
-    const size_t o_fix = carve((T + 1) * 4);
-    h->ws_bytes = off;
-    e = cudaMalloc(&h->ws, h->ws_bytes);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        int rc = fail(nullptr, BEAM_ERR_OOM, "workspace of %zu bytes: %s", h->ws_bytes,
-                      cudaGetErrorString(e));
-        delete h;
-        return rc;
-    }
-    char *b = static_cast<char *>(h->ws);
-    h->partial = reinterpret_cast<float *>(b + o_partial);
-    h->idx = reinterpret_cast<int32_t *>(b + o_idx);
-    h->w = reinterpret_cast<float *>(b + o_w);
-    h->block_cnt = reinterpret_cast<int32_t *>(b + o_bcnt);
-    h->block_base = reinterpret_cast<int32_t *>(b + o_bbase);
-    h->rank = reinterpret_cast<int32_t *>(b + o_rank);
-    h->counts = reinterpret_cast<int32_t *>(b + o_counts);
-    h->offsets = reinterpret_cast<int32_t *>(b + o_offsets);
-    h->tile_off = reinterpret_cast<int32_t *>(b + o_tile);
-    h->pair_row = reinterpret_cast<int32_t *>(b + o_prow);
-    h->row_pair = reinterpret_cast<int32_t *>(b + o_rpair);
-    h->xp = reinterpret_cast<__nv_bfloat16 *>(b + o_xp);
-    h->hbuf = reinterpret_cast<__nv_bfloat16 *>(b + o_h);
-    h->ybuf = reinterpret_cast<__nv_bfloat16 *>(b + o_y);
-    h->status = reinterpret_cast<int *>(b + o_status);
-    h->x_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_xs);
-    h->out_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_os);
-    h->res_stage = reinterpret_cast<float *>(b + o_rs);
-    h->wcat = reinterpret_cast<__nv_bfloat16 *>(b + o_wcat);
-    h->fix_count = reinterpret_cast<int *>(b + o_fix);
-    h->fix_list = h->fix_count + 1;
-    e = cudaMemset(h->fix_count, 0, sizeof(int));
-    e = cudaMemset(h->status, 0, sizeof(int));
-    if (e == cudaSuccess) e = prepare_grouped_gemm(n_experts);
-    if (e == cudaSuccess) e = prepare_dispatch(n_experts);
-    if (e == cudaSuccess) e = prepare_router_mma();
-    if (e == cudaSuccess) e = prepare_router_fix(hidden);
-    // the router weight's bf16 pieces for the tensor-core router (the weight
-    // is borrowed and must not change while the handle lives)
-    if (e == cudaSuccess) e = launch_router_split(router_w, n_experts, hidden, h->wcat, 0);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(0);
-    if (e != cudaSuccess) {
-        int rc = cuda_fail(nullptr, e, "workspace / kernel set-up");
-        cudaFree(h->ws);
-        delete h;
-        return rc;
-    }
-
-    bool ok = make_map(&h->tm_wcat, h->wcat, E, 3 * (uint64_t)hidden, 128) &&
-              make_map(&h->tm_gate, w_gate, E * inter, hidden, 128) &&
-              make_map(&h->tm_up, w_up, E * inter, hidden, 128) &&
-              make_map(&h->tm_down, w_down, E * hidden, inter, 128);
-    for (int i = 0; i < 6 && ok; ++i)
-        ok = make_map(&h->tm_xp.m[i], h->xp, P, hidden, 8u << i) &&
-             make_map(&h->tm_h.m[i], h->hbuf, P, inter, 8u << i);
-    if (!ok) {
-        cudaFree(h->ws);
-        delete h;
-        return fail(nullptr, BEAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-    }
-    *out = h;
-    return BEAM_OK;
+    beam_moe *h = new beam_moe();
+    h->dense = 1;
+    h->H = hidden;
+    h->E = 1;
+    h->I = inter;
+    h->n_group = 1;
+    h->topk_group = 1;
+    h->top_k = 1;
+    h->scaling = 1.0f;
+    h->gamma = post_norm_w;
+    h->w_gate = static_cast<const __nv_bfloat16 *>(w_gate);
+    h->w_up = static_cast<const __nv_bfloat16 *>(w_up);
+    h->w_down = static_cast<const __nv_bfloat16 *>(w_down);
+    h->eps = norm_eps;
+    h->max_tokens = max_tokens;
+    return finish_create(h, out);
 }
 
 int beam_moe_route(beam_moe_t h, void *stream, const void *x, int T, int32_t *topk_idx,
                    float *topk_w)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
+    if (h->dense) return fail(h, BEAM_ERR_UNSUPPORTED, "a dense layer has no router");
     h->err[0] = 0;
     int rc = check_tokens(h, x, T);
     if (rc != BEAM_OK) return rc;
@@ -578,6 +825,7 @@ int beam_moe_route(beam_moe_t h, void *stream, const void *x, int T, int32_t *to
 int beam_moe_router_logits(beam_moe_t h, void *stream, const void *x, int T, float *logits)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
+    if (h->dense) return fail(h, BEAM_ERR_UNSUPPORTED, "a dense layer has no router");
     h->err[0] = 0;
     int rc = check_tokens(h, x, T);
     if (rc != BEAM_OK) return rc;
@@ -591,6 +839,7 @@ int beam_moe_route_logits(beam_moe_t h, void *stream, const float *logits, int T
                           const float *expert_bias, int32_t *topk_idx, float *topk_w)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
+    if (h->dense) return fail(h, BEAM_ERR_UNSUPPORTED, "a dense layer has no router");
     h->err[0] = 0;
     if (T < 0 || T > h->max_tokens)
         return fail(h, BEAM_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->max_tokens);
@@ -715,6 +964,8 @@ int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host)
     plan_host[4] = p.router_tc;
     plan_host[5] = p.router_slices;
     plan_host[6] = p.gather;
+    plan_host[7] = p.ksplit_gate_up;
+    plan_host[8] = p.ksplit_down;
     return BEAM_OK;
 }
 

@@ -2,6 +2,7 @@
 // depth-scaled residual update fused in.
 //
 //   o[t]   = routed_scaling * sum_j w[t,j] * y[row(t,j)]     (bf16 y, fp32 sum, slot order)
+//            (dense layer: o[t] = sum_s y_s[t] over FP32 split-K slices, in slice order)
 //   out[t] = bf16_rn(o[t])
 //   n[t]   = o[t] / sqrt(mean(o[t]^2) + eps) * gamma          (if gamma)
 //   stream[t] <- sqrt((k-1)/k) * stream[t] + n[t] / sqrt(k)
@@ -24,7 +25,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a)
     const int nvec = a.H / 4;
     int rows[32];
     float wts[32];
-    for (int j = 0; j < a.top_k; ++j) {
+    const int nsum = a.y_f32 ? 0 : a.top_k;   // expert slots (none for FP32 slices)
+    for (int j = 0; j < nsum; ++j) {
         rows[j] = a.pair_row[(size_t)t * a.top_k + j];
         wts[j] = a.w[(size_t)t * a.top_k + j];
     }
@@ -35,7 +37,17 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a)
         const int i = tid + v * kCombThreads;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (i < nvec) {
-            for (int j = 0; j < a.top_k; ++j) {
+            if (a.y_f32) {
+                for (int sl = 0; sl < a.nslice; ++sl) {
+                    const float4 y = reinterpret_cast<const float4 *>(
+                        a.y_f32 + (size_t)sl * (size_t)a.slice_stride + (size_t)t * a.H)[i];
+                    acc.x += y.x;
+                    acc.y += y.y;
+                    acc.z += y.z;
+                    acc.w += y.w;
+                }
+            }
+            for (int j = 0; j < nsum; ++j) {
                 const uint2 raw = reinterpret_cast<const uint2 *>(a.y + (size_t)rows[j] * a.H)[i];
                 const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
                 const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));

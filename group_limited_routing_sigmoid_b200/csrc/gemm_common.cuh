@@ -17,7 +17,13 @@ constexpr int kStagingWarpBytes = 2048;                // one 32-row x CH-column
 constexpr int kStagingBytes = kEpiWarps * kStagingWarpBytes;
 constexpr int kStageBudget = kMaxDynSmem - 1024 - kBarrierBytes - kTableBytes - kStagingBytes;
 
-enum Epi { kSwiGLU = 0, kStoreBF16 = 1 };   // gate|up with SwiGLU; plain (down)
+// Epilogues: gate|up with SwiGLU; plain bf16 (down); FP32 partial sums of a
+// K slice, gate and up side by side (kGateUpF32) or one matrix (kStoreF32).
+enum Epi { kSwiGLU = 0, kStoreBF16 = 1, kGateUpF32 = 2, kStoreF32 = 3 };
+
+// Whether the second A tile holds the same weight rows of a second matrix
+// (gate|up) rather than the next 128 rows of the same one (paired down).
+constexpr bool same_rows(int epi) { return epi == kSwiGLU || epi == kGateUpF32; }
 
 constexpr int pow2_at_least(int v, int lo)
 {
@@ -140,6 +146,27 @@ __device__ __forceinline__ void epilogue_block(uint32_t taddr, int nrows, int ro
             }
         }
         __syncwarp();
+    }
+}
+
+// FP32 partial sums of one accumulator (32 TMEM lanes of this warp,
+// `nrows` columns): TMEM lane l is output column l of the warp's 32, TMEM
+// column j is token row j, so each store instruction of the warp writes one
+// row's 32 consecutive floats (128 bytes).  Chunks of 16 columns alternate
+// between the two warps of a quadrant.
+//   out:   this warp's first output column in token row 0
+//   ldo:   output row stride in elements
+__device__ __forceinline__ void epilogue_f32(uint32_t taddr, int nrows, int row0, int half, int lane,
+                                             float *out, int ldo)
+{
+#pragma unroll 1
+    for (int c0 = half * 16; c0 < nrows; c0 += 32) {
+        uint32_t v[16];
+        tmem_ld16(taddr + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (c0 + j < nrows) out[(size_t)(row0 + c0 + j) * ldo + lane] = __uint_as_float(v[j]);
     }
 }
 

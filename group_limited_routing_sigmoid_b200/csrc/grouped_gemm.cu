@@ -57,7 +57,8 @@ struct Cfg {
     static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
     static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS, 32);
     static constexpr int CH = BN >= 32 ? 32 : 16;           // epilogue columns per chunk
-    static constexpr int ROWS_PER_ITEM = EPI == kSwiGLU ? kBM : NUM_A * kBM;
+    static constexpr int ROWS_PER_ITEM = same_rows(EPI) ? kBM : NUM_A * kBM;
+    static constexpr bool F32 = EPI == kGateUpF32 || EPI == kStoreF32;   // split-K partials
     static constexpr int SMEM_BYTES =
         1024 + STAGES * STAGE_BYTES + kStagingBytes + kBarrierBytes + kTableBytes;
     static_assert(STAGES >= 2, "pipeline needs two stages");
@@ -65,7 +66,8 @@ struct Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
     static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of the next tile");
     static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory");
-    static_assert(EPI == kStoreBF16 || NUM_A == 2, "SwiGLU needs the gate and up tiles");
+    static_assert(!same_rows(EPI) || NUM_A == 2, "gate|up needs the gate and up tiles");
+    static_assert(!F32 || (EPI == kStoreF32 ? NUM_A == 1 : true), "FP32 down: one tile");
     static_assert(32 * CH * 2 <= kStagingWarpBytes, "staging block");
 };
 
@@ -123,8 +125,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     const int WT = p.R / C::ROWS_PER_ITEM;
-    const int total = WT * s_tile[p.E];
-    const int KB = p.K / kBK;
+    const int S = C::F32 ? p.ksplit : 1;          // K slices per (weight tile, token tile)
+    const int total = WT * s_tile[p.E] * S;
+    const int KB = p.K / kBK / S;                 // K steps of one slice
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -140,13 +143,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         long long issued = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const Item it = decode_item(item / S, WT, p.E, s_counts, s_offsets, s_tile);
+            const int kb0 = (item % S) * KB;
             const int a_row = it.e * p.R + it.wt * C::ROWS_PER_ITEM;
             const int n_load = (it.nrows + 15) & ~15;
             const uint32_t bytes = NUM_A * C::A_BYTES + n_load * (kBK * 2);
             int tok[G][4];
             if (gather) gather_tokens<G>(p, it, 0, n_load >> 2, lane, tok);
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = kb0; kb < kb0 + KB; ++kb) {
                 bool got = true;
                 if (lane == 0 || gather) got = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl);
                 ok = __all_sync(0xffffffffu, got);
@@ -159,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(sa, &tmA0, kb * kBK, a_row, fb, pol_w);
                     if (NUM_A == 2) {
                         // gate|up: the up matrix at the same rows; down: the next 128 rows
-                        const int a_row1 = EPI == kSwiGLU ? a_row : a_row + kBM;
+                        const int a_row1 = same_rows(EPI) ? a_row : a_row + kBM;
                         tma_load_2d(sa + C::A_BYTES, &tmA1, kb * kBK, a_row1, fb, pol_w);
                     }
                     if (!gather) {
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool issued_any = false;
         int iter = 0;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++iter) {
-            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const Item it = decode_item(item / S, WT, p.E, s_counts, s_offsets, s_tile);
             const int n_mma = (it.nrows + 15) & ~15;
             const uint32_t idesc = umma_idesc_bf16_f32(kBM, n_mma);
             const int acc = iter % C::NBUF;
@@ -270,10 +274,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.ctl);
             if (!__all_sync(0xffffffffu, ok)) break;   // warp-uniform from here on
             tc_fence_after();
-            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const Item it = decode_item(item / S, WT, p.E, s_counts, s_offsets, s_tile);
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
-            if constexpr (EPI == kSwiGLU) {
+            if constexpr (C::F32) {
+                float *out = p.out_f32 + (size_t)(item % S) * (size_t)p.slice_stride;
+                const int col0 = it.wt * kBM + quad * 32;
+                if constexpr (EPI == kGateUpF32) {
+                    epilogue_f32(taddr, it.nrows, it.row0, half, lane, out + col0, 2 * p.R);
+                    epilogue_f32(taddr + BN, it.nrows, it.row0, half, lane, out + p.R + col0, 2 * p.R);
+                } else {
+                    epilogue_f32(taddr, it.nrows, it.row0, half, lane, out + col0, p.R);
+                }
+            } else if constexpr (EPI == kSwiGLU) {
                 const int col0 = it.wt * C::ROWS_PER_ITEM + quad * 32;
                 epilogue_block<EPI, C::CH, BN>(taddr, it.nrows, it.row0, half, lane, stg,
                                                p.out + col0, p.R);
@@ -332,6 +345,13 @@ cudaError_t launch_kind(GemmKind kind, const CUtensorMap &a0, const CUtensorMap 
             return launch<BN, 1, kStoreBF16>(a0, a1, b, args, grid, stream);
         case GemmKind::kDownPaired:
             return launch<BN, 2, kStoreBF16>(a0, a1, b, args, grid, stream);
+        case GemmKind::kGateUpF32:
+        case GemmKind::kDownF32:
+            if constexpr (BN <= 64) {
+                if (kind == GemmKind::kGateUpF32) return launch<BN, 2, kGateUpF32>(a0, a1, b, args, grid, stream);
+                return launch<BN, 1, kStoreF32>(a0, a1, b, args, grid, stream);
+            }
+            return cudaErrorInvalidValue;
     }
     return cudaErrorInvalidValue;
 }
@@ -350,12 +370,19 @@ cudaError_t prepare_grouped_gemm(int E)
     if ((err = set_smem<BN, 2, kSwiGLU>()) != cudaSuccess) return err;       \
     if ((err = set_smem<BN, 1, kStoreBF16>()) != cudaSuccess) return err;    \
     if ((err = set_smem<BN, 2, kStoreBF16>()) != cudaSuccess) return err;
+#define BEAM_PREP_F32(BN)                                                    \
+    if ((err = set_smem<BN, 2, kGateUpF32>()) != cudaSuccess) return err;    \
+    if ((err = set_smem<BN, 1, kStoreF32>()) != cudaSuccess) return err;
     BEAM_PREP(16)
     BEAM_PREP(32)
     BEAM_PREP(64)
     BEAM_PREP(128)
     BEAM_PREP(256)
+    BEAM_PREP_F32(16)
+    BEAM_PREP_F32(32)
+    BEAM_PREP_F32(64)
 #undef BEAM_PREP
+#undef BEAM_PREP_F32
     return prepare_grouped_gemm_pair();
 }
 

@@ -89,6 +89,12 @@ struct GemmArgs {
     const int32_t *row_pair;     // [P]
     int top_k;
     int gather;
+    // split-K (single-CTA kernel, FP32-partials kinds only): work item i takes
+    // K slice i % ksplit and writes its FP32 partial sums to
+    // out_f32 + slice * slice_stride
+    int ksplit;
+    float *out_f32;
+    long long slice_stride;
     WaitCtl ctl;
 };
 
@@ -103,7 +109,10 @@ struct BoxMaps {
 enum class GemmKind {
     kGateUp,       // gate and up tiles, SwiGLU epilogue, bf16 out
     kDown,         // one 128-row tile, bf16 out
-    kDownPaired    // two consecutive 128-row tiles sharing the token tile, bf16 out
+    kDownPaired,   // two consecutive 128-row tiles sharing the token tile, bf16 out
+    kGateUpF32,    // gate and up tiles, FP32 partial sums out ([slice][P][2R]: gate, then up);
+                   // single-CTA kernel, token tiles of up to 64 rows
+    kDownF32       // one 128-row tile, FP32 partial sums out ([slice][P][R]); as above
 };
 // BN: largest token tile (16..256, power of two).
 cudaError_t launch_grouped_gemm(GemmKind kind, int BN, const CUtensorMap &a0,
@@ -125,6 +134,12 @@ int gemm_pair_max_ctas();   // CTAs of the pair kernels that can be resident at 
 // ---------------------------------------------------------------- combine
 struct CombineArgs {
     const __nv_bfloat16 *y;      // [P, H] expert outputs
+    // instead of y (dense layer, top_k == 1, unit weight): FP32 partial sums
+    // of nslice split-K slices [nslice][T][H], slice_stride elements apart,
+    // summed in slice order
+    const float *y_f32;
+    int nslice;
+    long long slice_stride;
     const int32_t *pair_row;     // [P]
     const float *w;              // [T, top_k]
     int T, H, top_k;
@@ -136,6 +151,13 @@ struct CombineArgs {
     float keep, add;             // sqrt((k-1)/k), 1/sqrt(k)
 };
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream);
+
+// ------------------------------------------------------------- dense layer
+cudaError_t launch_dense_setup(int T, int tiles, int32_t *counts, int32_t *offsets,
+                               int32_t *tile_off, int32_t *pair_row, int32_t *row_pair, float *w,
+                               cudaStream_t stream);
+cudaError_t launch_dense_swiglu(const float *part, int S, long long slice_stride, int T, int I,
+                                __nv_bfloat16 *h, cudaStream_t stream);
 
 // ------------------------------------------------------------- self-check
 cudaError_t launch_wait_timeout_check(WaitCtl ctl, cudaStream_t stream);

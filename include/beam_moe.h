@@ -99,6 +99,29 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
                     int max_tokens);
 
 /*
+ * Create a handle for one dense SwiGLU MLP layer (Beam's first three layers;
+ * launch blog "Introducing Beam", section "Mixture of Experts"):
+ *   out = W_down . bf16(silu(W_gate . x) * (W_up . x))   (SwiGLU product in FP32)
+ * with the same optional post-norm and depth-scaled residual update as the
+ * sparse block, and no routing or routed scaling.
+ *
+ * hidden        H (Beam: 5120).  Multiple of 128, at most 8192.
+ * inter         intermediate size of the layer.  Multiple of 128.
+ * w_gate, w_up  bf16 [inter, H];  w_down  bf16 [H, inter].
+ * post_norm_w, norm_eps, max_tokens: as beam_moe_create.
+ * The handle takes beam_moe_forward, beam_moe_forward_host,
+ * beam_moe_launch_plan, beam_moe_set_gemm_tuning (tile_rows, ctas,
+ * cta_pairs and down_pair apply), the status, wait-limit and profiling
+ * calls, and beam_moe_destroy; the routing calls return
+ * BEAM_ERR_UNSUPPORTED.  Token tiles of up to 64 rows split the GEMMs' K
+ * range into slices whose FP32 partial sums are added in slice order.
+ * Allocates device memory; launches nothing.
+ */
+int beam_moe_create_dense(beam_moe_t *out, int hidden, int inter, const void *w_gate,
+                          const void *w_up, const void *w_down, const float *post_norm_w,
+                          float norm_eps, int max_tokens);
+
+/*
  * Route T tokens: the router step alone.
  * x         bf16 [T, H].
  * topk_idx  int32 [T, top_k] (out): chosen experts, in descending biased
@@ -212,13 +235,14 @@ int beam_moe_router_stats(beam_moe_t h, void *stream, int32_t *rederived_host);
 
 /*
  * The launch configuration a forward pass of T tokens (0 <= T <= max_tokens)
- * uses under the handle's current tuning, written to plan_host (int32 [7],
+ * uses under the handle's current tuning, written to plan_host (int32 [9],
  * host): {largest token tile of the grouped GEMMs (rows), 1 if
  * they run on CTA pairs (cta_group::2), CTAs per grouped GEMM, 1 if the down
  * projection takes two weight blocks per work item, 1 if the router logits
  * run on the tensor cores (with exact re-derivation of thin-margin tokens),
- * K slices of the router logits, 1 if the gate|up GEMM gathers token rows
- * from x}.  A function of T and the tuning only; launches nothing.
+ * K slices of the router logits (0 for a dense layer), 1 if the gate|up GEMM
+ * gathers token rows from x, K slices of the gate|up GEMM and of the down
+ * GEMM (dense layers; 1 = no split)}.  A function of T and the tuning only; launches nothing.
  * Returns BEAM_ERR_INVALID_ARG for a NULL pointer or T out of range.
  */
 int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host);

@@ -160,3 +160,45 @@ def check_block(wl: W.Workload, d: dict, moe, sample: Optional[torch.Tensor] = N
             delta = (s_out - keep_f * s_in)[keep]
             rep.res_rel_fro, rep.res_max_abs_over_rms = errors(delta, res.contrib[keep])
     return rep
+
+
+def check_dense(wl, d, moe, T: Optional[int] = None, sample: Optional[torch.Tensor] = None) -> Report:
+    """The dense SwiGLU layer (a handle from beam_moe_create_dense): run the
+    CUDA forward on d['x'][:T] and compare the sampled tokens with the oracle's
+    dense_block under the block's output tolerances (no routing to compare)."""
+    x = d["x"] if T is None else d["x"][:T]
+    T = x.shape[0]
+    dev = x.device
+    rep = Report()
+    stream_in = None
+    if wl.residual_k:
+        stream_in = d["stream"][:T].clone()
+        stream_dev = stream_in.clone()
+        out = moe.forward(x, residual=stream_dev, k=wl.residual_k)
+    else:
+        out = moe.forward(x)
+    torch.cuda.synchronize(dev)
+    assert moe.get_status() == 0, "device-side wait ran out"
+    if sample is None:
+        sample = torch.arange(T)
+    sample = sample[sample < T]
+    s_dev = sample.to(dev)
+    gamma = None if d.get("gamma") is None else d["gamma"].cpu().numpy()
+    t0 = time.time()
+    res = oracle.dense_block(W.bf16_bits(x.index_select(0, s_dev)), W.bf16_bits(d["w_gate"][0]),
+                             W.bf16_bits(d["w_up"][0]), W.bf16_bits(d["w_down"][0]), gamma=gamma,
+                             eps=wl.norm_eps,
+                             stream=None if stream_in is None else stream_in.index_select(0, s_dev).cpu().numpy(),
+                             kstep=wl.residual_k)
+    rep.oracle_seconds = time.time() - t0
+    rep.tokens = len(sample)
+    if out is not None:
+        got = bf16_to_f64(out.index_select(0, s_dev))
+        ref = oracle.bf16_to_f64(res.out)
+        rep.rel_fro, rep.max_abs_over_rms, rep.max_abs_over_rms_raw, rep.ulp_neighbours = bf16_errors(got, ref)
+    if stream_in is not None:
+        keep_f = math.sqrt((wl.residual_k - 1) / wl.residual_k)
+        s_out = stream_dev.index_select(0, s_dev).cpu().double().numpy()
+        s_in = stream_in.index_select(0, s_dev).cpu().double().numpy()
+        rep.res_rel_fro, rep.res_max_abs_over_rms = errors(s_out - keep_f * s_in, res.contrib)
+    return rep
