@@ -205,7 +205,8 @@ def run_ours(args):
     if wl.post_norm:
         weights["gamma"] = batches[0]["gamma"]
     moe = BeamMoE.from_workload(wl, weights)
-    moe.set_gemm_tuning(0, args.gemm_tile, args.down_pair, args.cta_pairs, args.router, args.gather)
+    moe.set_gemm_tuning(0, args.gemm_tile, args.down_pair, args.cta_pairs, args.router, args.gather,
+                        args.token_stages)
     outs = [torch.empty(T, H, dtype=torch.bfloat16, device=dev) for _ in range(2)]
     streams = [b["stream"] for b in batches]
 
@@ -445,6 +446,8 @@ def main():
     ap.add_argument("--gemm-tile", type=int, default=0, help="largest GEMM token tile (0 = auto)")
     ap.add_argument("--gather", type=int, default=-1,
                     help="gate|up token rows gathered from x: -1 auto (tiles <= 32 rows), 0 never, 1 always")
+    ap.add_argument("--token-stages", type=int, default=0,
+                    help="CTA-pair GEMMs: token-row ring depth (0 = default 3)")
     ap.add_argument("--down-pair", type=int, default=-1, help="paired down tiles: -1 auto, 0, 1")
     ap.add_argument("--cta-pairs", type=int, default=1, help="SM-pair GEMMs for large tiles: 1 or 0")
     ap.add_argument("--router", type=int, default=-1, help="router logits: -1 auto, 0 CUDA cores, 1 tensor cores")

@@ -64,7 +64,7 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_router_stats.argtypes = [P, P, P]
         lib.beam_moe_launch_plan.argtypes = [P, I, P]
         lib.beam_moe_set_wait_limit.argtypes = [P, ctypes.c_int64]
-        lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I, I, I, I]
+        lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I, I, I, I, I]
         lib.beam_moe_check_wait_timeout.argtypes = [P, P]
         lib.beam_moe_profile_begin.argtypes = [P, I]
         lib.beam_moe_profile_end.argtypes = [P, P, P]
@@ -277,10 +277,12 @@ class BeamMoE:
         self._check(library().beam_moe_set_wait_limit(self._h, int(limit_ns)))
 
     def set_gemm_tuning(self, ctas: int = 0, tile_rows: int = 0, down_pair: int = -1,
-                        cta_pairs: int = 1, router_mode: int = -1, gather_rows: int = -1):
+                        cta_pairs: int = 1, router_mode: int = -1, gather_rows: int = -1,
+                        token_stages: int = 0):
         self._check(library().beam_moe_set_gemm_tuning(self._h, int(ctas), int(tile_rows),
                                                         int(down_pair), int(cta_pairs),
-                                                        int(router_mode), int(gather_rows)))
+                                                        int(router_mode), int(gather_rows),
+                                                        int(token_stages)))
 
     STAGES = ("router", "dispatch", "gate_up_gemm", "down_gemm", "combine")
 

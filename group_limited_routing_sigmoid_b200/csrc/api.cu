@@ -53,6 +53,7 @@ struct beam_moe {
     int down_pair;                   // -1: auto, 0: single tiles, 1: paired tiles
     int use_pair;                    // 1: CTA-pair kernels for large token tiles (default)
     int gather_rows;                 // -1: auto (default), 0: never, 1: always
+    int token_stages;                // CTA-pair kernels: token-row ring depth (0: default)
     int last_T;
     std::vector<cudaEvent_t> prof_events;   // 6 per profiled forward pass
     int prof_max, prof_calls;
@@ -386,6 +387,8 @@ int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *o
     g.gather = 0;
     g.ctl.status = h->status;
     g.ctl.limit_ns = h->wait_limit_ns;
+    g.b_stages = h->token_stages;
+    g.a_stages = 0;
     const int grid1 = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
 
     g.K = h->H;
@@ -500,6 +503,8 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.tile_off = h->tile_off;
     g.ctl.status = h->status;
     g.ctl.limit_ns = h->wait_limit_ns;
+    g.b_stages = h->token_stages;
+    g.a_stages = 0;
     g.row_pair = h->row_pair;
     g.top_k = h->top_k;
     g.gather = plan.gather;
@@ -1044,7 +1049,7 @@ int beam_moe_profile_end(beam_moe_t h, float *stage_ms, int *calls)
 }
 
 int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair, int cta_pairs,
-                             int router_mode, int gather_rows)
+                             int router_mode, int gather_rows, int token_stages)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
     if (ctas < 0 || ctas > 65535) return fail(h, BEAM_ERR_INVALID_ARG, "ctas outside [0, 65535]");
@@ -1057,6 +1062,9 @@ int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pai
         return fail(h, BEAM_ERR_INVALID_ARG, "router_mode outside [-1, 2]");
     if (gather_rows < -1 || gather_rows > 1)
         return fail(h, BEAM_ERR_INVALID_ARG, "gather_rows outside [-1, 1]");
+    if (token_stages != 0 && (token_stages < 2 || token_stages > 8))
+        return fail(h, BEAM_ERR_INVALID_ARG, "token_stages must be 0 or in [2, 8]");
+    h->token_stages = token_stages;
     h->router_mode = router_mode;
     h->gather_rows = gather_rows;
     h->gemm_ctas = ctas;

@@ -7,18 +7,26 @@
 // of the pair holds weight rows r*128 .. r*128+127 (its half of the MMA's
 // M = 256) and token rows r*N/2 .. r*N/2+N/2-1 (its half of N); the MMA,
 // issued by CTA 0, reads both CTAs' shared memory and writes each CTA's TMEM
-// (128 lanes, its weight rows, all N token columns).  Per SM this halves the
-// token bytes of every stage, so more stages fit in shared memory and more
-// weight bytes are in flight for the same MMA work.
+// (128 lanes, its weight rows, all N token columns).
+//
+// Two rings.  The weight tiles stream from HBM with a loaded latency of a
+// few microseconds, the token rows come from L2 (an expert's token tile is
+// reused by all of its weight blocks) with about a third of that.  So the
+// weights get a ring of their own, as deep as shared memory allows, and the
+// token rows a shallow one; each has its own producer warp, so neither ring
+// waits on the other's slots.  With 256-token tiles this keeps 4 weight
+// stages (128 KB per SM) in flight instead of 3 in one shared ring.
 //
 // Synchronisation (every wait bounded):
-//   full[s]    in CTA 0: CTA 0's producer expects the bytes of both CTAs;
-//              both CTAs' TMA loads complete on it;
-//   empty[s]   in each CTA: the MMA's completion, multicast to both;
+//   fullA[s], fullB[s]  in CTA 0: CTA 0's producers expect the bytes of both
+//                       CTAs; both CTAs' TMA loads complete on them;
+//   emptyA[s], emptyB[s] in each CTA: the MMAs' completion, multicast to both;
 //   tfull[a]   in each CTA: accumulator ready, multicast to both;
 //   tempty[a]  in CTA 0: both CTAs' epilogue threads arrive;
 //   drain      in each CTA: all MMAs complete, before TMEM is released.
-// Only local TMA loads (no multicast).
+// Only local TMA loads (no multicast).  The expert tables are read from
+// global memory (a few hundred bytes, L1-resident), which leaves their
+// shared memory to the rings.
 #include "gemm_common.cuh"
 
 namespace beam {
@@ -27,35 +35,64 @@ using namespace gemm;
 
 namespace {
 
+constexpr int kPairThreads = kThreads + 32;     // + warp 10: token-row producer
+constexpr int kPairMaxStages = 16;              // barrier slots per ring
+constexpr int kPairBarrierBytes = 1024;
+constexpr int kPairRingBytes = kMaxDynSmem - 1024 - kPairBarrierBytes - kStagingBytes;
+constexpr int kPairDefaultBStages = 3;
+
 template <int BN, int NUM_A, int EPI>
 struct PairCfg {
     static constexpr int HALF = BN / 2;                    // token rows per CTA, at most
-    static constexpr int A_BYTES = kBM * kBK * 2;
-    static constexpr int B_BYTES = HALF * kBK * 2;
-    static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
-    static constexpr int STAGES_FIT = kStageBudget / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
+    static constexpr int A_BYTES = kBM * kBK * 2;          // one 128 x 64 weight tile
+    static constexpr int A_STAGE = NUM_A * A_BYTES;
+    static constexpr int B_STAGE = HALF * kBK * 2;
     static constexpr int ACC_COLS = NUM_A * BN;            // per CTA: 128 lanes x N per matrix
     static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
     static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS, 32);
     static constexpr int CH = 32;
     static constexpr int ROWS_PER_ITEM = 2 * kBM * (EPI == kSwiGLU ? 1 : NUM_A);
-    static constexpr int SMEM_BYTES =
-        1024 + STAGES * STAGE_BYTES + kStagingBytes + kBarrierBytes + kTableBytes;
-    static_assert(STAGES >= 2, "pipeline needs two stages");
+    static constexpr int SMEM_BYTES = kMaxDynSmem;
     static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair UMMA N");
-    static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of the next tile");
-    static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory");
+    static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0, "stages keep 1024-byte alignment");
+    static_assert(kPairRingBytes >= 2 * A_STAGE + 2 * B_STAGE, "two stages per ring");
     static_assert(EPI == kStoreBF16 || NUM_A == 2, "SwiGLU needs the gate and up tiles");
+    static_assert(4 * kPairMaxStages * 8 + 5 * 8 + 4 <= kPairBarrierBytes, "barrier block");
 };
 
 constexpr uint16_t kPairMask = 0x3;
 
+__device__ __forceinline__ void ring_next(int &s, uint32_t &ph, int n)
+{
+    if (++s == n) {
+        s = 0;
+        ph ^= 1u;
+    }
+}
+
+// Wait (time-bounded, status ignored) for the last min(issued, n) copies a
+// ring's producer issued to land, so that no copy is in flight when the CTA
+// leaves after a failed wait.  CTA 0's barriers count both CTAs' copies.
+__device__ __forceinline__ void drain_ring(uint64_t *full, int s, uint32_t ph, long long issued,
+                                           int n, long long limit_ns)
+{
+    const long long m = issued < n ? issued : n;
+    for (long long j = 0; j < m; ++j) {
+        if (s == 0) {
+            s = n - 1;
+            ph ^= 1u;
+        } else {
+            --s;
+        }
+        mbar_wait_drain(smem_u32(&full[s]), ph, limit_ns);
+    }
+}
+
 }  // namespace
 
 template <int BN, int NUM_A, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
                              const __grid_constant__ CUtensorMap tmA1,
                              const __grid_constant__ BoxMaps tmB, GemmArgs p)
@@ -65,17 +102,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t *base_ptr = smem_raw + (base - raw_addr);
-    uint8_t *staging = base_ptr + C::STAGES * C::STAGE_BYTES;
-    uint8_t *bar_ptr = staging + kStagingBytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(bar_ptr);
-    uint64_t *empty = full + C::STAGES;
-    uint64_t *tfull = empty + C::STAGES;
+    const int SA = p.a_stages, SB = p.b_stages;            // ring depths (host-checked)
+    const uint32_t ring_b = base + (uint32_t)(SA * C::A_STAGE);
+    uint8_t *staging = base_ptr + SA * C::A_STAGE + SB * C::B_STAGE;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(staging + kStagingBytes);
+    uint64_t *fullA = bars;
+    uint64_t *emptyA = fullA + kPairMaxStages;
+    uint64_t *fullB = emptyA + kPairMaxStages;
+    uint64_t *emptyB = fullB + kPairMaxStages;
+    uint64_t *tfull = emptyB + kPairMaxStages;
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
-    int *s_counts = reinterpret_cast<int *>(bar_ptr + kBarrierBytes);
-    int *s_offsets = s_counts + p.E;
-    int *s_tile = s_offsets + (p.E + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -83,11 +121,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
 
-    load_tables(p, s_counts, s_offsets, s_tile);
     if (warp == 0 && lane == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);
-            mbar_init(smem_u32(&empty[s]), 1);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(smem_u32(&fullA[s]), 1);
+            mbar_init(smem_u32(&emptyA[s]), 1);
+        }
+        for (int s = 0; s < SB; ++s) {
+            mbar_init(smem_u32(&fullB[s]), 1);
+            mbar_init(smem_u32(&emptyB[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
@@ -111,57 +152,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     const int WT = p.R / C::ROWS_PER_ITEM;
-    const int total = WT * s_tile[p.E];
+    const int total = WT * __ldg(&p.tile_off[p.E]);
     const int KB = p.K / kBK;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        // Lane 0 loads the weight tiles (and the token rows from the sorted
-        // buffer); with gathering, every lane also issues its gather4 copies
-        // of token rows straight from x.
-        const uint64_t pol_w = l2_policy_evict_first();
-        const uint64_t pol_x = l2_policy_evict_last();
+        if (lane == 0) {
+            // -------------------------------------------- weight producer
+            const uint64_t pol_w = l2_policy_evict_first();   // weights: streamed once
+            int sa = 0;
+            uint32_t pa = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int item = pair; item < total && ok; item += npairs) {
+                const Item it = decode_item(item, WT, p.E, p.counts, p.offsets, p.tile_off);
+                // A rows of this CTA: its 128-row half of each 256-row block
+                const int a_base = it.e * p.R + it.wt * C::ROWS_PER_ITEM + (int)rank * kBM;
+                // gate|up: the up matrix at the same rows; down: the next 256-row block
+                const int a_row1 = EPI == kSwiGLU ? a_base : a_base + 2 * kBM;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(smem_u32(&emptyA[sa]), pa ^ 1u, p.ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t dst = base + (uint32_t)(sa * C::A_STAGE);
+                    const uint32_t f_local = smem_u32(&fullA[sa]);
+                    const uint32_t f = mapa_shared(f_local, 0);   // CTA 0's barrier
+                    if (rank == 0) mbar_arrive_expect_tx(f_local, 2u * C::A_STAGE);
+                    tma_load_2d_pair(dst, &tmA0, kb * kBK, a_base, f, pol_w);
+                    if (NUM_A == 2) tma_load_2d_pair(dst + C::A_BYTES, &tmA1, kb * kBK, a_row1, f, pol_w);
+                    ++issued;
+                    ring_next(sa, pa, SA);
+                }
+            }
+            if (!ok && rank == 0) drain_ring(fullA, sa, pa, issued, SA, p.ctl.limit_ns);
+        }
+    } else if (warp == kPairThreads / 32 - 1) {
+        // ------------------------------------------------ token-row producer
+        // Lane 0 loads boxes of the sorted rows; with gathering every lane
+        // issues its gather4 copies of rows straight from x.
+        const uint64_t pol_x = l2_policy_evict_last();    // activations: reused across tiles
         constexpr int G = (C::HALF / 4 + 31) / 32;          // gather4 copies per lane, at most
         const bool gather = EPI == kSwiGLU && p.gather != 0;
-        int stage = 0;
-        uint32_t phase = 0;
+        int sb = 0;
+        uint32_t pb = 0;
         long long issued = 0;
         bool ok = true;
         for (int item = pair; item < total && ok; item += npairs) {
-            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const Item it = decode_item(item, WT, p.E, p.counts, p.offsets, p.tile_off);
             const int n_mma = (it.nrows + 15) & ~15;
             const int half = n_mma >> 1;                    // this CTA's token rows
             const int b_row = it.row0 + (int)rank * half;
-            // A rows of this CTA: its 128-row half of each 256-row block
-            const int a_base = it.e * p.R + it.wt * C::ROWS_PER_ITEM + (int)rank * kBM;
-            const uint32_t pair_bytes = 2u * (NUM_A * C::A_BYTES + half * (kBK * 2));
+            const uint32_t pair_bytes = 2u * (uint32_t)(half * (kBK * 2));
             int tok[G][4];
             if (gather) gather_tokens<G>(p, it, (int)rank * half, half >> 2, lane, tok);
             for (int kb = 0; kb < KB; ++kb) {
                 bool got = true;
-                if (lane == 0 || gather) got = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl);
+                if (lane == 0 || gather) got = mbar_wait(smem_u32(&emptyB[sb]), pb ^ 1u, p.ctl);
                 ok = __all_sync(0xffffffffu, got);
                 if (!ok) break;
-                const uint32_t sa = base + stage * C::STAGE_BYTES;
-                const uint32_t sb = sa + NUM_A * C::A_BYTES;
-                const uint32_t fb_local = smem_u32(&full[stage]);
-                const uint32_t fb = mapa_shared(fb_local, 0);   // CTA 0's barrier
+                const uint32_t dst = ring_b + (uint32_t)(sb * C::B_STAGE);
+                const uint32_t f_local = smem_u32(&fullB[sb]);
+                const uint32_t f = mapa_shared(f_local, 0);   // CTA 0's barrier
                 if (lane == 0) {
-                    if (rank == 0) mbar_arrive_expect_tx(fb_local, pair_bytes);
-                    tma_load_2d_pair(sa, &tmA0, kb * kBK, a_base, fb, pol_w);
-                    if (NUM_A == 2) {
-                        // gate|up: the up matrix at the same rows; down: the next 256-row block
-                        const int a_row1 = EPI == kSwiGLU ? a_base : a_base + 2 * kBM;
-                        tma_load_2d_pair(sa + C::A_BYTES, &tmA1, kb * kBK, a_row1, fb, pol_w);
-                    }
+                    if (rank == 0) mbar_arrive_expect_tx(f_local, pair_bytes);
                     if (!gather) {
                         int off = 0;
 #pragma unroll
                         for (int bi = 4; bi >= 0; --bi) {   // boxes of 128, 64, 32, 16, 8 rows
                             const int hgt = 8 << bi;
                             if (hgt <= C::HALF && half - off >= hgt) {
-                                tma_load_2d_pair(sb + off * (kBK * 2), &tmB.m[bi], kb * kBK,
-                                                 b_row + off, fb, pol_x);
+                                tma_load_2d_pair(dst + off * (kBK * 2), &tmB.m[bi], kb * kBK,
+                                                 b_row + off, f, pol_x);
                                 off += hgt;
                             }
                         }
@@ -172,42 +233,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int g = 0; g < G; ++g) {
                         const int op = lane + 32 * g;
                         if (op < (half >> 2))
-                            tma_gather4_pair(sb + op * (4 * kBK * 2), &tmB.gather, kb * kBK,
-                                             tok[g][0], tok[g][1], tok[g][2], tok[g][3], fb, pol_x);
+                            tma_gather4_pair(dst + op * (4 * kBK * 2), &tmB.gather, kb * kBK,
+                                             tok[g][0], tok[g][1], tok[g][2], tok[g][3], f, pol_x);
                     }
                 }
                 ++issued;
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                ring_next(sb, pb, SB);
             }
         }
-        if (!ok && lane == 0 && rank == 0) {
-            // Let both CTAs' copies in flight land (CTA 0's barrier counts
-            // both) before the pair leaves; time-bounded, status ignored.
-            long long n = issued < C::STAGES ? issued : C::STAGES;
-            int s = stage;
-            uint32_t ph = phase;
-            for (long long j = 0; j < n; ++j) {
-                if (s == 0) {
-                    s = C::STAGES - 1;
-                    ph ^= 1u;
-                } else {
-                    --s;
-                }
-                mbar_wait_drain(smem_u32(&full[s]), ph, p.ctl.limit_ns);
-            }
-        }
+        if (!ok && lane == 0 && rank == 0) drain_ring(fullB, sb, pb, issued, SB, p.ctl.limit_ns);
     } else if (warp == 1 && lane == 0 && rank == 0) {
         // ------------------------------------------------ UMMA issuer (CTA 0)
-        int stage = 0;
-        uint32_t phase = 0;
+        int sa = 0, sb = 0;
+        uint32_t pa = 0, pb = 0;
         bool ok = true;
         bool issued_any = false;
         int iter = 0;
         for (int item = pair; item < total && ok; item += npairs, ++iter) {
-            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const Item it = decode_item(item, WT, p.E, p.counts, p.offsets, p.tile_off);
             const int n_mma = (it.nrows + 15) & ~15;
             const uint32_t idesc = umma_idesc_bf16_f32(2 * kBM, n_mma);
             const int acc = iter % C::NBUF;
@@ -219,28 +262,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(smem_u32(&full[stage]), phase, p.ctl)) {
+                if (!mbar_wait(smem_u32(&fullA[sa]), pa, p.ctl) ||
+                    !mbar_wait(smem_u32(&fullB[sb]), pb, p.ctl)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sa = base + stage * C::STAGE_BYTES;
-                const uint32_t sb = sa + NUM_A * C::A_BYTES;
+                const uint32_t a_addr = base + (uint32_t)(sa * C::A_STAGE);
+                const uint32_t b_addr = ring_b + (uint32_t)(sb * C::B_STAGE);
 #pragma unroll
                 for (int k = 0; k < kBK / 16; ++k) {
-                    const uint64_t bdesc = umma_desc_sw128(sb + k * 32);
+                    const uint64_t bdesc = umma_desc_sw128(b_addr + k * 32);
                     const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-                    umma_bf16_pair(d0, umma_desc_sw128(sa + k * 32), bdesc, idesc, accum);
+                    umma_bf16_pair(d0, umma_desc_sw128(a_addr + k * 32), bdesc, idesc, accum);
                     if (NUM_A == 2)
-                        umma_bf16_pair(d0 + BN, umma_desc_sw128(sa + C::A_BYTES + k * 32), bdesc,
+                        umma_bf16_pair(d0 + BN, umma_desc_sw128(a_addr + C::A_BYTES + k * 32), bdesc,
                                        idesc, accum);
                     issued_any = true;
                 }
-                umma_commit_pair(smem_u32(&empty[stage]), kPairMask);
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                umma_commit_pair(smem_u32(&emptyA[sa]), kPairMask);
+                umma_commit_pair(smem_u32(&emptyB[sb]), kPairMask);
+                ring_next(sa, pa, SA);
+                ring_next(sb, pb, SB);
             }
             if (!ok) break;
             umma_commit_pair(smem_u32(&tfull[acc]), kPairMask);
@@ -260,7 +303,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const bool ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.ctl);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const Item it = decode_item(item, WT, p.E, p.counts, p.offsets, p.tile_off);
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
             if constexpr (EPI == kSwiGLU) {
@@ -314,8 +357,16 @@ template <int BN, int NUM_A, int EPI>
 cudaError_t launch_pair(const CUtensorMap &a0, const CUtensorMap &a1, const BoxMaps &b,
                         const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    grouped_gemm_pair_kernel<BN, NUM_A, EPI>
-        <<<grid, kThreads, PairCfg<BN, NUM_A, EPI>::SMEM_BYTES, stream>>>(a0, a1, b, args);
+    using C = PairCfg<BN, NUM_A, EPI>;
+    // ring depths: the token rows' ring as asked (default 3), the weights'
+    // ring as deep as the rest of shared memory allows
+    GemmArgs a = args;
+    a.b_stages = args.b_stages > 0 ? args.b_stages : kPairDefaultBStages;
+    if (a.b_stages < 2 || a.b_stages > kPairMaxStages) return cudaErrorInvalidValue;
+    a.a_stages = (kPairRingBytes - a.b_stages * C::B_STAGE) / C::A_STAGE;
+    if (a.a_stages > kPairMaxStages) a.a_stages = kPairMaxStages;
+    if (a.a_stages < 2) return cudaErrorInvalidValue;
+    grouped_gemm_pair_kernel<BN, NUM_A, EPI><<<grid, kPairThreads, C::SMEM_BYTES, stream>>>(a0, a1, b, a);
     return cudaGetLastError();
 }
 
@@ -354,7 +405,7 @@ cudaError_t prepare_grouped_gemm_pair()
     // of one GPC), so that the persistent grid is fully resident.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
     cfg.dynamicSmemBytes = PairCfg<256, 2, kSwiGLU>::SMEM_BYTES;
     cfg.numAttrs = 0;   // the cluster shape comes from the kernel's __cluster_dims__
     int clusters = 0;

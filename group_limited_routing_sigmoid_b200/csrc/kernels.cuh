@@ -95,6 +95,10 @@ struct GemmArgs {
     int ksplit;
     float *out_f32;
     long long slice_stride;
+    // CTA-pair kernel: depth of the token-row ring (0 = default); the weight
+    // ring's depth is derived at launch (a_stages)
+    int b_stages;
+    int a_stages;
     WaitCtl ctl;
 };
 

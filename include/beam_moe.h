@@ -295,9 +295,12 @@ int beam_moe_set_wait_limit(beam_moe_t h, int64_t limit_ns);
  *                 sorted buffer and the GEMM loads boxes of it; -1
  *                 (default): gather when token tiles are at most 32 rows
  *                 (the gathers of a large tile outlast its MMAs).
+ * token_stages    CTA-pair kernels: depth of the token-row ring, 2..8, or 0
+ *                 for the default (3); the weight ring takes the rest of
+ *                 shared memory.
  */
 int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair,
-                             int cta_pairs, int router_mode, int gather_rows);
+                             int cta_pairs, int router_mode, int gather_rows, int token_stages);
 
 /*
  * Per-stage timing of forward passes, for measurement.  After
