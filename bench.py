@@ -236,7 +236,6 @@ def run_ours(args):
 
     stream = torch.cuda.current_stream(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    moe.profile_begin(args.steps)
     sampler = ClockSampler(local)
     if ws > 1:
         dist.barrier()
@@ -250,11 +249,21 @@ def run_ours(args):
     if ws > 1:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
-    calls, stage_ms = moe.profile_end()
     rederived = moe.router_stats()
     if moe.get_status() != 0:
         raise SystemExit("a device-side wait ran out during the timed region")
     ms_max = max_over_ranks(ms, dist, dev)
+
+    # per-stage device times: the same steps again with the library's CUDA
+    # events around each stage (kept out of the headline region: an event
+    # between two kernels stops the second from starting early)
+    stage_steps = min(args.steps, 50)
+    moe.profile_begin(stage_steps)
+    for i in range(stage_steps):
+        step(args.warmup + i)
+    calls, stage_ms = moe.profile_end()
+    if moe.get_status() != 0:
+        raise SystemExit("a device-side wait ran out during the stage-timed steps")
 
     # end to end through the host-buffer entry point (pinned buffers)
     x_host = [b["x"].cpu().pin_memory() for b in batches]
@@ -282,7 +291,7 @@ def run_ours(args):
     # roofline of the dominant kernel
     pk = peaks()
     steps_done = args.steps
-    d_mean = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(steps_done)) / steps_done
+    d_mean = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(stage_steps)) / stage_steps
     P = T * k
     gate_up_ms = stage_ms["gate_up_gemm"] / max(calls, 1)
     if args.workload in HBM_BOUND:
@@ -308,7 +317,8 @@ def run_ours(args):
                           if plan["cta_pairs"] else
                           "gate_up_gemm (grouped_gemm_kernel<%d,2,0>, grid %d)") % (plan["tile_rows"], plan["grid"])
     roof["traffic"] = ncu_traffic(args.workload)
-    step_bytes = (d_mean * 3 * H * I * 2 + (0 if dense else E * H * 4) + T * H * 4
+    d_steps = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(steps_done)) / steps_done
+    step_bytes = (d_steps * 3 * H * I * 2 + (0 if dense else E * H * 4) + T * H * 4
                   + (T * H * 8 if wl.residual_k else 0))
     stage_avg = {kname: round(v / max(calls, 1), 4) for kname, v in stage_ms.items()}
 
@@ -329,8 +339,8 @@ def run_ours(args):
                    "n_group": wl.n_group, "topk_group": wl.topk_group, "top_k": k, "inter": I,
                    "routed_scaling": wl.routed_scaling, "residual_k": wl.residual_k,
                    "post_norm": wl.post_norm, "token_batches": TOKEN_BATCHES,
-                   "distinct_experts_per_step": round(d_mean, 2),
-                   "l2": f"inputs larger than L2: each step streams {d_mean * 3 * H * I * 2 / 1e9:.1f} GB of expert weights",
+                   "distinct_experts_per_step": round(d_steps, 2),
+                   "l2": f"inputs larger than L2: each step streams {d_steps * 3 * H * I * 2 / 1e9:.1f} GB of expert weights",
                    "parallelism": f"{ws} independent replicas (data parallel, no collective on the data path)"},
         "hbm_fraction_whole_step": round(step_bytes / (ms_max / steps_done * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
         "stage_ms": stage_avg,

@@ -199,14 +199,13 @@ int run_router(beam_moe *h, cudaStream_t s, const void *x, int T, int32_t *idx, 
         m.kb_per_slice = 3 * h->H / 64 / m.nslice;
         m.kb_per_h = h->H / 64;
         m.partial = h->partial;
+        m.fix_count = h->fix_count;   // the kernel zeroes the re-derivation count
         m.ctl.status = h->status;
         m.ctl.limit_ns = h->wait_limit_ns;
         const int items = ((h->E + router_mma_experts_per_tile() - 1) / router_mma_experts_per_tile()) *
                           ((T + router_mma_tokens_per_tile() - 1) / router_mma_tokens_per_tile()) *
                           m.nslice;
-        e = cudaMemsetAsync(h->fix_count, 0, sizeof(int), s);
-        if (e == cudaSuccess)
-            e = launch_router_mma(h->tm_wcat, tmx, m, items < h->num_sms ? items : h->num_sms, s);
+        e = launch_router_mma(h->tm_wcat, tmx, m, items < h->num_sms ? items : h->num_sms, s);
         if (e == cudaSuccess) {
             // select on the tensor-core logits, listing tokens whose margins
             // are too thin for their accumulation error ...

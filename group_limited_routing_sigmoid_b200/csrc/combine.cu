@@ -20,6 +20,8 @@ constexpr int kMaxVec = 8;   // float4 per thread: H <= 8 * 4 * 256 = 8192
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int t = blockIdx.x;
     const int tid = threadIdx.x;
     const int nvec = a.H / 4;
@@ -113,8 +115,7 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream)
 {
     if (a.H % 4 != 0 || a.H > kMaxVec * 4 * kCombThreads || a.top_k > 32)
         return cudaErrorInvalidValue;
-    combine_kernel<<<a.T, kCombThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3(a.T), dim3(kCombThreads), 0, stream, a);
 }
 
 // ---------------------------------------------------------------------------

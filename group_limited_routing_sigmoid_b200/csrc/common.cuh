@@ -149,6 +149,20 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// Programmatic dependent launch.  pdl_launch_dependents lets the next kernel
+// on the stream be scheduled now (its blocks run their set-up while this one
+// finishes); pdl_wait returns once the previous kernel has completed and its
+// memory operations are visible.  Both are no-ops for a kernel that was not
+// launched as a programmatic dependent.  Every kernel here calls pdl_wait
+// before it reads anything an earlier kernel wrote, so completion passes down
+// the chain.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t l2_policy_evict_first()
 {
     uint64_t p;

@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(256) dense_setup_kernel(int T, int tiles, int3
                                                           int32_t *pair_row, int32_t *row_pair,
                                                           float *w)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     if (t == 0) {
         counts[0] = T;
@@ -39,6 +41,8 @@ __global__ void __launch_bounds__(256) dense_swiglu_kernel(const float *__restri
                                                            long long slice_stride, int T, int I,
                                                            __nv_bfloat16 *__restrict__ h)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // float4 index in [T, I]
     const int nq = I / 4;
     if (q >= (long long)T * nq) return;
@@ -66,18 +70,16 @@ cudaError_t launch_dense_setup(int T, int tiles, int32_t *counts, int32_t *offse
                                int32_t *tile_off, int32_t *pair_row, int32_t *row_pair, float *w,
                                cudaStream_t stream)
 {
-    dense_setup_kernel<<<(T + 255) / 256, 256, 0, stream>>>(T, tiles, counts, offsets, tile_off,
-                                                            pair_row, row_pair, w);
-    return cudaGetLastError();
+    return launch_pdl(dense_setup_kernel, dim3((T + 255) / 256), dim3(256), 0, stream, T, tiles,
+                      counts, offsets, tile_off, pair_row, row_pair, w);
 }
 
 cudaError_t launch_dense_swiglu(const float *part, int S, long long slice_stride, int T, int I,
                                 __nv_bfloat16 *h, cudaStream_t stream)
 {
     const long long n = (long long)T * (I / 4);
-    dense_swiglu_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(part, S, slice_stride, T,
-                                                                         I, h);
-    return cudaGetLastError();
+    return launch_pdl(dense_swiglu_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, stream,
+                      part, S, slice_stride, T, I, h);
 }
 
 }  // namespace beam

@@ -16,6 +16,8 @@ __global__ void __launch_bounds__(kDispatchBlock) dispatch_count_kernel(
     const int32_t *__restrict__ idx, int P, int E, int32_t *__restrict__ block_cnt,
     int32_t *__restrict__ rank)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     extern __shared__ int32_t wcnt[];   // [32 warps][E]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
@@ -46,6 +48,8 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
     int32_t *__restrict__ block_base, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ tile_off)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ int32_t wsum_c[32], wsum_t[32];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
     int run = 0;
@@ -112,6 +116,8 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
     const __nv_bfloat16 *__restrict__ x, int P, int H, int E, int top_k,
     int32_t *__restrict__ pair_row, int32_t *__restrict__ row_pair, __nv_bfloat16 *__restrict__ xp)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (p >= P) return;
     const int lane = threadIdx.x & 31;
@@ -134,6 +140,8 @@ __global__ void __launch_bounds__(256) dispatch_rows_kernel(
     const int32_t *__restrict__ block_base, const int32_t *__restrict__ offsets, int P, int E,
     int32_t *__restrict__ pair_row, int32_t *__restrict__ row_pair)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int p = blockIdx.x * blockDim.x + threadIdx.x;
     if (p >= P) return;
     const int e = idx[p];
@@ -153,23 +161,19 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t stream)
     const int P = a.T * a.top_k;
     const int nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
     const size_t smem = sizeof(int32_t) * 32 * (size_t)a.E;
-    dispatch_count_kernel<<<nblk, kDispatchBlock, smem, stream>>>(a.idx, P, a.E, a.block_cnt,
-                                                                  a.rank);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_pdl(dispatch_count_kernel, dim3(nblk), dim3(kDispatchBlock), smem,
+                                 stream, a.idx, P, a.E, a.block_cnt, a.rank);
     if (err != cudaSuccess) return err;
     const int threads = ((a.E + 31) / 32) * 32;
-    dispatch_scan_kernel<<<1, threads, 0, stream>>>(a.block_cnt, nblk, a.E, a.tile_rows,
-                                                    a.block_base, a.counts, a.offsets, a.tile_off);
-    err = cudaGetLastError();
+    err = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(threads), 0, stream, a.block_cnt, nblk,
+                     a.E, a.tile_rows, a.block_base, a.counts, a.offsets, a.tile_off);
     if (err != cudaSuccess) return err;
     if (a.copy_rows)
-        dispatch_permute_kernel<<<(P + 7) / 8, 256, 0, stream>>>(
-            a.idx, a.rank, a.block_base, a.offsets, a.x, P, a.H, a.E, a.top_k, a.pair_row,
-            a.row_pair, a.xp);
-    else
-        dispatch_rows_kernel<<<(P + 255) / 256, 256, 0, stream>>>(
-            a.idx, a.rank, a.block_base, a.offsets, P, a.E, a.pair_row, a.row_pair);
-    return cudaGetLastError();
+        return launch_pdl(dispatch_permute_kernel, dim3((P + 7) / 8), dim3(256), 0, stream, a.idx,
+                          a.rank, a.block_base, a.offsets, a.x, P, a.H, a.E, a.top_k, a.pair_row,
+                          a.row_pair, a.xp);
+    return launch_pdl(dispatch_rows_kernel, dim3((P + 255) / 256), dim3(256), 0, stream, a.idx,
+                      a.rank, a.block_base, a.offsets, P, a.E, a.pair_row, a.row_pair);
 }
 
 }  // namespace beam

@@ -99,7 +99,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    load_tables(p, s_counts, s_offsets, s_tile);
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
@@ -119,6 +118,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
+    pdl_launch_dependents();
+    pdl_wait();   // set-up above overlaps the previous kernel; data from here on
+    load_tables(p, s_counts, s_offsets, s_tile);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -329,9 +331,8 @@ template <int BN, int NUM_A, int EPI>
 cudaError_t launch(const CUtensorMap &a0, const CUtensorMap &a1, const BoxMaps &b,
                    const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    grouped_gemm_kernel<BN, NUM_A, EPI>
-        <<<grid, kThreads, Cfg<BN, NUM_A, EPI>::SMEM_BYTES, stream>>>(a0, a1, b, args);
-    return cudaGetLastError();
+    return launch_pdl(grouped_gemm_kernel<BN, NUM_A, EPI>, dim3(grid), dim3(kThreads),
+                      Cfg<BN, NUM_A, EPI>::SMEM_BYTES, stream, a0, a1, b, args);
 }
 
 template <int BN>

@@ -144,6 +144,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish_pair();
     }
+    pdl_launch_dependents();
+    pdl_wait();   // set-up above overlaps the previous kernel; data from here on
     tc_fence_before();
     __syncthreads();
     __syncwarp();
@@ -366,8 +368,8 @@ cudaError_t launch_pair(const CUtensorMap &a0, const CUtensorMap &a1, const BoxM
     a.a_stages = (kPairRingBytes - a.b_stages * C::B_STAGE) / C::A_STAGE;
     if (a.a_stages > kPairMaxStages) a.a_stages = kPairMaxStages;
     if (a.a_stages < 2) return cudaErrorInvalidValue;
-    grouped_gemm_pair_kernel<BN, NUM_A, EPI><<<grid, kPairThreads, C::SMEM_BYTES, stream>>>(a0, a1, b, a);
-    return cudaGetLastError();
+    return launch_pdl(grouped_gemm_pair_kernel<BN, NUM_A, EPI>, dim3(grid), dim3(kPairThreads),
+                      C::SMEM_BYTES, stream, a0, a1, b, a);
 }
 
 template <int BN>

@@ -6,6 +6,26 @@
 namespace beam {
 
 // ----------------------------------------------------------------- router
+// Launch `kernel` on `stream` as a programmatic dependent of the previous
+// kernel there (it may start while that one finishes; it waits for it with
+// pdl_wait before touching its results).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 struct RouterArgs {
     const __nv_bfloat16 *x;   // [T, H]
     const float *router_w;    // [E, H]
@@ -44,6 +64,7 @@ struct RouterMmaArgs {
     int kb_per_slice;    // 64-wide K steps per slice
     int kb_per_h;        // H / 64 (the token operand wraps around every H)
     float *partial;      // [nslice, T, E]
+    int *fix_count;      // zeroed by the kernel (the re-derivation list's length), or nullptr
     WaitCtl ctl;
 };
 cudaError_t launch_router_split(const float *w, int E, int H, __nv_bfloat16 *wcat, cudaStream_t s);

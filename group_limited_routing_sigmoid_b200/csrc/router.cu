@@ -31,6 +31,8 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16 
                                                             int H, int E, int kslice,
                                                             float *__restrict__ partial)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ __align__(16) float xs[kLK][kLT + 4];
     __shared__ __align__(16) float ws[kLK][kLE + 4];
     const int tid = threadIdx.x;
@@ -160,6 +162,8 @@ __global__ void __launch_bounds__(256) router_select_kernel(
     int top_k, const float *__restrict__ bias, int32_t *__restrict__ idx_out,
     float *__restrict__ w_out, float *__restrict__ logits_out, SelectExtra ex)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int lpg = (E / n_group) / EPL;   // lanes per group (power of two)
     const int my_group = lane / lpg;
@@ -296,22 +300,26 @@ __global__ void __launch_bounds__(256) router_select_kernel(
 
 // ---------------------------------------------------------------------------
 // Exact-path logits for listed tokens: FP32 dot products on CUDA cores.
-// A work unit is (8 listed tokens, 32 experts): the tokens' rows are staged
-// in shared memory as bf16, each warp takes 4 experts, the lanes split K
+// A work unit is (8 listed tokens, 16 experts): the tokens' rows are staged
+// in shared memory as bf16, each warp takes one expert, the lanes split K
 // (lane l reads the 16-byte chunks l, l+32, ... of the weight row, so every
 // load is 512 contiguous bytes), and the 8 per-lane sums (chains of at most
 // 256 terms, folded) are combined by a shuffle tree: logits[slot][e] for
 // list slots 0..*count-1.
 // ---------------------------------------------------------------------------
 constexpr int kFixTokens = 8;
-constexpr int kFixExperts = 32;
+constexpr int kFixExperts = 16;  // one per warp
+constexpr int kFixThreads = 32 * kFixExperts;
+constexpr int kFixLoads = 8;     // weight vectors in flight per lane
 
-__global__ void __launch_bounds__(256) router_fix_kernel(const __nv_bfloat16 *__restrict__ x,
+__global__ void __launch_bounds__(kFixThreads) router_fix_kernel(const __nv_bfloat16 *__restrict__ x,
                                                          const float *__restrict__ w, int H, int E,
                                                          int T, const int *__restrict__ list,
                                                          const int *__restrict__ count,
                                                          float *__restrict__ logits)
 {
+    pdl_launch_dependents();
+    pdl_wait();
     extern __shared__ __align__(16) __nv_bfloat16 xs[];   // [kFixTokens][H]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n = min(*count, T);
@@ -328,34 +336,47 @@ __global__ void __launch_bounds__(256) router_fix_kernel(const __nv_bfloat16 *__
             reinterpret_cast<uint4 *>(xs + (size_t)j * H)[q] = v;
         }
         __syncthreads();
-        for (int m = 0; m < kFixExperts / 8; ++m) {
-            const int e = c * kFixExperts + warp * (kFixExperts / 8) + m;
-            if (e >= E) break;
+        {
+            const int e = c * kFixExperts + warp;
+            if (e >= E) continue;
             const float4 *wr = reinterpret_cast<const float4 *>(w + (size_t)e * H);
             float acc[kFixTokens], tot[kFixTokens];
 #pragma unroll
             for (int j = 0; j < kFixTokens; ++j) acc[j] = tot[j] = 0.f;
             int terms = 0;
-            for (int q = lane; q < H / 4; q += 32) {
-                const float4 wv = wr[q];
+            // kFixLoads weight vectors in flight per lane; the sums take them
+            // in the same order (q = lane, lane + 32, ...) and fold at the
+            // same points as a one-at-a-time loop would
+            for (int q0 = lane; q0 < H / 4; q0 += 32 * kFixLoads) {
+                float4 wv[kFixLoads];
 #pragma unroll
-                for (int j = 0; j < kFixTokens; ++j) {
-                    const __nv_bfloat162 *p2 =
-                        reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)j * H + 4 * q);
-                    const float2 a = __bfloat1622float2(p2[0]);
-                    const float2 b = __bfloat1622float2(p2[1]);
-                    acc[j] = fmaf(wv.x, a.x, acc[j]);
-                    acc[j] = fmaf(wv.y, a.y, acc[j]);
-                    acc[j] = fmaf(wv.z, b.x, acc[j]);
-                    acc[j] = fmaf(wv.w, b.y, acc[j]);
+                for (int u = 0; u < kFixLoads; ++u) {
+                    const int q = q0 + 32 * u;
+                    wv[u] = q < H / 4 ? wr[q] : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-                terms += 4;
-                if (terms == 256) {
-                    terms = 0;
+#pragma unroll
+                for (int u = 0; u < kFixLoads; ++u) {
+                    const int q = q0 + 32 * u;
+                    if (q >= H / 4) break;
 #pragma unroll
                     for (int j = 0; j < kFixTokens; ++j) {
-                        tot[j] += acc[j];
-                        acc[j] = 0.f;
+                        const __nv_bfloat162 *p2 =
+                            reinterpret_cast<const __nv_bfloat162 *>(xs + (size_t)j * H + 4 * q);
+                        const float2 a = __bfloat1622float2(p2[0]);
+                        const float2 b = __bfloat1622float2(p2[1]);
+                        acc[j] = fmaf(wv[u].x, a.x, acc[j]);
+                        acc[j] = fmaf(wv[u].y, a.y, acc[j]);
+                        acc[j] = fmaf(wv[u].z, b.x, acc[j]);
+                        acc[j] = fmaf(wv[u].w, b.y, acc[j]);
+                    }
+                    terms += 4;
+                    if (terms == 256) {
+                        terms = 0;
+#pragma unroll
+                        for (int j = 0; j < kFixTokens; ++j) {
+                            tot[j] += acc[j];
+                            acc[j] = 0.f;
+                        }
                     }
                 }
             }
@@ -392,18 +413,17 @@ cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream)
     const int ns = a.nslice;
     const int kslice = a.H / ns;
     dim3 grid((a.T + kLT - 1) / kLT, (a.E + kLE - 1) / kLE, ns);
-    router_logits_kernel<<<grid, 256, 0, stream>>>(a.x, a.router_w, a.T, a.H, a.E, kslice,
-                                                   a.partial);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_pdl(router_logits_kernel, grid, dim3(256), 0, stream, a.x, a.router_w,
+                                 a.T, a.H, a.E, kslice, a.partial);
     if (err != cudaSuccess) return err;
     const int warps = 8;
     dim3 sgrid((a.T + warps - 1) / warps);
     const int epl = a.E / 32;
 #define BEAM_SELECT(EPLV)                                                                        \
     case EPLV:                                                                                   \
-        router_select_kernel<EPLV><<<sgrid, warps * 32, 0, stream>>>(                            \
-            a.partial, ns, a.T, a.E, a.n_group, a.topk_group, a.top_k, a.bias, a.idx, a.w,       \
-            a.logits_out, SelectExtra{});                                                        \
+        err = launch_pdl(router_select_kernel<EPLV>, sgrid, dim3(warps * 32), 0, stream,         \
+                         a.partial, ns, a.T, a.E, a.n_group, a.topk_group, a.top_k, a.bias, a.idx, \
+                         a.w, a.logits_out, SelectExtra{});                                      \
         break;
     switch (epl) {
         BEAM_SELECT(1)
@@ -416,7 +436,7 @@ cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream)
             return cudaErrorInvalidValue;
     }
 #undef BEAM_SELECT
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace beam
@@ -505,6 +525,9 @@ __global__ void __launch_bounds__(192, 1)
         tmem_alloc(smem_u32(tmem_slot), 2 * kRAccCols);
         tmem_relinquish();
     }
+    pdl_launch_dependents();
+    pdl_wait();   // set-up above overlaps the previous kernel; data from here on
+    if (p.fix_count && blockIdx.x == 0 && threadIdx.x == 0) *p.fix_count = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -646,7 +669,8 @@ cudaError_t prepare_router_mma()
 cudaError_t launch_router_mma(const CUtensorMap &tmW, const CUtensorMap &tmX, const RouterMmaArgs &a,
                               int grid, cudaStream_t stream)
 {
-    router_mma_kernel<<<grid, 192, kRSmem, stream>>>(tmW, tmX, a);
+    cudaError_t e = launch_pdl(router_mma_kernel, dim3(grid), dim3(192), kRSmem, stream, tmW, tmX, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -660,11 +684,12 @@ cudaError_t launch_router_select(const RouterArgs &a, const SelectExtra &ex, int
     int blocks = (a.T + warps - 1) / warps;
     if (max_blocks > 0 && blocks > max_blocks) blocks = max_blocks;
     const int epl = a.E / 32;
+    cudaError_t err = cudaSuccess;
 #define BEAM_SELECT2(EPLV)                                                                       \
     case EPLV:                                                                                   \
-        router_select_kernel<EPLV><<<blocks, warps * 32, 0, stream>>>(                           \
-            a.partial, a.nslice, a.T, a.E, a.n_group, a.topk_group, a.top_k, a.bias, a.idx, a.w, \
-            a.logits_out, ex);                                                                   \
+        err = launch_pdl(router_select_kernel<EPLV>, dim3(blocks), dim3(warps * 32), 0, stream,  \
+                         a.partial, a.nslice, a.T, a.E, a.n_group, a.topk_group, a.top_k, a.bias, \
+                         a.idx, a.w, a.logits_out, ex);                                          \
         break;
     switch (epl) {
         BEAM_SELECT2(1)
@@ -677,7 +702,7 @@ cudaError_t launch_router_select(const RouterArgs &a, const SelectExtra &ex, int
             return cudaErrorInvalidValue;
     }
 #undef BEAM_SELECT2
-    return cudaGetLastError();
+    return err;
 }
 
 cudaError_t prepare_router_fix(int H)
@@ -690,8 +715,9 @@ cudaError_t launch_router_fix(const __nv_bfloat16 *x, const float *w, int H, int
                               const int *list, const int *count, float *logits, int grid,
                               cudaStream_t stream)
 {
-    router_fix_kernel<<<grid, 256, kFixTokens * (size_t)H * 2, stream>>>(x, w, H, E, T, list, count,
-                                                                       logits);
+    cudaError_t e = launch_pdl(router_fix_kernel, dim3(grid), dim3(kFixThreads),
+                               kFixTokens * (size_t)H * 2, stream, x, w, H, E, T, list, count, logits);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
