@@ -14,115 +14,138 @@
 namespace beam {
 
 namespace {
-constexpr int kCombThreads = 256;
-constexpr int kMaxVec = 8;   // float4 per thread: H <= 8 * 4 * 256 = 8192
+constexpr int kCombVecs = 2;            // 16-byte vectors (8 hidden values each) per thread
+constexpr int kCombMaxThreads = 512;    // H <= 8 * kCombVecs * 512 = 8192
+constexpr int kCombBatch = 4;           // expert slots whose loads are in flight together
+
+__device__ __forceinline__ void unpack8(const uint4 &raw, float (&v)[8])
+{
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
 }  // namespace
 
-__global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a)
+// Block per token; thread q takes the 16-byte vectors q and q + blockDim.x of
+// the row (8 hidden values each).  The loads of kCombBatch expert slots of a
+// vector are issued before their sums, which take the slots in order (FP32
+// FMA), so every value is the same slot-order sum.
+__global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
 {
     pdl_launch_dependents();
     pdl_wait();
+    __shared__ int rows[32];
+    __shared__ float wts[32];
+    __shared__ float red[kCombMaxThreads / 32];
     const int t = blockIdx.x;
     const int tid = threadIdx.x;
-    const int nvec = a.H / 4;
-    int rows[32];
-    float wts[32];
+    const int nvec = a.H / 8;
     const int nsum = a.y_f32 ? 0 : a.top_k;   // expert slots (none for FP32 slices)
-    for (int j = 0; j < nsum; ++j) {
-        rows[j] = a.pair_row[(size_t)t * a.top_k + j];
-        wts[j] = a.w[(size_t)t * a.top_k + j];
+    if (tid < nsum) {
+        rows[tid] = a.pair_row[(size_t)t * a.top_k + tid];
+        wts[tid] = a.w[(size_t)t * a.top_k + tid];
     }
-    float4 o[kMaxVec];
+    __syncthreads();
+
+    float acc[kCombVecs][8];
     float ss = 0.f;
 #pragma unroll
-    for (int v = 0; v < kMaxVec; ++v) {
-        const int i = tid + v * kCombThreads;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < nvec) {
-            if (a.y_f32) {
-                for (int sl = 0; sl < a.nslice; ++sl) {
-                    const float4 y = reinterpret_cast<const float4 *>(
-                        a.y_f32 + (size_t)sl * (size_t)a.slice_stride + (size_t)t * a.H)[i];
-                    acc.x += y.x;
-                    acc.y += y.y;
-                    acc.z += y.z;
-                    acc.w += y.w;
+    for (int v = 0; v < kCombVecs; ++v) {
+        const int q = tid + v * blockDim.x;   // vector index in the row
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[v][i] = 0.f;
+        if (q >= nvec) continue;
+        if (a.y_f32) {
+            for (int sl = 0; sl < a.nslice; ++sl) {
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    a.y_f32 + (size_t)sl * (size_t)a.slice_stride + (size_t)t * a.H + 8 * q);
+                const float4 lo = src[0], hi = src[1];
+                acc[v][0] += lo.x; acc[v][1] += lo.y; acc[v][2] += lo.z; acc[v][3] += lo.w;
+                acc[v][4] += hi.x; acc[v][5] += hi.y; acc[v][6] += hi.z; acc[v][7] += hi.w;
+            }
+        }
+        for (int j0 = 0; j0 < nsum; j0 += kCombBatch) {
+            uint4 raw[kCombBatch];
+#pragma unroll
+            for (int j = 0; j < kCombBatch; ++j)
+                if (j0 + j < nsum)
+                    raw[j] = reinterpret_cast<const uint4 *>(a.y + (size_t)rows[j0 + j] * a.H)[q];
+#pragma unroll
+            for (int j = 0; j < kCombBatch; ++j) {
+                if (j0 + j < nsum) {
+                    float y[8];
+                    unpack8(raw[j], y);
+                    const float wj = wts[j0 + j];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[v][i] = fmaf(wj, y[i], acc[v][i]);
                 }
             }
-            for (int j = 0; j < nsum; ++j) {
-                const uint2 raw = reinterpret_cast<const uint2 *>(a.y + (size_t)rows[j] * a.H)[i];
-                const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-                const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
-                const float4 y = make_float4(lo.x, lo.y, hi.x, hi.y);
-                acc.x = fmaf(wts[j], y.x, acc.x);
-                acc.y = fmaf(wts[j], y.y, acc.y);
-                acc.z = fmaf(wts[j], y.z, acc.z);
-                acc.w = fmaf(wts[j], y.w, acc.w);
-            }
-            acc.x *= a.scaling;
-            acc.y *= a.scaling;
-            acc.z *= a.scaling;
-            acc.w *= a.scaling;
-            if (a.out) {
-                __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-                __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-                uint2 packed;
-                packed.x = *reinterpret_cast<uint32_t *>(&lo);
-                packed.y = *reinterpret_cast<uint32_t *>(&hi);
-                reinterpret_cast<uint2 *>(a.out + (size_t)t * a.H)[i] = packed;
-            }
-            ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
         }
-        o[v] = acc;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[v][i] *= a.scaling;
+        if (a.out) {
+            uint4 packed;
+            __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&packed);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[v][2 * i], acc[v][2 * i + 1]);
+            reinterpret_cast<uint4 *>(a.out + (size_t)t * a.H)[q] = packed;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss += acc[v][i] * acc[v][i];
     }
     if (!a.residual) return;
 
     float scale = 1.0f;
     if (a.gamma) {
-        __shared__ float red[kCombThreads / 32];
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         if ((tid & 31) == 0) red[tid >> 5] = ss;
         __syncthreads();
         float tot = 0.f;
-#pragma unroll
-        for (int wv = 0; wv < kCombThreads / 32; ++wv) tot += red[wv];
+        const int nw = (blockDim.x + 31) >> 5;
+        for (int wv = 0; wv < nw; ++wv) tot += red[wv];
         scale = 1.0f / sqrtf(tot / (float)a.H + a.eps);
     }
-    float *st = a.residual + (size_t)t * a.H;
 #pragma unroll
-    for (int v = 0; v < kMaxVec; ++v) {
-        const int i = tid + v * kCombThreads;
-        if (i >= nvec) continue;
-        float4 s = reinterpret_cast<float4 *>(st)[i];
-        float4 n = o[v];
-        if (a.gamma) {
-            const float4 g = reinterpret_cast<const float4 *>(a.gamma)[i];
-            n.x = n.x * scale * g.x;
-            n.y = n.y * scale * g.y;
-            n.z = n.z * scale * g.z;
-            n.w = n.w * scale * g.w;
+    for (int v = 0; v < kCombVecs; ++v) {
+        const int q = tid + v * blockDim.x;
+        if (q >= nvec) continue;
+        float4 *st = reinterpret_cast<float4 *>(a.residual + (size_t)t * a.H + 8 * q);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            float4 sv = st[h2];
+            float n[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) n[i] = acc[v][4 * h2 + i];
+            if (a.gamma) {
+                const float4 g = reinterpret_cast<const float4 *>(a.gamma + 8 * q)[h2];
+                n[0] = n[0] * scale * g.x;
+                n[1] = n[1] * scale * g.y;
+                n[2] = n[2] * scale * g.z;
+                n[3] = n[3] * scale * g.w;
+            }
+            sv.x = fmaf(a.keep, sv.x, n[0] * a.add);
+            sv.y = fmaf(a.keep, sv.y, n[1] * a.add);
+            sv.z = fmaf(a.keep, sv.z, n[2] * a.add);
+            sv.w = fmaf(a.keep, sv.w, n[3] * a.add);
+            st[h2] = sv;
         }
-        s.x = fmaf(a.keep, s.x, n.x * a.add);
-        s.y = fmaf(a.keep, s.y, n.y * a.add);
-        s.z = fmaf(a.keep, s.z, n.z * a.add);
-        s.w = fmaf(a.keep, s.w, n.w * a.add);
-        reinterpret_cast<float4 *>(st)[i] = s;
     }
 }
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream)
 {
-    if (a.H % 4 != 0 || a.H > kMaxVec * 4 * kCombThreads || a.top_k > 32)
-        return cudaErrorInvalidValue;
-    return launch_pdl(combine_kernel, dim3(a.T), dim3(kCombThreads), 0, stream, a);
+    if (a.H % 8 != 0 || a.top_k > 32) return cudaErrorInvalidValue;
+    const int nvec = a.H / 8;
+    const int threads = ((nvec + kCombVecs - 1) / kCombVecs + 31) / 32 * 32;
+    if (threads > kCombMaxThreads) return cudaErrorInvalidValue;
+    return launch_pdl(combine_kernel, dim3(a.T), dim3(threads), 0, stream, a);
 }
 
-// ---------------------------------------------------------------------------
-// Failure-detection self-check: one thread waits on a barrier that nothing
-// completes.  The bounded wait must give up, record the timeout in the status
-// word and let the kernel return.
-// ---------------------------------------------------------------------------
 __global__ void wait_timeout_check_kernel(WaitCtl ctl)
 {
     __shared__ __align__(8) uint64_t bar;
