@@ -21,12 +21,13 @@ BEAM_ERR_UNSUPPORTED = -2
 BEAM_ERR_CUDA = -3
 BEAM_ERR_OOM = -4
 BEAM_ERR_TIMEOUT = -5
+BEAM_ERR_CHECK = -6
 
 # every entry point declared in include/beam_moe.h
 SYMBOLS = (
     "beam_moe_create", "beam_moe_create_dense", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_route_logits",
     "beam_moe_forward",
-    "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_launch_plan",
+    "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_launch_plan", "beam_moe_set_checks", "beam_moe_debug_corrupt_routing",
     "beam_moe_get_status",
     "beam_moe_set_wait_limit", "beam_moe_set_gemm_tuning", "beam_moe_profile_begin",
     "beam_moe_profile_end", "beam_moe_check_wait_timeout", "beam_moe_last_error",
@@ -63,6 +64,8 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_get_status.argtypes = [P, P]
         lib.beam_moe_router_stats.argtypes = [P, P, P]
         lib.beam_moe_launch_plan.argtypes = [P, I, P]
+        lib.beam_moe_set_checks.argtypes = [P, I]
+        lib.beam_moe_debug_corrupt_routing.argtypes = [P, I]
         lib.beam_moe_set_wait_limit.argtypes = [P, ctypes.c_int64]
         lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I, I, I, I, I]
         lib.beam_moe_check_wait_timeout.argtypes = [P, P]
@@ -269,6 +272,17 @@ class BeamMoE:
         keys = ("tile_rows", "cta_pairs", "grid", "down_paired", "router_tensor_cores", "router_slices",
                 "gather_rows", "ksplit_gate_up", "ksplit_down")
         return dict(zip(keys, (int(v) for v in p)))
+
+    def set_checks(self, on: bool = True):
+        """Checked mode: validate routing and dispatch tables on the device."""
+        self._check(library().beam_moe_set_checks(self._h, int(bool(on))))
+
+    def debug_corrupt_routing(self, passes: int = 1):
+        """Test hook (checked mode only): corrupt the next passes' routing."""
+        self._check(library().beam_moe_debug_corrupt_routing(self._h, int(passes)))
+
+    def last_error(self) -> str:
+        return library().beam_moe_last_error(self._h).decode()
 
     def get_status(self, stream=None) -> int:
         return library().beam_moe_get_status(self._h, _stream(stream))

@@ -54,6 +54,9 @@ struct beam_moe {
     int use_pair;                    // 1: CTA-pair kernels for large token tiles (default)
     int gather_rows;                 // -1: auto (default), 0: never, 1: always
     int token_stages;                // CTA-pair kernels: token-row ring depth (0: default)
+    int checks;                      // 1: validate routing and dispatch tables on the device
+    int corrupt_next;                // test hook: forward passes left whose routing is corrupted
+    int *check_where;                // device: first index a check failed at
     int last_T;
     std::vector<cudaEvent_t> prof_events;   // 6 per profiled forward pass
     int prof_max, prof_calls;
@@ -439,6 +442,7 @@ int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *o
 
     if (plan.ksplit_down > 1 || residual) {
         CombineArgs c;
+        c.status = h->status;
         c.y = h->ybuf;
         c.y_f32 = plan.ksplit_down > 1 ? h->split : nullptr;
         c.nslice = plan.ksplit_down;
@@ -470,10 +474,21 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     prof_mark(h, s, 0);
     int rc = run_router(h, s, x, T, h->idx, h->w, nullptr);
     if (rc != BEAM_OK) return rc;
+    if (h->checks) {
+        cudaError_t ce = cudaSuccess;
+        if (h->corrupt_next > 0) {
+            --h->corrupt_next;
+            ce = launch_corrupt_routing(h->idx, h->E, s);
+        }
+        if (ce == cudaSuccess)
+            ce = launch_check_routing(h->idx, h->w, T, h->E, h->top_k, h->status, h->check_where, s);
+        if (ce != cudaSuccess) return cuda_fail(h, ce, "routing check launch");
+    }
     prof_mark(h, s, 1);
     const ForwardPlan plan = plan_forward(h, T);
     const int BN = plan.tile_rows;
     DispatchArgs d;
+    d.status = h->status;
     d.idx = h->idx;
     d.x = static_cast<const __nv_bfloat16 *>(x);
     d.T = T;
@@ -492,6 +507,9 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     d.xp = h->xp;
     d.copy_rows = !plan.gather;
     cudaError_t e = launch_dispatch(d, s);
+    if (e == cudaSuccess && h->checks)
+        e = launch_check_dispatch(h->idx, h->counts, h->offsets, h->tile_off, h->pair_row,
+                                  h->row_pair, T * h->top_k, h->E, BN, h->status, h->check_where, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "dispatch launch");
     prof_mark(h, s, 2);
 
@@ -542,6 +560,7 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     prof_mark(h, s, 4);
 
     CombineArgs c;
+    c.status = h->status;
     c.y = h->ybuf;
     c.y_f32 = nullptr;
     c.nslice = 0;
@@ -673,8 +692,10 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     h->wcat = reinterpret_cast<__nv_bfloat16 *>(b + o_wcat);
     h->fix_count = reinterpret_cast<int *>(b + o_fix);
     h->fix_list = h->fix_count + 1;
+    h->check_where = h->status + 1;
     e = cudaMemset(h->fix_count, 0, sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(h->check_where, 0x7f, sizeof(int));
     if (e == cudaSuccess) e = prepare_grouped_gemm(n_experts);
     if (e == cudaSuccess) e = prepare_dispatch(n_experts);
     if (!h->dense) {
@@ -977,13 +998,36 @@ int beam_moe_get_status(beam_moe_t h, void *stream)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    int v = 0;
+    int v[2] = {0, 0};   // the status word and the first index a check failed at
     cudaError_t e = cudaStreamSynchronize(s);
-    if (e == cudaSuccess) e = cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost);
-    if (e == cudaSuccess && v != 0) e = cudaMemset(h->status, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemcpy(v, h->status, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && v[0] != 0) e = cudaMemset(h->status, 0, sizeof(int));
+    if (e == cudaSuccess && v[0] != 0) e = cudaMemset(h->check_where, 0x7f, sizeof(int));
     if (e != cudaSuccess) return cuda_fail(h, e, "status read");
-    if (v != 0) fail(h, v, "device-side wait ran out (status %d)", v);
-    return v;
+    if (v[0] == BEAM_ERR_CHECK)
+        fail(h, v[0], "checked mode: validation failed at index %d (T*top_k: the dispatch tables)", v[1]);
+    else if (v[0] != 0)
+        fail(h, v[0], "device-side wait ran out (status %d)", v[0]);
+    return v[0];
+}
+
+int beam_moe_set_checks(beam_moe_t h, int on)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    if (on < 0 || on > 1) return fail(h, BEAM_ERR_INVALID_ARG, "checks must be 0 or 1");
+    h->checks = on;
+    if (!on) h->corrupt_next = 0;
+    return BEAM_OK;
+}
+
+int beam_moe_debug_corrupt_routing(beam_moe_t h, int passes)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    if (h->dense) return fail(h, BEAM_ERR_UNSUPPORTED, "a dense layer has no router");
+    if (!h->checks) return fail(h, BEAM_ERR_INVALID_ARG, "corrupted routing needs checked mode");
+    if (passes < 0) return fail(h, BEAM_ERR_INVALID_ARG, "passes < 0");
+    h->corrupt_next = passes;
+    return BEAM_OK;
 }
 
 int beam_moe_set_wait_limit(beam_moe_t h, int64_t limit_ns)

@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
 {
     pdl_launch_dependents();
     pdl_wait();
+    if (a.status && status_is_set(a.status)) return;   // a check failed earlier in this pass
     __shared__ int rows[32];
     __shared__ float wts[32];
     __shared__ float red[kCombMaxThreads / 32];

@@ -11,6 +11,7 @@ namespace beam {
 
 // Device status codes (same values as beam_status in beam_moe.h).
 constexpr int kStatusTimeout = -5;
+constexpr int kStatusCheck = -6;   // a checked-mode validation failed
 
 // Control block every kernel with a wait receives.
 struct WaitCtl {

@@ -13,11 +13,12 @@ namespace beam {
 // every pair gets its rank among the block's pairs of the same expert
 // (ordered by pair index).
 __global__ void __launch_bounds__(kDispatchBlock) dispatch_count_kernel(
-    const int32_t *__restrict__ idx, int P, int E, int32_t *__restrict__ block_cnt,
+    const int *status, const int32_t *__restrict__ idx, int P, int E, int32_t *__restrict__ block_cnt,
     int32_t *__restrict__ rank)
 {
     pdl_launch_dependents();
     pdl_wait();
+    if (status_is_set(status)) return;   // a check failed earlier in this pass
     extern __shared__ int32_t wcnt[];   // [32 warps][E]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
@@ -44,12 +45,13 @@ __global__ void __launch_bounds__(kDispatchBlock) dispatch_count_kernel(
 // One block, thread e = expert: per-block bases, expert counts, exclusive
 // offsets and the prefix of token tiles of BN rows.
 __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
-    const int32_t *__restrict__ block_cnt, int nblk, int E, int BN,
+    const int *status, const int32_t *__restrict__ block_cnt, int nblk, int E, int BN,
     int32_t *__restrict__ block_base, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ tile_off)
 {
     pdl_launch_dependents();
     pdl_wait();
+    if (status_is_set(status)) return;   // a check failed earlier in this pass
     __shared__ int32_t wsum_c[32], wsum_t[32];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
     int run = 0;
@@ -111,13 +113,14 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
 // One warp per pair: its row in the sorted buffer, the maps both ways, and
 // the copy of the token's hidden vector (16-byte vectors).
 __global__ void __launch_bounds__(256) dispatch_permute_kernel(
-    const int32_t *__restrict__ idx, const int32_t *__restrict__ rank,
+    const int *status, const int32_t *__restrict__ idx, const int32_t *__restrict__ rank,
     const int32_t *__restrict__ block_base, const int32_t *__restrict__ offsets,
     const __nv_bfloat16 *__restrict__ x, int P, int H, int E, int top_k,
     int32_t *__restrict__ pair_row, int32_t *__restrict__ row_pair, __nv_bfloat16 *__restrict__ xp)
 {
     pdl_launch_dependents();
     pdl_wait();
+    if (status_is_set(status)) return;   // a check failed earlier in this pass
     const int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (p >= P) return;
     const int lane = threadIdx.x & 31;
@@ -136,12 +139,13 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
 // The maps only, a thread per pair: used when the gate|up GEMM gathers its
 // token rows from x, so no sorted copy of x is made.
 __global__ void __launch_bounds__(256) dispatch_rows_kernel(
-    const int32_t *__restrict__ idx, const int32_t *__restrict__ rank,
+    const int *status, const int32_t *__restrict__ idx, const int32_t *__restrict__ rank,
     const int32_t *__restrict__ block_base, const int32_t *__restrict__ offsets, int P, int E,
     int32_t *__restrict__ pair_row, int32_t *__restrict__ row_pair)
 {
     pdl_launch_dependents();
     pdl_wait();
+    if (status_is_set(status)) return;   // a check failed earlier in this pass
     const int p = blockIdx.x * blockDim.x + threadIdx.x;
     if (p >= P) return;
     const int e = idx[p];
@@ -162,17 +166,17 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t stream)
     const int nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
     const size_t smem = sizeof(int32_t) * 32 * (size_t)a.E;
     cudaError_t err = launch_pdl(dispatch_count_kernel, dim3(nblk), dim3(kDispatchBlock), smem,
-                                 stream, a.idx, P, a.E, a.block_cnt, a.rank);
+                                 stream, a.status, a.idx, P, a.E, a.block_cnt, a.rank);
     if (err != cudaSuccess) return err;
     const int threads = ((a.E + 31) / 32) * 32;
-    err = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(threads), 0, stream, a.block_cnt, nblk,
+    err = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(threads), 0, stream, a.status, a.block_cnt, nblk,
                      a.E, a.tile_rows, a.block_base, a.counts, a.offsets, a.tile_off);
     if (err != cudaSuccess) return err;
     if (a.copy_rows)
-        return launch_pdl(dispatch_permute_kernel, dim3((P + 7) / 8), dim3(256), 0, stream, a.idx,
+        return launch_pdl(dispatch_permute_kernel, dim3((P + 7) / 8), dim3(256), 0, stream, a.status, a.idx,
                           a.rank, a.block_base, a.offsets, a.x, P, a.H, a.E, a.top_k, a.pair_row,
                           a.row_pair, a.xp);
-    return launch_pdl(dispatch_rows_kernel, dim3((P + 255) / 256), dim3(256), 0, stream, a.idx,
+    return launch_pdl(dispatch_rows_kernel, dim3((P + 255) / 256), dim3(256), 0, stream, a.status, a.idx,
                       a.rank, a.block_base, a.offsets, P, a.E, a.pair_row, a.row_pair);
 }
 

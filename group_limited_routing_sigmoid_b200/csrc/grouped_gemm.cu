@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int WT = p.R / C::ROWS_PER_ITEM;
     const int S = C::F32 ? p.ksplit : 1;          // K slices per (weight tile, token tile)
-    const int total = WT * s_tile[p.E] * S;
+    // no work while the status word is set (a failed check or wait)
+    const int total = status_is_set(p.ctl.status) ? 0 : WT * s_tile[p.E] * S;
     const int KB = p.K / kBK / S;                 // K steps of one slice
 
     if (warp == 0) {

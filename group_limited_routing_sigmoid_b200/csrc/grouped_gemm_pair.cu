@@ -154,7 +154,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     const int WT = p.R / C::ROWS_PER_ITEM;
-    const int total = WT * __ldg(&p.tile_off[p.E]);
+    // no work while the status word is set (a failed check or wait)
+    const int total = status_is_set(p.ctl.status) ? 0 : WT * __ldg(&p.tile_off[p.E]);
     const int KB = p.K / kBK;
 
     if (warp == 0) {

@@ -78,6 +78,7 @@ int router_mma_experts_per_tile();
 constexpr int kDispatchBlock = 1024;   // pairs per counting block
 
 struct DispatchArgs {
+    const int *status;           // the handle's status word: no work while it is set
     const int32_t *idx;          // [P] expert of pair p = t*top_k + j
     const __nv_bfloat16 *x;      // [T, H]
     int T, H, E, top_k;
@@ -158,6 +159,7 @@ int gemm_pair_max_ctas();   // CTAs of the pair kernels that can be resident at 
 
 // ---------------------------------------------------------------- combine
 struct CombineArgs {
+    const int *status;           // the handle's status word: no work while it is set
     const __nv_bfloat16 *y;      // [P, H] expert outputs
     // instead of y (dense layer, top_k == 1, unit weight): FP32 partial sums
     // of nslice split-K slices [nslice][T][H], slice_stride elements apart,
@@ -176,6 +178,18 @@ struct CombineArgs {
     float keep, add;             // sqrt((k-1)/k), 1/sqrt(k)
 };
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream);
+
+// ------------------------------------------------------------- checked mode
+// Validation of the routing and of the dispatch tables (see checks.cu); a
+// failure records kStatusCheck and the first failing index in *where.
+cudaError_t launch_check_routing(const int32_t *idx, const float *w, int T, int E, int top_k,
+                                 int *status, int *where, cudaStream_t stream);
+cudaError_t launch_check_dispatch(const int32_t *idx, const int32_t *counts,
+                                  const int32_t *offsets, const int32_t *tile_off,
+                                  const int32_t *pair_row, const int32_t *row_pair, int P, int E,
+                                  int tile_rows, int *status, int *where, cudaStream_t stream);
+// Test hook: write an out-of-range expert into slot 0 of the routing.
+cudaError_t launch_corrupt_routing(int32_t *idx, int E, cudaStream_t stream);
 
 // ------------------------------------------------------------- dense layer
 cudaError_t launch_dense_setup(int T, int tiles, int32_t *counts, int32_t *offsets,

@@ -59,7 +59,8 @@ typedef enum {
     BEAM_ERR_UNSUPPORTED = -2, /* valid for the method, not for these kernels */
     BEAM_ERR_CUDA = -3,        /* a CUDA runtime / driver call failed          */
     BEAM_ERR_OOM = -4,         /* workspace allocation failed                  */
-    BEAM_ERR_TIMEOUT = -5      /* a bounded device-side wait ran out           */
+    BEAM_ERR_TIMEOUT = -5,     /* a bounded device-side wait ran out           */
+    BEAM_ERR_CHECK = -6        /* a checked-mode validation failed             */
 } beam_status;
 
 /*
@@ -249,11 +250,35 @@ int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host);
 
 /*
  * Synchronise `stream`, then return and clear the device status word:
- * BEAM_OK, or BEAM_ERR_TIMEOUT when a bounded in-kernel wait ran out since
- * the last call.  While the word is set, kernels of this handle stop at
- * their next wait, so results of calls made meanwhile are not valid.
+ * BEAM_OK, BEAM_ERR_TIMEOUT when a bounded in-kernel wait ran out, or
+ * BEAM_ERR_CHECK when a checked-mode validation failed, since the last call.
+ * While the word is set, kernels of this handle skip their work (or stop at
+ * their next wait), so results of calls made meanwhile are not valid.
  */
 int beam_moe_get_status(beam_moe_t h, void *stream);
+
+/*
+ * Checked mode (off by default), the stand-in for a memory checker.  With
+ * on = 1 every forward pass of this handle also validates, on the device:
+ * each token's experts (in [0, E), none twice, weights in (0, 1]); the
+ * dispatch tables (offsets from 0 growing by the counts to T*top_k, token
+ * tiles per expert = ceil(count / tile)); every pair's row inside its
+ * expert's range, with the two row maps inverse.  A failure records
+ * BEAM_ERR_CHECK in the status word (no trap); every later kernel of the
+ * pass then skips its work, so none indexes memory with a bad expert or row.
+ * beam_moe_get_status returns it, with the first failing index (a token for
+ * the routing check, a pair, or T*top_k for the tables) in
+ * beam_moe_last_error.  Costs two small kernels per forward pass.
+ */
+int beam_moe_set_checks(beam_moe_t h, int on);
+
+/*
+ * Test hook for checked mode: the next `passes` forward passes overwrite
+ * slot 0 of token 0's routing with the expert index n_experts (out of range)
+ * before the checks run.  BEAM_ERR_INVALID_ARG unless checked mode is on;
+ * BEAM_ERR_UNSUPPORTED on a dense layer.
+ */
+int beam_moe_debug_corrupt_routing(beam_moe_t h, int passes);
 
 /*
  * Set the limit of every in-kernel wait of this handle, in nanoseconds

@@ -77,6 +77,8 @@ def test_calls_on_null_handle_fail_cleanly(lib):
     assert lib.beam_moe_destroy(None) == binding.BEAM_ERR_INVALID_ARG
     assert lib.beam_moe_get_status(None, None) == binding.BEAM_ERR_INVALID_ARG
     assert lib.beam_moe_launch_plan(None, 1, None) == binding.BEAM_ERR_INVALID_ARG
+    assert lib.beam_moe_set_checks(None, 1) == binding.BEAM_ERR_INVALID_ARG
+    assert lib.beam_moe_debug_corrupt_routing(None, 1) == binding.BEAM_ERR_INVALID_ARG
     assert lib.beam_moe_route_logits(None, None, None, 1, None, None, None) == binding.BEAM_ERR_INVALID_ARG
 
 
