@@ -154,6 +154,14 @@ def max_over_ranks(value: float, dist, device) -> float:
     return float(t.item())
 
 
+def workload_config(name: str, wl) -> dict:
+    """The workload's identity and shape (the same keys on both arms)."""
+    return {"workload": f"beam_{name}", "T": wl.T, "hidden": wl.hidden, "n_experts": wl.n_experts,
+            "n_group": wl.n_group, "topk_group": wl.topk_group, "top_k": wl.top_k,
+            "inter": wl.inter, "routed_scaling": wl.routed_scaling, "residual_k": wl.residual_k,
+            "post_norm": wl.post_norm}
+
+
 def kernels_per_forward(plan: dict, dense: bool, residual: bool) -> int:
     """Kernels of this library one forward pass launches, from its launch plan."""
     if dense:
@@ -335,10 +343,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded random weights and tokens of the Beam block shape)",
-        "config": {"workload": f"beam_{args.workload}", "T": T, "hidden": H, "n_experts": E,
-                   "n_group": wl.n_group, "topk_group": wl.topk_group, "top_k": k, "inter": I,
-                   "routed_scaling": wl.routed_scaling, "residual_k": wl.residual_k,
-                   "post_norm": wl.post_norm, "token_batches": TOKEN_BATCHES,
+        "config": {**workload_config(args.workload, wl), "token_batches": TOKEN_BATCHES,
                    "distinct_experts_per_step": round(d_steps, 2),
                    "l2": f"inputs larger than L2: each step streams {d_steps * 3 * H * I * 2 / 1e9:.1f} GB of expert weights",
                    "parallelism": f"{ws} independent replicas (data parallel, no collective on the data path)"},
@@ -433,8 +438,7 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded random weights and tokens of the Beam block shape)",
-        "config": {"workload": f"beam_{args.workload}", "T": wl.T, "hidden": wl.hidden,
-                   "n_experts": wl.n_experts, "top_k": wl.top_k, "inter": wl.inter},
+        "config": workload_config(args.workload, wl),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
                          "sample": f"{per_step} token per step (all {wl.top_k} experts), tokens "
                                    f"cycled through one {wl.T}-token batch"},

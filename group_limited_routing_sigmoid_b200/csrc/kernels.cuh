@@ -5,7 +5,7 @@
 
 namespace beam {
 
-// ----------------------------------------------------------------- router
+// ----------------------------------------------------------------- launch
 // Launch `kernel` on `stream` as a programmatic dependent of the previous
 // kernel there (it may start while that one finishes; it waits for it with
 // pdl_wait before touching its results).
@@ -26,6 +26,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// ----------------------------------------------------------------- router
 struct RouterArgs {
     const __nv_bfloat16 *x;   // [T, H]
     const float *router_w;    // [E, H]
