@@ -62,3 +62,18 @@ def test_block_on_other_layouts(E, G, KG, K):
     rep = check_block(wl, d, moe)
     assert rep.ok(), rep
     moe.close()
+
+
+def test_largest_supported_shapes():
+    """The kernels' size limits at once: hidden 8192, 1024 experts (32 per
+    lane in the selection) in 16 groups of 64, top-32 (the largest top_k),
+    every token through the whole block."""
+    wl = dataclasses.replace(W.WORKLOADS["tiny"], name="max", T=48, hidden=8192, n_experts=1024,
+                             n_group=16, topk_group=4, top_k=32, inter=128)
+    g = W.generator(wl, "cuda")
+    d = W.make_weights(wl, "cuda", g)
+    d.update(W.make_tokens(wl, "cuda", g))
+    moe = BeamMoE.from_workload(wl, d, max_tokens=wl.T)
+    rep = check_block(wl, d, moe)
+    assert rep.ok(), rep
+    moe.close()
