@@ -325,6 +325,10 @@ def run_ours(args):
                           if plan["cta_pairs"] else
                           "gate_up_gemm (grouped_gemm_kernel<%d,2,0>, grid %d)") % (plan["tile_rows"], plan["grid"])
     roof["traffic"] = ncu_traffic(args.workload)
+    # the nominal datasheet peaks beside the measured ones (context, not the denominator)
+    nominal = 8000.0 if roof["bound"] == "hbm" else 2250.0
+    roof["nominal_peak"] = nominal
+    roof["frac_of_nominal"] = round(roof["achieved"] / nominal, 4)
     d_steps = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(steps_done)) / steps_done
     step_bytes = (d_steps * 3 * H * I * 2 + (0 if dense else E * H * 4) + T * H * 4
                   + (T * H * 8 if wl.residual_k else 0))
