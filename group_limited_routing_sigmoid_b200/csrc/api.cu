@@ -65,7 +65,7 @@ struct beam_moe {
 
 namespace {
 
-char g_create_err[512] = "";
+thread_local char g_create_err[512] = "";   // per calling thread
 
 int fail(beam_moe *h, int code, const char *fmt, ...)
 {

@@ -350,7 +350,8 @@ int beam_moe_check_wait_timeout(beam_moe_t h, void *stream);
 /* Text of the last host-side error on this handle ("" if none). */
 const char *beam_moe_last_error(beam_moe_t h);
 
-/* Text of the last error of a beam_moe_create call that returned no handle. */
+/* Text of the last error of a beam_moe_create / beam_moe_create_dense call
+ * that returned no handle, on the calling thread. */
 const char *beam_moe_create_error(void);
 
 /* Free the workspace and the handle.  Synchronises the handle's device. */
