@@ -27,7 +27,7 @@ import ctypes
 import os
 import subprocess
 from dataclasses import dataclass
-from typing import Callable, Dict, Iterable, Optional
+from typing import Callable, Optional
 
 import numpy as np
 

@@ -8,7 +8,6 @@ normalised to 1.  No GPU."""
 import itertools
 
 import numpy as np
-import pytest
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
 from scipy.special import expit

@@ -7,7 +7,6 @@ import dataclasses
 
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from group_limited_routing_sigmoid_b200 import workloads as W
