@@ -49,3 +49,22 @@ def test_two_rank_host_logic():
     assert r0[1] != r1[1]                      # each rank its own tokens
     assert r0[2] == r1[2] == 15.0              # slowest rank's time on both
     assert r0[3] == r1[3] == 2 * 4 * 64 / 15e-3
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """`bench.py --impl reference` launched the way a multi-GPU run is: rank 0
+    alone times the oracle and prints one JSON line; every rank exits 0."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py",
+           "--impl", "reference", "--gpus", "2", "--steps", "2", "--warmup", "3", "--workload", "tiny"]
+    res = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["config"]["workload"] == "beam_tiny"
