@@ -272,25 +272,31 @@ def run_ours(args):
     if moe.get_status() != 0:
         raise SystemExit("a device-side wait ran out during the stage-timed steps")
 
-    # end to end through the host-buffer entry point (pinned buffers)
+    # end to end through the host-buffer entry points (pinned buffers): each
+    # step copies its batch in and its result out; the pipelined call lets a
+    # step's copies overlap its neighbours' compute
     x_host = [b["x"].cpu().pin_memory() for b in batches]
-    out_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    out_host = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     res_host = [s.cpu().pin_memory() for s in streams] if wl.residual_k else None
     e2e_steps = max(3, min(args.steps, 50))
 
     def e2e_step(i):
         j = i % TOKEN_BATCHES
-        moe.forward_host(x_host[j], out_host=out_host,
-                         residual_host=res_host[j] if res_host else None, k=max(1, wl.residual_k))
+        moe.forward_host_async(x_host[j], out_host=out_host[i & 1],
+                               residual_host=res_host[j] if res_host else None,
+                               k=max(1, wl.residual_k))
 
     for i in range(args.warmup):
         e2e_step(i)
+    moe.host_join()
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     ev0.record(stream)
+    moe.host_fence()          # the first copy in starts after ev0
     for i in range(e2e_steps):
         e2e_step(i)
+    moe.host_join()           # ev1 after the last copy out
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)

@@ -27,7 +27,9 @@ BEAM_ERR_CHECK = -6
 SYMBOLS = (
     "beam_moe_create", "beam_moe_create_dense", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_route_logits",
     "beam_moe_forward",
-    "beam_moe_forward_host", "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_launch_plan", "beam_moe_set_checks", "beam_moe_debug_corrupt_routing",
+    "beam_moe_forward_host", "beam_moe_forward_host_async", "beam_moe_host_join",
+    "beam_moe_host_fence",
+    "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_launch_plan", "beam_moe_set_checks", "beam_moe_debug_corrupt_routing",
     "beam_moe_get_status",
     "beam_moe_set_wait_limit", "beam_moe_set_gemm_tuning", "beam_moe_profile_begin",
     "beam_moe_profile_end", "beam_moe_check_wait_timeout", "beam_moe_last_error",
@@ -60,6 +62,9 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_route_logits.argtypes = [P, P, P, I, P, P, P]
         lib.beam_moe_forward.argtypes = [P, P, P, I, P, P, I]
         lib.beam_moe_forward_host.argtypes = [P, P, P, I, P, P, I]
+        lib.beam_moe_forward_host_async.argtypes = [P, P, P, I, P, P, I]
+        lib.beam_moe_host_join.argtypes = [P, P]
+        lib.beam_moe_host_fence.argtypes = [P, P]
         lib.beam_moe_dispatch_info.argtypes = [P, P, I, P, P, P]
         lib.beam_moe_get_status.argtypes = [P, P]
         lib.beam_moe_router_stats.argtypes = [P, P, P]
@@ -248,6 +253,22 @@ class BeamMoE:
         self._check(library().beam_moe_forward_host(self._h, _stream(stream), _ptr(x_host), T,
                                                      _ptr(out_host), _ptr(residual_host), int(k)))
         return out_host
+
+    def forward_host_async(self, x_host: torch.Tensor, out_host: Optional[torch.Tensor] = None,
+                           residual_host: Optional[torch.Tensor] = None, k: int = 1, stream=None):
+        """Pipelined host-buffer pass: returns at once; host_join + a stream
+        synchronise before reading the results."""
+        assert not x_host.is_cuda and x_host.dtype == torch.bfloat16 and x_host.is_contiguous()
+        T = x_host.shape[0]
+        self._check(library().beam_moe_forward_host_async(self._h, _stream(stream), _ptr(x_host), T,
+                                                           _ptr(out_host), _ptr(residual_host), int(k)))
+        return out_host
+
+    def host_join(self, stream=None):
+        self._check(library().beam_moe_host_join(self._h, _stream(stream)))
+
+    def host_fence(self, stream=None):
+        self._check(library().beam_moe_host_fence(self._h, _stream(stream)))
 
     def dispatch_info(self, T: int, stream=None):
         counts = np.empty(self.n_experts, np.int32)

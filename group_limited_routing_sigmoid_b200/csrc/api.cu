@@ -36,8 +36,15 @@ struct beam_moe {
     __nv_bfloat16 *hbuf;     // [P, I]
     __nv_bfloat16 *ybuf;     // [P, H]
     int *status;             // device status word
-    __nv_bfloat16 *x_stage, *out_stage;
-    float *res_stage;
+    // host-buffer path: two staging slots, so one call's copies overlap the
+    // neighbouring calls' compute; a copy-in and a copy-out stream; per slot
+    // the events copy-in done, compute done, copy-out done
+    __nv_bfloat16 *x_stage[2], *out_stage[2];
+    float *res_stage[2];
+    cudaStream_t copy_in, copy_out;
+    cudaEvent_t ev_in[2], ev_comp[2], ev_out[2];
+    cudaEvent_t ev_fence;            // host_fence: the caller's stream position
+    int host_slot;
 
     CUtensorMap tm_gate, tm_up, tm_down;
     CUtensorMap tm_wcat;             // router weight as three bf16 pieces [E, 3H]
@@ -593,6 +600,18 @@ int check_tokens(beam_moe *h, const void *x, int T)
     return BEAM_OK;
 }
 
+void release_host_path(beam_moe *h)
+{
+    for (int i = 0; i < 2; ++i) {
+        if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+        if (h->ev_comp[i]) cudaEventDestroy(h->ev_comp[i]);
+        if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+    }
+    if (h->ev_fence) cudaEventDestroy(h->ev_fence);
+    if (h->copy_in) cudaStreamDestroy(h->copy_in);
+    if (h->copy_out) cudaStreamDestroy(h->copy_out);
+}
+
 // Device set-up common to both handle kinds: workspace, kernel attributes,
 // the router weight's bf16 pieces (sparse blocks) and the tensor maps.
 int finish_create(beam_moe *h, beam_moe_t *out)
@@ -655,9 +674,12 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     const size_t o_h = carve(P * inter * 2);
     const size_t o_y = carve(P * hidden * 2);
     const size_t o_status = carve(256);
-    const size_t o_xs = carve(T * hidden * 2);
-    const size_t o_os = carve(T * hidden * 2);
-    const size_t o_rs = carve(T * hidden * 4);
+    size_t o_xs[2], o_os[2], o_rs[2];
+    for (int i = 0; i < 2; ++i) {
+        o_xs[i] = carve(T * hidden * 2);
+        o_os[i] = carve(T * hidden * 2);
+        o_rs[i] = carve(T * hidden * 4);
+    }
     const size_t o_wcat = carve(h->dense ? 0 : E * 3 * (size_t)hidden * 2);
     const size_t o_fix = carve((T + 1) * 4);
     h->ws_bytes = off;
@@ -686,9 +708,11 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     h->hbuf = reinterpret_cast<__nv_bfloat16 *>(b + o_h);
     h->ybuf = reinterpret_cast<__nv_bfloat16 *>(b + o_y);
     h->status = reinterpret_cast<int *>(b + o_status);
-    h->x_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_xs);
-    h->out_stage = reinterpret_cast<__nv_bfloat16 *>(b + o_os);
-    h->res_stage = reinterpret_cast<float *>(b + o_rs);
+    for (int i = 0; i < 2; ++i) {
+        h->x_stage[i] = reinterpret_cast<__nv_bfloat16 *>(b + o_xs[i]);
+        h->out_stage[i] = reinterpret_cast<__nv_bfloat16 *>(b + o_os[i]);
+        h->res_stage[i] = reinterpret_cast<float *>(b + o_rs[i]);
+    }
     h->wcat = reinterpret_cast<__nv_bfloat16 *>(b + o_wcat);
     h->fix_count = reinterpret_cast<int *>(b + o_fix);
     h->fix_list = h->fix_count + 1;
@@ -725,6 +749,21 @@ int finish_create(beam_moe *h, beam_moe_t *out)
         cudaFree(h->ws);
         delete h;
         return fail(nullptr, BEAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    }
+    e = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fence, cudaEventDisableTiming);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+        e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_comp[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) {
+        int rc = cuda_fail(nullptr, e, "host-path streams / events");
+        release_host_path(h);
+        cudaFree(h->ws);
+        delete h;
+        return rc;
     }
     *out = h;
     return BEAM_OK;
@@ -911,8 +950,8 @@ int beam_moe_forward(beam_moe_t h, void *stream, const void *x, int T, void *out
     return run_forward(h, static_cast<cudaStream_t>(stream), x, T, out, residual, k);
 }
 
-int beam_moe_forward_host(beam_moe_t h, void *stream, const void *x_host, int T, void *out_host,
-                          float *residual_host, int k)
+int beam_moe_forward_host_async(beam_moe_t h, void *stream, const void *x_host, int T,
+                                void *out_host, float *residual_host, int k)
 {
     if (!h) return BEAM_ERR_INVALID_ARG;
     h->err[0] = 0;
@@ -921,25 +960,68 @@ int beam_moe_forward_host(beam_moe_t h, void *stream, const void *x_host, int T,
     if (T == 0) return BEAM_OK;
     if (!out_host && !residual_host)
         return fail(h, BEAM_ERR_INVALID_ARG, "out_host and residual_host are both NULL");
-    if (T > 0 && !x_host) return fail(h, BEAM_ERR_INVALID_ARG, "x_host is NULL");
+    if (!x_host) return fail(h, BEAM_ERR_INVALID_ARG, "x_host is NULL");
     if (residual_host && k < 1) return fail(h, BEAM_ERR_INVALID_ARG, "residual step k must be >= 1");
-    if (T == 0) return BEAM_OK;
     int rc = check_device(h);
     if (rc != BEAM_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int slot = h->host_slot;
     const size_t n = (size_t)T * h->H;
-    cudaError_t e = cudaMemcpyAsync(h->x_stage, x_host, n * 2, cudaMemcpyHostToDevice, s);
+    // copy in once this slot's previous pass has read its inputs and its
+    // previous results have left
+    cudaError_t e = cudaStreamWaitEvent(h->copy_in, h->ev_comp[slot], 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_in, h->ev_out[slot], 0);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(h->x_stage[slot], x_host, n * 2, cudaMemcpyHostToDevice, h->copy_in);
     if (e == cudaSuccess && residual_host)
-        e = cudaMemcpyAsync(h->res_stage, residual_host, n * 4, cudaMemcpyHostToDevice, s);
+        e = cudaMemcpyAsync(h->res_stage[slot], residual_host, n * 4, cudaMemcpyHostToDevice,
+                            h->copy_in);
+    if (e == cudaSuccess) e = cudaEventRecord(h->ev_in[slot], h->copy_in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, h->ev_in[slot], 0);
     if (e != cudaSuccess) return cuda_fail(h, e, "host-to-device copy");
-    rc = run_forward(h, s, h->x_stage, T, out_host ? h->out_stage : nullptr,
-                     residual_host ? h->res_stage : nullptr, k);
+    rc = run_forward(h, s, h->x_stage[slot], T, out_host ? h->out_stage[slot] : nullptr,
+                     residual_host ? h->res_stage[slot] : nullptr, k);
     if (rc != BEAM_OK) return rc;
-    if (out_host) e = cudaMemcpyAsync(out_host, h->out_stage, n * 2, cudaMemcpyDeviceToHost, s);
+    e = cudaEventRecord(h->ev_comp[slot], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->ev_comp[slot], 0);
+    if (e == cudaSuccess && out_host)
+        e = cudaMemcpyAsync(out_host, h->out_stage[slot], n * 2, cudaMemcpyDeviceToHost, h->copy_out);
     if (e == cudaSuccess && residual_host)
-        e = cudaMemcpyAsync(residual_host, h->res_stage, n * 4, cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "device-to-host copy");
+        e = cudaMemcpyAsync(residual_host, h->res_stage[slot], n * 4, cudaMemcpyDeviceToHost,
+                            h->copy_out);
+    if (e == cudaSuccess) e = cudaEventRecord(h->ev_out[slot], h->copy_out);
+    if (e != cudaSuccess) return cuda_fail(h, e, "device-to-host copy");
+    h->host_slot = slot ^ 1;
+    return BEAM_OK;
+}
+
+int beam_moe_host_fence(beam_moe_t h, void *stream)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    cudaError_t e = cudaEventRecord(h->ev_fence, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_in, h->ev_fence, 0);
+    return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "fence of the host-buffer copies");
+}
+
+int beam_moe_host_join(beam_moe_t h, void *stream)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamWaitEvent(s, h->ev_out[0], 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, h->ev_out[1], 0);
+    return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "join of the host-buffer copies");
+}
+
+int beam_moe_forward_host(beam_moe_t h, void *stream, const void *x_host, int T, void *out_host,
+                          float *residual_host, int k)
+{
+    int rc = beam_moe_forward_host_async(h, stream, x_host, T, out_host, residual_host, k);
+    if (rc != BEAM_OK) return rc;
+    if (T == 0) return BEAM_OK;
+    rc = beam_moe_host_join(h, stream);
+    if (rc != BEAM_OK) return rc;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "host-buffer pass");
 }
 
 int beam_moe_dispatch_info(beam_moe_t h, void *stream, int T, int32_t *counts_host,
@@ -1140,6 +1222,7 @@ int beam_moe_destroy(beam_moe_t h)
     if (prev != h->device) cudaSetDevice(h->device);
     cudaError_t e = cudaDeviceSynchronize();
     prof_release(h);
+    release_host_path(h);
     if (h->ws) cudaFree(h->ws);
     if (prev >= 0 && prev != h->device) cudaSetDevice(prev);
     delete h;

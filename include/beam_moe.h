@@ -203,14 +203,40 @@ int beam_moe_forward(beam_moe_t h, void *stream, const void *x, int T, void *out
 
 /*
  * beam_moe_forward with HOST buffers: copies x_host (and residual_host) to
- * the handle's device staging buffers, runs the forward pass and copies the
- * results back, all on `stream`, then waits for the stream.  Pinned host
- * memory gives asynchronous copies; pageable memory works too.
+ * one of the handle's two device staging slots, runs the forward pass on
+ * `stream` and copies the results back, then waits until they landed.
  * x_host bf16 [T, H]; out_host bf16 [T, H] or NULL; residual_host fp32
- * [T, H] (in/out) or NULL.  Synchronous: returns after the results landed.
+ * [T, H] (in/out) or NULL.  Pinned host memory gives asynchronous copies;
+ * pageable memory works too.  Synchronous.
  */
 int beam_moe_forward_host(beam_moe_t h, void *stream, const void *x_host, int T,
                           void *out_host, float *residual_host, int k);
+
+/*
+ * The same pass without waiting: a pipeline for a stream of host batches.
+ * The copy to the device runs on the handle's copy-in stream, the pass on
+ * `stream`, the copy back on its copy-out stream, ordered by events.  Calls
+ * alternate between two staging slots, so the copy-in of one call overlaps
+ * the compute of the previous call and the copy-out overlaps the next.  The
+ * host buffers must stay untouched until the results landed; call
+ * beam_moe_host_join (then synchronise `stream`) before reading out_host /
+ * residual_host.  Passes run in call order on `stream`; use one stream per
+ * handle.
+ */
+int beam_moe_forward_host_async(beam_moe_t h, void *stream, const void *x_host, int T,
+                                void *out_host, float *residual_host, int k);
+
+/*
+ * Make `stream` wait (without blocking the host) until every copy back of
+ * earlier beam_moe_forward_host_async calls has landed in host memory.
+ */
+int beam_moe_host_join(beam_moe_t h, void *stream);
+
+/*
+ * Make the copies of later beam_moe_forward_host_async calls start only
+ * after the work enqueued on `stream` so far (for instance a timing event).
+ */
+int beam_moe_host_fence(beam_moe_t h, void *stream);
 
 /*
  * Dispatch bookkeeping of the last forward pass on this handle (for checks):
