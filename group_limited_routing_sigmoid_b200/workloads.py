@@ -52,6 +52,7 @@ class Workload:
     expert_std: float = 0.02
     seed: int = 0
     sample: int = 0              # tokens the oracle checks (0 = all)
+    weight_format: str = "bf16"  # "bf16" or "nvfp4" (expert weights)
 
     def with_tokens(self, T: int) -> "Workload":
         return replace(self, T=T)
@@ -96,6 +97,11 @@ WORKLOADS: Dict[str, Workload] = {
                              topk_group=1, top_k=1, inter=20480, routed_scaling=1.0),
     "dense_prefill": Workload("dense_prefill", T=8192, hidden=5120, n_experts=1, n_group=1,
                               topk_group=1, top_k=1, inter=20480, routed_scaling=1.0, sample=256),
+    # NVFP4 expert weights (the 4-bit checkpoint format the pages recommend for
+    # Blackwell): the same draws, quantised by nvfp4_quantize
+    "tiny_nvfp4": Workload("tiny_nvfp4", T=64, hidden=256, n_experts=32, n_group=8, topk_group=4,
+                           top_k=8, inter=128, weight_format="nvfp4"),
+    "decode_nvfp4": Workload("decode_nvfp4", T=64, weight_format="nvfp4", **_BEAM),
 }
 
 
@@ -125,6 +131,55 @@ def make_weights(wl: Workload, device, g: Optional[torch.Generator] = None) -> D
         w_down[e] = (torch.randn(H, I, generator=g, device=device) * wl.expert_std).to(torch.bfloat16)
     return dict(router_w=router_w.contiguous(), bias=bias.contiguous(), w_gate=w_gate, w_up=w_up,
                 w_down=w_down, hot=hot)
+
+
+E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def nvfp4_quantize(w: torch.Tensor, global_scale: float):
+    """Round-to-nearest NVFP4 encoding of w [..., R, K] (K a multiple of 16)
+    with the given per-tensor scale: one E4M3 scale per 16 elements (the
+    block's absolute maximum / 6, over the tensor scale, rounded to E4M3 by
+    torch's cast) and each element's nearest E2M1 magnitude and its sign.
+    Returns codes uint8 [..., R, K/2] (element 2j in the low nibble of byte
+    j) and scales uint8 [..., R, K/16].  This makes synthetic inputs; the
+    block's arithmetic only ever decodes them."""
+    *lead, K = w.shape
+    blocks = w.float().reshape(*lead, K // 16, 16)
+    bscale = (blocks.abs().amax(-1) / 6.0 / global_scale).to(torch.float8_e4m3fn)
+    eff = bscale.float() * global_scale
+    q = torch.where(eff[..., None] > 0, blocks / eff[..., None].clamp_min(1e-30), torch.zeros_like(blocks))
+    mids = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], device=w.device)
+    mag = torch.bucketize(q.abs().clamp(max=6.0), mids)
+    code = (mag | ((q < 0).to(torch.int64) << 3)).reshape(*lead, K)
+    packed = (code[..., 0::2] | (code[..., 1::2] << 4)).to(torch.uint8)
+    return packed.contiguous(), bscale.view(torch.uint8).contiguous()
+
+
+def nvfp4_global_scale(w: torch.Tensor) -> float:
+    """The per-tensor scale that maps the tensor's absolute maximum to the
+    largest NVFP4 value (6 x 448)."""
+    amax = float(w.abs().max())
+    return amax / (6.0 * 448.0) if amax > 0 else 1.0
+
+
+def make_nvfp4_weights(wl: Workload, device, g: Optional[torch.Generator] = None) -> Dict[str, torch.Tensor]:
+    """make_weights, then the expert tensors in NVFP4: {gate,up,down}_codes,
+    _scales and _global (per tensor); the bf16 tensors are dropped."""
+    d = make_weights(wl, device, g)
+    for name in ("gate", "up", "down"):
+        w = d.pop("w_" + name)
+        gs = nvfp4_global_scale(w)
+        codes, scales = [], []
+        for e in range(w.shape[0]):        # per expert: bounded temporaries
+            c, s = nvfp4_quantize(w[e], gs)
+            codes.append(c)
+            scales.append(s)
+        d[name + "_codes"] = torch.stack(codes)
+        d[name + "_scales"] = torch.stack(scales)
+        d[name + "_global"] = gs
+        del w
+    return d
 
 
 def make_tokens(wl: Workload, device, g: torch.Generator, T: Optional[int] = None) -> Dict[str, torch.Tensor]:

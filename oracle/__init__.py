@@ -62,6 +62,12 @@ def _load():
         lib.oracle_route_logits.restype = I
         lib.oracle_expert_swiglu.argtypes = [I, I, I, P, P, P, P, P, P]
         lib.oracle_expert_swiglu.restype = None
+        lib.oracle_expert_swiglu_nvfp4.argtypes = [I, I, I, P, P, P, P, P, P, P, D, D, D, P, P]
+        lib.oracle_expert_swiglu_nvfp4.restype = None
+        lib.oracle_e2m1_value.argtypes = [ctypes.c_uint]
+        lib.oracle_e2m1_value.restype = D
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint]
+        lib.oracle_e4m3_value.restype = D
         lib.oracle_combine.argtypes = [I, I, I, P, P, D, P, P]
         lib.oracle_combine.restype = None
         lib.oracle_post_norm_residual.argtypes = [I, I, P, P, D, I, P, P, P]
@@ -196,6 +202,48 @@ def expert_swiglu(x_bits: np.ndarray, w_gate_bits: np.ndarray, w_up_bits: np.nda
     return (y, h) if want_h else y
 
 
+def e2m1_value(code: int) -> float:
+    """An E2M1 code (4 bits) -> its value (the C decoder, from the format's definition)."""
+    return _load().oracle_e2m1_value(int(code))
+
+
+def e4m3_value(byte: int) -> float:
+    """An FP8 E4M3 byte -> its value (the C decoder)."""
+    return _load().oracle_e4m3_value(int(byte))
+
+
+@dataclass
+class Nvfp4Matrix:
+    """One NVFP4 weight tensor: codes uint8 [..., R, K/2] (element 2j in the low
+    nibble of byte j), scales uint8 [..., R, K/16] (E4M3), a per-tensor scale."""
+    codes: np.ndarray
+    scales: np.ndarray
+    global_scale: float
+
+
+def expert_swiglu_nvfp4(x_bits: np.ndarray, gate: Nvfp4Matrix, up: Nvfp4Matrix,
+                        down: Nvfp4Matrix, want_h: bool = False):
+    """One SwiGLU expert with NVFP4 matrices (gate, up [I, H], down [H, I])."""
+    lib = _load()
+    x = _u16(x_bits)
+    n, H = x.shape
+    I = gate.codes.shape[0]
+    u8 = lambda a: np.ascontiguousarray(a, dtype=np.uint8)
+    gc, gs, uc, us, dc, ds = (u8(gate.codes), u8(gate.scales), u8(up.codes), u8(up.scales),
+                              u8(down.codes), u8(down.scales))
+    assert gc.shape == (I, H // 2) and gs.shape == (I, H // 16)
+    assert uc.shape == (I, H // 2) and us.shape == (I, H // 16)
+    assert dc.shape == (H, I // 2) and ds.shape == (H, I // 16)
+    y = np.empty((n, H), np.float64)
+    h = np.empty((n, I), np.uint16) if want_h else None
+    if n:
+        lib.oracle_expert_swiglu_nvfp4(n, H, I, _ptr(x), _ptr(gc), _ptr(gs), _ptr(uc), _ptr(us),
+                                       _ptr(dc), _ptr(ds), float(gate.global_scale),
+                                       float(up.global_scale), float(down.global_scale),
+                                       _ptr(y), _ptr(h))
+    return (y, h) if want_h else y
+
+
 def combine(y: np.ndarray, w: np.ndarray, scale: float):
     """o = scale * sum_j w_j y_j in slot order; returns (o float64 [T,H], out bf16 bits [T,H])."""
     lib = _load()
@@ -253,8 +301,9 @@ def moe_block(x_bits: np.ndarray, router_w: np.ndarray, bias: np.ndarray,
     """The block's forward pass on the tokens in ``x_bits``.
 
     ``fetch_expert(e)`` returns expert e's (w_gate [I,H], w_up [I,H],
-    w_down [H,I]) bf16 bit patterns; it is called once per expert that the
-    tokens route to, so that the caller can stream large weight sets.
+    w_down [H,I]) as bf16 bit patterns or as three Nvfp4Matrix; it is called
+    once per expert that the tokens route to, so that the caller can stream
+    large weight sets.
     Steps: route; for every (token, slot) run the slot's expert; combine in
     slot order x routed_scaling; round to bf16; optionally post-norm and
     residual update at step ``kstep``.
@@ -266,8 +315,11 @@ def moe_block(x_bits: np.ndarray, router_w: np.ndarray, bias: np.ndarray,
     experts = sorted(set(int(e) for e in r.idx.reshape(-1)))
     for e in experts:
         tt, jj = np.nonzero(r.idx == e)
-        wg, wu, wd = fetch_expert(e)
-        ye = expert_swiglu(np.ascontiguousarray(x[tt]), wg, wu, wd)
+        mats = fetch_expert(e)
+        if isinstance(mats[0], Nvfp4Matrix):
+            ye = expert_swiglu_nvfp4(np.ascontiguousarray(x[tt]), *mats)
+        else:
+            ye = expert_swiglu(np.ascontiguousarray(x[tt]), *mats)
         y[tt, jj, :] = ye
         if on_expert is not None:
             on_expert(e, len(tt))

@@ -328,6 +328,98 @@ void oracle_expert_swiglu(int n, int H, int I, const uint16_t *x,
 }
 
 /* ------------------------------------------------------------------ */
+/* One SwiGLU expert with NVFP4 weights                                 */
+/* ------------------------------------------------------------------ */
+
+/*
+ * NVFP4 weights (the 4-bit checkpoint format the Beam pages name for
+ * Blackwell GPUs): 4-bit E2M1 elements, one FP8 E4M3 scale per 16
+ * consecutive elements of a row, one FP32 scale per tensor:
+ *   w[r][k] = e2m1(code[r][k]) * e4m3(scale[r][k / 16]) * global.
+ * Codes: two per byte, element 2j in the low nibble of byte j of the row.
+ * Both small formats are decoded from their definitions: E2M1 is sign,
+ * 2 exponent bits (bias 1), 1 mantissa bit, exponent 0 subnormal (m * 0.5);
+ * E4M3 is sign, 4 exponent bits (bias 7), 3 mantissa bits, exponent 0
+ * subnormal (m / 8 * 2^-6), all-ones exponent and mantissa NaN, no infinity.
+ */
+double oracle_e2m1_value(unsigned code)
+{
+    const int sgn = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    const double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sgn ? -v : v;
+}
+
+double oracle_e4m3_value(unsigned byte)
+{
+    const int sgn = (byte >> 7) & 1, e = (byte >> 3) & 15, m = byte & 7;
+    double v;
+    if (e == 15 && m == 7) v = NAN;
+    else if (e == 0) v = ldexp(m / 8.0, -6);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* Row r of an NVFP4 matrix with K columns, decoded into w[0..K-1]. */
+static void nvfp4_row(const uint8_t *codes, const uint8_t *scales, double global, int K, size_t r,
+                      double *w)
+{
+    const uint8_t *c = codes + r * (size_t)(K / 2);
+    const uint8_t *sc = scales + r * (size_t)(K / 16);
+    for (int k = 0; k < K; ++k) {
+        const unsigned code = (k & 1) ? (c[k / 2] >> 4) & 15u : c[k / 2] & 15u;
+        w[k] = oracle_e2m1_value(code) * oracle_e4m3_value(sc[k / 16]) * global;
+    }
+}
+
+/*
+ * oracle_expert_swiglu with the expert's three matrices in NVFP4:
+ * gate, up [I, H] and down [H, I] as codes (uint8, K/2 per row), scales
+ * (uint8, K/16 per row) and a per-tensor scale.  Same arithmetic otherwise:
+ * double sums in index order, the SwiGLU product rounded to FP32 then bf16.
+ */
+void oracle_expert_swiglu_nvfp4(int n, int H, int I, const uint16_t *x,
+                                const uint8_t *gate_codes, const uint8_t *gate_scales,
+                                const uint8_t *up_codes, const uint8_t *up_scales,
+                                const uint8_t *down_codes, const uint8_t *down_scales,
+                                double gate_global, double up_global, double down_global,
+                                double *y, uint16_t *h_out)
+{
+    double *hv = (double *)malloc(sizeof(double) * (size_t)I);
+    for (int r = 0; r < n; ++r) {
+        const uint16_t *xr = x + (size_t)r * H;
+#pragma omp parallel for schedule(static)
+        for (int i = 0; i < I; ++i) {
+            double *wg = (double *)malloc(sizeof(double) * (size_t)H);
+            double *wu = (double *)malloc(sizeof(double) * (size_t)H);
+            nvfp4_row(gate_codes, gate_scales, gate_global, H, (size_t)i, wg);
+            nvfp4_row(up_codes, up_scales, up_global, H, (size_t)i, wu);
+            double g = 0.0, u = 0.0;
+            for (int h = 0; h < H; ++h) {
+                double xv = oracle_bf16_to_double(xr[h]);
+                g += xv * wg[h];
+                u += xv * wu[h];
+            }
+            float p32 = (float)(silu(g) * u);
+            uint16_t hb = oracle_double_to_bf16((double)p32);
+            hv[i] = oracle_bf16_to_double(hb);
+            if (h_out) h_out[(size_t)r * I + i] = hb;
+            free(wg);
+            free(wu);
+        }
+#pragma omp parallel for schedule(static)
+        for (int h = 0; h < H; ++h) {
+            double *wd = (double *)malloc(sizeof(double) * (size_t)I);
+            nvfp4_row(down_codes, down_scales, down_global, I, (size_t)h, wd);
+            double acc = 0.0;
+            for (int i = 0; i < I; ++i) acc += hv[i] * wd[i];
+            y[(size_t)r * H + h] = acc;
+            free(wd);
+        }
+    }
+    free(hv);
+}
+
+/* ------------------------------------------------------------------ */
 /* Combine                                                              */
 /* ------------------------------------------------------------------ */
 
