@@ -34,7 +34,8 @@ from group_limited_routing_sigmoid_b200 import workloads as W  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (Beam shape, bf16) and % of HBM / tensor-core roofline"
 # workloads whose dominant kernel streams weights (roofline against HBM)
-HBM_BOUND = ("decode", "tiny", "decode_small", "dense_decode", "dense_tiny")
+HBM_BOUND = ("decode", "tiny", "decode_small", "dense_decode", "dense_tiny", "decode_nvfp4",
+             "tiny_nvfp4", "decode_small_nvfp4")
 TOKEN_BATCHES = 8           # distinct token batches cycled through the steps
 
 
@@ -158,7 +159,7 @@ def workload_config(name: str, wl) -> dict:
     return {"workload": f"beam_{name}", "T": wl.T, "hidden": wl.hidden, "n_experts": wl.n_experts,
             "n_group": wl.n_group, "topk_group": wl.topk_group, "top_k": wl.top_k,
             "inter": wl.inter, "routed_scaling": wl.routed_scaling, "residual_k": wl.residual_k,
-            "post_norm": wl.post_norm}
+            "post_norm": wl.post_norm, "expert_weights": wl.weight_format}
 
 
 def kernels_per_forward(plan: dict, dense: bool, residual: bool) -> int:
@@ -172,6 +173,16 @@ def kernels_per_forward(plan: dict, dense: bool, residual: bool) -> int:
     # exact re-derivation, selection of the re-derived tokens; dispatch:
     # count, scan, permute or row maps; the two GEMMs; combine
     return (4 if plan["router_tensor_cores"] else 2) + 3 + 2 + 1
+
+
+def expert_weight_bytes(wl) -> float:
+    """Bytes per expert weight as stored: bf16, or NVFP4 (4-bit element plus
+    an 8-bit scale per 16 elements)."""
+    return 0.5625 if wl.weight_format == "nvfp4" else 2.0
+
+
+def make_weights(wl, dev, g):
+    return W.make_nvfp4_weights(wl, dev, g) if wl.weight_format == "nvfp4" else W.make_weights(wl, dev, g)
 
 
 def whole_job_tokens_per_s(world: int, steps: int, T: int, ms_max: float) -> float:
@@ -204,7 +215,8 @@ def run_ours(args):
     wl = W.WORKLOADS[args.workload]
     T, H, I, E, k = wl.T, wl.hidden, wl.inter, wl.n_experts, wl.top_k
     g = W.generator(wl, dev)
-    weights = W.make_weights(wl, dev, g)
+    weights = make_weights(wl, dev, g)
+    wb = expert_weight_bytes(wl)
     # distinct token batches per rank (weights identical on every rank)
     tg = torch.Generator(device=dev)
     tg.manual_seed(token_seed(wl, rank))
@@ -308,7 +320,7 @@ def run_ours(args):
     P = T * k
     gate_up_ms = stage_ms["gate_up_gemm"] / max(calls, 1)
     if args.workload in HBM_BOUND:
-        alg_bytes = d_mean * 2 * I * H * 2 + P * H * 2 + P * I * 2
+        alg_bytes = d_mean * 2 * I * H * wb + P * H * 2 + P * I * 2
         achieved = alg_bytes / (gate_up_ms * 1e-3) / 1e9
         roof = {"bound": "hbm",
                 "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -325,6 +337,9 @@ def run_ours(args):
     if plan["ksplit_gate_up"] > 1:
         roof["kernel"] = ("gate_up_gemm (grouped_gemm_kernel<%d,2,2>, split-K %d, + dense_swiglu_kernel)"
                           % (plan["tile_rows"], plan["ksplit_gate_up"]))
+    elif wl.weight_format == "nvfp4":
+        roof["kernel"] = ("gate_up_gemm (grouped_gemm_fp4_kernel<%d,2,0>, NVFP4 weights, grid %d)"
+                          % (plan["tile_rows"], plan["grid"]))
     else:
         roof["kernel"] = ("gate_up_gemm (grouped_gemm_pair_kernel<%d,2,0>, CTA pairs, grid %d)"
                           if plan["cta_pairs"] else
@@ -335,7 +350,7 @@ def run_ours(args):
     roof["nominal_peak"] = nominal
     roof["frac_of_nominal"] = round(roof["achieved"] / nominal, 4)
     d_steps = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(steps_done)) / steps_done
-    step_bytes = (d_steps * 3 * H * I * 2 + (0 if dense else E * H * 4) + T * H * 4
+    step_bytes = (d_steps * 3 * H * I * wb + (0 if dense else E * H * 4) + T * H * 4
                   + (T * H * 8 if wl.residual_k else 0))
     stage_avg = {kname: round(v / max(calls, 1), 4) for kname, v in stage_ms.items()}
 
@@ -354,7 +369,7 @@ def run_ours(args):
         "data": "synthetic (seeded random weights and tokens of the Beam block shape)",
         "config": {**workload_config(args.workload, wl), "token_batches": TOKEN_BATCHES,
                    "distinct_experts_per_step": round(d_steps, 2),
-                   "l2": f"inputs larger than L2: each step streams {d_steps * 3 * H * I * 2 / 1e9:.1f} GB of expert weights",
+                   "l2": f"inputs larger than L2: each step streams {d_steps * 3 * H * I * wb / 1e9:.1f} GB of expert weights",
                    "parallelism": f"{ws} independent replicas (data parallel, no collective on the data path)"},
         "hbm_fraction_whole_step": round(step_bytes / (ms_max / steps_done * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
         "stage_ms": stage_avg,
@@ -397,8 +412,13 @@ def _oracle_on_tokens(wl, weights, x, n_tokens):
     r = oracle.route(xs, rw, bias, wl.n_group, wl.topk_group, wl.top_k)
     cache = {}
     for e in sorted(set(int(v) for v in r.idx.reshape(-1))):
-        cache[e] = (W.bf16_bits(weights["w_gate"][e]), W.bf16_bits(weights["w_up"][e]),
-                    W.bf16_bits(weights["w_down"][e]))
+        if wl.weight_format == "nvfp4":
+            cache[e] = tuple(oracle.Nvfp4Matrix(weights[n + "_codes"][e].cpu().numpy(),
+                                                weights[n + "_scales"][e].cpu().numpy(),
+                                                weights[n + "_global"]) for n in ("gate", "up", "down"))
+        else:
+            cache[e] = (W.bf16_bits(weights["w_gate"][e]), W.bf16_bits(weights["w_up"][e]),
+                        W.bf16_bits(weights["w_down"][e]))
     t0 = time.perf_counter()
     oracle.moe_block(xs, rw, bias, cache.__getitem__, wl.n_group, wl.topk_group, wl.top_k,
                      wl.routed_scaling, gamma=gamma, eps=wl.norm_eps, stream=stream, kstep=wl.residual_k)
@@ -426,7 +446,7 @@ def run_reference(args):
     wl = W.WORKLOADS[args.workload]
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     g = W.generator(wl, dev)
-    weights = W.make_weights(wl, dev, g)
+    weights = make_weights(wl, dev, g)
     tg = torch.Generator(device=dev)
     tg.manual_seed(token_seed(wl, 0))
     x = W.make_tokens(wl, dev, tg)["x"]

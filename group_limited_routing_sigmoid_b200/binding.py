@@ -25,7 +25,8 @@ BEAM_ERR_CHECK = -6
 
 # every entry point declared in include/beam_moe.h
 SYMBOLS = (
-    "beam_moe_create", "beam_moe_create_dense", "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_route_logits",
+    "beam_moe_create", "beam_moe_create_dense", "beam_moe_create_nvfp4", "beam_nvfp4_dequant",
+    "beam_moe_route", "beam_moe_route_static", "beam_moe_router_logits", "beam_moe_route_logits",
     "beam_moe_forward",
     "beam_moe_forward_host", "beam_moe_forward_host_async", "beam_moe_host_join",
     "beam_moe_host_fence",
@@ -59,6 +60,9 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_router_logits.argtypes = [P, P, P, I, P]
         lib.beam_moe_route_static.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P]
         lib.beam_moe_create_dense.argtypes = [P, I, I, P, P, P, P, ctypes.c_float, I]
+        lib.beam_moe_create_nvfp4.argtypes = [ctypes.POINTER(P), I, I, I, I, I, I, F, P, P,
+                                              P, P, F, P, P, F, P, P, F, P, F, I]
+        lib.beam_nvfp4_dequant.argtypes = [P, P, P, ctypes.c_int64, I, P]
         lib.beam_moe_route_logits.argtypes = [P, P, P, I, P, P, P]
         lib.beam_moe_forward.argtypes = [P, P, P, I, P, P, I]
         lib.beam_moe_forward_host.argtypes = [P, P, P, I, P, P, I]
@@ -126,6 +130,22 @@ def route_static(x: torch.Tensor, router_w: torch.Tensor, expert_bias: torch.Ten
     return idx, w
 
 
+def nvfp4_dequant(codes: torch.Tensor, scales: torch.Tensor, stream=None) -> torch.Tensor:
+    """beam_nvfp4_dequant: codes uint8 [..., K/2], scales uint8 [..., K/16] ->
+    bf16 [..., K], each element times its block scale (no per-tensor scale)."""
+    _dev(codes, torch.uint8, "codes")
+    _dev(scales, torch.uint8, "scales")
+    K = codes.shape[-1] * 2
+    rows = codes.numel() // max(codes.shape[-1], 1)
+    if scales.shape[:-1] != codes.shape[:-1] or scales.shape[-1] * 16 != K:
+        raise ValueError("scales must be [..., K/16] for codes [..., K/2]")
+    out = torch.empty(*codes.shape[:-1], K, dtype=torch.bfloat16, device=codes.device)
+    rc = library().beam_nvfp4_dequant(_stream(stream), _ptr(codes), _ptr(scales), rows, K, _ptr(out))
+    if rc != BEAM_OK:
+        raise BeamMoEError(rc, "beam_nvfp4_dequant rejected the call")
+    return out
+
+
 class BeamMoE:
     """One MoE block on the current CUDA device (borrows the weight tensors)."""
 
@@ -181,10 +201,53 @@ class BeamMoE:
         return self
 
     @classmethod
+    def nvfp4(cls, hidden: int, n_experts: int, inter: int, n_group: int, topk_group: int,
+              top_k: int, routed_scaling: float, router_w: torch.Tensor, expert_bias: torch.Tensor,
+              gate: Tuple[torch.Tensor, torch.Tensor, float], up: Tuple[torch.Tensor, torch.Tensor, float],
+              down: Tuple[torch.Tensor, torch.Tensor, float],
+              post_norm_w: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
+              max_tokens: int = 64) -> "BeamMoE":
+        """A block with NVFP4 expert weights (beam_moe_create_nvfp4): each of
+        gate, up, down is (codes uint8 [E, R, K/2], scales uint8 [E, R, K/16],
+        per-tensor scale).  The handle keeps its own copy of the weights."""
+        lib = library()
+        _dev(router_w, torch.float32, "router_w")
+        _dev(expert_bias, torch.float32, "expert_bias")
+        for n, (c, sc, _) in (("gate", gate), ("up", up), ("down", down)):
+            _dev(c, torch.uint8, n + "_codes")
+            _dev(sc, torch.uint8, n + "_scales")
+        if post_norm_w is not None:
+            _dev(post_norm_w, torch.float32, "post_norm_w")
+        self = cls.__new__(cls)
+        self._keep = (router_w, expert_bias, post_norm_w)
+        self.hidden, self.n_experts, self.inter = hidden, n_experts, inter
+        self.top_k = top_k
+        self.max_tokens = max_tokens
+        self.device = router_w.device
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            rc = lib.beam_moe_create_nvfp4(
+                ctypes.byref(h), hidden, n_experts, inter, n_group, topk_group, top_k,
+                float(routed_scaling), _ptr(router_w), _ptr(expert_bias),
+                _ptr(gate[0]), _ptr(gate[1]), float(gate[2]), _ptr(up[0]), _ptr(up[1]), float(up[2]),
+                _ptr(down[0]), _ptr(down[1]), float(down[2]), _ptr(post_norm_w), float(norm_eps),
+                max_tokens)
+        if rc != BEAM_OK:
+            raise BeamMoEError(rc, lib.beam_moe_create_error().decode())
+        self._h = h
+        return self
+
+    @classmethod
     def from_workload(cls, wl, weights, max_tokens: Optional[int] = None) -> "BeamMoE":
         if wl.n_experts == 1:
             return cls.dense(wl.hidden, wl.inter, weights["w_gate"][0], weights["w_up"][0],
                              weights["w_down"][0], weights.get("gamma"), wl.norm_eps,
+                             max_tokens or wl.T)
+        if getattr(wl, "weight_format", "bf16") == "nvfp4":
+            t = lambda n: (weights[n + "_codes"], weights[n + "_scales"], weights[n + "_global"])
+            return cls.nvfp4(wl.hidden, wl.n_experts, wl.inter, wl.n_group, wl.topk_group, wl.top_k,
+                             wl.routed_scaling, weights["router_w"], weights["bias"], t("gate"),
+                             t("up"), t("down"), weights.get("gamma"), wl.norm_eps,
                              max_tokens or wl.T)
         return cls(wl.hidden, wl.n_experts, wl.inter, wl.n_group, wl.topk_group, wl.top_k,
                    wl.routed_scaling, weights["router_w"], weights["bias"], weights["w_gate"],

@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "beam_moe.h"
+#include "fp4.cuh"
 #include "kernels.cuh"
 
 using namespace beam;
@@ -27,6 +28,13 @@ struct beam_moe {
     void *ws;
     size_t ws_bytes;
     int dense;               // 1: dense SwiGLU MLP (one expert, no router)
+    int fp4;                 // 1: NVFP4 expert weights
+    // NVFP4: the caller's row-major tensors (read at create only), the
+    // tiled copy the GEMMs stream (owned), and its operand sets
+    const uint8_t *fp4_codes_in[3], *fp4_scales_in[3];
+    float fp4_global[3];
+    uint8_t *fp4_buf;
+    Fp4Operands fp4_gate_up, fp4_down;
     float *partial;          // [nslice_max * T_max * E]
     float *split;            // dense layers: FP32 split-K partial sums
     int32_t *idx;            // [P]
@@ -338,6 +346,15 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
     p.gather = h->gather_rows < 0 ? (p.tile_rows <= 32 ? 1 : 0) : h->gather_rows;
     p.ksplit_gate_up = 1;
     p.ksplit_down = 1;
+    if (h->fp4) {
+        // NVFP4 weights: the single-CTA kernel with token tiles of up to 128
+        // rows from the sorted copy, one weight block per down item
+        if (p.tile_rows > 128) p.tile_rows = 128;
+        p.cta_pairs = 0;
+        p.grid = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
+        p.down_paired = 0;
+        p.gather = 0;
+    }
     if (h->dense) {
         // one expert: with decode-sized T the weight tiles alone give too few
         // work items, so K is split and FP32 partial sums are reduced after
@@ -550,10 +567,13 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.K = h->H;
     g.R = h->I;
     g.out = h->hbuf;
-    e = use_pair ? launch_grouped_gemm_pair(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx, g,
-                                            grid, s)
-                 : launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx, g,
-                                       grid, s);
+    if (h->fp4)
+        e = launch_grouped_gemm_fp4(GemmKind::kGateUp, BN, h->fp4_gate_up, *bx, g, grid, s);
+    else
+        e = use_pair ? launch_grouped_gemm_pair(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx,
+                                                g, grid, s)
+                     : launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx, g,
+                                           grid, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "gate/up GEMM launch");
     prof_mark(h, s, 3);
     g.K = h->I;
@@ -561,8 +581,11 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.out = h->ybuf;
     g.gather = 0;
     const GemmKind dk = plan.down_paired ? GemmKind::kDownPaired : GemmKind::kDown;
-    e = use_pair ? launch_grouped_gemm_pair(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s)
-                 : launch_grouped_gemm(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s);
+    if (h->fp4)
+        e = launch_grouped_gemm_fp4(GemmKind::kDown, BN, h->fp4_down, h->tm_h, g, grid, s);
+    else
+        e = use_pair ? launch_grouped_gemm_pair(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s)
+                     : launch_grouped_gemm(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "down GEMM launch");
     prof_mark(h, s, 4);
 
@@ -722,6 +745,46 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     if (e == cudaSuccess) e = cudaMemset(h->check_where, 0x7f, sizeof(int));
     if (e == cudaSuccess) e = prepare_grouped_gemm(n_experts);
     if (e == cudaSuccess) e = prepare_dispatch(n_experts);
+    if (e == cudaSuccess && h->fp4) {
+        // the tiled copy of the three NVFP4 tensors (gate, up: [E*I, H];
+        // down: [E*H, I]), made once on the legacy default stream
+        const long long rows[3] = {(long long)E * inter, (long long)E * inter, (long long)E * hidden};
+        const int kdim[3] = {hidden, hidden, inter};
+        size_t code_off[3], scale_off[3], total = 0;
+        for (int i = 0; i < 3; ++i) {
+            code_off[i] = total;
+            total = align_up(total + (size_t)rows[i] * kdim[i] / 2, 256);
+            scale_off[i] = total;
+            total = align_up(total + (size_t)rows[i] * kdim[i] / 16, 256);
+        }
+        e = cudaMalloc(&h->fp4_buf, total);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            h->fp4_buf = nullptr;
+            int rc = fail(nullptr, BEAM_ERR_OOM, "NVFP4 weight copy of %zu bytes: %s", total,
+                          cudaGetErrorString(e));
+            cudaFree(h->ws);
+            delete h;
+            return rc;
+        }
+        Fp4Tensor t[3];
+        for (int i = 0; i < 3 && e == cudaSuccess; ++i) {
+            t[i].codes = h->fp4_buf + code_off[i];
+            t[i].scales = h->fp4_buf + scale_off[i];
+            t[i].global = h->fp4_global[i];
+            e = launch_fp4_repack(h->fp4_codes_in[i], h->fp4_scales_in[i], rows[i], kdim[i],
+                                  h->fp4_buf + code_off[i], h->fp4_buf + scale_off[i], 0);
+        }
+        h->fp4_gate_up.a[0] = t[0];
+        h->fp4_gate_up.a[1] = t[1];
+        h->fp4_gate_up.row_tiles = inter / kFp4TileRows;
+        h->fp4_gate_up.k_steps = hidden / kFp4TileK;
+        h->fp4_down.a[0] = t[2];
+        h->fp4_down.a[1] = t[2];
+        h->fp4_down.row_tiles = hidden / kFp4TileRows;
+        h->fp4_down.k_steps = inter / kFp4TileK;
+        if (e == cudaSuccess) e = prepare_grouped_gemm_fp4();
+    }
     if (!h->dense) {
         if (e == cudaSuccess) e = prepare_router_mma();
         if (e == cudaSuccess) e = prepare_router_fix(hidden);
@@ -732,20 +795,22 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     if (e == cudaSuccess) e = cudaStreamSynchronize(0);
     if (e != cudaSuccess) {
         int rc = cuda_fail(nullptr, e, "workspace / kernel set-up");
+        if (h->fp4_buf) cudaFree(h->fp4_buf);
         cudaFree(h->ws);
         delete h;
         return rc;
     }
 
-    bool ok = make_map(&h->tm_gate, h->w_gate, E * inter, hidden, 128) &&
-              make_map(&h->tm_up, h->w_up, E * inter, hidden, 128) &&
-              make_map(&h->tm_down, h->w_down, E * hidden, inter, 128);
+    bool ok = h->fp4 || (make_map(&h->tm_gate, h->w_gate, E * inter, hidden, 128) &&
+                         make_map(&h->tm_up, h->w_up, E * inter, hidden, 128) &&
+                         make_map(&h->tm_down, h->w_down, E * hidden, inter, 128));
     if (!h->dense) ok = ok && make_map(&h->tm_wcat, h->wcat, E, 3 * (uint64_t)hidden, 128);
     for (int i = 0; i < 6 && ok; ++i) {
         ok = make_map(&h->tm_h.m[i], h->hbuf, P, inter, 8u << i);
         if (ok && !h->dense) ok = make_map(&h->tm_xp.m[i], h->xp, P, hidden, 8u << i);
     }
     if (!ok) {
+        if (h->fp4_buf) cudaFree(h->fp4_buf);
         cudaFree(h->ws);
         delete h;
         return fail(nullptr, BEAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
@@ -761,12 +826,72 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     if (e != cudaSuccess) {
         int rc = cuda_fail(nullptr, e, "host-path streams / events");
         release_host_path(h);
+        if (h->fp4_buf) cudaFree(h->fp4_buf);
         cudaFree(h->ws);
         delete h;
         return rc;
     }
     *out = h;
     return BEAM_OK;
+}
+
+// Argument checks shared by the sparse-block create calls: shapes, routing
+// parameters, the router and norm pointers.
+int check_sparse_args(int hidden, int n_experts, int inter, int n_group, int topk_group, int top_k,
+                      float routed_scaling, const float *router_w, const float *expert_bias,
+                      const float *post_norm_w, float norm_eps, int max_tokens)
+{
+    if (hidden <= 0 || n_experts <= 0 || inter <= 0 || n_group <= 0 || max_tokens < 1)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "sizes must be positive");
+    if (n_experts % n_group != 0)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "n_experts %% n_group != 0");
+    const int gsize = n_experts / n_group;
+    if (gsize < 2) return fail(nullptr, BEAM_ERR_INVALID_ARG, "group size must be >= 2");
+    if (topk_group < 1 || topk_group > n_group)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "topk_group outside [1, n_group]");
+    if (top_k < 1 || top_k > topk_group * gsize)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "top_k outside [1, topk_group * group size]");
+    if (!(routed_scaling == routed_scaling) || !(norm_eps >= 0.f))
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "routed_scaling / norm_eps not valid");
+    if (!router_w || !expert_bias)
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "weight pointer is NULL");
+    if (!aligned16(router_w) || !aligned16(expert_bias) || (post_norm_w && !aligned16(post_norm_w)))
+        return fail(nullptr, BEAM_ERR_INVALID_ARG, "weight pointers must be 16-byte aligned");
+    if (hidden % 128 != 0 || inter % 128 != 0)
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "hidden and inter must be multiples of 128");
+    if (hidden > 8192)
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "hidden > 8192");
+    if (n_experts % 32 != 0 || n_experts > 1024 || !is_pow2(n_experts / 32))
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED,
+                    "n_experts must be 32 x a power of two, at most 1024");
+    const int epl = n_experts / 32;
+    if (gsize % epl != 0 || !is_pow2(gsize / epl) || n_group > 32)
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "group size not supported by the router kernel");
+    if (top_k > 32) return fail(nullptr, BEAM_ERR_UNSUPPORTED, "top_k > 32");
+    if ((long long)max_tokens * top_k > (1LL << 30))
+        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "max_tokens * top_k too large");
+    return BEAM_OK;
+}
+
+beam_moe *new_sparse_handle(int hidden, int n_experts, int inter, int n_group, int topk_group,
+                            int top_k, float routed_scaling, const float *router_w,
+                            const float *expert_bias, const float *post_norm_w, float norm_eps,
+                            int max_tokens)
+{
+    beam_moe *h = new beam_moe();   // value-initialised: every plain field starts at zero
+    h->H = hidden;
+    h->E = n_experts;
+    h->I = inter;
+    h->n_group = n_group;
+    h->topk_group = topk_group;
+    h->top_k = top_k;
+    h->scaling = routed_scaling;
+    h->router_w = router_w;
+    h->bias = expert_bias;
+    h->gamma = post_norm_w;
+    h->eps = norm_eps;
+    h->max_tokens = max_tokens;
+    return h;
 }
 
 }  // namespace
@@ -783,54 +908,68 @@ int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n
     g_create_err[0] = 0;
     if (!out) return fail(nullptr, BEAM_ERR_INVALID_ARG, "out is NULL");
     *out = nullptr;
-    if (hidden <= 0 || n_experts <= 0 || inter <= 0 || n_group <= 0 || max_tokens < 1)
-        return fail(nullptr, BEAM_ERR_INVALID_ARG, "sizes must be positive");
-    if (n_experts % n_group != 0)
-        return fail(nullptr, BEAM_ERR_INVALID_ARG, "n_experts %% n_group != 0");
-    const int gsize = n_experts / n_group;
-    if (gsize < 2) return fail(nullptr, BEAM_ERR_INVALID_ARG, "group size must be >= 2");
-    if (topk_group < 1 || topk_group > n_group)
-        return fail(nullptr, BEAM_ERR_INVALID_ARG, "topk_group outside [1, n_group]");
-    if (top_k < 1 || top_k > topk_group * gsize)
-        return fail(nullptr, BEAM_ERR_INVALID_ARG, "top_k outside [1, topk_group * group size]");
-    if (!(routed_scaling == routed_scaling) || !(norm_eps >= 0.f))
-        return fail(nullptr, BEAM_ERR_INVALID_ARG, "routed_scaling / norm_eps not valid");
-    if (!router_w || !expert_bias || !w_gate || !w_up || !w_down)
+    int rc = check_sparse_args(hidden, n_experts, inter, n_group, topk_group, top_k, routed_scaling,
+                               router_w, expert_bias, post_norm_w, norm_eps, max_tokens);
+    if (rc != BEAM_OK) return rc;
+    if (!w_gate || !w_up || !w_down)
         return fail(nullptr, BEAM_ERR_INVALID_ARG, "weight pointer is NULL");
-    if (!aligned16(router_w) || !aligned16(expert_bias) || !aligned16(w_gate) || !aligned16(w_up) ||
-        !aligned16(w_down) || (post_norm_w && !aligned16(post_norm_w)))
+    if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down))
         return fail(nullptr, BEAM_ERR_INVALID_ARG, "weight pointers must be 16-byte aligned");
-    if (hidden % 128 != 0 || inter % 128 != 0)
-        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "hidden and inter must be multiples of 128");
-    if (hidden > 8192)
-        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "hidden > 8192");
-    if (n_experts % 32 != 0 || n_experts > 1024 || !is_pow2(n_experts / 32))
-        return fail(nullptr, BEAM_ERR_UNSUPPORTED,
-                    "n_experts must be 32 x a power of two, at most 1024");
-    const int epl = n_experts / 32;
-    if (gsize % epl != 0 || !is_pow2(gsize / epl) || n_group > 32)
-        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "group size not supported by the router kernel");
-    if (top_k > 32) return fail(nullptr, BEAM_ERR_UNSUPPORTED, "top_k > 32");
-    if ((long long)max_tokens * top_k > (1LL << 30))
-        return fail(nullptr, BEAM_ERR_UNSUPPORTED, "max_tokens * top_k too large");
-
-    beam_moe *h = new beam_moe();   // value-initialised: every plain field starts at zero
-    h->H = hidden;
-    h->E = n_experts;
-    h->I = inter;
-    h->n_group = n_group;
-    h->topk_group = topk_group;
-    h->top_k = top_k;
-    h->scaling = routed_scaling;
-    h->router_w = router_w;
-    h->bias = expert_bias;
-    h->gamma = post_norm_w;
+    beam_moe *h = new_sparse_handle(hidden, n_experts, inter, n_group, topk_group, top_k,
+                                    routed_scaling, router_w, expert_bias, post_norm_w, norm_eps,
+                                    max_tokens);
     h->w_gate = static_cast<const __nv_bfloat16 *>(w_gate);
     h->w_up = static_cast<const __nv_bfloat16 *>(w_up);
     h->w_down = static_cast<const __nv_bfloat16 *>(w_down);
-    h->eps = norm_eps;
-    h->max_tokens = max_tokens;
     return finish_create(h, out);
+}
+
+int beam_moe_create_nvfp4(beam_moe_t *out, int hidden, int n_experts, int inter, int n_group,
+                          int topk_group, int top_k, float routed_scaling, const float *router_w,
+                          const float *expert_bias, const uint8_t *gate_codes,
+                          const uint8_t *gate_scales, float gate_global, const uint8_t *up_codes,
+                          const uint8_t *up_scales, float up_global, const uint8_t *down_codes,
+                          const uint8_t *down_scales, float down_global, const float *post_norm_w,
+                          float norm_eps, int max_tokens)
+{
+    g_create_err[0] = 0;
+    if (!out) return fail(nullptr, BEAM_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    int rc = check_sparse_args(hidden, n_experts, inter, n_group, topk_group, top_k, routed_scaling,
+                               router_w, expert_bias, post_norm_w, norm_eps, max_tokens);
+    if (rc != BEAM_OK) return rc;
+    const uint8_t *ptrs[6] = {gate_codes, gate_scales, up_codes, up_scales, down_codes, down_scales};
+    for (const uint8_t *q : ptrs) {
+        if (!q) return fail(nullptr, BEAM_ERR_INVALID_ARG, "NVFP4 tensor pointer is NULL");
+        if (!aligned16(q))
+            return fail(nullptr, BEAM_ERR_INVALID_ARG, "NVFP4 tensor pointers must be 16-byte aligned");
+    }
+    const float gl[3] = {gate_global, up_global, down_global};
+    for (float g : gl)
+        if (!(std::isfinite(g)))
+            return fail(nullptr, BEAM_ERR_INVALID_ARG, "per-tensor scales must be finite");
+    beam_moe *h = new_sparse_handle(hidden, n_experts, inter, n_group, topk_group, top_k,
+                                    routed_scaling, router_w, expert_bias, post_norm_w, norm_eps,
+                                    max_tokens);
+    h->fp4 = 1;
+    for (int i = 0; i < 3; ++i) {
+        h->fp4_codes_in[i] = ptrs[2 * i];
+        h->fp4_scales_in[i] = ptrs[2 * i + 1];
+        h->fp4_global[i] = gl[i];
+    }
+    return finish_create(h, out);
+}
+
+int beam_nvfp4_dequant(void *stream, const uint8_t *codes, const uint8_t *scales, long long rows,
+                       int K, void *out)
+{
+    if (rows < 0 || K <= 0 || K % 16 != 0) return BEAM_ERR_INVALID_ARG;
+    if (rows == 0) return BEAM_OK;
+    if (!codes || !scales || !out || !aligned16(codes) || !aligned16(out)) return BEAM_ERR_INVALID_ARG;
+    const cudaError_t e = launch_fp4_dequant(codes, scales, rows * (long long)K,
+                                             static_cast<__nv_bfloat16 *>(out),
+                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BEAM_OK : BEAM_ERR_CUDA;
 }
 
 int beam_moe_create_dense(beam_moe_t *out, int hidden, int inter, const void *w_gate,
@@ -1224,6 +1363,7 @@ int beam_moe_destroy(beam_moe_t h)
     prof_release(h);
     release_host_path(h);
     if (h->ws) cudaFree(h->ws);
+    if (h->fp4_buf) cudaFree(h->fp4_buf);
     if (prev >= 0 && prev != h->device) cudaSetDevice(prev);
     delete h;
     return e == cudaSuccess ? BEAM_OK : BEAM_ERR_CUDA;

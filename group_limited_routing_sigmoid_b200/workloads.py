@@ -102,6 +102,10 @@ WORKLOADS: Dict[str, Workload] = {
     "tiny_nvfp4": Workload("tiny_nvfp4", T=64, hidden=256, n_experts=32, n_group=8, topk_group=4,
                            top_k=8, inter=128, weight_format="nvfp4"),
     "decode_nvfp4": Workload("decode_nvfp4", T=64, weight_format="nvfp4", **_BEAM),
+    # profiling-sized NVFP4 case: 32 Beam-shaped experts (0.7 GB of weights), 8 tokens
+    "decode_small_nvfp4": Workload("decode_small_nvfp4", T=8, hidden=5120, n_experts=32, n_group=8,
+                                   topk_group=4, top_k=8, inter=2560, routed_scaling=2.5,
+                                   weight_format="nvfp4"),
 }
 
 

@@ -123,6 +123,52 @@ int beam_moe_create_dense(beam_moe_t *out, int hidden, int inter, const void *w_
                           float norm_eps, int max_tokens);
 
 /*
+ * Create a handle for one MoE block whose expert weights are NVFP4, the
+ * 4-bit format the Beam launch blog recommends for Blackwell GPUs (launch
+ * blog "Introducing Beam", section "Mixture of Experts"): each weight is an
+ * E2M1 element times the FP8 E4M3 scale of its block of 16 consecutive
+ * elements along the row, times one FP32 scale per tensor.
+ *
+ * Arguments as beam_moe_create, with each expert tensor given as
+ *   *_codes   uint8 [E, R, K/2]: element 2j of a row in the low nibble of
+ *             byte j, 2j + 1 in the high nibble (a nibble: sign bit 3,
+ *             exponent bits 2..1 with bias 1, mantissa bit 0);
+ *   *_scales  uint8 [E, R, K/16]: E4M3 scale of elements 16b .. 16b + 15;
+ *   *_global  the tensor's FP32 scale (finite);
+ * with R = inter, K = hidden for gate and up, R = hidden, K = inter for
+ * down.  Device pointers, 16-byte aligned, read during this call only: the
+ * handle allocates and keeps its own tiled copy (0.5625 bytes per weight)
+ * made by kernels on the legacy default stream, which this call waits for.
+ * The grouped GEMMs decode the weights to bf16 (exact: an E2M1 x E4M3
+ * product has at most 6 significant bits) for the tensor cores and apply the
+ * per-tensor scales to the FP32 accumulators.
+ * The handle takes the same calls as a bf16 handle.  Differences: token
+ * tiles of at most 128 rows (tile_rows 256 acts as 128); the cta_pairs,
+ * gather_rows, token_stages and down_pair tunings are ignored (single-CTA
+ * kernels over the sorted activations).  Errors as beam_moe_create, and
+ * BEAM_ERR_OOM if the tiled copy cannot be allocated.
+ */
+int beam_moe_create_nvfp4(beam_moe_t *out, int hidden, int n_experts, int inter, int n_group,
+                          int topk_group, int top_k, float routed_scaling, const float *router_w,
+                          const float *expert_bias, const uint8_t *gate_codes,
+                          const uint8_t *gate_scales, float gate_global, const uint8_t *up_codes,
+                          const uint8_t *up_scales, float up_global, const uint8_t *down_codes,
+                          const uint8_t *down_scales, float down_global, const float *post_norm_w,
+                          float norm_eps, int max_tokens);
+
+/*
+ * Decode rows x K NVFP4 elements (codes uint8 [rows, K/2], scales uint8
+ * [rows, K/16], laid out as for beam_moe_create_nvfp4) to bf16 [rows, K]:
+ * each element times its block scale, exact; no per-tensor scale.  The same
+ * decode the NVFP4 grouped GEMMs run.  Device pointers; codes and out
+ * 16-byte aligned.  K a positive multiple of 16, rows >= 0 (0: nothing to
+ * do).  Needs no handle.  Asynchronous on `stream`.  Returns
+ * BEAM_ERR_INVALID_ARG for bad arguments, BEAM_ERR_CUDA if the launch fails.
+ */
+int beam_nvfp4_dequant(void *stream, const uint8_t *codes, const uint8_t *scales, long long rows,
+                       int K, void *out);
+
+/*
  * Route T tokens: the router step alone.
  * x         bf16 [T, H].
  * topk_idx  int32 [T, top_k] (out): chosen experts, in descending biased

@@ -125,6 +125,10 @@ def check_block(wl: W.Workload, d: dict, moe, sample: Optional[torch.Tensor] = N
     gamma = None if d.get("gamma") is None else d["gamma"].cpu().numpy()
 
     def fetch(e):
+        if "gate_codes" in d:   # NVFP4 expert weights
+            return tuple(oracle.Nvfp4Matrix(d[n + "_codes"][e].cpu().numpy(),
+                                            d[n + "_scales"][e].cpu().numpy(), d[n + "_global"])
+                         for n in ("gate", "up", "down"))
         return (W.bf16_bits(d["w_gate"][e]), W.bf16_bits(d["w_up"][e]), W.bf16_bits(d["w_down"][e]))
 
     t0 = time.time()

@@ -1,0 +1,95 @@
+"""NVFP4 expert weights (beam_moe_create_nvfp4) against the oracle's NVFP4
+expert: the decode the GEMMs run, bit for bit, over every code byte and
+every finite scale byte; the block over ragged token counts, every token
+tile, fewer CTAs than work items, and the post-norm and residual update; and
+the Beam decode shape (H=5120, 256 experts, I=2560, 64 tokens) in full."""
+import dataclasses
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from group_limited_routing_sigmoid_b200 import workloads as W
+from group_limited_routing_sigmoid_b200.binding import BeamMoE, nvfp4_dequant
+from group_limited_routing_sigmoid_b200.build import build
+
+from parity import check_block
+
+pytestmark = pytest.mark.gpu
+
+
+def setup_module(_):
+    build(quiet=True)
+
+
+def _log(case, rep, plan):
+    path = os.environ.get("BEAM_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": case, **rep.__dict__, "plan": plan}) + "\n")
+
+
+def test_dequant_is_exact_for_every_code_and_scale():
+    # rows of 512 elements: every code byte twice per row; one scale byte per
+    # 16-element block, cycling through the 254 finite E4M3 bytes
+    finite = np.array([b for b in range(256) if b not in (0x7F, 0xFF)], np.uint8)
+    rows, K = 254, 512
+    codes = np.tile(np.concatenate([np.arange(256, dtype=np.uint8)] * 1), (rows, 1))
+    scales = finite[(np.arange(rows)[:, None] + np.arange(K // 16)[None, :] * 7) % len(finite)]
+    got = nvfp4_dequant(torch.from_numpy(codes).cuda(), torch.from_numpy(scales.astype(np.uint8)).cuda())
+    torch.cuda.synchronize()
+    e2m1 = np.array([oracle.e2m1_value(c) for c in range(16)])
+    e4m3 = np.array([oracle.e4m3_value(b) for b in range(256)])
+    c = codes.astype(np.int64)
+    nib = np.stack([c & 15, c >> 4], axis=-1).reshape(rows, K)
+    ref = e2m1[nib] * np.repeat(e4m3[scales], 16, axis=1)
+    # the products have at most 6 significant bits: exact in bf16
+    ref_bits = W.bf16_bits(torch.from_numpy(ref).to(torch.bfloat16))
+    assert np.array_equal(oracle.bf16_to_f64(ref_bits), ref)
+    got_bits = W.bf16_bits(got.cpu())
+    # equal as values (a zero may carry either sign)
+    np.testing.assert_array_equal(oracle.bf16_to_f64(got_bits), ref)
+
+
+# (T, GEMM CTAs (0 = one per SM), largest token tile (0 = auto), post-norm + residual)
+CASES = [(1, 0, 0, False), (5, 0, 0, False), (64, 0, 0, False), (64, 7, 0, False),
+         (300, 0, 0, False), (300, 0, 16, False), (300, 0, 32, False), (1000, 0, 64, False),
+         (1000, 0, 128, False), (1000, 0, 256, False), (1000, 3, 0, False), (64, 0, 0, True),
+         (300, 0, 0, True)]
+
+
+@pytest.mark.parametrize("T,ctas,tile,resid", CASES)
+def test_nvfp4_block(T, ctas, tile, resid):
+    wl = W.WORKLOADS["tiny_nvfp4"]
+    if resid:
+        wl = dataclasses.replace(wl, post_norm=True, residual_k=20)
+    g = W.generator(wl, "cuda")
+    d = W.make_nvfp4_weights(wl, "cuda", g)
+    d.update(W.make_tokens(wl, "cuda", g, T=T))
+    moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    moe.set_gemm_tuning(ctas, tile, -1, 1)
+    plan = moe.launch_plan(T)
+    assert plan["cta_pairs"] == 0 and plan["gather_rows"] == 0 and plan["tile_rows"] <= 128
+    rep = check_block(wl, d, moe)
+    _log(f"nvfp4_T{T}_ctas{ctas}_tile{tile}_resid{resid}", rep, plan)
+    assert rep.ok(), rep
+    if resid:
+        assert rep.res_rel_fro is not None
+    moe.close()
+
+
+def test_nvfp4_beam_decode():
+    wl = W.WORKLOADS["decode_nvfp4"]
+    g = W.generator(wl, "cuda")
+    d = W.make_nvfp4_weights(wl, "cuda", g)
+    d.update(W.make_tokens(wl, "cuda", g))
+    moe = BeamMoE.from_workload(wl, d)
+    rep = check_block(wl, d, moe)
+    _log("beam_decode_nvfp4", rep, moe.launch_plan(wl.T))
+    assert rep.ok(), rep
+    moe.close()
+    del d, moe
+    torch.cuda.empty_cache()
