@@ -11,6 +11,12 @@ rank runs its own replica on its own batches (tokens are independent: weak
 scaling, no data-path collective); ``value`` is all ranks' tokens over the
 slowest rank's device time.
 
+``--workload`` picks one of the seeded workloads: the Beam block at decode
+(``decode``, the default) and prefill sizes, skewed routing, the long
+sequence with post-norm and residual, the dense layers, and the same decode
+batch with NVFP4 expert weights (``decode_nvfp4``, whose HBM roofline counts
+0.5625 bytes per weight).
+
 ``--impl reference`` times the plain CPU oracle on the host cores instead,
 one bounded sample of tokens per step (rank 0 only).
 """

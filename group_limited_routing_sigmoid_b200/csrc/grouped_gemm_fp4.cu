@@ -14,17 +14,21 @@
 //                 by the block scale: every product has at most 6
 //                 significant bits, so it is exact) and writes it to TMEM
 //                 lane r with tcgen05.st;
-//   warp 1        MMA issuer: A (the decoded weights) from TMEM, four stages
-//                 deep, B (the token rows) from the shared-memory stage;
+//   warps 1, 22   MMA issuers (lane 0): A (the decoded weights) from TMEM,
+//                 four stages deep, B (the token rows) from the shared-memory
+//                 stage.  gate|up: warp 1 issues the gate MMAs and warp 22
+//                 the up MMAs; down: warp 1 alone.  At 16-row token tiles
+//                 the issuing thread, not the tensor pipe, sets the pace (an
+//                 issued MMA of this shape is ~100 cycles of issue for a few
+//                 cycles of tensor work), so two issuers cut the gate|up time
+//                 by about a tenth; splitting down the same way was slower;
 //   warps 2..5    epilogue, one per quadrant: as the bf16 kernel, with the
 //                 FP32 accumulators first multiplied by the per-tensor scales.
 //
-// Accumulator chains: an MMA that adds into an accumulator waits for the
-// previous MMA into it, so a token tile of 16 rows (an MMA of a few cycles of
-// tensor-core work) would leave the tensor core waiting on that dependence.
-// Small tiles therefore spread the four K sub-steps of a stage over CHAINS
-// independent accumulators per matrix, which the epilogue adds in chain order
-// in FP32.
+// Accumulator chains: small tiles spread the four K sub-steps of a stage over
+// CHAINS independent accumulators per matrix, so consecutive MMAs never add
+// into the same accumulator; the epilogue adds the chains in chain order in
+// FP32.
 //
 // Why TMEM for A: a decode token tile has 16 rows, so each MMA reads a
 // 128 x 16 weight block for a 16 x 16 token block.  Staging the decoded

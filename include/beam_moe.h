@@ -28,7 +28,9 @@
  * Memory.  Every tensor argument is a DEVICE pointer unless its name ends in
  * _host.  The caller owns all of them.  Weights are borrowed by the handle and
  * must stay valid and unchanged until beam_moe_destroy.  The handle owns only
- * its workspace (sized by max_tokens at create time) and its TMA descriptors.
+ * its workspace (sized by max_tokens at create time) and its TMA descriptors
+ * (an NVFP4 handle also owns its tiled copy of the expert weights, whose
+ * inputs are read at create only).
  * Device pointers must be 16-byte aligned.  Layouts are row-major, C order.
  *
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL: the legacy
