@@ -784,6 +784,8 @@ int finish_create(beam_moe *h, beam_moe_t *out)
         h->fp4_down.row_tiles = hidden / kFp4TileRows;
         h->fp4_down.k_steps = inter / kFp4TileK;
         if (e == cudaSuccess) e = prepare_grouped_gemm_fp4();
+        for (int i = 0; i < 3; ++i)   // read at create only: not kept
+            h->fp4_codes_in[i] = h->fp4_scales_in[i] = nullptr;
     }
     if (!h->dense) {
         if (e == cudaSuccess) e = prepare_router_mma();
