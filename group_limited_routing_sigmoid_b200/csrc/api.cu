@@ -767,7 +767,7 @@ int finish_create(beam_moe *h, beam_moe_t *out)
             delete h;
             return rc;
         }
-        Fp4Tensor t[3];
+        Fp4Tensor t[3] = {};
         for (int i = 0; i < 3 && e == cudaSuccess; ++i) {
             t[i].codes = h->fp4_buf + code_off[i];
             t[i].scales = h->fp4_buf + scale_off[i];
