@@ -43,6 +43,11 @@ METRIC = "MoE-layer tokens/s (Beam shape, bf16) and % of HBM / tensor-core roofl
 HBM_BOUND = ("decode", "tiny", "decode_small", "dense_decode", "dense_tiny", "decode_nvfp4",
              "tiny_nvfp4", "decode_small_nvfp4")
 TOKEN_BATCHES = 8           # distinct token batches cycled through the steps
+MIN_WINDOWS = 5             # headline windows of --steps steps, at least
+MAX_WINDOWS = 200
+TIMED_SPAN_S = 2.0          # headline windows cover about this much device time
+STAGE_WINDOWS = 7           # stage-timed windows (median per stage)
+E2E_WINDOWS = 7             # host-buffer windows (median)
 
 
 def peaks():
@@ -261,34 +266,53 @@ def run_ours(args):
 
     stream = torch.cuda.current_stream(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local)
-    if ws > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    with sampler:
+
+    def window(first: int, n: int, fn) -> float:
+        """Device time (ms) of n steps fn(first + i), bracketed by a barrier
+        and a synchronize on both sides; the slowest rank's time."""
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
         ev0.record(stream)
-        for i in range(args.steps):
-            step(args.warmup + i)
+        for i in range(n):
+            fn(first + i)
         ev1.record(stream)
         torch.cuda.synchronize(dev)
-    if ws > 1:
-        dist.barrier()
-    ms = ev0.elapsed_time(ev1)
+        if ws > 1:
+            dist.barrier()
+        return max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
+
+    # headline: windows of exactly --steps steps each, enough of them (at
+    # least MIN_WINDOWS) that the timed span covers TIMED_SPAN_S seconds of
+    # clock samples; every rank takes the same number (decided from the
+    # slowest rank's first window)
+    sampler = ClockSampler(local)
+    win_ms = []
+    with sampler:
+        win_ms.append(window(args.warmup, args.steps, step))
+        n_win = max(MIN_WINDOWS, min(MAX_WINDOWS, int(TIMED_SPAN_S * 1e3 / max(win_ms[0], 1e-3)) + 1))
+        for w in range(1, n_win):
+            win_ms.append(window(args.warmup + w * args.steps, args.steps, step))
     rederived = moe.router_stats()
     if moe.get_status() != 0:
         raise SystemExit("a device-side wait ran out during the timed region")
-    ms_max = max_over_ranks(ms, dist, dev)
+    ms_max = statistics.median(win_ms)
 
-    # per-stage device times: the same steps again with the library's CUDA
-    # events around each stage (kept out of the headline region: an event
-    # between two kernels stops the second from starting early)
+    # per-stage device times: windows of the same steps again with the
+    # library's CUDA events around each stage (kept out of the headline
+    # region: an event between two kernels stops the second from starting
+    # early); each stage's per-launch time is the median over the windows
     stage_steps = min(args.steps, 50)
-    moe.profile_begin(stage_steps)
-    for i in range(stage_steps):
-        step(args.warmup + i)
-    calls, stage_ms = moe.profile_end()
+    stage_windows = []
+    for w in range(min(n_win, STAGE_WINDOWS)):
+        moe.profile_begin(stage_steps)
+        for i in range(stage_steps):
+            step(args.warmup + i)
+        calls, st = moe.profile_end()
+        stage_windows.append({kname: v / max(calls, 1) for kname, v in st.items()})
     if moe.get_status() != 0:
         raise SystemExit("a device-side wait ran out during the stage-timed steps")
+    stage_med = {kname: statistics.median(sw[kname] for sw in stage_windows) for kname in stage_windows[0]}
 
     # end to end through the host-buffer entry points (pinned buffers): each
     # step copies its batch in and its result out; the pipelined call lets a
@@ -304,27 +328,33 @@ def run_ours(args):
                                residual_host=res_host[j] if res_host else None,
                                k=max(1, wl.residual_k))
 
+    def e2e_window(first: int, n: int) -> float:
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        moe.host_fence()          # the first copy in starts after ev0
+        for i in range(n):
+            e2e_step(first + i)
+        moe.host_join()           # ev1 after the last copy out
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        if ws > 1:
+            dist.barrier()
+        return max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
+
     for i in range(args.warmup):
         e2e_step(i)
     moe.host_join()
-    if ws > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    ev0.record(stream)
-    moe.host_fence()          # the first copy in starts after ev0
-    for i in range(e2e_steps):
-        e2e_step(i)
-    moe.host_join()           # ev1 after the last copy out
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
+    e2e_win = [e2e_window(w * e2e_steps, e2e_steps) for w in range(min(n_win, E2E_WINDOWS))]
+    e2e_ms = statistics.median(e2e_win)
 
     # roofline of the dominant kernel
     pk = peaks()
     steps_done = args.steps
     d_mean = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(stage_steps)) / stage_steps
     P = T * k
-    gate_up_ms = stage_ms["gate_up_gemm"] / max(calls, 1)
+    gate_up_ms = stage_med["gate_up_gemm"]
     if args.workload in HBM_BOUND:
         alg_bytes = d_mean * 2 * I * H * wb + P * H * 2 + P * I * 2
         achieved = alg_bytes / (gate_up_ms * 1e-3) / 1e9
@@ -355,10 +385,14 @@ def run_ours(args):
     nominal = 8000.0 if roof["bound"] == "hbm" else 2250.0
     roof["nominal_peak"] = nominal
     roof["frac_of_nominal"] = round(roof["achieved"] / nominal, 4)
-    d_steps = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(steps_done)) / steps_done
+    timed = n_win * steps_done
+    d_steps = sum(distinct[(args.warmup + i) % TOKEN_BATCHES] for i in range(timed)) / timed
     step_bytes = (d_steps * 3 * H * I * wb + (0 if dense else E * H * 4) + T * H * 4
                   + (T * H * 8 if wl.residual_k else 0))
-    stage_avg = {kname: round(v / max(calls, 1), 4) for kname, v in stage_ms.items()}
+    stage_avg = {kname: round(v, 4) for kname, v in stage_med.items()}
+    gu = sorted(sw["gate_up_gemm"] for sw in stage_windows)
+    roof["launch_ms_min"], roof["launch_ms_max"] = round(gu[0], 4), round(gu[-1], 4)
+    roof["launch_ms_windows"] = len(gu)
 
     line = {
         "metric": METRIC,
@@ -368,6 +402,11 @@ def run_ours(args):
         "steps": steps_done,
         "warmup": args.warmup,
         "ms_per_step": round(ms_max / steps_done, 4),
+        "ms_per_step_min": round(min(win_ms) / steps_done, 4),
+        "ms_per_step_max": round(max(win_ms) / steps_done, 4),
+        "windows": n_win,
+        "timing": (f"median of {n_win} windows of {steps_done} steps, each bracketed by a barrier "
+                   f"and a synchronize; CUDA events on the launching stream; max over ranks per window"),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -382,9 +421,11 @@ def run_ours(args):
         "router_tokens_rederived_last_step": rederived,
         "clocks": sampler.report(),
         "e2e": {"value": round(whole_job_tokens_per_s(ws, e2e_steps, T, e2e_ms), 1), "unit": "tokens/s",
+                "windows": len(e2e_win), "steps_per_window": e2e_steps,
                 "h2d_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0),
                 "d2h_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0)},
-        "gpu_launches": kernels_per_forward(plan, dense, bool(wl.residual_k)) * steps_done,
+        "gpu_launches": kernels_per_forward(plan, dense, bool(wl.residual_k)) * steps_done * n_win,
+        "gpu_launches_per_step": kernels_per_forward(plan, dense, bool(wl.residual_k)),
         "roofline": roof,
         "launch_plan": plan,
     }

@@ -351,10 +351,10 @@ class BeamMoE:
 
     def launch_plan(self, T: int) -> dict:
         """The kernels and launch shapes a forward pass of T tokens uses."""
-        p = (ctypes.c_int32 * 9)()
+        p = (ctypes.c_int32 * 10)()
         self._check(library().beam_moe_launch_plan(self._h, int(T), ctypes.cast(p, ctypes.c_void_p)))
         keys = ("tile_rows", "cta_pairs", "grid", "down_paired", "router_tensor_cores", "router_slices",
-                "gather_rows", "ksplit_gate_up", "ksplit_down")
+                "gather_rows", "ksplit_gate_up", "ksplit_down", "y_f32")
         return dict(zip(keys, (int(v) for v in p)))
 
     def set_checks(self, on: bool = True):

@@ -42,7 +42,8 @@ struct beam_moe {
     int32_t *block_cnt, *block_base, *rank, *counts, *offsets, *tile_off, *pair_row, *row_pair;
     __nv_bfloat16 *xp;       // [P, H]
     __nv_bfloat16 *hbuf;     // [P, I]
-    __nv_bfloat16 *ybuf;     // [P, H]
+    __nv_bfloat16 *ybuf;     // [P, H] bf16 expert outputs, or
+    float *y32;              // [P, H] FP32 expert outputs (same memory; sparse blocks)
     int *status;             // device status word
     // host-buffer path: two staging slots, so one call's copies overlap the
     // neighbouring calls' compute; a copy-in and a copy-out stream; per slot
@@ -68,6 +69,7 @@ struct beam_moe {
     int down_pair;                   // -1: auto, 0: single tiles, 1: paired tiles
     int use_pair;                    // 1: CTA-pair kernels for large token tiles (default)
     int gather_rows;                 // -1: auto (default), 0: never, 1: always
+    int y_mode;                      // 1: FP32 expert outputs y (default), 0: bf16 y
     int token_stages;                // CTA-pair kernels: token-row ring depth (0: default)
     int checks;                      // 1: validate routing and dispatch tables on the device
     int corrupt_next;                // test hook: forward passes left whose routing is corrupted
@@ -246,7 +248,10 @@ int run_router(beam_moe *h, cudaStream_t s, const void *x, int T, int32_t *idx, 
             e = launch_router_select(b, ex, 4 * h->num_sms, s);
         }
     } else {
-        a.nslice = router_slices(T, h->H, h->E, h->num_sms);   // the workspace holds nslice * T rows
+        // the workspace holds nslice * T rows of either path
+        const int ns_small = router_small_slices(T, h->H, h->E, h->num_sms);
+        a.small = ns_small > 0;
+        a.nslice = ns_small > 0 ? ns_small : router_slices(T, h->H, h->E, h->num_sms);
         e = launch_router(a, s);
     }
     return e == cudaSuccess ? BEAM_OK : cuda_fail(h, e, "router launch");
@@ -271,6 +276,7 @@ struct ForwardPlan {
     int gather;        // 1: gate|up gathers token rows from x; no sorted copy
     int ksplit_gate_up;   // dense layers: K slices of the gate|up GEMM (1: fused SwiGLU)
     int ksplit_down;      // dense layers: K slices of the down GEMM
+    int y_f32;            // 1: the down GEMM writes the expert outputs y in FP32
 };
 
 // Split-K slices for a GEMM of `items` work items and KB K steps: the fewest
@@ -346,14 +352,20 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
     p.gather = h->gather_rows < 0 ? (p.tile_rows <= 32 ? 1 : 0) : h->gather_rows;
     p.ksplit_gate_up = 1;
     p.ksplit_down = 1;
+    // Expert outputs y in FP32: the combine then rounds only once, to the
+    // block's bf16 output.  The single-CTA FP32 down GEMM takes one weight
+    // block per item.
+    p.y_f32 = !h->dense && !h->fp4 && h->y_mode != 0;
+    if (p.y_f32 && !p.cta_pairs) p.down_paired = 0;
     if (h->fp4) {
         // NVFP4 weights: the single-CTA kernel with token tiles of up to 128
-        // rows from the sorted copy, one weight block per down item
+        // rows from the sorted copy, one weight block per down item, bf16 y
         if (p.tile_rows > 128) p.tile_rows = 128;
         p.cta_pairs = 0;
         p.grid = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
         p.down_paired = 0;
         p.gather = 0;
+        p.y_f32 = 0;
     }
     if (h->dense) {
         // one expert: with decode-sized T the weight tiles alone give too few
@@ -365,8 +377,9 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
         return p;
     }
     p.router_tc = router_on_tensor_cores(h, T);
+    const int ns_small = router_small_slices(T, h->H, h->E, h->num_sms);
     p.router_slices = p.router_tc ? router_mma_slices(T, h->H, h->E, h->num_sms)
-                                  : router_slices(T, h->H, h->E, h->num_sms);
+                                  : (ns_small > 0 ? ns_small : router_slices(T, h->H, h->E, h->num_sms));
     return p;
 }
 
@@ -468,6 +481,7 @@ int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *o
         CombineArgs c;
         c.status = h->status;
         c.y = h->ybuf;
+        c.y32 = nullptr;
         c.y_f32 = plan.ksplit_down > 1 ? h->split : nullptr;
         c.nslice = plan.ksplit_down;
         c.slice_stride = (long long)T * h->H;
@@ -579,8 +593,12 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.K = h->I;
     g.R = h->H;
     g.out = h->ybuf;
+    g.out_f32 = plan.y_f32 ? h->y32 : nullptr;
     g.gather = 0;
-    const GemmKind dk = plan.down_paired ? GemmKind::kDownPaired : GemmKind::kDown;
+    GemmKind dk = plan.down_paired ? GemmKind::kDownPaired : GemmKind::kDown;
+    if (plan.y_f32)
+        dk = use_pair ? (plan.down_paired ? GemmKind::kDownPairedY32 : GemmKind::kDownY32)
+                      : GemmKind::kDownF32;
     if (h->fp4)
         e = launch_grouped_gemm_fp4(GemmKind::kDown, BN, h->fp4_down, h->tm_h, g, grid, s);
     else
@@ -591,7 +609,8 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
 
     CombineArgs c;
     c.status = h->status;
-    c.y = h->ybuf;
+    c.y = plan.y_f32 ? nullptr : h->ybuf;
+    c.y32 = plan.y_f32 ? h->y32 : nullptr;
     c.y_f32 = nullptr;
     c.nslice = 0;
     c.slice_stride = 0;
@@ -646,6 +665,7 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     h->use_pair = 1;
     h->gather_rows = -1;
     h->router_mode = -1;
+    h->y_mode = 1;
 
     cudaError_t e = cudaGetDevice(&h->device);
     if (e == cudaSuccess)
@@ -670,6 +690,8 @@ int finish_create(beam_moe *h, beam_moe_t *out)
             }
             continue;
         }
+        const size_t r0 = (size_t)router_small_slices(t, hidden, n_experts, h->num_sms) * t;
+        if (r0 > partial_rows) partial_rows = r0;
         const size_t r1 = (size_t)router_slices(t, hidden, n_experts, h->num_sms) * t;
         const size_t r2 = (size_t)router_mma_slices(t, hidden, n_experts, h->num_sms) * t;
         if (r1 > partial_rows) partial_rows = r1;
@@ -695,7 +717,7 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     const size_t o_rpair = carve(P * 4);
     const size_t o_xp = carve(h->dense ? 0 : P * hidden * 2);   // dense: the GEMM reads x
     const size_t o_h = carve(P * inter * 2);
-    const size_t o_y = carve(P * hidden * 2);
+    const size_t o_y = carve(P * hidden * (h->dense ? 2 : 4));   // bf16 or FP32 y
     const size_t o_status = carve(256);
     size_t o_xs[2], o_os[2], o_rs[2];
     for (int i = 0; i < 2; ++i) {
@@ -730,6 +752,7 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     h->xp = reinterpret_cast<__nv_bfloat16 *>(b + o_xp);
     h->hbuf = reinterpret_cast<__nv_bfloat16 *>(b + o_h);
     h->ybuf = reinterpret_cast<__nv_bfloat16 *>(b + o_y);
+    h->y32 = reinterpret_cast<float *>(b + o_y);
     h->status = reinterpret_cast<int *>(b + o_status);
     for (int i = 0; i < 2; ++i) {
         h->x_stage[i] = reinterpret_cast<__nv_bfloat16 *>(b + o_xs[i]);
@@ -789,6 +812,7 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     }
     if (!h->dense) {
         if (e == cudaSuccess) e = prepare_router_mma();
+        if (e == cudaSuccess) e = prepare_router_small();
         if (e == cudaSuccess) e = prepare_router_fix(hidden);
         // the router weight's bf16 pieces for the tensor-core router (the
         // weight is borrowed and must not change while the handle lives)
@@ -1214,6 +1238,7 @@ int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host)
     plan_host[6] = p.gather;
     plan_host[7] = p.ksplit_gate_up;
     plan_host[8] = p.ksplit_down;
+    plan_host[9] = p.y_f32;
     return BEAM_OK;
 }
 

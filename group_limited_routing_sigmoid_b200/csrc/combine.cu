@@ -1,7 +1,8 @@
 // Combine of the Beam MoE block, with the optional post-norm and
 // depth-scaled residual update fused in.
 //
-//   o[t]   = routed_scaling * sum_j w[t,j] * y[row(t,j)]     (bf16 y, fp32 sum, slot order)
+//   o[t]   = routed_scaling * sum_j w[t,j] * y[row(t,j)]     (FP32 or bf16 y, FP32 sum,
+//                                                             slot order)
 //            (dense layer: o[t] = sum_s y_s[t] over FP32 split-K slices, in slice order)
 //   out[t] = bf16_rn(o[t])
 //   n[t]   = o[t] / sqrt(mean(o[t]^2) + eps) * gamma          (if gamma)
@@ -46,6 +47,7 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
     const int tid = threadIdx.x;
     const int nvec = a.H / 8;
     const int nsum = a.y_f32 ? 0 : a.top_k;   // expert slots (none for FP32 slices)
+    const bool wide = a.y32 != nullptr;        // FP32 expert outputs
     if (tid < nsum) {
         rows[tid] = a.pair_row[(size_t)t * a.top_k + tid];
         wts[tid] = a.w[(size_t)t * a.top_k + tid];
@@ -69,20 +71,44 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
                 acc[v][4] += hi.x; acc[v][5] += hi.y; acc[v][6] += hi.z; acc[v][7] += hi.w;
             }
         }
-        for (int j0 = 0; j0 < nsum; j0 += kCombBatch) {
-            uint4 raw[kCombBatch];
+        if (wide) {
+            for (int j0 = 0; j0 < nsum; j0 += kCombBatch) {
+                float4 lo[kCombBatch], hi[kCombBatch];
 #pragma unroll
-            for (int j = 0; j < kCombBatch; ++j)
-                if (j0 + j < nsum)
-                    raw[j] = reinterpret_cast<const uint4 *>(a.y + (size_t)rows[j0 + j] * a.H)[q];
+                for (int j = 0; j < kCombBatch; ++j)
+                    if (j0 + j < nsum) {
+                        const float4 *src = reinterpret_cast<const float4 *>(
+                            a.y32 + (size_t)rows[j0 + j] * a.H + 8 * q);
+                        lo[j] = src[0];
+                        hi[j] = src[1];
+                    }
 #pragma unroll
-            for (int j = 0; j < kCombBatch; ++j) {
-                if (j0 + j < nsum) {
-                    float y[8];
-                    unpack8(raw[j], y);
-                    const float wj = wts[j0 + j];
+                for (int j = 0; j < kCombBatch; ++j) {
+                    if (j0 + j < nsum) {
+                        const float y[8] = {lo[j].x, lo[j].y, lo[j].z, lo[j].w,
+                                            hi[j].x, hi[j].y, hi[j].z, hi[j].w};
+                        const float wj = wts[j0 + j];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[v][i] = fmaf(wj, y[i], acc[v][i]);
+                        for (int i = 0; i < 8; ++i) acc[v][i] = fmaf(wj, y[i], acc[v][i]);
+                    }
+                }
+            }
+        } else {
+            for (int j0 = 0; j0 < nsum; j0 += kCombBatch) {
+                uint4 raw[kCombBatch];
+#pragma unroll
+                for (int j = 0; j < kCombBatch; ++j)
+                    if (j0 + j < nsum)
+                        raw[j] = reinterpret_cast<const uint4 *>(a.y + (size_t)rows[j0 + j] * a.H)[q];
+#pragma unroll
+                for (int j = 0; j < kCombBatch; ++j) {
+                    if (j0 + j < nsum) {
+                        float y[8];
+                        unpack8(raw[j], y);
+                        const float wj = wts[j0 + j];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[v][i] = fmaf(wj, y[i], acc[v][i]);
+                    }
                 }
             }
         }

@@ -348,12 +348,12 @@ cudaError_t launch_kind(GemmKind kind, const CUtensorMap &a0, const CUtensorMap 
         case GemmKind::kDownPaired:
             return launch<BN, 2, kStoreBF16>(a0, a1, b, args, grid, stream);
         case GemmKind::kGateUpF32:
-        case GemmKind::kDownF32:
-            if constexpr (BN <= 64) {
-                if (kind == GemmKind::kGateUpF32) return launch<BN, 2, kGateUpF32>(a0, a1, b, args, grid, stream);
-                return launch<BN, 1, kStoreF32>(a0, a1, b, args, grid, stream);
-            }
+            if constexpr (BN <= 64) return launch<BN, 2, kGateUpF32>(a0, a1, b, args, grid, stream);
             return cudaErrorInvalidValue;
+        case GemmKind::kDownF32:
+            return launch<BN, 1, kStoreF32>(a0, a1, b, args, grid, stream);
+        default:
+            break;
     }
     return cudaErrorInvalidValue;
 }
@@ -371,10 +371,10 @@ cudaError_t prepare_grouped_gemm(int E)
 #define BEAM_PREP(BN)                                                        \
     if ((err = set_smem<BN, 2, kSwiGLU>()) != cudaSuccess) return err;       \
     if ((err = set_smem<BN, 1, kStoreBF16>()) != cudaSuccess) return err;    \
-    if ((err = set_smem<BN, 2, kStoreBF16>()) != cudaSuccess) return err;
-#define BEAM_PREP_F32(BN)                                                    \
-    if ((err = set_smem<BN, 2, kGateUpF32>()) != cudaSuccess) return err;    \
+    if ((err = set_smem<BN, 2, kStoreBF16>()) != cudaSuccess) return err;    \
     if ((err = set_smem<BN, 1, kStoreF32>()) != cudaSuccess) return err;
+#define BEAM_PREP_F32(BN)                                                    \
+    if ((err = set_smem<BN, 2, kGateUpF32>()) != cudaSuccess) return err;
     BEAM_PREP(16)
     BEAM_PREP(32)
     BEAM_PREP(64)

@@ -57,7 +57,8 @@ struct PairCfg {
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair UMMA N");
     static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0, "stages keep 1024-byte alignment");
     static_assert(kPairRingBytes >= 2 * A_STAGE + 2 * B_STAGE, "two stages per ring");
-    static_assert(EPI == kStoreBF16 || NUM_A == 2, "SwiGLU needs the gate and up tiles");
+    static_assert(EPI != kSwiGLU || NUM_A == 2, "SwiGLU needs the gate and up tiles");
+    static_assert(EPI == kSwiGLU || EPI == kStoreBF16 || EPI == kStoreF32, "pair epilogues");
     static_assert(4 * kPairMaxStages * 8 + 5 * 8 + 4 <= kPairBarrierBytes, "barrier block");
 };
 
@@ -313,6 +314,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 const int col0 = it.wt * C::ROWS_PER_ITEM + (int)rank * kBM + quad * 32;
                 epilogue_block<EPI, C::CH, BN>(taddr, it.nrows, it.row0, half_sel, lane, stg,
                                                p.out + col0, p.R);
+            } else if constexpr (EPI == kStoreF32) {
+                // FP32 expert outputs: TMEM lane = output column, so each
+                // warp store is one token row's 32 consecutive floats
+#pragma unroll 1
+                for (int a = 0; a < NUM_A; ++a) {
+                    const int col0 =
+                        it.wt * C::ROWS_PER_ITEM + a * 2 * kBM + (int)rank * kBM + quad * 32;
+                    epilogue_f32(taddr + a * BN, it.nrows, it.row0, half_sel, lane,
+                                 p.out_f32 + col0, p.R);
+                }
             } else {
 #pragma unroll 1
                 for (int a = 0; a < NUM_A; ++a) {
@@ -384,6 +395,12 @@ cudaError_t launch_pair_kind(GemmKind kind, const CUtensorMap &a0, const CUtenso
             return launch_pair<BN, 1, kStoreBF16>(a0, a1, b, args, grid, stream);
         case GemmKind::kDownPaired:
             return launch_pair<BN, 2, kStoreBF16>(a0, a1, b, args, grid, stream);
+        case GemmKind::kDownY32:
+            return launch_pair<BN, 1, kStoreF32>(a0, a1, b, args, grid, stream);
+        case GemmKind::kDownPairedY32:
+            return launch_pair<BN, 2, kStoreF32>(a0, a1, b, args, grid, stream);
+        default:
+            break;
     }
     return cudaErrorInvalidValue;
 }
@@ -399,7 +416,9 @@ cudaError_t prepare_grouped_gemm_pair()
 #define BEAM_PREP_PAIR(BN)                                                        \
     if ((err = set_smem_pair<BN, 2, kSwiGLU>()) != cudaSuccess) return err;       \
     if ((err = set_smem_pair<BN, 1, kStoreBF16>()) != cudaSuccess) return err;    \
-    if ((err = set_smem_pair<BN, 2, kStoreBF16>()) != cudaSuccess) return err;
+    if ((err = set_smem_pair<BN, 2, kStoreBF16>()) != cudaSuccess) return err;    \
+    if ((err = set_smem_pair<BN, 1, kStoreF32>()) != cudaSuccess) return err;     \
+    if ((err = set_smem_pair<BN, 2, kStoreF32>()) != cudaSuccess) return err;
     BEAM_PREP_PAIR(64)
     BEAM_PREP_PAIR(128)
     BEAM_PREP_PAIR(256)

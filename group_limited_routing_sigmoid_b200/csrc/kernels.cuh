@@ -32,13 +32,16 @@ struct RouterArgs {
     const float *router_w;    // [E, H]
     const float *bias;        // [E]
     int T, H, E, n_group, topk_group, top_k;
-    int nslice;               // K slices of the logits (router_slices)
+    int nslice;               // K slices of the logits (router_slices or router_small_slices)
+    int small = 0;            // 1: the small-batch logits kernel (T <= 64)
     float *partial;           // [nslice, T, E] workspace
     int32_t *idx;             // [T, top_k]
     float *w;                 // [T, top_k]
     float *logits_out;        // [T, E] or nullptr
 };
 int router_slices(int T, int H, int E, int num_sms);
+int router_small_slices(int T, int H, int E, int num_sms);   // 0: the small path does not apply
+cudaError_t prepare_router_small();
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream);          // SIMT logits + selection
 
 // Selection extras: a decision-margin check that lists tokens for the exact
@@ -139,7 +142,10 @@ enum class GemmKind {
     kDownPaired,   // two consecutive 128-row tiles sharing the token tile, bf16 out
     kGateUpF32,    // gate and up tiles, FP32 partial sums out ([slice][P][2R]: gate, then up);
                    // single-CTA kernel, token tiles of up to 64 rows
-    kDownF32       // one 128-row tile, FP32 partial sums out ([slice][P][R]); as above
+    kDownF32,      // one 128-row tile, FP32 partial sums out ([slice][P][R]); as above
+                   // (ksplit 1: FP32 expert outputs y)
+    kDownY32,      // CTA-pair kernel: one 256-row block, FP32 expert outputs y ([P][R])
+    kDownPairedY32 // CTA-pair kernel: two 256-row blocks sharing the token tile, FP32 y
 };
 // BN: largest token tile (16..256, power of two).
 cudaError_t launch_grouped_gemm(GemmKind kind, int BN, const CUtensorMap &a0,
@@ -161,7 +167,9 @@ int gemm_pair_max_ctas();   // CTAs of the pair kernels that can be resident at 
 // ---------------------------------------------------------------- combine
 struct CombineArgs {
     const int *status;           // the handle's status word: no work while it is set
-    const __nv_bfloat16 *y;      // [P, H] expert outputs
+    const __nv_bfloat16 *y;      // [P, H] expert outputs (bf16), or
+    const float *y32;            // [P, H] expert outputs (FP32); exactly one of y, y32 is set
+                                 // for a sparse block
     // instead of y (dense layer, top_k == 1, unit weight): FP32 partial sums
     // of nslice split-K slices [nslice][T][H], slice_stride elements apart,
     // summed in slice order

@@ -145,6 +145,111 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16 
 }
 
 // ---------------------------------------------------------------------------
+// Logits for small batches (T <= 64, decode): a block per (16 experts, K
+// slice of width ks), all tokens.  The block stages its whole slice of x
+// (T rows of ks bf16) and of the router matrix (16 rows of ks floats) in
+// shared memory with every 16-byte copy in flight at once, so the slice
+// costs one memory round trip rather than one per K stage.  Warp w then sums
+// K range [w*ks/8, (w+1)*ks/8) for all 64 x 16 outputs: lane l holds tokens
+// (l & 7) + 8i and experts (l >> 3) + 4j (the rows a load instruction reads
+// are consecutive, so the padded rows fall in distinct banks).  The eight
+// warps' sums are added in warp order into partial[slice][t][e]; the
+// selection adds the slices in slice order.
+// ---------------------------------------------------------------------------
+constexpr int kSmallT = 64;     // tokens per block (the largest T of this path)
+constexpr int kSmallE = 16;     // experts per block
+constexpr int kSmallMaxK = 640; // widest K slice (shared memory)
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__global__ void __launch_bounds__(256) router_logits_small_kernel(
+    const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w, int T, int H, int E, int ks,
+    float *__restrict__ partial)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    extern __shared__ __align__(16) uint8_t small_smem[];
+    const int xstride = ks + 8;   // bf16 per staged token row (16 bytes of padding)
+    const int wstride = ks + 4;   // floats per staged expert row (16 bytes of padding)
+    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(small_smem);
+    float *ws = reinterpret_cast<float *>(small_smem + (size_t)kSmallT * xstride * 2);
+    const int e0 = blockIdx.x * kSmallE;
+    const int k0 = blockIdx.y * ks;
+    const int xv = ks / 8, wv = ks / 4;   // 16-byte vectors per row
+    for (int i = threadIdx.x; i < T * xv; i += blockDim.x) {
+        const int t = i / xv, q = i - t * xv;
+        cp_async16(xs + (size_t)t * xstride + 8 * q, x + (size_t)t * H + k0 + 8 * q);
+    }
+    for (int i = threadIdx.x; i < kSmallE * wv; i += blockDim.x) {
+        const int r = i / wv, q = i - r * wv;
+        cp_async16(ws + (size_t)r * wstride + 4 * q, w + (size_t)(e0 + r) * H + k0 + 4 * q);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tg = lane & 7, eg = lane >> 3;
+    const int kw = ks / 8;
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    // rows of tokens >= T are never written: their sums are not stored
+    for (int k = warp * kw; k < (warp + 1) * kw; k += 8) {
+        float wf[4][8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 *p = reinterpret_cast<const float4 *>(ws + (size_t)(eg + 4 * j) * wstride + k);
+            const float4 a = p[0], b = p[1];
+            wf[j][0] = a.x; wf[j][1] = a.y; wf[j][2] = a.z; wf[j][3] = a.w;
+            wf[j][4] = b.x; wf[j][5] = b.y; wf[j][6] = b.z; wf[j][7] = b.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint4 raw = *reinterpret_cast<const uint4 *>(xs + (size_t)(tg + 8 * i) * xstride + k);
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+            float xf[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = __bfloat1622float2(h2[q]);
+                xf[2 * q] = f.x;
+                xf[2 * q + 1] = f.y;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[i][j] = fmaf(xf[q], wf[j][q], acc[i][j]);
+        }
+    }
+    __syncthreads();   // every warp is done with the staged rows
+    float *red = reinterpret_cast<float *>(small_smem);   // [8 warps][64 tokens][16 experts]
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            red[((size_t)warp * kSmallT + tg + 8 * i) * kSmallE + eg + 4 * j] = acc[i][j];
+    __syncthreads();
+    const int t = threadIdx.x >> 2, ec = (threadIdx.x & 3) * 4;
+    if (t < T) {
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int wv2 = 0; wv2 < 8; ++wv2) {
+            const float4 v = *reinterpret_cast<const float4 *>(red + ((size_t)wv2 * kSmallT + t) * kSmallE + ec);
+            sum.x += v.x;
+            sum.y += v.y;
+            sum.z += v.z;
+            sum.w += v.w;
+        }
+        *reinterpret_cast<float4 *>(partial + ((size_t)blockIdx.y * T + t) * E + e0 + ec) = sum;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Selection: one warp per token; lane l owns experts l*EPL .. l*EPL+EPL-1,
 // so a group of g experts spans g/EPL consecutive lanes.  Grid-stride over
 // the tokens.  Optional extras (SelectExtra):
@@ -179,7 +284,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(
         float l[EPL];
 #pragma unroll
         for (int m = 0; m < EPL; ++m) l[m] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
         for (int q = 0; q < nslice; ++q) {
             const float *src = partial + ((size_t)q * T + r) * E + e_base;
             if constexpr (EPL % 4 == 0) {
@@ -408,13 +513,52 @@ int router_slices(int T, int H, int E, int num_sms)
     return ns;
 }
 
+// Small-batch path: the fewest K slices (each a multiple of 64 wide and at
+// most kSmallMaxK) whose blocks cover every SM; 0 when the path does not
+// apply (T > 64, or H or E off its grid).
+int router_small_slices(int T, int H, int E, int num_sms)
+{
+    if (T < 1 || T > kSmallT || E % kSmallE != 0 || H % 64 != 0) return 0;
+    int best = 0;
+    for (int ns = 1; ns <= H / 64; ++ns) {
+        if (H % (ns * 64) != 0 || H / ns > kSmallMaxK) continue;
+        best = ns;
+        if ((E / kSmallE) * ns >= num_sms) break;
+    }
+    return best;
+}
+
+// Staged rows, or the warps' sums that reuse them, whichever is larger.
+static size_t small_smem_bytes(int ks)
+{
+    const size_t staged = (size_t)kSmallT * (ks + 8) * 2 + (size_t)kSmallE * (ks + 4) * 4;
+    const size_t red = (size_t)8 * kSmallT * kSmallE * 4;
+    return staged > red ? staged : red;
+}
+
+cudaError_t prepare_router_small()
+{
+    return cudaFuncSetAttribute(router_logits_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)small_smem_bytes(kSmallMaxK));
+}
+
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream)
 {
     const int ns = a.nslice;
     const int kslice = a.H / ns;
-    dim3 grid((a.T + kLT - 1) / kLT, (a.E + kLE - 1) / kLE, ns);
-    cudaError_t err = launch_pdl(router_logits_kernel, grid, dim3(256), 0, stream, a.x, a.router_w,
-                                 a.T, a.H, a.E, kslice, a.partial);
+    cudaError_t err;
+    if (a.small) {
+        if (a.T > kSmallT || a.E % kSmallE != 0 || kslice % 64 != 0 || kslice > kSmallMaxK ||
+            kslice * ns != a.H)
+            return cudaErrorInvalidValue;
+        const size_t smem = small_smem_bytes(kslice);
+        err = launch_pdl(router_logits_small_kernel, dim3(a.E / kSmallE, ns), dim3(256), smem, stream,
+                         a.x, a.router_w, a.T, a.H, a.E, kslice, a.partial);
+    } else {
+        dim3 grid((a.T + kLT - 1) / kLT, (a.E + kLE - 1) / kLE, ns);
+        err = launch_pdl(router_logits_kernel, grid, dim3(256), 0, stream, a.x, a.router_w, a.T, a.H,
+                         a.E, kslice, a.partial);
+    }
     if (err != cudaSuccess) return err;
     const int warps = 8;
     dim3 sgrid((a.T + warps - 1) / warps);

@@ -66,7 +66,12 @@ typedef enum {
 } beam_status;
 
 /*
- * Create a handle for one MoE block.
+ * Create a handle for one MoE block: the router (sigmoid scores, per-expert
+ * bias, n_group groups scored by their two best biased scores, topk_group
+ * groups kept, top_k experts chosen) and E SwiGLU experts, as the launch blog
+ * "Introducing Beam", section "Mixture of Experts", and the transformers
+ * page "Beam", section "Overview", "Sparse MoE" bullet, define them; the
+ * optional post-norm as in the blog's section "Residual Stream".
  *
  * hidden        H, hidden size (Beam: 5120).  Must be a multiple of 128.
  * n_experts     E (Beam: 256).  Must be a multiple of 32 and at most 1024.
@@ -92,8 +97,11 @@ typedef enum {
  * (group size)/(E/32) a power of two, n_group <= 32.
  * On success *out receives the handle.  Allocates device memory and launches
  * one kernel on the legacy default stream (splitting router_w into the bf16
- * pieces the tensor-core router uses), waiting for it.  The current CUDA
- * device at create time is the handle's device.
+ * pieces the tensor-core router uses), waiting for it: the handle's one
+ * derived weight is then complete before create returns, so the first call
+ * may come on any stream, or inside a stream capture, with no ordering
+ * against create.  The current CUDA device at create time is the handle's
+ * device.
  */
 int beam_moe_create(beam_moe_t *out, int hidden, int n_experts, int inter, int n_group,
                     int topk_group, int top_k, float routed_scaling, const float *router_w,
@@ -171,7 +179,11 @@ int beam_nvfp4_dequant(void *stream, const uint8_t *codes, const uint8_t *scales
                        int K, void *out);
 
 /*
- * Route T tokens: the router step alone.
+ * Route T tokens: the router step alone (launch blog "Introducing Beam",
+ * section "Mixture of Experts": sigmoid scores plus the expert bias, groups
+ * scored by the sum of their two best scores, the best groups kept, the top
+ * experts chosen inside them, their weights normalised; transformers page
+ * "Beam", "Sparse MoE" bullet and the FP32 router paragraph).
  * x         bf16 [T, H].
  * topk_idx  int32 [T, top_k] (out): chosen experts, in descending biased
  *           score, ties to the lower index.
@@ -200,6 +212,9 @@ int beam_moe_route(beam_moe_t h, void *stream, const void *x, int T, int32_t *to
  * race and give undefined results; calls ordered on one stream are safe.
  * Nothing in the array needs clearing: each call writes every element it
  * reads.  No cudaMalloc, cudaFree or allocating library call is made.
+ * The array's device address is looked up once per device and kept for the
+ * life of the process, so this entry point does not support cudaDeviceReset:
+ * after a reset the kept address belongs to the destroyed context.
  * Arguments as beam_moe_create / beam_moe_route: x bf16 [T, H], router_w fp32
  * [E, H], expert_bias fp32 [E] (16-byte aligned device pointers), topk_idx
  * int32 [T, top_k] and topk_w fp32 [T, top_k] (device, out).  hidden must be
@@ -235,7 +250,11 @@ int beam_moe_route_logits(beam_moe_t h, void *stream, const float *logits, int T
                           const float *expert_bias, int32_t *topk_idx, float *topk_w);
 
 /*
- * Forward pass of the block for T tokens.
+ * Forward pass of the block for T tokens: routing, the chosen experts'
+ * SwiGLU MLPs and their weighted sum scaled by routed_scaling (launch blog
+ * "Introducing Beam", section "Mixture of Experts"), and optionally the
+ * post-norm and the depth-scaled residual update (same blog, section
+ * "Residual Stream"; transformers page "Beam", "Overview").
  * x         bf16 [T, H].
  * out       bf16 [T, H] (out): routed_scaling * sum_j w_j * expert_j(x),
  *           rounded to nearest even; may be NULL when residual is given.
@@ -310,14 +329,16 @@ int beam_moe_router_stats(beam_moe_t h, void *stream, int32_t *rederived_host);
 
 /*
  * The launch configuration a forward pass of T tokens (0 <= T <= max_tokens)
- * uses under the handle's current tuning, written to plan_host (int32 [9],
+ * uses under the handle's current tuning, written to plan_host (int32 [10],
  * host): {largest token tile of the grouped GEMMs (rows), 1 if
  * they run on CTA pairs (cta_group::2), CTAs per grouped GEMM, 1 if the down
  * projection takes two weight blocks per work item, 1 if the router logits
  * run on the tensor cores (with exact re-derivation of thin-margin tokens),
  * K slices of the router logits (0 for a dense layer), 1 if the gate|up GEMM
  * gathers token rows from x, K slices of the gate|up GEMM and of the down
- * GEMM (dense layers; 1 = no split)}.  A function of T and the tuning only; launches nothing.
+ * GEMM (dense layers; 1 = no split), 1 if the down GEMM stores the expert
+ * outputs in FP32 (else bf16)}.  A function of T and the tuning only;
+ * launches nothing.
  * Returns BEAM_ERR_INVALID_ARG for a NULL pointer or T out of range.
  */
 int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host);

@@ -8,15 +8,16 @@ Tolerances (the block's stated bar):
     score order, so a token whose chosen experts contain a near-tie (two
     neighbours in that order closer than 1e-6) must match as a set, and its
     order is exempt (counted in ``order_exempt``);
+  * combine weights (before x routed_scaling): max abs error <= 1e-5, on
+    every token whose set matches; where the order is exempt the two sides'
+    slots are paired by expert id first;
   * outputs: relative Frobenius error <= 5e-3 and max abs error <= 2e-2 x
-    the RMS of the oracle output.  Both sides round to bf16; where the two
-    bf16 values are neighbours (at most one bf16 ulp of the oracle value
-    apart) the pair is a rounding-boundary case -- two valid roundings of
-    values that differ by far less than the tolerance -- and it is counted
-    (``ulp_neighbours``) rather than held to the max-abs bound.  At 5 sigma one
-    bf16 ulp is already ~2e-2 x RMS, so without this any large sample would
-    fail on correct roundings.  The Frobenius bound covers every element;
-  * combine weights (before x routed_scaling): max abs error <= 1e-5.
+    the RMS of the oracle output, both measured against the oracle's exact
+    (fp64, unrounded) combined output, over every element of every compared
+    token.  A correct bf16 output is then off by at most half a bf16 ulp
+    plus its own arithmetic error.  The count of elements whose bf16 value
+    is a neighbour (one ulp away) of the oracle's own bf16 rounding is kept
+    as a diagnostic only (``ulp_neighbours``).
 With a residual stream, the update's contribution
     stream_out - sqrt((k-1)/k) * stream_in
 is compared with the oracle's n / sqrt(k) under the output tolerances.
@@ -50,7 +51,6 @@ class Report:
     w_max_err: float = 0.0
     rel_fro: float = 0.0
     max_abs_over_rms: float = 0.0
-    max_abs_over_rms_raw: float = 0.0
     ulp_neighbours: int = 0
     res_rel_fro: Optional[float] = None
     res_max_abs_over_rms: Optional[float] = None
@@ -80,15 +80,28 @@ def bf16_ulp(v: np.ndarray) -> np.ndarray:
     return 2.0 ** (e - 7)
 
 
-def bf16_errors(got: np.ndarray, ref: np.ndarray):
-    """(rel_fro, max_abs/rms over non-neighbour pairs, raw max_abs/rms, neighbours)."""
-    rel, raw = errors(got, ref)
-    d = np.abs(got - ref)
-    neighbour = (d > 0) & (d <= bf16_ulp(ref) * (1 + 1e-12))
-    rms = math.sqrt(float((ref ** 2).mean()))
-    rest = d[~neighbour]
-    mx = float(rest.max() / max(rms, 1e-300)) if rest.size else 0.0
-    return rel, mx, raw, int(neighbour.sum())
+def bf16_errors(got: np.ndarray, exact: np.ndarray, rounded: np.ndarray):
+    """(rel_fro, max_abs/rms, neighbours) of bf16 outputs ``got`` against the
+    oracle's exact values ``exact``; ``neighbours`` counts the elements that
+    sit one bf16 ulp from the oracle's own bf16 rounding ``rounded`` (a
+    diagnostic, not part of the bound)."""
+    rel, mx = errors(got, exact)
+    d = np.abs(got - rounded)
+    neighbour = (d > 0) & (d <= bf16_ulp(rounded) * (1 + 1e-12))
+    return rel, mx, int(neighbour.sum())
+
+
+def paired_weight_error(ig: np.ndarray, wg: np.ndarray, io: np.ndarray, wo: np.ndarray) -> float:
+    """Max abs weight error of tokens whose expert sets match but whose slot
+    order may differ: each side's slots sorted by expert id, then compared."""
+    if ig.size == 0:
+        return 0.0
+    og = np.argsort(ig, axis=1, kind="stable")
+    oo = np.argsort(io, axis=1, kind="stable")
+    a = np.take_along_axis(ig, og, 1)
+    b = np.take_along_axis(io, oo, 1)
+    assert (a == b).all(), "paired weights need matching expert sets"
+    return float(np.abs(np.take_along_axis(wg, og, 1) - np.take_along_axis(wo, oo, 1)).max())
 
 
 def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
@@ -151,12 +164,15 @@ def check_block(wl: W.Workload, d: dict, moe, sample: Optional[torch.Tensor] = N
     rep.set_mismatch = int(sum(set(a.tolist()) != set(b.tolist()) for a, b in zip(ig[keep], r.idx[keep])))
     if ordered.any():
         rep.w_max_err = float(np.abs(wg[ordered] - r.w[ordered]).max())
+    swapped = keep & ~ordered
+    if swapped.any() and rep.set_mismatch == 0:
+        rep.w_max_err = max(rep.w_max_err, paired_weight_error(ig[swapped], wg[swapped],
+                                                               r.idx[swapped], r.w[swapped]))
     if keep.any():
         if out is not None:
             got = bf16_to_f64(out.index_select(0, s_dev))[keep]
-            ref = oracle.bf16_to_f64(res.out)[keep]
-            (rep.rel_fro, rep.max_abs_over_rms, rep.max_abs_over_rms_raw,
-             rep.ulp_neighbours) = bf16_errors(got, ref)
+            rep.rel_fro, rep.max_abs_over_rms, rep.ulp_neighbours = bf16_errors(
+                got, res.o[keep], oracle.bf16_to_f64(res.out)[keep])
         if stream_in is not None:
             keep_f = math.sqrt((wl.residual_k - 1) / wl.residual_k)
             s_out = stream_dev.index_select(0, s_dev).cpu().double().numpy()
@@ -198,8 +214,8 @@ def check_dense(wl, d, moe, T: Optional[int] = None, sample: Optional[torch.Tens
     rep.tokens = len(sample)
     if out is not None:
         got = bf16_to_f64(out.index_select(0, s_dev))
-        ref = oracle.bf16_to_f64(res.out)
-        rep.rel_fro, rep.max_abs_over_rms, rep.max_abs_over_rms_raw, rep.ulp_neighbours = bf16_errors(got, ref)
+        rep.rel_fro, rep.max_abs_over_rms, rep.ulp_neighbours = bf16_errors(
+            got, res.o, oracle.bf16_to_f64(res.out))
     if stream_in is not None:
         keep_f = math.sqrt((wl.residual_k - 1) / wl.residual_k)
         s_out = stream_dev.index_select(0, s_dev).cpu().double().numpy()

@@ -235,6 +235,7 @@ def test_launch_plan_follows_tokens_per_expert_and_tuning():
     assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"],
             p["gather_rows"]) == (16, 0, 0, 0, 1)
     assert p["grid"] == torch.cuda.get_device_properties(0).multi_processor_count
+    assert p["y_f32"] == 1
     p = moe.launch_plan(wl.T)
     assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"]) == (256, 1, 1, 1)
     assert p["grid"] % 2 == 0 and p["router_slices"] >= 1
