@@ -35,6 +35,9 @@ __device__ __forceinline__ void unpack8(const uint4 &raw, float (&v)[8])
 // the row (8 hidden values each).  The loads of kCombBatch expert slots of a
 // vector are issued before their sums, which take the slots in order (FP32
 // FMA), so every value is the same slot-order sum.
+// WIDE: FP32 expert outputs (a.y32), all top_k slots' loads in flight at
+// once; otherwise bf16 outputs (a.y) or the dense layer's FP32 slices.
+template <bool WIDE>
 __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
 {
     pdl_launch_dependents();
@@ -47,7 +50,7 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
     const int tid = threadIdx.x;
     const int nvec = a.H / 8;
     const int nsum = a.y_f32 ? 0 : a.top_k;   // expert slots (none for FP32 slices)
-    const bool wide = a.y32 != nullptr;        // FP32 expert outputs
+    constexpr bool wide = WIDE;                // FP32 expert outputs
     if (tid < nsum) {
         rows[tid] = a.pair_row[(size_t)t * a.top_k + tid];
         wts[tid] = a.w[(size_t)t * a.top_k + tid];
@@ -62,20 +65,12 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[v][i] = 0.f;
         if (q >= nvec) continue;
-        if (a.y_f32) {
-            for (int sl = 0; sl < a.nslice; ++sl) {
-                const float4 *src = reinterpret_cast<const float4 *>(
-                    a.y_f32 + (size_t)sl * (size_t)a.slice_stride + (size_t)t * a.H + 8 * q);
-                const float4 lo = src[0], hi = src[1];
-                acc[v][0] += lo.x; acc[v][1] += lo.y; acc[v][2] += lo.z; acc[v][3] += lo.w;
-                acc[v][4] += hi.x; acc[v][5] += hi.y; acc[v][6] += hi.z; acc[v][7] += hi.w;
-            }
-        }
-        if (wide) {
-            for (int j0 = 0; j0 < nsum; j0 += kCombBatch) {
-                float4 lo[kCombBatch], hi[kCombBatch];
+        if constexpr (wide) {
+            constexpr int B = 8;   // slots in flight
+            for (int j0 = 0; j0 < nsum; j0 += B) {
+                float4 lo[B], hi[B];
 #pragma unroll
-                for (int j = 0; j < kCombBatch; ++j)
+                for (int j = 0; j < B; ++j)
                     if (j0 + j < nsum) {
                         const float4 *src = reinterpret_cast<const float4 *>(
                             a.y32 + (size_t)rows[j0 + j] * a.H + 8 * q);
@@ -83,7 +78,7 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
                         hi[j] = src[1];
                     }
 #pragma unroll
-                for (int j = 0; j < kCombBatch; ++j) {
+                for (int j = 0; j < B; ++j) {
                     if (j0 + j < nsum) {
                         const float y[8] = {lo[j].x, lo[j].y, lo[j].z, lo[j].w,
                                             hi[j].x, hi[j].y, hi[j].z, hi[j].w};
@@ -94,6 +89,15 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
                 }
             }
         } else {
+            if (a.y_f32) {
+                for (int sl = 0; sl < a.nslice; ++sl) {
+                    const float4 *src = reinterpret_cast<const float4 *>(
+                        a.y_f32 + (size_t)sl * (size_t)a.slice_stride + (size_t)t * a.H + 8 * q);
+                    const float4 lo = src[0], hi = src[1];
+                    acc[v][0] += lo.x; acc[v][1] += lo.y; acc[v][2] += lo.z; acc[v][3] += lo.w;
+                    acc[v][4] += hi.x; acc[v][5] += hi.y; acc[v][6] += hi.z; acc[v][7] += hi.w;
+                }
+            }
             for (int j0 = 0; j0 < nsum; j0 += kCombBatch) {
                 uint4 raw[kCombBatch];
 #pragma unroll
@@ -170,7 +174,8 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream)
     const int nvec = a.H / 8;
     const int threads = ((nvec + kCombVecs - 1) / kCombVecs + 31) / 32 * 32;
     if (threads > kCombMaxThreads) return cudaErrorInvalidValue;
-    return launch_pdl(combine_kernel, dim3(a.T), dim3(threads), 0, stream, a);
+    if (a.y32) return launch_pdl(combine_kernel<true>, dim3(a.T), dim3(threads), 0, stream, a);
+    return launch_pdl(combine_kernel<false>, dim3(a.T), dim3(threads), 0, stream, a);
 }
 
 __global__ void wait_timeout_check_kernel(WaitCtl ctl)

@@ -14,10 +14,16 @@ Tolerances (the block's stated bar):
   * outputs: relative Frobenius error <= 5e-3 and max abs error <= 2e-2 x
     the RMS of the oracle output, both measured against the oracle's exact
     (fp64, unrounded) combined output, over every element of every compared
-    token.  A correct bf16 output is then off by at most half a bf16 ulp
-    plus its own arithmetic error.  The count of elements whose bf16 value
-    is a neighbour (one ulp away) of the oracle's own bf16 rounding is kept
-    as a diagnostic only (``ulp_neighbours``).
+    token.  A correct bf16 output is then off by at most half a bf16 spacing
+    plus its own arithmetic error.  That half spacing alone exceeds
+    2e-2 x RMS for elements above about 5.1 x RMS, where no bf16 value meets
+    the bound: there (and only there) an element may be off by its half
+    spacing plus GRID_SLACK x RMS, the allowance for an exact value within
+    that distance of a rounding midpoint.  Such elements are counted
+    (``grid_limited``); ``max_abs_over_rms`` is the raw largest error and
+    ``max_abs_over_bound`` the asserted one (<= 1).  The count of elements
+    whose bf16 value is a neighbour (one spacing away) of the oracle's own
+    bf16 rounding is kept as a diagnostic only (``ulp_neighbours``).
 With a residual stream, the update's contribution
     stream_out - sqrt((k-1)/k) * stream_in
 is compared with the oracle's n / sqrt(k) under the output tolerances.
@@ -38,6 +44,7 @@ from group_limited_routing_sigmoid_b200 import workloads as W
 NEAR_TIE = 1e-6
 REL_FRO = 5e-3
 MAX_ABS_RMS = 2e-2
+GRID_SLACK = 1e-3
 W_ABS = 1e-5
 
 
@@ -51,6 +58,8 @@ class Report:
     w_max_err: float = 0.0
     rel_fro: float = 0.0
     max_abs_over_rms: float = 0.0
+    max_abs_over_bound: float = 0.0
+    grid_limited: int = 0
     ulp_neighbours: int = 0
     res_rel_fro: Optional[float] = None
     res_max_abs_over_rms: Optional[float] = None
@@ -60,7 +69,7 @@ class Report:
     def ok(self) -> bool:
         good = (self.idx_mismatch == 0 and self.set_mismatch == 0 and self.w_max_err <= W_ABS
                 and self.rel_fro <= REL_FRO
-                and self.max_abs_over_rms <= MAX_ABS_RMS)
+                and self.max_abs_over_bound <= 1.0)
         if self.res_rel_fro is not None:
             good = good and self.res_rel_fro <= REL_FRO and self.res_max_abs_over_rms <= MAX_ABS_RMS
         return good
@@ -80,15 +89,30 @@ def bf16_ulp(v: np.ndarray) -> np.ndarray:
     return 2.0 ** (e - 7)
 
 
+def bf16_half_spacing(v: np.ndarray) -> np.ndarray:
+    """Half the distance between the two bf16 values around v: the largest
+    error of a correctly rounded bf16 value (just below a power of two the
+    spacing below is the one that counts, which the floor of log2 gives)."""
+    return bf16_ulp(v) / 2
+
+
 def bf16_errors(got: np.ndarray, exact: np.ndarray, rounded: np.ndarray):
-    """(rel_fro, max_abs/rms, neighbours) of bf16 outputs ``got`` against the
-    oracle's exact values ``exact``; ``neighbours`` counts the elements that
-    sit one bf16 ulp from the oracle's own bf16 rounding ``rounded`` (a
-    diagnostic, not part of the bound)."""
+    """(rel_fro, max_abs/rms, max_abs/bound, grid_limited, neighbours) of bf16
+    outputs ``got`` against the oracle's exact values ``exact``.  The bound of
+    an element is MAX_ABS_RMS x RMS, or its half bf16 spacing plus
+    GRID_SLACK x RMS where that is larger (``grid_limited`` counts those);
+    ``neighbours`` counts the elements one bf16 spacing from the oracle's own
+    rounding ``rounded`` (a diagnostic, not part of the bound)."""
     rel, mx = errors(got, exact)
-    d = np.abs(got - rounded)
-    neighbour = (d > 0) & (d <= bf16_ulp(rounded) * (1 + 1e-12))
-    return rel, mx, int(neighbour.sum())
+    rms = math.sqrt(float((exact.astype(np.float64) ** 2).mean()))
+    half = bf16_half_spacing(exact)
+    grid = half + GRID_SLACK * rms > MAX_ABS_RMS * rms
+    bound = np.where(grid, half + GRID_SLACK * rms, MAX_ABS_RMS * rms)
+    d = np.abs(got - exact)
+    over = float((d / np.maximum(bound, 1e-300)).max()) if d.size else 0.0
+    e = np.abs(got - rounded)
+    neighbour = (e > 0) & (e <= bf16_ulp(rounded) * (1 + 1e-12))
+    return rel, mx, over, int(grid.sum()), int(neighbour.sum())
 
 
 def paired_weight_error(ig: np.ndarray, wg: np.ndarray, io: np.ndarray, wo: np.ndarray) -> float:
@@ -171,8 +195,8 @@ def check_block(wl: W.Workload, d: dict, moe, sample: Optional[torch.Tensor] = N
     if keep.any():
         if out is not None:
             got = bf16_to_f64(out.index_select(0, s_dev))[keep]
-            rep.rel_fro, rep.max_abs_over_rms, rep.ulp_neighbours = bf16_errors(
-                got, res.o[keep], oracle.bf16_to_f64(res.out)[keep])
+            (rep.rel_fro, rep.max_abs_over_rms, rep.max_abs_over_bound, rep.grid_limited,
+             rep.ulp_neighbours) = bf16_errors(got, res.o[keep], oracle.bf16_to_f64(res.out)[keep])
         if stream_in is not None:
             keep_f = math.sqrt((wl.residual_k - 1) / wl.residual_k)
             s_out = stream_dev.index_select(0, s_dev).cpu().double().numpy()
@@ -214,8 +238,8 @@ def check_dense(wl, d, moe, T: Optional[int] = None, sample: Optional[torch.Tens
     rep.tokens = len(sample)
     if out is not None:
         got = bf16_to_f64(out.index_select(0, s_dev))
-        rep.rel_fro, rep.max_abs_over_rms, rep.ulp_neighbours = bf16_errors(
-            got, res.o, oracle.bf16_to_f64(res.out))
+        (rep.rel_fro, rep.max_abs_over_rms, rep.max_abs_over_bound, rep.grid_limited,
+         rep.ulp_neighbours) = bf16_errors(got, res.o, oracle.bf16_to_f64(res.out))
     if stream_in is not None:
         keep_f = math.sqrt((wl.residual_k - 1) / wl.residual_k)
         s_out = stream_dev.index_select(0, s_dev).cpu().double().numpy()
