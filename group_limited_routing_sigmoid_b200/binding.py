@@ -32,7 +32,8 @@ SYMBOLS = (
     "beam_moe_host_fence",
     "beam_moe_dispatch_info", "beam_moe_router_stats", "beam_moe_launch_plan", "beam_moe_set_checks", "beam_moe_debug_corrupt_routing",
     "beam_moe_get_status",
-    "beam_moe_set_wait_limit", "beam_moe_set_gemm_tuning", "beam_moe_profile_begin",
+    "beam_moe_set_wait_limit", "beam_moe_set_gemm_tuning", "beam_moe_set_gate_up_layout",
+    "beam_moe_profile_begin",
     "beam_moe_profile_end", "beam_moe_check_wait_timeout", "beam_moe_last_error",
     "beam_moe_create_error", "beam_moe_destroy",
 )
@@ -77,6 +78,7 @@ def library() -> ctypes.CDLL:
         lib.beam_moe_debug_corrupt_routing.argtypes = [P, I]
         lib.beam_moe_set_wait_limit.argtypes = [P, ctypes.c_int64]
         lib.beam_moe_set_gemm_tuning.argtypes = [P, I, I, I, I, I, I, I]
+        lib.beam_moe_set_gate_up_layout.argtypes = [P, I]
         lib.beam_moe_check_wait_timeout.argtypes = [P, P]
         lib.beam_moe_profile_begin.argtypes = [P, I]
         lib.beam_moe_profile_end.argtypes = [P, P, P]
@@ -351,10 +353,10 @@ class BeamMoE:
 
     def launch_plan(self, T: int) -> dict:
         """The kernels and launch shapes a forward pass of T tokens uses."""
-        p = (ctypes.c_int32 * 10)()
+        p = (ctypes.c_int32 * 11)()
         self._check(library().beam_moe_launch_plan(self._h, int(T), ctypes.cast(p, ctypes.c_void_p)))
         keys = ("tile_rows", "cta_pairs", "grid", "down_paired", "router_tensor_cores", "router_slices",
-                "gather_rows", "ksplit_gate_up", "ksplit_down", "y_f32")
+                "gather_rows", "ksplit_gate_up", "ksplit_down", "y_f32", "gate_up_interleaved")
         return dict(zip(keys, (int(v) for v in p)))
 
     def set_checks(self, on: bool = True):
@@ -383,6 +385,10 @@ class BeamMoE:
                                                         int(token_stages)))
 
     STAGES = ("router", "dispatch", "gate_up_gemm", "down_gemm", "combine")
+
+    def set_gate_up_layout(self, layout: int = -1):
+        """0: separate gate and up tiles, 1: interleaved, -1: automatic."""
+        self._check(library().beam_moe_set_gate_up_layout(self._h, int(layout)))
 
     def profile_begin(self, max_calls: int):
         self._check(library().beam_moe_profile_begin(self._h, int(max_calls)))

@@ -56,6 +56,7 @@ struct beam_moe {
     int host_slot;
 
     CUtensorMap tm_gate, tm_up, tm_down;
+    CUtensorMap tm_gate16, tm_up16;  // the same with 16-row boxes (interleaved gate|up tiles)
     CUtensorMap tm_wcat;             // router weight as three bf16 pieces [E, 3H]
     __nv_bfloat16 *wcat;
     int router_mode;                 // -1: auto, 0: FP32 SIMT, 1: tensor cores, 2: 1 + every token re-derived
@@ -70,6 +71,7 @@ struct beam_moe {
     int use_pair;                    // 1: CTA-pair kernels for large token tiles (default)
     int gather_rows;                 // -1: auto (default), 0: never, 1: always
     int y_mode;                      // 1: FP32 expert outputs y (default), 0: bf16 y
+    int gu_layout;                   // -1: auto, 0: separate gate and up tiles, 1: interleaved
     int token_stages;                // CTA-pair kernels: token-row ring depth (0: default)
     int checks;                      // 1: validate routing and dispatch tables on the device
     int corrupt_next;                // test hook: forward passes left whose routing is corrupted
@@ -277,6 +279,7 @@ struct ForwardPlan {
     int ksplit_gate_up;   // dense layers: K slices of the gate|up GEMM (1: fused SwiGLU)
     int ksplit_down;      // dense layers: K slices of the down GEMM
     int y_f32;            // 1: the down GEMM writes the expert outputs y in FP32
+    int gu_interleaved;   // 1: CTA-pair gate|up with interleaved gate and up rows per tile
 };
 
 // Split-K slices for a GEMM of `items` work items and KB K steps: the fewest
@@ -357,6 +360,11 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
     // block per item.
     p.y_f32 = !h->dense && !h->fp4 && h->y_mode != 0;
     if (p.y_f32 && !p.cta_pairs) p.down_paired = 0;
+    // Interleaved gate|up tiles for 256-token tiles on CTA pairs: one
+    // accumulator of N columns instead of two, so two fit TMEM and the
+    // epilogue of one item overlaps the next item's MMAs.
+    p.gu_interleaved = p.cta_pairs && p.tile_rows == 256 && h->I % 128 == 0 && h->gu_layout != 0;
+    if (h->gu_layout == 1) p.gu_interleaved = p.cta_pairs && h->I % 128 == 0;
     if (h->fp4) {
         // NVFP4 weights: the single-CTA kernel with token tiles of up to 128
         // rows from the sorted copy, one weight block per down item, bf16 y
@@ -366,6 +374,7 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
         p.down_paired = 0;
         p.gather = 0;
         p.y_f32 = 0;
+        p.gu_interleaved = 0;
     }
     if (h->dense) {
         // one expert: with decode-sized T the weight tiles alone give too few
@@ -374,6 +383,7 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
         p.router_tc = 0;
         p.router_slices = 0;
         dense_splits(h, T, p.tile_rows, &p.ksplit_gate_up, &p.ksplit_down);
+        if (p.ksplit_gate_up > 1) p.gu_interleaved = 0;   // the split kernel has its own epilogue
         return p;
     }
     p.router_tc = router_on_tensor_cores(h, T);
@@ -445,7 +455,10 @@ int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *o
         g.out = h->hbuf;
         g.out_f32 = nullptr;
         g.slice_stride = 0;
-        e = plan.cta_pairs
+        e = plan.gu_interleaved
+                ? launch_grouped_gemm_pair(GemmKind::kGateUpI, BN, h->tm_gate16, h->tm_up16, h->tm_x,
+                                           g, plan.grid, s)
+            : plan.cta_pairs
                 ? launch_grouped_gemm_pair(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_x, g,
                                            plan.grid, s)
                 : launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, h->tm_x, g,
@@ -584,10 +597,13 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     if (h->fp4)
         e = launch_grouped_gemm_fp4(GemmKind::kGateUp, BN, h->fp4_gate_up, *bx, g, grid, s);
     else
-        e = use_pair ? launch_grouped_gemm_pair(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx,
-                                                g, grid, s)
-                     : launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx, g,
-                                           grid, s);
+        e = plan.gu_interleaved
+                ? launch_grouped_gemm_pair(GemmKind::kGateUpI, BN, h->tm_gate16, h->tm_up16, *bx, g,
+                                           grid, s)
+            : use_pair ? launch_grouped_gemm_pair(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx,
+                                                  g, grid, s)
+                       : launch_grouped_gemm(GemmKind::kGateUp, BN, h->tm_gate, h->tm_up, *bx, g,
+                                             grid, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "gate/up GEMM launch");
     prof_mark(h, s, 3);
     g.K = h->I;
@@ -666,6 +682,7 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     h->gather_rows = -1;
     h->router_mode = -1;
     h->y_mode = 1;
+    h->gu_layout = -1;
 
     cudaError_t e = cudaGetDevice(&h->device);
     if (e == cudaSuccess)
@@ -829,6 +846,8 @@ int finish_create(beam_moe *h, beam_moe_t *out)
 
     bool ok = h->fp4 || (make_map(&h->tm_gate, h->w_gate, E * inter, hidden, 128) &&
                          make_map(&h->tm_up, h->w_up, E * inter, hidden, 128) &&
+                         make_map(&h->tm_gate16, h->w_gate, E * inter, hidden, 16) &&
+                         make_map(&h->tm_up16, h->w_up, E * inter, hidden, 16) &&
                          make_map(&h->tm_down, h->w_down, E * hidden, inter, 128));
     if (!h->dense) ok = ok && make_map(&h->tm_wcat, h->wcat, E, 3 * (uint64_t)hidden, 128);
     for (int i = 0; i < 6 && ok; ++i) {
@@ -1239,6 +1258,7 @@ int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host)
     plan_host[7] = p.ksplit_gate_up;
     plan_host[8] = p.ksplit_down;
     plan_host[9] = p.y_f32;
+    plan_host[10] = p.gu_interleaved;
     return BEAM_OK;
 }
 
@@ -1362,6 +1382,14 @@ int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pai
     h->tile_rows = tile_rows;
     h->down_pair = down_pair;
     h->use_pair = cta_pairs;
+    return BEAM_OK;
+}
+
+int beam_moe_set_gate_up_layout(beam_moe_t h, int layout)
+{
+    if (!h) return BEAM_ERR_INVALID_ARG;
+    if (layout < -1 || layout > 1) return fail(h, BEAM_ERR_INVALID_ARG, "layout outside [-1, 1]");
+    h->gu_layout = layout;
     return BEAM_OK;
 }
 

@@ -18,8 +18,11 @@ constexpr int kStagingBytes = kEpiWarps * kStagingWarpBytes;
 constexpr int kStageBudget = kMaxDynSmem - 1024 - kBarrierBytes - kTableBytes - kStagingBytes;
 
 // Epilogues: gate|up with SwiGLU; plain bf16 (down); FP32 partial sums of a
-// K slice, gate and up side by side (kGateUpF32) or one matrix (kStoreF32).
-enum Epi { kSwiGLU = 0, kStoreBF16 = 1, kGateUpF32 = 2, kStoreF32 = 3 };
+// K slice, gate and up side by side (kGateUpF32) or one matrix (kStoreF32);
+// gate|up with SwiGLU from one interleaved weight tile (kSwiGLUI, CTA-pair
+// kernel): in each 32-row quarter of the tile, rows 0-15 are 16 gate rows
+// and rows 16-31 the up rows of the same intermediate indices.
+enum Epi { kSwiGLU = 0, kStoreBF16 = 1, kGateUpF32 = 2, kStoreF32 = 3, kSwiGLUI = 4 };
 
 // Whether the second A tile holds the same weight rows of a second matrix
 // (gate|up) rather than the next 128 rows of the same one (paired down).
@@ -143,6 +146,48 @@ __device__ __forceinline__ void epilogue_block(uint32_t taddr, int nrows, int ro
             if (c0 + j < nrows) {
                 const uint4 val = *reinterpret_cast<const uint4 *>(stg + v * 16);
                 *reinterpret_cast<uint4 *>(out + (size_t)(row0 + c0 + j) * ldo + part * 8) = val;
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// SwiGLU epilogue of an interleaved gate|up accumulator (kSwiGLUI): TMEM
+// lanes 0-15 of this warp's quarter hold gate rows, lanes 16-31 the up rows
+// of the same 16 intermediate indices.  Per chunk of 32 token columns, lane l
+// and lane l ^ 16 swap half their columns, so lane l < 16 holds gate and up
+// of columns 0-15 and lane l + 16 those of columns 16-31 for intermediate
+// index l; the 16 x 32 bf16 results go through the warp's staging block to
+// 32-byte row stores.
+//   out:   first output element of this warp's 16 intermediate columns (token row 0)
+__device__ __forceinline__ void epilogue_swiglu_interleaved(uint32_t taddr, int nrows, int row0,
+                                                            int half, int lane, uint8_t *stg,
+                                                            __nv_bfloat16 *out, int ldo)
+{
+    __nv_bfloat16 *sh = reinterpret_cast<__nv_bfloat16 *>(stg);   // [32 tokens][16 columns]
+    const bool up_lane = lane >= 16;
+    const int icol = lane & 15;
+#pragma unroll 1
+    for (int c0 = half * 32; c0 < nrows; c0 += 64) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint32_t send = up_lane ? v[j] : v[16 + j];
+            const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 16);
+            const float g = __uint_as_float(up_lane ? recv : v[j]);
+            const float u = __uint_as_float(up_lane ? v[16 + j] : recv);
+            const int tok = up_lane ? 16 + j : j;
+            sh[tok * 16 + icol] = __float2bfloat16_rn(silu_f32(g) * u);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int w = lane; w < 64; w += 32) {
+            const int tok = w >> 1, part = w & 1;
+            if (c0 + tok < nrows) {
+                const uint4 val = *reinterpret_cast<const uint4 *>(stg + tok * 32 + part * 16);
+                *reinterpret_cast<uint4 *>(out + (size_t)(row0 + c0 + tok) * ldo + part * 8) = val;
             }
         }
         __syncwarp();

@@ -51,14 +51,19 @@ struct PairCfg {
     static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
     static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS, 32);
     static constexpr int CH = 32;
-    static constexpr int ROWS_PER_ITEM = 2 * kBM * (EPI == kSwiGLU ? 1 : NUM_A);
+    // weight rows of one matrix per item: gate|up 256 (128 per CTA, both
+    // matrices), interleaved gate|up 128 (64 gate + 64 up rows per CTA),
+    // down 256 per weight block
+    static constexpr int ROWS_PER_ITEM = EPI == kSwiGLUI ? kBM : 2 * kBM * (EPI == kSwiGLU ? 1 : NUM_A);
     static constexpr int SMEM_BYTES = kMaxDynSmem;
     static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair UMMA N");
     static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0, "stages keep 1024-byte alignment");
     static_assert(kPairRingBytes >= 2 * A_STAGE + 2 * B_STAGE, "two stages per ring");
     static_assert(EPI != kSwiGLU || NUM_A == 2, "SwiGLU needs the gate and up tiles");
-    static_assert(EPI == kSwiGLU || EPI == kStoreBF16 || EPI == kStoreF32, "pair epilogues");
+    static_assert(EPI == kSwiGLU || EPI == kStoreBF16 || EPI == kStoreF32 || EPI == kSwiGLUI,
+                  "pair epilogues");
+    static_assert(EPI != kSwiGLUI || NUM_A == 1, "one interleaved tile holds gate and up");
     static_assert(4 * kPairMaxStages * 8 + 5 * 8 + 4 <= kPairBarrierBytes, "barrier block");
 };
 
@@ -170,7 +175,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             for (int item = pair; item < total && ok; item += npairs) {
                 const Item it = decode_item(item, WT, p.E, p.counts, p.offsets, p.tile_off);
                 // A rows of this CTA: its 128-row half of each 256-row block
-                const int a_base = it.e * p.R + it.wt * C::ROWS_PER_ITEM + (int)rank * kBM;
+                // (interleaved gate|up: its 64 intermediate rows of the 128)
+                const int a_base = it.e * p.R + it.wt * C::ROWS_PER_ITEM +
+                                   (int)rank * (EPI == kSwiGLUI ? kBM / 2 : kBM);
                 // gate|up: the up matrix at the same rows; down: the next 256-row block
                 const int a_row1 = EPI == kSwiGLU ? a_base : a_base + 2 * kBM;
                 for (int kb = 0; kb < KB; ++kb) {
@@ -182,8 +189,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     const uint32_t f_local = smem_u32(&fullA[sa]);
                     const uint32_t f = mapa_shared(f_local, 0);   // CTA 0's barrier
                     if (rank == 0) mbar_arrive_expect_tx(f_local, 2u * C::A_STAGE);
-                    tma_load_2d_pair(dst, &tmA0, kb * kBK, a_base, f, pol_w);
-                    if (NUM_A == 2) tma_load_2d_pair(dst + C::A_BYTES, &tmA1, kb * kBK, a_row1, f, pol_w);
+                    if constexpr (EPI == kSwiGLUI) {
+                        // 16-row boxes: gate rows to rows 32q..32q+15 of the
+                        // tile, the same up rows to 32q+16..32q+31
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            tma_load_2d_pair(dst + (uint32_t)(32 * q) * (kBK * 2), &tmA0, kb * kBK,
+                                             a_base + 16 * q, f, pol_w);
+                            tma_load_2d_pair(dst + (uint32_t)(32 * q + 16) * (kBK * 2), &tmA1,
+                                             kb * kBK, a_base + 16 * q, f, pol_w);
+                        }
+                    } else {
+                        tma_load_2d_pair(dst, &tmA0, kb * kBK, a_base, f, pol_w);
+                        if (NUM_A == 2)
+                            tma_load_2d_pair(dst + C::A_BYTES, &tmA1, kb * kBK, a_row1, f, pol_w);
+                    }
                     ++issued;
                     ring_next(sa, pa, SA);
                 }
@@ -196,7 +216,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         // issues its gather4 copies of rows straight from x.
         const uint64_t pol_x = l2_policy_evict_last();    // activations: reused across tiles
         constexpr int G = (C::HALF / 4 + 31) / 32;          // gather4 copies per lane, at most
-        const bool gather = EPI == kSwiGLU && p.gather != 0;
+        const bool gather = (EPI == kSwiGLU || EPI == kSwiGLUI) && p.gather != 0;
         int sb = 0;
         uint32_t pb = 0;
         long long issued = 0;
@@ -314,6 +334,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 const int col0 = it.wt * C::ROWS_PER_ITEM + (int)rank * kBM + quad * 32;
                 epilogue_block<EPI, C::CH, BN>(taddr, it.nrows, it.row0, half_sel, lane, stg,
                                                p.out + col0, p.R);
+            } else if constexpr (EPI == kSwiGLUI) {
+                const int col0 = it.wt * C::ROWS_PER_ITEM + (int)rank * (kBM / 2) + quad * 16;
+                epilogue_swiglu_interleaved(taddr, it.nrows, it.row0, half_sel, lane, stg,
+                                            p.out + col0, p.R);
             } else if constexpr (EPI == kStoreF32) {
                 // FP32 expert outputs: TMEM lane = output column, so each
                 // warp store is one token row's 32 consecutive floats
@@ -395,6 +419,8 @@ cudaError_t launch_pair_kind(GemmKind kind, const CUtensorMap &a0, const CUtenso
             return launch_pair<BN, 1, kStoreBF16>(a0, a1, b, args, grid, stream);
         case GemmKind::kDownPaired:
             return launch_pair<BN, 2, kStoreBF16>(a0, a1, b, args, grid, stream);
+        case GemmKind::kGateUpI:
+            return launch_pair<BN, 1, kSwiGLUI>(a0, a1, b, args, grid, stream);
         case GemmKind::kDownY32:
             return launch_pair<BN, 1, kStoreF32>(a0, a1, b, args, grid, stream);
         case GemmKind::kDownPairedY32:
@@ -418,6 +444,7 @@ cudaError_t prepare_grouped_gemm_pair()
     if ((err = set_smem_pair<BN, 1, kStoreBF16>()) != cudaSuccess) return err;    \
     if ((err = set_smem_pair<BN, 2, kStoreBF16>()) != cudaSuccess) return err;    \
     if ((err = set_smem_pair<BN, 1, kStoreF32>()) != cudaSuccess) return err;     \
+    if ((err = set_smem_pair<BN, 1, kSwiGLUI>()) != cudaSuccess) return err;      \
     if ((err = set_smem_pair<BN, 2, kStoreF32>()) != cudaSuccess) return err;
     BEAM_PREP_PAIR(64)
     BEAM_PREP_PAIR(128)

@@ -144,6 +144,8 @@ enum class GemmKind {
                    // single-CTA kernel, token tiles of up to 64 rows
     kDownF32,      // one 128-row tile, FP32 partial sums out ([slice][P][R]); as above
                    // (ksplit 1: FP32 expert outputs y)
+    kGateUpI,      // CTA-pair kernel: one interleaved tile (64 gate + 64 up rows per CTA,
+                   // 16-row box maps), SwiGLU epilogue, bf16 out; one accumulator of N columns
     kDownY32,      // CTA-pair kernel: one 256-row block, FP32 expert outputs y ([P][R])
     kDownPairedY32 // CTA-pair kernel: two 256-row blocks sharing the token tile, FP32 y
 };

@@ -329,7 +329,7 @@ int beam_moe_router_stats(beam_moe_t h, void *stream, int32_t *rederived_host);
 
 /*
  * The launch configuration a forward pass of T tokens (0 <= T <= max_tokens)
- * uses under the handle's current tuning, written to plan_host (int32 [10],
+ * uses under the handle's current tuning, written to plan_host (int32 [11],
  * host): {largest token tile of the grouped GEMMs (rows), 1 if
  * they run on CTA pairs (cta_group::2), CTAs per grouped GEMM, 1 if the down
  * projection takes two weight blocks per work item, 1 if the router logits
@@ -337,8 +337,9 @@ int beam_moe_router_stats(beam_moe_t h, void *stream, int32_t *rederived_host);
  * K slices of the router logits (0 for a dense layer), 1 if the gate|up GEMM
  * gathers token rows from x, K slices of the gate|up GEMM and of the down
  * GEMM (dense layers; 1 = no split), 1 if the down GEMM stores the expert
- * outputs in FP32 (else bf16)}.  A function of T and the tuning only;
- * launches nothing.
+ * outputs in FP32 (else bf16), 1 if the gate|up GEMM runs on interleaved
+ * gate and up tiles (see beam_moe_set_gate_up_layout)}.  A function of T and
+ * the tuning only; launches nothing.
  * Returns BEAM_ERR_INVALID_ARG for a NULL pointer or T out of range.
  */
 int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host);
@@ -421,6 +422,22 @@ int beam_moe_set_wait_limit(beam_moe_t h, int64_t limit_ns);
  */
 int beam_moe_set_gemm_tuning(beam_moe_t h, int ctas, int tile_rows, int down_pair,
                              int cta_pairs, int router_mode, int gather_rows, int token_stages);
+
+/*
+ * Layout of the gate|up GEMM's weight tiles on CTA pairs (results do not
+ * depend on it; a layout choice, not a change of the method):
+ *   0   separate tiles: each CTA holds 128 gate rows and the same 128 up
+ *       rows, in two accumulators of N columns each;
+ *   1   interleaved tiles: each CTA's 128-row tile holds 64 gate rows and
+ *       the same 64 up rows in 16-row groups, one accumulator of N columns,
+ *       so two accumulators fit tensor memory even at 256-token tiles and
+ *       one work item's epilogue overlaps the next item's MMAs; needs inter
+ *       a multiple of 128;
+ *  -1   (default) interleaved for 256-row token tiles, separate otherwise.
+ * Ignored where the gate|up GEMM does not run on CTA pairs.  Returns
+ * BEAM_ERR_INVALID_ARG for a layout outside [-1, 1].
+ */
+int beam_moe_set_gate_up_layout(beam_moe_t h, int layout);
 
 /*
  * Per-stage timing of forward passes, for measurement.  After

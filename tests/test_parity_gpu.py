@@ -89,6 +89,27 @@ def test_small_block(T, ctas, tile, pair, pairs, router, gather):
     moe.close()
 
 
+# (T, largest token tile, gathered rows, gate|up layout): CTA pairs; layout 0
+# keeps separate gate and up tiles, 1 interleaves them (the default for
+# 256-row tiles), at every pair tile size and with gathered rows too
+LAYOUT_CASES = [(1024, 256, 0, 0), (1024, 256, 0, 1), (3000, 256, 0, 0), (3000, 256, 1, 1),
+                (1024, 128, 0, 1), (777, 64, 0, 1), (130, 256, 0, 1)]
+
+
+@pytest.mark.parametrize("T,tile,gather,layout", LAYOUT_CASES)
+def test_small_block_gate_up_layouts(T, tile, gather, layout):
+    wl = W.WORKLOADS["small"]
+    d = _inputs(wl, T)
+    moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    moe.set_gemm_tuning(0, tile, -1, 1, -1, gather)
+    moe.set_gate_up_layout(layout)
+    assert moe.launch_plan(T)["gate_up_interleaved"] == layout
+    rep = check_block(wl, d, moe)
+    _log(f"small_layout_T{T}_tile{tile}_gather{gather}_layout{layout}", rep)
+    assert rep.ok(), rep
+    moe.close()
+
+
 @pytest.mark.parametrize("norm", [True, False])
 def test_tiny_residual(norm):
     wl = dataclasses.replace(W.WORKLOADS["tiny"], post_norm=norm, residual_k=20)
@@ -235,9 +256,10 @@ def test_launch_plan_follows_tokens_per_expert_and_tuning():
     assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"],
             p["gather_rows"]) == (16, 0, 0, 0, 1)
     assert p["grid"] == torch.cuda.get_device_properties(0).multi_processor_count
-    assert p["y_f32"] == 1
+    assert p["y_f32"] == 1 and p["gate_up_interleaved"] == 0
     p = moe.launch_plan(wl.T)
     assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"]) == (256, 1, 1, 1)
+    assert p["gate_up_interleaved"] == 1
     assert p["grid"] % 2 == 0 and p["router_slices"] >= 1
     assert p["gather_rows"] == 0
     moe.set_gemm_tuning(6, 64, 0, 0, 0, 1)
