@@ -176,10 +176,8 @@ def workload_config(name: str, wl) -> dict:
 def kernels_per_forward(plan: dict, dense: bool, residual: bool) -> int:
     """Kernels of this library one forward pass launches, from its launch plan."""
     if dense:
-        # table set-up, gate|up (+ SwiGLU over split-K partials), down, combine
-        # (needed for split-K partials or the residual update)
-        return (1 + 1 + (plan["ksplit_gate_up"] > 1) + 1
-                + (plan["ksplit_down"] > 1 or residual))
+        # table set-up, gate|up, down, combine (only for the residual update)
+        return 1 + 1 + 1 + int(residual)
     # router: logits + selection (CUDA cores) or tensor-core logits, selection,
     # exact re-derivation, selection of the re-derived tokens; dispatch:
     # count, scan, permute or row maps; the two GEMMs; combine
@@ -291,6 +289,8 @@ def run_ours(args):
     with sampler:
         win_ms.append(window(args.warmup, args.steps, step))
         n_win = max(MIN_WINDOWS, min(MAX_WINDOWS, int(TIMED_SPAN_S * 1e3 / max(win_ms[0], 1e-3)) + 1))
+        if args.windows > 0:
+            n_win = max(MIN_WINDOWS, args.windows)
         for w in range(1, n_win):
             win_ms.append(window(args.warmup + w * args.steps, args.steps, step))
     rederived = moe.router_stats()
@@ -370,9 +370,9 @@ def run_ours(args):
                 "frac": round(achieved / pk["bf16_sus"], 4), "peak_source": pk["source"] + " sustained",
                 "algorithmic_flops_per_launch": flops, "launch_ms": round(gate_up_ms, 4)}
     plan = moe.launch_plan(T)
-    if plan["ksplit_gate_up"] > 1:
-        roof["kernel"] = ("gate_up_gemm (grouped_gemm_kernel<%d,2,2>, split-K %d, + dense_swiglu_kernel)"
-                          % (plan["tile_rows"], plan["ksplit_gate_up"]))
+    if plan["stream_k_gate_up"]:
+        roof["kernel"] = ("gate_up_gemm (dense_sk_kernel<%d,true>, stream-K, grid %d)"
+                          % (plan["tile_rows"], plan["grid"]))
     elif wl.weight_format == "nvfp4":
         roof["kernel"] = ("gate_up_gemm (grouped_gemm_fp4_kernel<%d,2,0>, NVFP4 weights, grid %d)"
                           % (plan["tile_rows"], plan["grid"]))
@@ -533,6 +533,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=128,
                     help="tokens in the CPU-baseline sample (about 10 s of oracle work at the decode shape)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--windows", type=int, default=0,
+                    help="headline windows (0 = enough for about 2 s of device time; at least 5)")
     ap.add_argument("--gemm-tile", type=int, default=0, help="largest GEMM token tile (0 = auto)")
     ap.add_argument("--gather", type=int, default=-1,
                     help="gate|up token rows gathered from x: -1 auto (tiles <= 32 rows), 0 never, 1 always")

@@ -356,7 +356,7 @@ class BeamMoE:
         p = (ctypes.c_int32 * 11)()
         self._check(library().beam_moe_launch_plan(self._h, int(T), ctypes.cast(p, ctypes.c_void_p)))
         keys = ("tile_rows", "cta_pairs", "grid", "down_paired", "router_tensor_cores", "router_slices",
-                "gather_rows", "ksplit_gate_up", "ksplit_down", "y_f32", "gate_up_interleaved")
+                "gather_rows", "stream_k_gate_up", "stream_k_down", "y_f32", "gate_up_interleaved")
         return dict(zip(keys, (int(v) for v in p)))
 
     def set_checks(self, on: bool = True):

@@ -36,7 +36,9 @@ struct beam_moe {
     uint8_t *fp4_buf;
     Fp4Operands fp4_gate_up, fp4_down;
     float *partial;          // [nslice_max * T_max * E]
-    float *split;            // dense layers: FP32 split-K partial sums
+    float *sk_part;          // dense layers: stream-K slots, two per CTA
+    int *sk_cnt;             // dense layers: stream-K arrival counter per tile
+    int sk_cnt_n;
     int32_t *idx;            // [P]
     float *w;                // [P]
     int32_t *block_cnt, *block_base, *rank, *counts, *offsets, *tile_off, *pair_row, *row_pair;
@@ -276,46 +278,21 @@ struct ForwardPlan {
     int router_tc;     // 1: tensor-core logits with exact re-derivation
     int router_slices; // K slices of the router logits
     int gather;        // 1: gate|up gathers token rows from x; no sorted copy
-    int ksplit_gate_up;   // dense layers: K slices of the gate|up GEMM (1: fused SwiGLU)
-    int ksplit_down;      // dense layers: K slices of the down GEMM
+    int stream_k;         // dense layers: 1 = both GEMMs stream-K (decode-sized token tiles)
     int y_f32;            // 1: the down GEMM writes the expert outputs y in FP32
     int gu_interleaved;   // 1: CTA-pair gate|up with interleaved gate and up rows per tile
 };
 
-// Split-K slices for a GEMM of `items` work items and KB K steps: the fewest
-// slices (dividing KB, at least 8 steps each) that give three work items per
-// SM, or the most such slices when none does; 1 when the items suffice.
-int split_for(long long items, int KB, int num_sms)
-{
-    int best = 1;
-    for (int d = 1; d <= KB / 8; ++d) {
-        if (KB % d) continue;
-        best = d;
-        if (items * d >= 3LL * num_sms) break;
-    }
-    return best;
-}
+// Dense layers: stream-K for token tiles of up to 64 rows (decode-sized
+// batches), where the weight tiles alone give too few work items to spread
+// evenly over the SMs.
+bool dense_stream_k(const beam_moe *h, int BN) { return h->dense && BN <= 64; }
 
-// Dense layers: K slices of the gate|up and down GEMMs for T tokens in tiles
-// of BN rows (none above 64 rows: there the token tiles give work enough).
-void dense_splits(const beam_moe *h, int T, int BN, int *s_gate_up, int *s_down)
+// Stream-K grid of a dense GEMM: every SM, or the tuning's CTA count.
+int dense_sk_grid(const beam_moe *h)
 {
-    *s_gate_up = *s_down = 1;
-    if (BN > 64) return;
-    const long long tiles = (T + BN - 1) / BN;
-    *s_gate_up = split_for(tiles * (h->I / 128), h->H / 64, h->num_sms);
-    *s_down = split_for(tiles * (h->H / 128), h->I / 64, h->num_sms);
-}
-
-// FP32 partial sums the split GEMMs of T tokens in BN-row tiles write.
-size_t dense_split_floats(const beam_moe *h, int T, int BN)
-{
-    int a, b;
-    dense_splits(h, T, BN, &a, &b);
-    size_t n = 0;
-    if (a > 1) n = (size_t)a * T * 2 * h->I;
-    if (b > 1 && (size_t)b * T * h->H > n) n = (size_t)b * T * h->H;
-    return n;
+    const int g = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
+    return g < h->num_sms ? g : h->num_sms;
 }
 
 // Dense layers: the smallest power-of-two token tile (16..256) that holds T.
@@ -353,18 +330,19 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
     // large token tiles the gathers of a stage outlast its MMAs.  Automatic
     // only for tiles of up to 32 rows, where the weight stream sets the pace.
     p.gather = h->gather_rows < 0 ? (p.tile_rows <= 32 ? 1 : 0) : h->gather_rows;
-    p.ksplit_gate_up = 1;
-    p.ksplit_down = 1;
+    p.stream_k = 0;
     // Expert outputs y in FP32: the combine then rounds only once, to the
     // block's bf16 output.  The single-CTA FP32 down GEMM takes one weight
     // block per item.
     p.y_f32 = !h->dense && !h->fp4 && h->y_mode != 0;
     if (p.y_f32 && !p.cta_pairs) p.down_paired = 0;
-    // Interleaved gate|up tiles for 256-token tiles on CTA pairs: one
-    // accumulator of N columns instead of two, so two fit TMEM and the
-    // epilogue of one item overlaps the next item's MMAs.
-    p.gu_interleaved = p.cta_pairs && p.tile_rows == 256 && h->I % 128 == 0 && h->gu_layout != 0;
-    if (h->gu_layout == 1) p.gu_interleaved = p.cta_pairs && h->I % 128 == 0;
+    // Interleaved gate|up tiles on CTA pairs (on request only): one
+    // accumulator of N columns instead of two, so two fit TMEM and one
+    // item's epilogue overlaps the next item's MMAs; but each token tile is
+    // then loaded for 128 intermediate rows instead of 256, and the extra
+    // token-row traffic costs more than the overlap gains (measured at the
+    // Beam prefill shape: gate|up 4.30 -> 5.87 ms).
+    p.gu_interleaved = h->gu_layout == 1 && p.cta_pairs && h->I % 128 == 0;
     if (h->fp4) {
         // NVFP4 weights: the single-CTA kernel with token tiles of up to 128
         // rows from the sorted copy, one weight block per down item, bf16 y
@@ -382,8 +360,13 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
         p.gather = 0;
         p.router_tc = 0;
         p.router_slices = 0;
-        dense_splits(h, T, p.tile_rows, &p.ksplit_gate_up, &p.ksplit_down);
-        if (p.ksplit_gate_up > 1) p.gu_interleaved = 0;   // the split kernel has its own epilogue
+        p.stream_k = dense_stream_k(h, p.tile_rows);
+        if (p.stream_k) {
+            p.cta_pairs = 0;
+            p.gu_interleaved = 0;
+            p.down_paired = 0;
+            p.grid = dense_sk_grid(h);
+        }
         return p;
     }
     p.router_tc = router_on_tensor_cores(h, T);
@@ -401,9 +384,8 @@ void finish_profile(beam_moe *h, cudaStream_t s, int T)
 }
 
 // The dense SwiGLU MLP: the grouped GEMMs over one expert of T rows that
-// reads x directly; split-K partial sums when the plan asks for them; the
-// combine only where something is left to do (split partials to sum, or
-// the post-norm and residual update).  Stage marks as the sparse block's,
+// reads x directly, stream-K for decode-sized token tiles; the combine only
+// for the post-norm and residual update.  Stage marks as the sparse block's,
 // with empty router and a table set-up in place of the dispatch.
 int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *out,
                       float *residual, int k)
@@ -414,7 +396,8 @@ int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *o
     const int BN = plan.tile_rows;
     const int tiles = (T + BN - 1) / BN;
     cudaError_t e = launch_dense_setup(T, tiles, h->counts, h->offsets, h->tile_off, h->pair_row,
-                                       h->row_pair, h->w, s);
+                                       h->row_pair, h->w, plan.stream_k ? h->sk_cnt : nullptr,
+                                       h->sk_cnt_n, s);
     if (e != cudaSuccess) return cuda_fail(h, e, "dense set-up launch");
     prof_mark(h, s, 2);
     if (h->tm_x_ptr != x || h->tm_x_T != T) {
@@ -438,23 +421,18 @@ int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *o
     g.ctl.limit_ns = h->wait_limit_ns;
     g.b_stages = h->token_stages;
     g.a_stages = 0;
-    const int grid1 = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
+    g.out_f32 = nullptr;
+    // counters of the gate|up tiles, then of the down tiles
+    const int nt = (T + BN - 1) / BN;
+    int *cnt_gu = h->sk_cnt, *cnt_d = h->sk_cnt + (size_t)(h->I / 128) * nt;
 
     g.K = h->H;
     g.R = h->I;
-    if (plan.ksplit_gate_up > 1) {
-        g.ksplit = plan.ksplit_gate_up;
-        g.out = nullptr;
-        g.out_f32 = h->split;
-        g.slice_stride = (long long)T * 2 * h->I;
-        e = launch_grouped_gemm(GemmKind::kGateUpF32, BN, h->tm_gate, h->tm_up, h->tm_x, g, grid1, s);
-        if (e == cudaSuccess)
-            e = launch_dense_swiglu(h->split, g.ksplit, g.slice_stride, T, h->I, h->hbuf, s);
+    g.out = h->hbuf;
+    if (plan.stream_k) {
+        e = launch_dense_sk(true, BN, h->tm_gate, h->tm_up, h->tm_x, g, T, h->sk_part, cnt_gu,
+                            plan.grid, s);
     } else {
-        g.ksplit = 1;
-        g.out = h->hbuf;
-        g.out_f32 = nullptr;
-        g.slice_stride = 0;
         e = plan.gu_interleaved
                 ? launch_grouped_gemm_pair(GemmKind::kGateUpI, BN, h->tm_gate16, h->tm_up16, h->tm_x,
                                            g, plan.grid, s)
@@ -469,18 +447,12 @@ int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *o
 
     g.K = h->I;
     g.R = h->H;
-    if (plan.ksplit_down > 1) {
-        g.ksplit = plan.ksplit_down;
-        g.out = nullptr;
-        g.out_f32 = h->split;
-        g.slice_stride = (long long)T * h->H;
-        e = launch_grouped_gemm(GemmKind::kDownF32, BN, h->tm_down, h->tm_down, h->tm_h, g, grid1, s);
+    // without a residual the down projection's bf16 rows are the output
+    g.out = residual ? h->ybuf : static_cast<__nv_bfloat16 *>(out);
+    if (plan.stream_k) {
+        e = launch_dense_sk(false, BN, h->tm_down, h->tm_down, h->tm_h, g, T, h->sk_part, cnt_d,
+                            plan.grid, s);
     } else {
-        // without a residual the down projection's bf16 rows are the output
-        g.ksplit = 1;
-        g.out = residual ? h->ybuf : static_cast<__nv_bfloat16 *>(out);
-        g.out_f32 = nullptr;
-        g.slice_stride = 0;
         const GemmKind dk = plan.down_paired ? GemmKind::kDownPaired : GemmKind::kDown;
         e = plan.cta_pairs ? launch_grouped_gemm_pair(dk, BN, h->tm_down, h->tm_down, h->tm_h, g,
                                                       plan.grid, s)
@@ -490,14 +462,11 @@ int run_forward_dense(beam_moe *h, cudaStream_t s, const void *x, int T, void *o
     if (e != cudaSuccess) return cuda_fail(h, e, "down GEMM launch");
     prof_mark(h, s, 4);
 
-    if (plan.ksplit_down > 1 || residual) {
+    if (residual) {
         CombineArgs c;
         c.status = h->status;
         c.y = h->ybuf;
         c.y32 = nullptr;
-        c.y_f32 = plan.ksplit_down > 1 ? h->split : nullptr;
-        c.nslice = plan.ksplit_down;
-        c.slice_stride = (long long)T * h->H;
         c.pair_row = h->pair_row;
         c.w = h->w;
         c.T = T;
@@ -576,9 +545,7 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     g.row_pair = h->row_pair;
     g.top_k = h->top_k;
     g.gather = plan.gather;
-    g.ksplit = 1;
     g.out_f32 = nullptr;
-    g.slice_stride = 0;
     // token rows of the gate|up GEMM: x itself, four rows per gather4 copy,
     // or boxes of the sorted copy
     BoxMaps bx_local;
@@ -627,9 +594,6 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     c.status = h->status;
     c.y = plan.y_f32 ? nullptr : h->ybuf;
     c.y32 = plan.y_f32 ? h->y32 : nullptr;
-    c.y_f32 = nullptr;
-    c.nslice = 0;
-    c.slice_stride = 0;
     c.pair_row = h->pair_row;
     c.w = h->w;
     c.T = T;
@@ -698,15 +662,15 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     const size_t nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
     // router partial sums: the largest nslice(t) * t over t <= max_tokens, for
     // either router path; dense layers: the largest split-K partial sums
-    size_t partial_rows = 0, split_floats = 0;
-    for (int t = 1; t <= max_tokens; ++t) {
-        if (h->dense) {   // every token tile a tuning may ask for
-            for (int bn = 16; bn <= 64; bn <<= 1) {
-                const size_t n = dense_split_floats(h, t, bn);
-                if (n > split_floats) split_floats = n;
-            }
-            continue;
-        }
+    size_t partial_rows = 0;
+    // dense layers: stream-K slots (two per CTA, at the largest stream-K
+    // token tile) and an arrival counter per tile of either GEMM, for every
+    // token tile a tuning may ask for (16 rows: the most tiles)
+    const size_t sk_floats = h->dense ? dense_sk_part_floats(64, true, h->num_sms) : 0;
+    h->sk_cnt_n = h->dense ? (int)((size_t)(hidden > inter ? hidden : inter) / 128 * 2 *
+                                   ((size_t)(max_tokens + 15) / 16))
+                           : 0;
+    for (int t = 1; t <= max_tokens && !h->dense; ++t) {
         const size_t r0 = (size_t)router_small_slices(t, hidden, n_experts, h->num_sms) * t;
         if (r0 > partial_rows) partial_rows = r0;
         const size_t r1 = (size_t)router_slices(t, hidden, n_experts, h->num_sms) * t;
@@ -721,7 +685,8 @@ int finish_create(beam_moe *h, beam_moe_t *out)
         return o;
     };
     const size_t o_partial = carve(partial_rows * E * 4);
-    const size_t o_split = carve(split_floats * 4);
+    const size_t o_skpart = carve(sk_floats * 4);
+    const size_t o_skcnt = carve((size_t)h->sk_cnt_n * 4);
     const size_t o_idx = carve(P * 4);
     const size_t o_w = carve(P * 4);
     const size_t o_bcnt = carve(nblk * E * 4);
@@ -755,7 +720,8 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     }
     char *b = static_cast<char *>(h->ws);
     h->partial = reinterpret_cast<float *>(b + o_partial);
-    h->split = reinterpret_cast<float *>(b + o_split);
+    h->sk_part = reinterpret_cast<float *>(b + o_skpart);
+    h->sk_cnt = reinterpret_cast<int *>(b + o_skcnt);
     h->idx = reinterpret_cast<int32_t *>(b + o_idx);
     h->w = reinterpret_cast<float *>(b + o_w);
     h->block_cnt = reinterpret_cast<int32_t *>(b + o_bcnt);
@@ -785,6 +751,7 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     if (e == cudaSuccess) e = cudaMemset(h->check_where, 0x7f, sizeof(int));
     if (e == cudaSuccess) e = prepare_grouped_gemm(n_experts);
     if (e == cudaSuccess) e = prepare_dispatch(n_experts);
+    if (e == cudaSuccess && h->dense) e = prepare_dense_sk();
     if (e == cudaSuccess && h->fp4) {
         // the tiled copy of the three NVFP4 tensors (gate, up: [E*I, H];
         // down: [E*H, I]), made once on the legacy default stream
@@ -1255,8 +1222,8 @@ int beam_moe_launch_plan(beam_moe_t h, int T, int32_t *plan_host)
     plan_host[4] = p.router_tc;
     plan_host[5] = p.router_slices;
     plan_host[6] = p.gather;
-    plan_host[7] = p.ksplit_gate_up;
-    plan_host[8] = p.ksplit_down;
+    plan_host[7] = p.stream_k;
+    plan_host[8] = p.stream_k;
     plan_host[9] = p.y_f32;
     plan_host[10] = p.gu_interleaved;
     return BEAM_OK;

@@ -3,7 +3,6 @@
 //
 //   o[t]   = routed_scaling * sum_j w[t,j] * y[row(t,j)]     (FP32 or bf16 y, FP32 sum,
 //                                                             slot order)
-//            (dense layer: o[t] = sum_s y_s[t] over FP32 split-K slices, in slice order)
 //   out[t] = bf16_rn(o[t])
 //   n[t]   = o[t] / sqrt(mean(o[t]^2) + eps) * gamma          (if gamma)
 //   stream[t] <- sqrt((k-1)/k) * stream[t] + n[t] / sqrt(k)
@@ -36,7 +35,7 @@ __device__ __forceinline__ void unpack8(const uint4 &raw, float (&v)[8])
 // vector are issued before their sums, which take the slots in order (FP32
 // FMA), so every value is the same slot-order sum.
 // WIDE: FP32 expert outputs (a.y32), all top_k slots' loads in flight at
-// once; otherwise bf16 outputs (a.y) or the dense layer's FP32 slices.
+// once; otherwise bf16 outputs (a.y).
 template <bool WIDE>
 __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
 {
@@ -49,7 +48,7 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
     const int t = blockIdx.x;
     const int tid = threadIdx.x;
     const int nvec = a.H / 8;
-    const int nsum = a.y_f32 ? 0 : a.top_k;   // expert slots (none for FP32 slices)
+    const int nsum = a.top_k;                  // expert slots
     constexpr bool wide = WIDE;                // FP32 expert outputs
     if (tid < nsum) {
         rows[tid] = a.pair_row[(size_t)t * a.top_k + tid];
@@ -89,15 +88,6 @@ __global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
                 }
             }
         } else {
-            if (a.y_f32) {
-                for (int sl = 0; sl < a.nslice; ++sl) {
-                    const float4 *src = reinterpret_cast<const float4 *>(
-                        a.y_f32 + (size_t)sl * (size_t)a.slice_stride + (size_t)t * a.H + 8 * q);
-                    const float4 lo = src[0], hi = src[1];
-                    acc[v][0] += lo.x; acc[v][1] += lo.y; acc[v][2] += lo.z; acc[v][3] += lo.w;
-                    acc[v][4] += hi.x; acc[v][5] += hi.y; acc[v][6] += hi.z; acc[v][7] += hi.w;
-                }
-            }
             for (int j0 = 0; j0 < nsum; j0 += kCombBatch) {
                 uint4 raw[kCombBatch];
 #pragma unroll

@@ -17,16 +17,15 @@ constexpr int kStagingWarpBytes = 2048;                // one 32-row x CH-column
 constexpr int kStagingBytes = kEpiWarps * kStagingWarpBytes;
 constexpr int kStageBudget = kMaxDynSmem - 1024 - kBarrierBytes - kTableBytes - kStagingBytes;
 
-// Epilogues: gate|up with SwiGLU; plain bf16 (down); FP32 partial sums of a
-// K slice, gate and up side by side (kGateUpF32) or one matrix (kStoreF32);
+// Epilogues: gate|up with SwiGLU; plain bf16 (down); FP32 (kStoreF32);
 // gate|up with SwiGLU from one interleaved weight tile (kSwiGLUI, CTA-pair
 // kernel): in each 32-row quarter of the tile, rows 0-15 are 16 gate rows
 // and rows 16-31 the up rows of the same intermediate indices.
-enum Epi { kSwiGLU = 0, kStoreBF16 = 1, kGateUpF32 = 2, kStoreF32 = 3, kSwiGLUI = 4 };
+enum Epi { kSwiGLU = 0, kStoreBF16 = 1, kStoreF32 = 3, kSwiGLUI = 4 };
 
 // Whether the second A tile holds the same weight rows of a second matrix
 // (gate|up) rather than the next 128 rows of the same one (paired down).
-constexpr bool same_rows(int epi) { return epi == kSwiGLU || epi == kGateUpF32; }
+constexpr bool same_rows(int epi) { return epi == kSwiGLU; }
 
 constexpr int pow2_at_least(int v, int lo)
 {
@@ -194,7 +193,7 @@ __device__ __forceinline__ void epilogue_swiglu_interleaved(uint32_t taddr, int 
     }
 }
 
-// FP32 partial sums of one accumulator (32 TMEM lanes of this warp,
+// FP32 values of one accumulator (32 TMEM lanes of this warp,
 // `nrows` columns): TMEM lane l is output column l of the warp's 32, TMEM
 // column j is token row j, so each store instruction of the warp writes one
 // row's 32 consecutive floats (128 bytes).  Chunks of 16 columns alternate

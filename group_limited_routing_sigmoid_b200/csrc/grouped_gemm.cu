@@ -58,7 +58,7 @@ struct Cfg {
     static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS, 32);
     static constexpr int CH = BN >= 32 ? 32 : 16;           // epilogue columns per chunk
     static constexpr int ROWS_PER_ITEM = same_rows(EPI) ? kBM : NUM_A * kBM;
-    static constexpr bool F32 = EPI == kGateUpF32 || EPI == kStoreF32;   // split-K partials
+    static constexpr bool F32 = EPI == kStoreF32;   // FP32 expert outputs
     static constexpr int SMEM_BYTES =
         1024 + STAGES * STAGE_BYTES + kStagingBytes + kBarrierBytes + kTableBytes;
     static_assert(STAGES >= 2, "pipeline needs two stages");
@@ -67,7 +67,7 @@ struct Cfg {
     static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment of the next tile");
     static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory");
     static_assert(!same_rows(EPI) || NUM_A == 2, "gate|up needs the gate and up tiles");
-    static_assert(!F32 || (EPI == kStoreF32 ? NUM_A == 1 : true), "FP32 down: one tile");
+    static_assert(!F32 || NUM_A == 1, "FP32 down: one tile");
     static_assert(32 * CH * 2 <= kStagingWarpBytes, "staging block");
 };
 
@@ -127,10 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     const int WT = p.R / C::ROWS_PER_ITEM;
-    const int S = C::F32 ? p.ksplit : 1;          // K slices per (weight tile, token tile)
     // no work while the status word is set (a failed check or wait)
-    const int total = status_is_set(p.ctl.status) ? 0 : WT * s_tile[p.E] * S;
-    const int KB = p.K / kBK / S;                 // K steps of one slice
+    const int total = status_is_set(p.ctl.status) ? 0 : WT * s_tile[p.E];
+    const int KB = p.K / kBK;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -146,8 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         long long issued = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const Item it = decode_item(item / S, WT, p.E, s_counts, s_offsets, s_tile);
-            const int kb0 = (item % S) * KB;
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const int kb0 = 0;
             const int a_row = it.e * p.R + it.wt * C::ROWS_PER_ITEM;
             const int n_load = (it.nrows + 15) & ~15;
             const uint32_t bytes = NUM_A * C::A_BYTES + n_load * (kBK * 2);
@@ -222,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool issued_any = false;
         int iter = 0;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++iter) {
-            const Item it = decode_item(item / S, WT, p.E, s_counts, s_offsets, s_tile);
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
             const int n_mma = (it.nrows + 15) & ~15;
             const uint32_t idesc = umma_idesc_bf16_f32(kBM, n_mma);
             const int acc = iter % C::NBUF;
@@ -277,18 +276,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.ctl);
             if (!__all_sync(0xffffffffu, ok)) break;   // warp-uniform from here on
             tc_fence_after();
-            const Item it = decode_item(item / S, WT, p.E, s_counts, s_offsets, s_tile);
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
             if constexpr (C::F32) {
-                float *out = p.out_f32 + (size_t)(item % S) * (size_t)p.slice_stride;
                 const int col0 = it.wt * kBM + quad * 32;
-                if constexpr (EPI == kGateUpF32) {
-                    epilogue_f32(taddr, it.nrows, it.row0, half, lane, out + col0, 2 * p.R);
-                    epilogue_f32(taddr + BN, it.nrows, it.row0, half, lane, out + p.R + col0, 2 * p.R);
-                } else {
-                    epilogue_f32(taddr, it.nrows, it.row0, half, lane, out + col0, p.R);
-                }
+                epilogue_f32(taddr, it.nrows, it.row0, half, lane, p.out_f32 + col0, p.R);
             } else if constexpr (EPI == kSwiGLU) {
                 const int col0 = it.wt * C::ROWS_PER_ITEM + quad * 32;
                 epilogue_block<EPI, C::CH, BN>(taddr, it.nrows, it.row0, half, lane, stg,
@@ -347,9 +340,6 @@ cudaError_t launch_kind(GemmKind kind, const CUtensorMap &a0, const CUtensorMap 
             return launch<BN, 1, kStoreBF16>(a0, a1, b, args, grid, stream);
         case GemmKind::kDownPaired:
             return launch<BN, 2, kStoreBF16>(a0, a1, b, args, grid, stream);
-        case GemmKind::kGateUpF32:
-            if constexpr (BN <= 64) return launch<BN, 2, kGateUpF32>(a0, a1, b, args, grid, stream);
-            return cudaErrorInvalidValue;
         case GemmKind::kDownF32:
             return launch<BN, 1, kStoreF32>(a0, a1, b, args, grid, stream);
         default:
@@ -373,18 +363,12 @@ cudaError_t prepare_grouped_gemm(int E)
     if ((err = set_smem<BN, 1, kStoreBF16>()) != cudaSuccess) return err;    \
     if ((err = set_smem<BN, 2, kStoreBF16>()) != cudaSuccess) return err;    \
     if ((err = set_smem<BN, 1, kStoreF32>()) != cudaSuccess) return err;
-#define BEAM_PREP_F32(BN)                                                    \
-    if ((err = set_smem<BN, 2, kGateUpF32>()) != cudaSuccess) return err;
     BEAM_PREP(16)
     BEAM_PREP(32)
     BEAM_PREP(64)
     BEAM_PREP(128)
     BEAM_PREP(256)
-    BEAM_PREP_F32(16)
-    BEAM_PREP_F32(32)
-    BEAM_PREP_F32(64)
 #undef BEAM_PREP
-#undef BEAM_PREP_F32
     return prepare_grouped_gemm_pair();
 }
 

@@ -115,12 +115,8 @@ struct GemmArgs {
     const int32_t *row_pair;     // [P]
     int top_k;
     int gather;
-    // split-K (single-CTA kernel, FP32-partials kinds only): work item i takes
-    // K slice i % ksplit and writes its FP32 partial sums to
-    // out_f32 + slice * slice_stride
-    int ksplit;
+    // FP32 outputs (kDownF32, kDownY32, kDownPairedY32): [P, R] instead of out
     float *out_f32;
-    long long slice_stride;
     // CTA-pair kernel: depth of the token-row ring (0 = default); the weight
     // ring's depth is derived at launch (a_stages)
     int b_stages;
@@ -140,10 +136,7 @@ enum class GemmKind {
     kGateUp,       // gate and up tiles, SwiGLU epilogue, bf16 out
     kDown,         // one 128-row tile, bf16 out
     kDownPaired,   // two consecutive 128-row tiles sharing the token tile, bf16 out
-    kGateUpF32,    // gate and up tiles, FP32 partial sums out ([slice][P][2R]: gate, then up);
-                   // single-CTA kernel, token tiles of up to 64 rows
-    kDownF32,      // one 128-row tile, FP32 partial sums out ([slice][P][R]); as above
-                   // (ksplit 1: FP32 expert outputs y)
+    kDownF32,      // one 128-row tile, FP32 expert outputs y ([P][R]) in out_f32
     kGateUpI,      // CTA-pair kernel: one interleaved tile (64 gate + 64 up rows per CTA,
                    // 16-row box maps), SwiGLU epilogue, bf16 out; one accumulator of N columns
     kDownY32,      // CTA-pair kernel: one 256-row block, FP32 expert outputs y ([P][R])
@@ -172,12 +165,6 @@ struct CombineArgs {
     const __nv_bfloat16 *y;      // [P, H] expert outputs (bf16), or
     const float *y32;            // [P, H] expert outputs (FP32); exactly one of y, y32 is set
                                  // for a sparse block
-    // instead of y (dense layer, top_k == 1, unit weight): FP32 partial sums
-    // of nslice split-K slices [nslice][T][H], slice_stride elements apart,
-    // summed in slice order
-    const float *y_f32;
-    int nslice;
-    long long slice_stride;
     const int32_t *pair_row;     // [P]
     const float *w;              // [T, top_k]
     int T, H, top_k;
@@ -205,9 +192,16 @@ cudaError_t launch_corrupt_routing(int32_t *idx, int E, cudaStream_t stream);
 // ------------------------------------------------------------- dense layer
 cudaError_t launch_dense_setup(int T, int tiles, int32_t *counts, int32_t *offsets,
                                int32_t *tile_off, int32_t *pair_row, int32_t *row_pair, float *w,
-                               cudaStream_t stream);
-cudaError_t launch_dense_swiglu(const float *part, int S, long long slice_stride, int T, int I,
-                                __nv_bfloat16 *h, cudaStream_t stream);
+                               int *cnt, int ncnt, cudaStream_t stream);
+// Stream-K GEMMs of a dense layer (dense_sk.cu): gate|up (SwiGLU to bf16 h)
+// or down (bf16 out), token tiles of BN = 16, 32 or 64 rows; `part` holds
+// dense_sk_part_floats(BN, gate_up, grid) floats; `cnt` one zeroed counter per
+// (weight tile, token tile).
+cudaError_t launch_dense_sk(bool gate_up, int BN, const CUtensorMap &a0, const CUtensorMap &a1,
+                            const BoxMaps &b, const GemmArgs &args, int T, float *part, int *cnt, int grid,
+                            cudaStream_t stream);
+size_t dense_sk_part_floats(int BN, bool gate_up, int grid);
+cudaError_t prepare_dense_sk();
 
 // ------------------------------------------------------------- self-check
 cudaError_t launch_wait_timeout_check(WaitCtl ctl, cudaStream_t stream);

@@ -39,7 +39,9 @@ def _log(case, rep, plan):
 DENSE_CASES = [(1, 0, 0, 1, False), (3, 0, 0, 1, False), (37, 5, 0, 1, False), (64, 0, 0, 1, False),
                (100, 0, 0, 1, False), (300, 0, 0, 1, False), (1000, 3, 0, 1, False),
                (1000, 0, 0, 0, False), (64, 0, 256, 1, False), (300, 0, 16, 1, False),
-               (64, 0, 0, 1, True), (300, 0, 0, 1, True), (300, 0, 16, 1, True)]
+               (64, 0, 0, 1, True), (300, 0, 0, 1, True), (300, 0, 16, 1, True),
+               (64, 7, 0, 1, False), (37, 1, 0, 1, False), (64, 0, 32, 1, False),
+               (200, 5, 16, 1, False)]
 
 
 @pytest.mark.parametrize("T,ctas,tile,pairs,resid", DENSE_CASES)
@@ -59,7 +61,7 @@ def test_dense_layer(T, ctas, tile, pairs, resid):
     moe.close()
 
 
-def test_dense_plan_splits_k_for_few_tokens():
+def test_dense_plan_streams_k_for_few_tokens():
     wl = W.WORKLOADS["dense_decode"]
     g = W.generator(wl, "cuda")
     # the plan depends on the shapes only: small stand-in weights of the right size are enough
@@ -68,10 +70,10 @@ def test_dense_plan_splits_k_for_few_tokens():
              w_down=torch.zeros(1, wl.hidden, wl.inter, dtype=torch.bfloat16, device="cuda"))
     moe = BeamMoE.from_workload(wl, w, max_tokens=8192)
     p = moe.launch_plan(64)
-    assert p["tile_rows"] == 64 and p["ksplit_gate_up"] > 1 and p["ksplit_down"] > 1
+    assert p["tile_rows"] == 64 and p["stream_k_gate_up"] == 1 and p["stream_k_down"] == 1
     assert p["router_tensor_cores"] == 0 and p["gather_rows"] == 0
     p = moe.launch_plan(8192)
-    assert p["tile_rows"] == 256 and p["ksplit_gate_up"] == 1 and p["ksplit_down"] == 1
+    assert p["tile_rows"] == 256 and p["stream_k_gate_up"] == 0 and p["stream_k_down"] == 0
     x = torch.zeros(4, wl.hidden, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(BeamMoEError) as err:
         moe.route(x)

@@ -90,8 +90,8 @@ def test_small_block(T, ctas, tile, pair, pairs, router, gather):
 
 
 # (T, largest token tile, gathered rows, gate|up layout): CTA pairs; layout 0
-# keeps separate gate and up tiles, 1 interleaves them (the default for
-# 256-row tiles), at every pair tile size and with gathered rows too
+# keeps separate gate and up tiles (the default), 1 interleaves them, at
+# every pair tile size and with gathered rows too
 LAYOUT_CASES = [(1024, 256, 0, 0), (1024, 256, 0, 1), (3000, 256, 0, 0), (3000, 256, 1, 1),
                 (1024, 128, 0, 1), (777, 64, 0, 1), (130, 256, 0, 1)]
 
@@ -259,7 +259,7 @@ def test_launch_plan_follows_tokens_per_expert_and_tuning():
     assert p["y_f32"] == 1 and p["gate_up_interleaved"] == 0
     p = moe.launch_plan(wl.T)
     assert (p["tile_rows"], p["cta_pairs"], p["down_paired"], p["router_tensor_cores"]) == (256, 1, 1, 1)
-    assert p["gate_up_interleaved"] == 1
+    assert p["gate_up_interleaved"] == 0
     assert p["grid"] % 2 == 0 and p["router_slices"] >= 1
     assert p["gather_rows"] == 0
     moe.set_gemm_tuning(6, 64, 0, 0, 0, 1)
