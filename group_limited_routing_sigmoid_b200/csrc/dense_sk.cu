@@ -296,7 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             float *slot = part + (size_t)(2 * b + (sg.first ? 0 : 1)) * C::PART;
 #pragma unroll 1
             for (int a = 0; a < C::NUM_A; ++a)
-                epilogue_f32(taddr + a * BN, nrows, 0, half, lane, slot + a * kBM + quad * 32, C::NUM_A * kBM);
+                epilogue_f32_staged(taddr + a * BN, nrows, 0, half, lane, stg, slot + a * kBM + quad * 32,
+                                    C::NUM_A * kBM);
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));   // TMEM is free again; the rest reads memory
             __threadfence();

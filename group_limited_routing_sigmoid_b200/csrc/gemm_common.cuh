@@ -193,24 +193,34 @@ __device__ __forceinline__ void epilogue_swiglu_interleaved(uint32_t taddr, int 
     }
 }
 
-// FP32 values of one accumulator (32 TMEM lanes of this warp,
-// `nrows` columns): TMEM lane l is output column l of the warp's 32, TMEM
-// column j is token row j, so each store instruction of the warp writes one
-// row's 32 consecutive floats (128 bytes).  Chunks of 16 columns alternate
-// between the two warps of a quadrant.
+// FP32 values of one accumulator (32 TMEM lanes of this warp = 32 output
+// columns, `nrows` token columns), transposed through the warp's staging
+// block so that each store is a 16-byte vector: chunks of 16 token rows
+// alternate between the two warps of a quadrant; a chunk is 16 rows x 128
+// bytes, four vectors per lane.
 //   out:   this warp's first output column in token row 0
 //   ldo:   output row stride in elements
-__device__ __forceinline__ void epilogue_f32(uint32_t taddr, int nrows, int row0, int half, int lane,
-                                             float *out, int ldo)
+__device__ __forceinline__ void epilogue_f32_staged(uint32_t taddr, int nrows, int row0, int half,
+                                                    int lane, uint8_t *stg, float *out, int ldo)
 {
+    float *sh = reinterpret_cast<float *>(stg);   // [16 token rows][32 columns]
 #pragma unroll 1
     for (int c0 = half * 16; c0 < nrows; c0 += 32) {
         uint32_t v[16];
         tmem_ld16(taddr + c0, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (c0 + j < nrows) out[(size_t)(row0 + c0 + j) * ldo + lane] = __uint_as_float(v[j]);
+        for (int j = 0; j < 16; ++j) sh[j * 32 + lane] = __uint_as_float(v[j]);
+        __syncwarp();
+#pragma unroll
+        for (int w = lane; w < 128; w += 32) {
+            const int j = w >> 3, part = w & 7;
+            if (c0 + j < nrows) {
+                const float4 val = *reinterpret_cast<const float4 *>(sh + j * 32 + part * 4);
+                *reinterpret_cast<float4 *>(out + (size_t)(row0 + c0 + j) * ldo + part * 4) = val;
+            }
+        }
+        __syncwarp();
     }
 }
 

@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
             if constexpr (C::F32) {
                 const int col0 = it.wt * kBM + quad * 32;
-                epilogue_f32(taddr, it.nrows, it.row0, half, lane, p.out_f32 + col0, p.R);
+                epilogue_f32_staged(taddr, it.nrows, it.row0, half, lane, stg, p.out_f32 + col0, p.R);
             } else if constexpr (EPI == kSwiGLU) {
                 const int col0 = it.wt * C::ROWS_PER_ITEM + quad * 32;
                 epilogue_block<EPI, C::CH, BN>(taddr, it.nrows, it.row0, half, lane, stg,

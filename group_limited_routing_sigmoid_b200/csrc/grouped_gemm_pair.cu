@@ -40,6 +40,7 @@ constexpr int kPairMaxStages = 16;              // barrier slots per ring
 constexpr int kPairBarrierBytes = 1024;
 constexpr int kPairRingBytes = kMaxDynSmem - 1024 - kPairBarrierBytes - kStagingBytes;
 constexpr int kPairDefaultBStages = 3;
+constexpr int kPairCh = 32;                     // epilogue token columns per chunk (bf16 paths)
 
 template <int BN, int NUM_A, int EPI>
 struct PairCfg {
@@ -50,7 +51,6 @@ struct PairCfg {
     static constexpr int ACC_COLS = NUM_A * BN;            // per CTA: 128 lanes x N per matrix
     static constexpr int NBUF = 2 * ACC_COLS <= 512 ? 2 : 1;
     static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS, 32);
-    static constexpr int CH = 32;
     // weight rows of one matrix per item: gate|up 256 (128 per CTA, both
     // matrices), interleaved gate|up 128 (64 gate + 64 up rows per CTA),
     // down 256 per weight block
@@ -68,6 +68,18 @@ struct PairCfg {
 };
 
 constexpr uint16_t kPairMask = 0x3;
+
+// K step of loop iteration kb for weight block wt of WT: each weight block
+// of an expert starts its K loop at its own offset (KB * wt / WT), so the
+// pairs working on one expert's token tile at the same time do not all ask
+// for the same token rows at once; the first to reach a stage brings it from
+// HBM and the others find it in L2.  Every role of the item walks the same
+// order; the sum over K is the same up to FP32 rounding order.
+__device__ __forceinline__ int k_step(int kb, int wt, int WT, int KB)
+{
+    int k = kb + (int)(((long long)KB * wt) / WT);
+    return k >= KB ? k - KB : k;
+}
 
 __device__ __forceinline__ void ring_next(int &s, uint32_t &ph, int n)
 {
@@ -181,6 +193,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 // gate|up: the up matrix at the same rows; down: the next 256-row block
                 const int a_row1 = EPI == kSwiGLU ? a_base : a_base + 2 * kBM;
                 for (int kb = 0; kb < KB; ++kb) {
+                    const int kr = k_step(kb, it.wt, WT, KB);
                     if (!mbar_wait(smem_u32(&emptyA[sa]), pa ^ 1u, p.ctl)) {
                         ok = false;
                         break;
@@ -194,15 +207,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         // tile, the same up rows to 32q+16..32q+31
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            tma_load_2d_pair(dst + (uint32_t)(32 * q) * (kBK * 2), &tmA0, kb * kBK,
+                            tma_load_2d_pair(dst + (uint32_t)(32 * q) * (kBK * 2), &tmA0, kr * kBK,
                                              a_base + 16 * q, f, pol_w);
                             tma_load_2d_pair(dst + (uint32_t)(32 * q + 16) * (kBK * 2), &tmA1,
-                                             kb * kBK, a_base + 16 * q, f, pol_w);
+                                             kr * kBK, a_base + 16 * q, f, pol_w);
                         }
                     } else {
-                        tma_load_2d_pair(dst, &tmA0, kb * kBK, a_base, f, pol_w);
+                        tma_load_2d_pair(dst, &tmA0, kr * kBK, a_base, f, pol_w);
                         if (NUM_A == 2)
-                            tma_load_2d_pair(dst + C::A_BYTES, &tmA1, kb * kBK, a_row1, f, pol_w);
+                            tma_load_2d_pair(dst + C::A_BYTES, &tmA1, kr * kBK, a_row1, f, pol_w);
                     }
                     ++issued;
                     ring_next(sa, pa, SA);
@@ -230,6 +243,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             int tok[G][4];
             if (gather) gather_tokens<G>(p, it, (int)rank * half, half >> 2, lane, tok);
             for (int kb = 0; kb < KB; ++kb) {
+                const int kr = k_step(kb, it.wt, WT, KB);
                 bool got = true;
                 if (lane == 0 || gather) got = mbar_wait(smem_u32(&emptyB[sb]), pb ^ 1u, p.ctl);
                 ok = __all_sync(0xffffffffu, got);
@@ -245,7 +259,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         for (int bi = 4; bi >= 0; --bi) {   // boxes of 128, 64, 32, 16, 8 rows
                             const int hgt = 8 << bi;
                             if (hgt <= C::HALF && half - off >= hgt) {
-                                tma_load_2d_pair(dst + off * (kBK * 2), &tmB.m[bi], kb * kBK,
+                                tma_load_2d_pair(dst + off * (kBK * 2), &tmB.m[bi], kr * kBK,
                                                  b_row + off, f, pol_x);
                                 off += hgt;
                             }
@@ -257,7 +271,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     for (int g = 0; g < G; ++g) {
                         const int op = lane + 32 * g;
                         if (op < (half >> 2))
-                            tma_gather4_pair(dst + op * (4 * kBK * 2), &tmB.gather, kb * kBK,
+                            tma_gather4_pair(dst + op * (4 * kBK * 2), &tmB.gather, kr * kBK,
                                              tok[g][0], tok[g][1], tok[g][2], tok[g][3], f, pol_x);
                     }
                 }
@@ -332,28 +346,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
             if constexpr (EPI == kSwiGLU) {
                 const int col0 = it.wt * C::ROWS_PER_ITEM + (int)rank * kBM + quad * 32;
-                epilogue_block<EPI, C::CH, BN>(taddr, it.nrows, it.row0, half_sel, lane, stg,
+                epilogue_block<EPI, kPairCh, BN>(taddr, it.nrows, it.row0, half_sel, lane, stg,
                                                p.out + col0, p.R);
             } else if constexpr (EPI == kSwiGLUI) {
                 const int col0 = it.wt * C::ROWS_PER_ITEM + (int)rank * (kBM / 2) + quad * 16;
                 epilogue_swiglu_interleaved(taddr, it.nrows, it.row0, half_sel, lane, stg,
                                             p.out + col0, p.R);
             } else if constexpr (EPI == kStoreF32) {
-                // FP32 expert outputs: TMEM lane = output column, so each
-                // warp store is one token row's 32 consecutive floats
+                // FP32 expert outputs through the staging block, 16-byte stores
 #pragma unroll 1
                 for (int a = 0; a < NUM_A; ++a) {
                     const int col0 =
                         it.wt * C::ROWS_PER_ITEM + a * 2 * kBM + (int)rank * kBM + quad * 32;
-                    epilogue_f32(taddr + a * BN, it.nrows, it.row0, half_sel, lane,
-                                 p.out_f32 + col0, p.R);
+                    epilogue_f32_staged(taddr + a * BN, it.nrows, it.row0, half_sel, lane, stg,
+                                        p.out_f32 + col0, p.R);
                 }
             } else {
 #pragma unroll 1
                 for (int a = 0; a < NUM_A; ++a) {
                     const int col0 =
                         it.wt * C::ROWS_PER_ITEM + a * 2 * kBM + (int)rank * kBM + quad * 32;
-                    epilogue_block<EPI, C::CH, 0>(taddr + a * BN, it.nrows, it.row0, half_sel,
+                    epilogue_block<EPI, kPairCh, 0>(taddr + a * BN, it.nrows, it.row0, half_sel,
                                                   lane, stg, p.out + col0, p.R);
                 }
             }
