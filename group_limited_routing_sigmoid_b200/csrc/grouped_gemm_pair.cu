@@ -69,18 +69,6 @@ struct PairCfg {
 
 constexpr uint16_t kPairMask = 0x3;
 
-// K step of loop iteration kb for weight block wt of WT: each weight block
-// of an expert starts its K loop at its own offset (KB * wt / WT), so the
-// pairs working on one expert's token tile at the same time do not all ask
-// for the same token rows at once; the first to reach a stage brings it from
-// HBM and the others find it in L2.  Every role of the item walks the same
-// order; the sum over K is the same up to FP32 rounding order.
-__device__ __forceinline__ int k_step(int kb, int wt, int WT, int KB)
-{
-    int k = kb + (int)(((long long)KB * wt) / WT);
-    return k >= KB ? k - KB : k;
-}
-
 __device__ __forceinline__ void ring_next(int &s, uint32_t &ph, int n)
 {
     if (++s == n) {
@@ -193,7 +181,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 // gate|up: the up matrix at the same rows; down: the next 256-row block
                 const int a_row1 = EPI == kSwiGLU ? a_base : a_base + 2 * kBM;
                 for (int kb = 0; kb < KB; ++kb) {
-                    const int kr = k_step(kb, it.wt, WT, KB);
                     if (!mbar_wait(smem_u32(&emptyA[sa]), pa ^ 1u, p.ctl)) {
                         ok = false;
                         break;
@@ -207,15 +194,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         // tile, the same up rows to 32q+16..32q+31
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            tma_load_2d_pair(dst + (uint32_t)(32 * q) * (kBK * 2), &tmA0, kr * kBK,
+                            tma_load_2d_pair(dst + (uint32_t)(32 * q) * (kBK * 2), &tmA0, kb * kBK,
                                              a_base + 16 * q, f, pol_w);
                             tma_load_2d_pair(dst + (uint32_t)(32 * q + 16) * (kBK * 2), &tmA1,
-                                             kr * kBK, a_base + 16 * q, f, pol_w);
+                                             kb * kBK, a_base + 16 * q, f, pol_w);
                         }
                     } else {
-                        tma_load_2d_pair(dst, &tmA0, kr * kBK, a_base, f, pol_w);
+                        tma_load_2d_pair(dst, &tmA0, kb * kBK, a_base, f, pol_w);
                         if (NUM_A == 2)
-                            tma_load_2d_pair(dst + C::A_BYTES, &tmA1, kr * kBK, a_row1, f, pol_w);
+                            tma_load_2d_pair(dst + C::A_BYTES, &tmA1, kb * kBK, a_row1, f, pol_w);
                     }
                     ++issued;
                     ring_next(sa, pa, SA);
@@ -243,7 +230,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             int tok[G][4];
             if (gather) gather_tokens<G>(p, it, (int)rank * half, half >> 2, lane, tok);
             for (int kb = 0; kb < KB; ++kb) {
-                const int kr = k_step(kb, it.wt, WT, KB);
                 bool got = true;
                 if (lane == 0 || gather) got = mbar_wait(smem_u32(&emptyB[sb]), pb ^ 1u, p.ctl);
                 ok = __all_sync(0xffffffffu, got);
@@ -259,7 +245,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                         for (int bi = 4; bi >= 0; --bi) {   // boxes of 128, 64, 32, 16, 8 rows
                             const int hgt = 8 << bi;
                             if (hgt <= C::HALF && half - off >= hgt) {
-                                tma_load_2d_pair(dst + off * (kBK * 2), &tmB.m[bi], kr * kBK,
+                                tma_load_2d_pair(dst + off * (kBK * 2), &tmB.m[bi], kb * kBK,
                                                  b_row + off, f, pol_x);
                                 off += hgt;
                             }
@@ -271,7 +257,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                     for (int g = 0; g < G; ++g) {
                         const int op = lane + 32 * g;
                         if (op < (half >> 2))
-                            tma_gather4_pair(dst + op * (4 * kBK * 2), &tmB.gather, kr * kBK,
+                            tma_gather4_pair(dst + op * (4 * kBK * 2), &tmB.gather, kb * kBK,
                                              tok[g][0], tok[g][1], tok[g][2], tok[g][3], f, pol_x);
                     }
                 }
