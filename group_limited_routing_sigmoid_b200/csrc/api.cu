@@ -356,7 +356,8 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
     }
     if (h->dense) {
         // one expert: with decode-sized T the weight tiles alone give too few
-        // work items, so K is split and FP32 partial sums are reduced after
+        // work items, so both GEMMs run stream-K (an equal run of K steps per
+        // CTA; tiles cut between CTAs are finished by the last to arrive)
         p.gather = 0;
         p.router_tc = 0;
         p.router_slices = 0;
@@ -661,7 +662,7 @@ int finish_create(beam_moe *h, beam_moe_t *out)
     const size_t T = (size_t)max_tokens, E = (size_t)n_experts, P = T * top_k;
     const size_t nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
     // router partial sums: the largest nslice(t) * t over t <= max_tokens, for
-    // either router path; dense layers: the largest split-K partial sums
+    // either router path
     size_t partial_rows = 0;
     // dense layers: stream-K slots (two per CTA, at the largest stream-K
     // token tile) and an arrival counter per tile of either GEMM, for every

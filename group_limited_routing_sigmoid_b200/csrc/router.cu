@@ -513,17 +513,27 @@ int router_slices(int T, int H, int E, int num_sms)
     return ns;
 }
 
-// Small-batch path: the fewest K slices (each a multiple of 64 wide and at
-// most kSmallMaxK) whose blocks cover every SM; 0 when the path does not
-// apply (T > 64, or H or E off its grid).
+// Small-batch path: the K slice count (each slice a multiple of 64 wide and
+// at most kSmallMaxK) with the shortest estimated kernel: the busiest SM's
+// blocks, each costing its slice width plus a fixed 128 for the staging
+// round trip and the warps' reduction.  A block's work does not depend on T
+// (its lanes cover 64 token rows), and two blocks sharing an SM share its
+// issue slots, so 160 blocks on 148 SMs take about twice as long as 128.
+// Ties go to fewer slices (less for the selection to add).  0 when the path
+// does not apply (T > 64, or H or E off its grid).
 int router_small_slices(int T, int H, int E, int num_sms)
 {
-    if (T < 1 || T > kSmallT || E % kSmallE != 0 || H % 64 != 0) return 0;
+    if (T < 1 || T > kSmallT || E % kSmallE != 0 || H % 64 != 0 || num_sms < 1) return 0;
     int best = 0;
+    long long best_cost = 0;
     for (int ns = 1; ns <= H / 64; ++ns) {
         if (H % (ns * 64) != 0 || H / ns > kSmallMaxK) continue;
-        best = ns;
-        if ((E / kSmallE) * ns >= num_sms) break;
+        const long long per_sm = ((long long)(E / kSmallE) * ns + num_sms - 1) / num_sms;
+        const long long cost = per_sm * (H / ns + 128);
+        if (best == 0 || cost < best_cost) {
+            best = ns;
+            best_cost = cost;
+        }
     }
     return best;
 }

@@ -90,7 +90,7 @@ WORKLOADS: Dict[str, Workload] = {
     # do not give the layers' intermediate size; 20480 (= 8 x 2560, the
     # routed width a token sees in a MoE layer) fits the pages' parameter
     # counts.  The router weight and bias are drawn (draw order) but unused.
-    # (dense_tiny: K long enough for split-K slices of at least 8 steps)
+    # (dense_tiny: K long enough that stream-K cuts tiles between CTAs)
     "dense_tiny": Workload("dense_tiny", T=64, hidden=1024, n_experts=1, n_group=1, topk_group=1,
                            top_k=1, inter=2048, routed_scaling=1.0),
     "dense_decode": Workload("dense_decode", T=64, hidden=5120, n_experts=1, n_group=1,

@@ -1,5 +1,5 @@
 """The dense SwiGLU MLP layer (beam_moe_create_dense) against the oracle's
-dense_block: split-K and fused paths, ragged token counts, the post-norm and
+dense_block: stream-K and grouped-GEMM paths, ragged token counts, the post-norm and
 residual update, and the Beam-shaped layer (H=5120, intermediate 20480)."""
 import dataclasses
 import json
