@@ -146,99 +146,135 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16 
 
 // ---------------------------------------------------------------------------
 // Logits for small batches (T <= 64, decode): a block per (16 experts, K
-// slice of width ks), all tokens.  The block stages its whole slice of x
-// (T rows of ks bf16) and of the router matrix (16 rows of ks floats) in
-// shared memory with every 16-byte copy in flight at once, so the slice
-// costs one memory round trip rather than one per K stage.  Warp w then sums
-// K range [w*ks/8, (w+1)*ks/8) for all 64 x 16 outputs: lane l holds tokens
-// (l & 7) + 8i and experts (l >> 3) + 4j (the rows a load instruction reads
-// are consecutive, so the padded rows fall in distinct banks).  The eight
-// warps' sums are added in warp order into partial[slice][t][e]; the
-// selection adds the slices in slice order.
+// slice of width ks), all tokens.  The block stages its slice of the router
+// matrix (16 rows of ks floats) with cp.async and its slice of x (T rows of
+// ks bf16, converted once to FP32; rows T..63 zero) in shared memory, so the
+// slice costs one memory round trip.  Each of the 16 warps then sums the K
+// range [w*ks/16, (w+1)*ks/16) for all 64 x 16 outputs: lane l holds tokens
+// (l & 7) + 8i and experts (l >> 3) + 4j.  The products go through packed
+// FP32 FMAs (fma.rn.f32x2), each output keeping two running sums, of its
+// even and of its odd K terms, added at the end.  The sixteen warps' sums are
+// added in warp order into partial[slice][t][e]; the selection adds the
+// slices in slice order.  The padded rows put the 8 rows one 128-bit load
+// instruction reads per quarter-warp in distinct banks.
 // ---------------------------------------------------------------------------
-constexpr int kSmallT = 64;     // tokens per block (the largest T of this path)
-constexpr int kSmallE = 16;     // experts per block
-constexpr int kSmallMaxK = 640; // widest K slice (shared memory)
+constexpr int kSmallT = 64;        // tokens per block (the largest T of this path)
+constexpr int kSmallE = 16;        // experts per block
+constexpr int kSmallMaxK = 640;    // widest K slice (shared memory)
+constexpr int kSmallWarps = 16;
+constexpr int kSmallThreads = 32 * kSmallWarps;
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
-__global__ void __launch_bounds__(256) router_logits_small_kernel(
+// d = a * b + c on two FP32 lanes at once (element 0 in the low word).
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ float pair_sum(uint64_t v)
+{
+    return __uint_as_float((uint32_t)v) + __uint_as_float((uint32_t)(v >> 32));
+}
+
+__global__ void __launch_bounds__(kSmallThreads, 1) router_logits_small_kernel(
     const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w, int T, int H, int E, int ks,
     float *__restrict__ partial)
 {
     pdl_launch_dependents();
     pdl_wait();
     extern __shared__ __align__(16) uint8_t small_smem[];
-    const int xstride = ks + 8;   // bf16 per staged token row (16 bytes of padding)
-    const int wstride = ks + 4;   // floats per staged expert row (16 bytes of padding)
-    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(small_smem);
-    float *ws = reinterpret_cast<float *>(small_smem + (size_t)kSmallT * xstride * 2);
+    const int stride = ks + 4;   // floats per staged row (16 bytes of padding)
+    float *xs = reinterpret_cast<float *>(small_smem);                 // [64][stride]
+    float *ws = xs + (size_t)kSmallT * stride;                         // [16][stride]
     const int e0 = blockIdx.x * kSmallE;
     const int k0 = blockIdx.y * ks;
-    const int xv = ks / 8, wv = ks / 4;   // 16-byte vectors per row
-    for (int i = threadIdx.x; i < T * xv; i += blockDim.x) {
-        const int t = i / xv, q = i - t * xv;
-        cp_async16(xs + (size_t)t * xstride + 8 * q, x + (size_t)t * H + k0 + 8 * q);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // router rows: one per warp, asynchronous
+    {
+        const float *src = w + (size_t)(e0 + warp) * H + k0;
+        float *dst = ws + (size_t)warp * stride;
+        for (int q = lane; q < ks / 4; q += 32) cp_async16(dst + 4 * q, src + 4 * q);
+        asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    for (int i = threadIdx.x; i < kSmallE * wv; i += blockDim.x) {
-        const int r = i / wv, q = i - r * wv;
-        cp_async16(ws + (size_t)r * wstride + 4 * q, w + (size_t)(e0 + r) * H + k0 + 4 * q);
+    // token rows: four per warp (rows warp + 16 r), every load of the four in
+    // flight before any is converted; rows T..63 are zero
+    {
+        constexpr int kRows = kSmallT / kSmallWarps;          // 4
+        constexpr int kPer = (kSmallMaxK / 8 + 31) / 32;      // 16-byte vectors per lane and row, at most
+        uint4 raw[kRows][kPer];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+            const int t = warp + kSmallWarps * r;
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int q = lane + 32 * u;
+                raw[r][u] = make_uint4(0, 0, 0, 0);
+                if (t < T && q < ks / 8)
+                    raw[r][u] = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + k0 + 8 * q);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+            float *dst = xs + (size_t)(warp + kSmallWarps * r) * stride;
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int q = lane + 32 * u;
+                if (q < ks / 8) {
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[r][u]);
+                    const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
+                    const float2 f2 = __bfloat1622float2(h2[2]), f3 = __bfloat1622float2(h2[3]);
+                    reinterpret_cast<float4 *>(dst + 8 * q)[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+                    reinterpret_cast<float4 *>(dst + 8 * q)[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+                }
+            }
+        }
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tg = lane & 7, eg = lane >> 3;
-    const int kw = ks / 8;
-    float acc[8][4];
+    const int kw = ks / kSmallWarps;   // a multiple of 4
+    uint64_t acc[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    // rows of tokens >= T are never written: their sums are not stored
-    for (int k = warp * kw; k < (warp + 1) * kw; k += 8) {
-        float wf[4][8];
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0ull;
+#pragma unroll 1
+    for (int k = warp * kw; k < (warp + 1) * kw; k += 4) {
+        ulonglong2 wv[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 *p = reinterpret_cast<const float4 *>(ws + (size_t)(eg + 4 * j) * wstride + k);
-            const float4 a = p[0], b = p[1];
-            wf[j][0] = a.x; wf[j][1] = a.y; wf[j][2] = a.z; wf[j][3] = a.w;
-            wf[j][4] = b.x; wf[j][5] = b.y; wf[j][6] = b.z; wf[j][7] = b.w;
-        }
+        for (int j = 0; j < 4; ++j)
+            wv[j] = *reinterpret_cast<const ulonglong2 *>(ws + (size_t)(eg + 4 * j) * stride + k);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(xs + (size_t)(tg + 8 * i) * xstride + k);
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-            float xf[8];
+            const ulonglong2 xv = *reinterpret_cast<const ulonglong2 *>(xs + (size_t)(tg + 8 * i) * stride + k);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float2 f = __bfloat1622float2(h2[q]);
-                xf[2 * q] = f.x;
-                xf[2 * q + 1] = f.y;
+            for (int j = 0; j < 4; ++j) {
+                acc[i][j] = fma_f32x2(xv.x, wv[j].x, acc[i][j]);
+                acc[i][j] = fma_f32x2(xv.y, wv[j].y, acc[i][j]);
             }
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int q = 0; q < 8; ++q) acc[i][j] = fmaf(xf[q], wf[j][q], acc[i][j]);
         }
     }
     __syncthreads();   // every warp is done with the staged rows
-    float *red = reinterpret_cast<float *>(small_smem);   // [8 warps][64 tokens][16 experts]
+    float *red = reinterpret_cast<float *>(small_smem);   // [16 warps][64 tokens][16 experts]
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            red[((size_t)warp * kSmallT + tg + 8 * i) * kSmallE + eg + 4 * j] = acc[i][j];
+            red[((size_t)warp * kSmallT + tg + 8 * i) * kSmallE + eg + 4 * j] = pair_sum(acc[i][j]);
     __syncthreads();
     const int t = threadIdx.x >> 2, ec = (threadIdx.x & 3) * 4;
     if (t < T) {
         float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int wv2 = 0; wv2 < 8; ++wv2) {
+        for (int wv2 = 0; wv2 < kSmallWarps; ++wv2) {
             const float4 v = *reinterpret_cast<const float4 *>(red + ((size_t)wv2 * kSmallT + t) * kSmallE + ec);
             sum.x += v.x;
             sum.y += v.y;
@@ -261,6 +297,139 @@ __global__ void __launch_bounds__(256) router_logits_small_kernel(
 //   token_list: select only the listed tokens, whose logits are the compact
 //     rows 0..*list_count-1 of `partial` (one slice).
 // ---------------------------------------------------------------------------
+// Candidate keys for the top-k: the biased score's bits made order-preserving
+// as an unsigned integer in the high word, ~expert in the low word, so that
+// the larger key is the larger score and, between equal scores, the lower
+// expert index (the ranking's tie rule).
+__device__ __forceinline__ uint64_t rank_key(float v, int e)
+{
+    uint32_t u = __float_as_uint(v);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((uint64_t)u << 32) | (uint32_t)~(uint32_t)e;
+}
+
+__device__ __forceinline__ float key_value(uint64_t k)
+{
+    uint32_t u = (uint32_t)(k >> 32);
+    u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+    return __uint_as_float(u);
+}
+
+__device__ __forceinline__ int key_expert(uint64_t k) { return (int)~(uint32_t)k; }
+
+// Larger key to a, smaller to b.
+__device__ __forceinline__ void key_cas(uint64_t &a, uint64_t &b)
+{
+    const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+    a = hi;
+    b = lo;
+}
+
+// Sorts 8 keys in descending order (Batcher's odd-even merge sort network).
+__device__ __forceinline__ void sort8_desc(uint64_t (&k)[8])
+{
+    key_cas(k[0], k[1]); key_cas(k[2], k[3]); key_cas(k[4], k[5]); key_cas(k[6], k[7]);
+    key_cas(k[0], k[2]); key_cas(k[1], k[3]); key_cas(k[4], k[6]); key_cas(k[5], k[7]);
+    key_cas(k[1], k[2]); key_cas(k[5], k[6]);
+    key_cas(k[0], k[4]); key_cas(k[1], k[5]); key_cas(k[2], k[6]); key_cas(k[3], k[7]);
+    key_cas(k[2], k[4]); key_cas(k[3], k[5]);
+    key_cas(k[1], k[2]); key_cas(k[3], k[4]); key_cas(k[5], k[6]);
+}
+
+// Top-8 selection for 8 experts per lane and top_k <= 8: each lane sorts its
+// 8 candidate keys, then five butterfly steps (partners lane ^ 1 .. lane ^
+// 16) each keep the 8 largest keys of the two lanes' sorted lists: the
+// elementwise maximum of one list and the other reversed holds them as a
+// bitonic sequence, which three compare-exchange steps sort.  Every lane
+// ends with the same ranked top 8: the ranking the one-at-a-time warp argmax
+// produces, with the same tie rule.  The chosen experts' unbiased scores are
+// fetched from their owner lanes, summed in rank order and normalised; the
+// margin check (ex.margin > 0) takes the gaps between neighbours in the
+// ranking of the top k + 1 candidates and the group gap, as in the general
+// path.
+__device__ __forceinline__ void select_top8(const float (&cand)[8], const float (&s)[8], int e_base,
+                                            int lane, int t, int T, int top_k, bool kept, float gs,
+                                            int32_t *__restrict__ idx_out, float *__restrict__ w_out,
+                                            const SelectExtra &ex)
+{
+    uint64_t k[8], loc[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) k[m] = rank_key(cand[m], e_base + m);
+    sort8_desc(k);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) loc[m] = k[m];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        uint64_t o[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) o[m] = __shfl_xor_sync(0xffffffffu, k[m], off);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) k[m] = k[m] > o[7 - m] ? k[m] : o[7 - m];
+        key_cas(k[0], k[4]); key_cas(k[1], k[5]); key_cas(k[2], k[6]); key_cas(k[3], k[7]);
+        key_cas(k[0], k[2]); key_cas(k[1], k[3]); key_cas(k[4], k[6]); key_cas(k[5], k[7]);
+        key_cas(k[0], k[1]); key_cas(k[2], k[3]); key_cas(k[4], k[5]); key_cas(k[6], k[7]);
+    }
+    // lane j < top_k takes the j-th ranked expert and its unbiased score
+    uint64_t mine = k[0];
+#pragma unroll
+    for (int m = 1; m < 8; ++m)
+        if (lane == m) mine = k[m];
+    const int my_idx = key_expert(mine);
+    const int owner = (my_idx >> 3) & 31, slot = my_idx & 7;
+    float my_s = 0.f;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const float v = __shfl_sync(0xffffffffu, s[m], owner);
+        if (slot == m) my_s = v;
+    }
+    float ssum = 0.f;
+    for (int j = 0; j < top_k; ++j) ssum += __shfl_sync(0xffffffffu, my_s, j);
+    if (lane < top_k) {
+        idx_out[(size_t)t * top_k + lane] = my_idx;
+        w_out[(size_t)t * top_k + lane] = my_s / ssum;
+    }
+    if (ex.margin > 0.f) {
+        // the (k+1)-th candidate: the 9th key when top_k is 8 (each lane's
+        // best key outside the top 8, then the warp's best of those)
+        uint64_t next = 0;
+        if (top_k < 8) {
+            next = __shfl_sync(0xffffffffu, mine, top_k);   // lane j holds the j-th ranked key
+        } else {
+            uint64_t c = 0;
+#pragma unroll
+            for (int m = 7; m >= 0; --m)
+                if (loc[m] < k[7]) c = loc[m];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+                const uint64_t o = __shfl_xor_sync(0xffffffffu, c, off);
+                c = o > c ? o : c;
+            }
+            next = c;
+        }
+        float min_gap = INFINITY, prev = key_value(k[0]);
+#pragma unroll
+        for (int m = 1; m < 8; ++m) {
+            if (m < top_k) {
+                const float v = key_value(k[m]);
+                min_gap = fminf(min_gap, prev - v);
+                prev = v;
+            }
+        }
+        min_gap = fminf(min_gap, prev - key_value(next));
+        float kmin = kept ? gs : INFINITY, dmax = kept ? -INFINITY : gs;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            kmin = fminf(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+            dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, off));
+        }
+        const float gap_group = kmin - dmax;
+        if (lane == 0 && !(fminf(gap_group, min_gap) >= ex.margin)) {
+            const int slot2 = atomicAdd(ex.fix_count, 1);
+            if (slot2 < T) ex.fix_list[slot2] = t;
+        }
+    }
+}
+
 template <int EPL>
 __global__ void __launch_bounds__(256) router_select_kernel(
     const float *__restrict__ partial, int nslice, int T, int E, int n_group, int topk_group,
@@ -275,6 +444,9 @@ __global__ void __launch_bounds__(256) router_select_kernel(
     const int e_base = lane * EPL;
     const int limit = ex.token_list ? min(*ex.list_count, T) : T;
     const int stride = gridDim.x * (blockDim.x >> 5);
+    float bias_r[EPL];   // the lane's experts' bias, the same for every token
+#pragma unroll
+    for (int m = 0; m < EPL; ++m) bias_r[m] = bias[e_base + m];
     for (int wi = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); wi < limit; wi += stride) {
         const int t = ex.token_list ? ex.token_list[wi] : wi;   // output row
         const int r = wi;                                         // logits row
@@ -307,7 +479,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(
             const int e = e_base + m;
             if (logits_out) logits_out[(size_t)t * E + e] = l[m];
             s[m] = 1.0f / (1.0f + expf(-l[m]));
-            b[m] = s[m] + bias[e];
+            b[m] = s[m] + bias_r[m];
         }
 
         // group score: sum of the group's two largest biased scores
@@ -342,6 +514,12 @@ __global__ void __launch_bounds__(256) router_select_kernel(
         float cand[EPL];
 #pragma unroll
         for (int m = 0; m < EPL; ++m) cand[m] = kept ? b[m] : -INFINITY;
+        if constexpr (EPL == 8) {
+            if (top_k <= 8) {
+                select_top8(cand, s, e_base, lane, t, T, top_k, kept, gs, idx_out, w_out, ex);
+                continue;
+            }
+        }
         uint32_t taken = 0;
         int my_idx = 0;
         float my_s = 0.f, ssum = 0.f, prev = INFINITY, min_gap = INFINITY;
@@ -541,8 +719,8 @@ int router_small_slices(int T, int H, int E, int num_sms)
 // Staged rows, or the warps' sums that reuse them, whichever is larger.
 static size_t small_smem_bytes(int ks)
 {
-    const size_t staged = (size_t)kSmallT * (ks + 8) * 2 + (size_t)kSmallE * (ks + 4) * 4;
-    const size_t red = (size_t)8 * kSmallT * kSmallE * 4;
+    const size_t staged = (size_t)(kSmallT + kSmallE) * (ks + 4) * 4;
+    const size_t red = (size_t)kSmallWarps * kSmallT * kSmallE * 4;
     return staged > red ? staged : red;
 }
 
@@ -562,7 +740,7 @@ cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream)
             kslice * ns != a.H)
             return cudaErrorInvalidValue;
         const size_t smem = small_smem_bytes(kslice);
-        err = launch_pdl(router_logits_small_kernel, dim3(a.E / kSmallE, ns), dim3(256), smem, stream,
+        err = launch_pdl(router_logits_small_kernel, dim3(a.E / kSmallE, ns), dim3(kSmallThreads), smem, stream,
                          a.x, a.router_w, a.T, a.H, a.E, kslice, a.partial);
     } else {
         dim3 grid((a.T + kLT - 1) / kLT, (a.E + kLE - 1) / kLE, ns);
@@ -570,7 +748,9 @@ cudaError_t launch_router(const RouterArgs &a, cudaStream_t stream)
                          a.E, kslice, a.partial);
     }
     if (err != cudaSuccess) return err;
-    const int warps = 8;
+    // the selection is a chain of dependent steps per token: few warps per
+    // block spread the tokens' warps over more SMs and scheduler slots
+    const int warps = a.small ? 2 : 8;
     dim3 sgrid((a.T + warps - 1) / warps);
     const int epl = a.E / 32;
 #define BEAM_SELECT(EPLV)                                                                        \
