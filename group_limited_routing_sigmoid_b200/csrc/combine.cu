@@ -14,8 +14,11 @@
 namespace beam {
 
 namespace {
-constexpr int kCombVecs = 2;            // 16-byte vectors (8 hidden values each) per thread
-constexpr int kCombMaxThreads = 512;    // H <= 8 * kCombVecs * 512 = 8192
+// 16-byte vectors (8 hidden values each) per thread: one while a row fits
+// 640 threads (H <= 5120: every load of a thread in flight at once), else two
+// (H <= 8192)
+constexpr int kCombOneVecThreads = 640;
+constexpr int kCombTwoVecThreads = 512;
 constexpr int kCombBatch = 4;           // expert slots whose loads are in flight together
 
 __device__ __forceinline__ void unpack8(const uint4 &raw, float (&v)[8])
@@ -30,15 +33,18 @@ __device__ __forceinline__ void unpack8(const uint4 &raw, float (&v)[8])
 }
 }  // namespace
 
-// Block per token; thread q takes the 16-byte vectors q and q + blockDim.x of
-// the row (8 hidden values each).  The loads of kCombBatch expert slots of a
+// Block per token; thread q takes the 16-byte vectors q (and q + blockDim.x
+// when VECS is 2) of the row (8 hidden values each).  The loads of kCombBatch expert slots of a
 // vector are issued before their sums, which take the slots in order (FP32
 // FMA), so every value is the same slot-order sum.
 // WIDE: FP32 expert outputs (a.y32), all top_k slots' loads in flight at
 // once; otherwise bf16 outputs (a.y).
-template <bool WIDE>
-__global__ void __launch_bounds__(kCombMaxThreads) combine_kernel(CombineArgs a)
+template <bool WIDE, int VECS>
+__global__ void __launch_bounds__(VECS == 1 ? kCombOneVecThreads : kCombTwoVecThreads)
+    combine_kernel(CombineArgs a)
 {
+    constexpr int kCombVecs = VECS;
+    constexpr int kCombMaxThreads = VECS == 1 ? kCombOneVecThreads : kCombTwoVecThreads;
     pdl_launch_dependents();
     pdl_wait();
     if (a.status && status_is_set(a.status)) return;   // a check failed earlier in this pass
@@ -162,10 +168,15 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t stream)
 {
     if (a.H % 8 != 0 || a.top_k > 32) return cudaErrorInvalidValue;
     const int nvec = a.H / 8;
-    const int threads = ((nvec + kCombVecs - 1) / kCombVecs + 31) / 32 * 32;
-    if (threads > kCombMaxThreads) return cudaErrorInvalidValue;
-    if (a.y32) return launch_pdl(combine_kernel<true>, dim3(a.T), dim3(threads), 0, stream, a);
-    return launch_pdl(combine_kernel<false>, dim3(a.T), dim3(threads), 0, stream, a);
+    const int one = (nvec + 31) / 32 * 32;
+    if (one <= kCombOneVecThreads) {
+        if (a.y32) return launch_pdl(combine_kernel<true, 1>, dim3(a.T), dim3(one), 0, stream, a);
+        return launch_pdl(combine_kernel<false, 1>, dim3(a.T), dim3(one), 0, stream, a);
+    }
+    const int two = ((nvec + 1) / 2 + 31) / 32 * 32;
+    if (two > kCombTwoVecThreads) return cudaErrorInvalidValue;
+    if (a.y32) return launch_pdl(combine_kernel<true, 2>, dim3(a.T), dim3(two), 0, stream, a);
+    return launch_pdl(combine_kernel<false, 2>, dim3(a.T), dim3(two), 0, stream, a);
 }
 
 __global__ void wait_timeout_check_kernel(WaitCtl ctl)
