@@ -172,12 +172,19 @@ int router_mma_slices(int T, int H, int E, int num_sms)
 {
     const int items = ((E + router_mma_experts_per_tile() - 1) / router_mma_experts_per_tile()) *
                       ((T + router_mma_tokens_per_tile() - 1) / router_mma_tokens_per_tile());
-    const int kb = 3 * H / 64;
+    // K slices of H (each at least 16 steps of 64): the fewest that minimise
+    // the busiest SM's K steps, (waves of items) x (steps per item)
+    const int kb = H / 64;
     int best = 1;
-    for (int d = 1; d <= kb / 16; ++d) {
+    long long best_cost = 0;
+    for (int d = 1; d <= kb / 16 || d == 1; ++d) {
         if (kb % d) continue;
-        best = d;
-        if (items * d >= 2 * num_sms) break;
+        const long long waves = ((long long)items * d + num_sms - 1) / num_sms;
+        const long long cost = waves * (kb / d);
+        if (d == 1 || cost < best_cost) {
+            best = d;
+            best_cost = cost;
+        }
     }
     return best;
 }
@@ -220,7 +227,7 @@ int run_router(beam_moe *h, cudaStream_t s, const void *x, int T, int32_t *idx, 
         m.T = T;
         m.E = h->E;
         m.nslice = router_mma_slices(T, h->H, h->E, h->num_sms);
-        m.kb_per_slice = 3 * h->H / 64 / m.nslice;
+        m.kb_per_slice = h->H / 64 / m.nslice;
         m.kb_per_h = h->H / 64;
         m.partial = h->partial;
         m.fix_count = h->fix_count;   // the kernel zeroes the re-derivation count

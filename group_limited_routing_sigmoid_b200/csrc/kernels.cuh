@@ -64,9 +64,9 @@ cudaError_t launch_router_fix(const __nv_bfloat16 *x, const float *w, int H, int
 // Tensor-core logits: W split into bf16 pieces (Wcat [E, 3H]) x tokens.
 struct RouterMmaArgs {
     int T, E;
-    int nslice;          // K slices of the concatenated 3H
+    int nslice;          // K slices of H
     int kb_per_slice;    // 64-wide K steps per slice
-    int kb_per_h;        // H / 64 (the token operand wraps around every H)
+    int kb_per_h;        // H / 64 (piece p's K step kb is Wcat column block p * kb_per_h + kb)
     float *partial;      // [nslice, T, E]
     int *fix_count;      // zeroed by the kernel (the re-derivation list's length), or nullptr
     WaitCtl ctl;

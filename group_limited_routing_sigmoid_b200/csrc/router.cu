@@ -784,9 +784,13 @@ namespace beam {
 // side as Wcat [E, 3H].  A product of a bf16 token value and a bf16 piece is
 // exact in FP32, so x . W = sum over k < 3H of Wcat[e,k] * x[t, k mod H] is
 // an FP32 sum of exact products: the tensor core accumulates it in TMEM.
-// Work items: (128-expert tile, BN-token tile, K slice); the MMA has the
-// experts as M (A = Wcat rows) and the tokens as N (B = x rows), and writes
-// partial[slice][t][e] like the SIMT kernel, so the selection is shared.
+// Work items: (128-expert tile, BN-token tile, K slice of H); the MMA has
+// the experts as M (A = Wcat rows) and the tokens as N (B = x rows), and
+// writes partial[slice][t][e] like the SIMT kernel, so the selection is
+// shared.  A pipeline stage holds one 64-wide K step of the token tile and
+// the same K step of all three pieces, so each token tile crosses into
+// shared memory once for the three pieces (the pieces' twelve MMAs per
+// stage go into one accumulator).
 // ---------------------------------------------------------------------------
 
 __global__ void router_split_kernel(const float *__restrict__ w, int n, __nv_bfloat16 *__restrict__ wcat,
@@ -818,8 +822,10 @@ namespace {
 constexpr int kRBM = 128;   // experts per tile (UMMA M)
 constexpr int kRBN = 128;   // tokens per tile (UMMA N)
 constexpr int kRBK = 64;
-constexpr int kRStageBytes = kRBM * kRBK * 2 + kRBN * kRBK * 2;
-constexpr int kRStages = 6;
+constexpr int kRPieces = 3;
+constexpr int kRTileA = kRBM * kRBK * 2;                 // one piece's weight tile
+constexpr int kRStageBytes = kRPieces * kRTileA + kRBN * kRBK * 2;
+constexpr int kRStages = 3;
 constexpr int kRAccCols = kRBN;
 constexpr int kRSmem = 1024 + kRStages * kRStageBytes + 256;
 }  // namespace
@@ -882,7 +888,7 @@ __global__ void __launch_bounds__(192, 1)
             const int mt = item % n_mt, rest = item / n_mt;
             const int s = rest % p.nslice, tt = rest / p.nslice;
             for (int j = 0; j < p.kb_per_slice; ++j) {
-                const int kb = s * p.kb_per_slice + j;   // over the concatenated 3H
+                const int kb = s * p.kb_per_slice + j;   // over H
                 if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, p.ctl)) {
                     ok = false;
                     break;
@@ -890,8 +896,10 @@ __global__ void __launch_bounds__(192, 1)
                 const uint32_t sa = base + stage * kRStageBytes;
                 const uint32_t fb = smem_u32(&full[stage]);
                 mbar_arrive_expect_tx(fb, kRStageBytes);
-                tma_load_2d(sa, &tmW, kb * kRBK, mt * kRBM, fb, pol);
-                tma_load_2d(sa + kRBM * kRBK * 2, &tmX, (kb % p.kb_per_h) * kRBK, tt * kRBN, fb, pol);
+#pragma unroll
+                for (int pc = 0; pc < kRPieces; ++pc)
+                    tma_load_2d(sa + pc * kRTileA, &tmW, (pc * p.kb_per_h + kb) * kRBK, mt * kRBM, fb, pol);
+                tma_load_2d(sa + kRPieces * kRTileA, &tmX, kb * kRBK, tt * kRBN, fb, pol);
                 ++issued;
                 if (++stage == kRStages) {
                     stage = 0;
@@ -935,13 +943,15 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 tc_fence_after();
                 const uint32_t sa = base + stage * kRStageBytes;
-                const uint32_t sb = sa + kRBM * kRBK * 2;
+                const uint32_t sb = sa + kRPieces * kRTileA;
 #pragma unroll
-                for (int k = 0; k < kRBK / 16; ++k) {
-                    umma_bf16(d, umma_desc_sw128(sa + k * 32), umma_desc_sw128(sb + k * 32), idesc,
-                              (j > 0 || k > 0) ? 1u : 0u);
-                    issued_any = true;
-                }
+                for (int pc = 0; pc < kRPieces; ++pc)
+#pragma unroll
+                    for (int k = 0; k < kRBK / 16; ++k) {
+                        umma_bf16(d, umma_desc_sw128(sa + pc * kRTileA + k * 32), umma_desc_sw128(sb + k * 32),
+                                  idesc, (j > 0 || pc > 0 || k > 0) ? 1u : 0u);
+                        issued_any = true;
+                    }
                 umma_commit(smem_u32(&empty[stage]));
                 if (++stage == kRStages) {
                     stage = 0;
