@@ -22,6 +22,7 @@ BEAM_ERR_CUDA = -3
 BEAM_ERR_OOM = -4
 BEAM_ERR_TIMEOUT = -5
 BEAM_ERR_CHECK = -6
+BEAM_ERR_RANGE = -7
 
 # every entry point declared in include/beam_moe.h
 SYMBOLS = (

@@ -12,6 +12,7 @@ namespace beam {
 // Device status codes (same values as beam_status in beam_moe.h).
 constexpr int kStatusTimeout = -5;
 constexpr int kStatusCheck = -6;   // a checked-mode validation failed
+constexpr int kStatusRange = -7;   // an NVFP4 GEMM met an activation beyond its f16 operand range
 
 // Control block every kernel with a wait receives.
 struct WaitCtl {
@@ -54,6 +55,13 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 __device__ __forceinline__ void fence_barrier_init()
 {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order this thread's generic-proxy writes to shared memory before later
+// async-proxy reads of them (TMA, tcgen05.mma operands).
+__device__ __forceinline__ void fence_view_async_shared()
+{
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
@@ -244,6 +252,12 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N)
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
+}
+
+// The same for f16 A and B (formats 0).
+__host__ __device__ constexpr uint32_t umma_idesc_f16_f32(int M, int N)
+{
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // D[tmem] (+)= A[smem desc] * B[smem desc]^T, issued by one thread.

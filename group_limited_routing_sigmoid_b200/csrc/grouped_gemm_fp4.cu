@@ -9,11 +9,16 @@
 //                 memory;
 //   warps 6..21   converters, four per TMEM lane quadrant: thread r of the
 //                 g-th warp of a quadrant decodes the g-th 16-element block
-//                 of weight row r of a stage to bf16 (hardware E2M1 -> f16
-//                 conversion, an exact re-encoding as bf16 and one multiply
-//                 by the block scale: every product has at most 6
-//                 significant bits, so it is exact) and writes it to TMEM
-//                 lane r with tcgen05.st;
+//                 of weight row r of a stage to f16 (hardware E2M1 -> f16
+//                 conversion and one f16 multiply by the block scale: every
+//                 product has at most 6 significant bits and lies between
+//                 2^-10 and 2688 in magnitude, so it is exact) and writes it
+//                 to TMEM lane r with tcgen05.st.  The converters also turn
+//                 the stage's token rows from bf16 into f16 times 2^-8 in
+//                 place (the MMA takes A and B of one type): exact for
+//                 every |x| from 2^-9 up to 65504 x 2^8, within 2^-17 below
+//                 that, and a larger value sets the status word
+//                 (BEAM_ERR_RANGE); the epilogue multiplies by 2^8 again;
 //   warps 1, 22   MMA issuers (lane 0): A (the decoded weights) from TMEM,
 //                 four stages deep, B (the token rows) from the shared-memory
 //                 stage.  gate|up: warp 1 issues the gate MMAs and warp 22
@@ -57,7 +62,9 @@ constexpr int kFp4AStages = 4;                             // decoded A tiles in
 constexpr int kFp4Ch = 16;                                 // epilogue columns per chunk
 constexpr int kFp4MaxRaw = 24;
 constexpr int kFp4BarrierBytes = 1024;
-constexpr int kFp4LutBytes = 256 * 2;                      // E4M3 byte -> bf16(scale x 2^112)
+constexpr int kFp4LutBytes = 256 * 2;                      // E4M3 byte -> f16 scale
+constexpr float kFp4TokenScale = 0.00390625f;              // 2^-8: token rows as f16
+constexpr float kFp4TokenUnscale = 256.0f;
 constexpr int kAColsPerTile = kBK / 2;                     // 64 bf16 of a row: 32 TMEM columns
 
 template <int BN, int NUM_A, int EPI>
@@ -247,6 +254,52 @@ __device__ __forceinline__ void fp4_decode4(uint32_t codes, uint32_t scale_bits,
     }
 }
 
+// The f16 encoding of an E4M3 value (exact: E4M3 values lie between 2^-9
+// and 448 in magnitude, all normal f16 numbers).
+__device__ __forceinline__ uint32_t fp4_scale_bits_f16(uint32_t byte)
+{
+    return __half_as_ushort(__float2half_rn(e4m3_float(byte)));
+}
+
+// Four code bytes (eight E2M1 elements, element 2j in the low nibble of byte
+// j) times one block scale, as four f16x2 words (element 2j in the low
+// half): the hardware converts a byte to two f16 values, one f16 multiply by
+// the scale (both halves of `scale2`) gives the exact product.
+__device__ __forceinline__ void fp4_decode4_f16(uint32_t codes, uint32_t scale2, uint32_t (&o)[4])
+{
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(codes));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o[i]) : "r"(h[i]), "r"(scale2));
+}
+
+// Token rows of a stage, bf16 -> f16 x 2^-8 in place: 32-bit words i of
+// `words` (two elements each; a row is 32 words), this thread taking every
+// `step`-th from `first`.  Returns false if a word of the first `valid_rows`
+// rows exceeds the f16 range.
+__device__ __forceinline__ bool fp4_tokens_to_f16(uint32_t *bw, int words, int valid_rows, int first,
+                                                  int step)
+{
+    bool fits = true;
+    for (int i = first; i < words; i += step) {
+        const uint32_t v = bw[i];
+        const float lo = __uint_as_float(v << 16) * kFp4TokenScale;
+        const float hi = __uint_as_float(v & 0xffff0000u) * kFp4TokenScale;
+        uint32_t f;
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(f) : "f"(hi), "f"(lo));
+        if ((i >> 5) < valid_rows && (fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f)) fits = false;
+        bw[i] = f;
+    }
+    return fits;
+}
+
 }  // namespace
 
 template <int BN, int NUM_A, int EPI>
@@ -300,7 +353,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
     }
     if (converter)
         for (int i = threadIdx.x - 32 * kFp4ConvFirst; i < 256; i += 32 * kFp4ConvWarps)
-            lut_s[i] = (uint16_t)fp4_scale_bits((uint32_t)i);
+            lut_s[i] = (uint16_t)fp4_scale_bits_f16((uint32_t)i);
     pdl_launch_dependents();
     pdl_wait();   // set-up above overlaps the previous kernel; data from here on
     load_tables(p, s_counts, s_offsets, s_tile);
@@ -384,13 +437,19 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         int rs = 0, cs = 0;
         uint32_t rp = 0, cp = 0;
         bool ok = true;
+        const int cidx = threadIdx.x - 32 * kFp4ConvFirst;   // 0 .. 32 * kFp4ConvWarps - 1
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
+            const int n_load = (it.nrows + 15) & ~15;
             for (int kb = 0; kb < KB; ++kb) {
                 const bool got = mbar_wait(smem_u32(&rfull[rs]), rp, p.ctl) &&
                                  mbar_wait(smem_u32(&cempty[cs]), cp ^ 1u, p.ctl);
                 ok = __all_sync(0xffffffffu, got);
                 if (!ok) break;
                 tc_fence_after();
+                if (!fp4_tokens_to_f16(reinterpret_cast<uint32_t *>(base_ptr + rs * C::RAW_STAGE),
+                                       n_load * (kBK / 2), it.nrows, cidx, 32 * kFp4ConvWarps))
+                    record_status(p.ctl.status, kStatusRange);
                 const uint8_t *raw = base_ptr + rs * C::RAW_STAGE + C::B_BYTES;
 #pragma unroll
                 for (int a = 0; a < NUM_A; ++a) {
@@ -400,14 +459,17 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                     const uint32_t sb =
                         lut_s[raw[NUM_A * kFp4CodeTile + a * kFp4ScaleTile + blk * kFp4TileRows + r]];
                     uint32_t lo[4], hi[4];
-                    fp4_decode4(c.x, sb, lo);
-                    fp4_decode4(c.y, sb, hi);
+                    fp4_decode4_f16(c.x, sb | (sb << 16), lo);
+                    fp4_decode4_f16(c.y, sb | (sb << 16), hi);
                     const uint32_t v[8] = {lo[0], lo[1], lo[2], lo[3], hi[0], hi[1], hi[2], hi[3]};
                     tmem_st8(lane_base + (uint32_t)((cs * NUM_A + a) * kAColsPerTile), v);
                 }
-                // every lane's stores complete, then one arrival for the warp
-                // (512 same-address arrivals a stage would serialise)
+                // every lane's stores complete (the token rows' generic
+                // writes made visible to the MMA's reads too), then one
+                // arrival for the warp (512 same-address arrivals a stage
+                // would serialise)
                 tmem_st_wait();
+                fence_view_async_shared();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&cfull[cs]));
@@ -427,7 +489,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++iter) {
             const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
             const int n_mma = (it.nrows + 15) & ~15;
-            const uint32_t idesc = umma_idesc_bf16_f32(kBM, n_mma);
+            const uint32_t idesc = umma_idesc_f16_f32(kBM, n_mma);
             const int acc = iter % C::NBUF;
             const uint32_t acc_phase = (uint32_t)(iter / C::NBUF) & 1u;
             if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, p.ctl)) {
@@ -487,11 +549,12 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
             const int col0 = it.wt * kBM + quad * 32;
             if constexpr (EPI == kSwiGLU)
                 fp4_epilogue_block<EPI, kFp4Ch, BN, C::CHAINS, NUM_A * BN>(
-                    taddr, it.nrows, it.row0, lane, stg, p.out + col0, p.R, w.a[0].global,
-                    w.a[1].global);
+                    taddr, it.nrows, it.row0, lane, stg, p.out + col0, p.R,
+                    w.a[0].global * kFp4TokenUnscale, w.a[1].global * kFp4TokenUnscale);
             else
                 fp4_epilogue_block<EPI, kFp4Ch, 0, C::CHAINS, NUM_A * BN>(
-                    taddr, it.nrows, it.row0, lane, stg, p.out + col0, p.R, w.a[0].global, 1.0f);
+                    taddr, it.nrows, it.row0, lane, stg, p.out + col0, p.R,
+                    w.a[0].global * kFp4TokenUnscale, 1.0f);
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
         }

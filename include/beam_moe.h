@@ -62,7 +62,9 @@ typedef enum {
     BEAM_ERR_CUDA = -3,        /* a CUDA runtime / driver call failed          */
     BEAM_ERR_OOM = -4,         /* workspace allocation failed                  */
     BEAM_ERR_TIMEOUT = -5,     /* a bounded device-side wait ran out           */
-    BEAM_ERR_CHECK = -6        /* a checked-mode validation failed             */
+    BEAM_ERR_CHECK = -6,       /* a checked-mode validation failed             */
+    BEAM_ERR_RANGE = -7        /* an NVFP4 forward met an activation above
+                                  65504 x 256 in magnitude (its f16 operands)  */
 } beam_status;
 
 /*
@@ -151,9 +153,13 @@ int beam_moe_create_dense(beam_moe_t *out, int hidden, int inter, const void *w_
  * down.  Device pointers, 16-byte aligned, read during this call only: the
  * handle allocates and keeps its own tiled copy (0.5625 bytes per weight)
  * made by kernels on the legacy default stream, which this call waits for.
- * The grouped GEMMs decode the weights to bf16 (exact: an E2M1 x E4M3
- * product has at most 6 significant bits) for the tensor cores and apply the
- * per-tensor scales to the FP32 accumulators.
+ * The grouped GEMMs decode the weights to f16 (exact: an E2M1 x E4M3
+ * product has at most 6 significant bits and lies between 2^-10 and 2688 in
+ * magnitude) for the tensor cores, take the bf16 activations as f16 times
+ * 2^-8 (exact for magnitudes from 2^-9 up to 65504 x 2^8, within 2^-17
+ * below that) and apply the per-tensor scales and 2^8 to the FP32
+ * accumulators.  An activation above 65504 x 2^8 in magnitude records
+ * BEAM_ERR_RANGE in the status word (beam_moe_get_status).
  * The handle takes the same calls as a bf16 handle.  Differences: token
  * tiles of at most 128 rows (tile_rows 256 acts as 128); the cta_pairs,
  * gather_rows, token_stages and down_pair tunings are ignored (single-CTA
@@ -171,8 +177,9 @@ int beam_moe_create_nvfp4(beam_moe_t *out, int hidden, int n_experts, int inter,
 /*
  * Decode rows x K NVFP4 elements (codes uint8 [rows, K/2], scales uint8
  * [rows, K/16], laid out as for beam_moe_create_nvfp4) to bf16 [rows, K]:
- * each element times its block scale, exact; no per-tensor scale.  The same
- * decode the NVFP4 grouped GEMMs run.  Device pointers; codes and out
+ * each element times its block scale, exact; no per-tensor scale.  The
+ * same products the NVFP4 grouped GEMMs give the tensor cores (as f16 there;
+ * both formats hold them exactly).  Device pointers; codes and out
  * 16-byte aligned.  K a positive multiple of 16, rows >= 0 (0: nothing to
  * do).  Needs no handle.  Asynchronous on `stream`.  Returns
  * BEAM_ERR_INVALID_ARG for bad arguments, BEAM_ERR_CUDA if the launch fails.

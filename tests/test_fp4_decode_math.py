@@ -60,3 +60,43 @@ def test_scale_zero_and_subnormals():
     np.testing.assert_array_equal(scale, np.arange(8) * 2.0 ** -9)
     s_val = _bf16_bits_to_f64(_to_bf16_bits(scale * 2.0 ** 112))
     np.testing.assert_array_equal(s_val, scale * 2.0 ** 112)
+
+
+# The GEMMs' f16 operands: the decoded weights and the token rows.
+
+def test_f16_products_are_exact_for_every_code_and_scale():
+    # every finite E4M3 scale is an f16 number, and so is every product with
+    # an E2M1 value (at most 6 significant bits, 2^-10 .. 2688 in magnitude)
+    finite = np.array([b for b in range(256) if b not in (0x7F, 0xFF)], np.uint8)
+    scale = torch.from_numpy(finite).view(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(scale.astype(np.float16).astype(np.float64), scale)
+    vals = np.array([_e2m1(c) for c in range(16)])
+    np.testing.assert_array_equal(vals.astype(np.float16).astype(np.float64), vals)
+    prod16 = vals.astype(np.float16)[:, None] * scale.astype(np.float16)[None, :]   # f16 multiply
+    np.testing.assert_array_equal(prod16.astype(np.float64), vals[:, None] * scale[None, :])
+    nz = np.abs(vals[:, None] * scale[None, :])
+    nz = nz[nz > 0]
+    assert nz.min() == 2.0 ** -10 and nz.max() == 6 * 448      # normal f16 numbers
+
+
+def _all_bf16() -> np.ndarray:
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    v = (bits << 16).view(np.float32).astype(np.float64)
+    return v[np.isfinite(v)]
+
+
+def test_token_rows_as_f16_times_2_pow_minus_8():
+    # bf16 -> f16(x * 2^-8), rounded to nearest: exact for 2^-9 <= |x| <=
+    # 65504 * 2^8, within 2^-17 of x * 2^-8 * 2^8 below 2^-9, and beyond the
+    # f16 range above 65504 * 2^8 (the kernels flag those)
+    x = _all_bf16()
+    y = (x * 2.0 ** -8).astype(np.float32).astype(np.float16).astype(np.float64) * 2.0 ** 8
+    a = np.abs(x)
+    inside = (a >= 2.0 ** -9) & (a <= 65504 * 2.0 ** 8)
+    np.testing.assert_array_equal(y[inside], x[inside])
+    small = a < 2.0 ** -9
+    assert np.all(np.abs(y[small] - x[small]) <= 2.0 ** -17)
+    big = a > 65504 * 2.0 ** 8
+    assert big.any() and np.all(np.isinf(y[big]))
+    # the bound is tight: something below 2^-9 does lose bits
+    assert np.any(y[small] != x[small])

@@ -2,7 +2,9 @@
 expert: the decode the GEMMs run, bit for bit, over every code byte and
 every finite scale byte; the block over ragged token counts, every token
 tile, fewer CTAs than work items, and the post-norm and residual update; and
-the Beam decode shape (H=5120, 256 experts, I=2560, 64 tokens) in full."""
+the Beam decode shape (H=5120, 256 experts, I=2560, 64 tokens) in full; and
+the status the GEMMs record for an activation beyond their f16 operands'
+range (65504 x 2^8)."""
 import dataclasses
 import json
 import os
@@ -13,7 +15,7 @@ import torch
 
 import oracle
 from group_limited_routing_sigmoid_b200 import workloads as W
-from group_limited_routing_sigmoid_b200.binding import BeamMoE, nvfp4_dequant
+from group_limited_routing_sigmoid_b200.binding import BEAM_ERR_RANGE, BeamMoE, nvfp4_dequant
 from group_limited_routing_sigmoid_b200.build import build
 
 from parity import check_block
@@ -93,3 +95,19 @@ def test_nvfp4_beam_decode():
     moe.close()
     del d, moe
     torch.cuda.empty_cache()
+
+
+def test_nvfp4_activation_beyond_f16_range_sets_status():
+    wl = W.WORKLOADS["tiny_nvfp4"]
+    g = W.generator(wl, "cuda")
+    d = W.make_nvfp4_weights(wl, "cuda", g)
+    d.update(W.make_tokens(wl, "cuda", g, T=8))
+    moe = BeamMoE.from_workload(wl, d, max_tokens=8)
+    x = d["x"].clone()
+    x[3, 5] = 2.0 ** 25                    # exact in bf16, above 65504 x 2^8
+    moe.forward(x)
+    assert moe.get_status() == BEAM_ERR_RANGE
+    # read and cleared above: an ordinary batch leaves it at zero
+    moe.forward(d["x"])
+    assert moe.get_status() == 0
+    moe.close()
