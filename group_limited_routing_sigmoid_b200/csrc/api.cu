@@ -341,7 +341,7 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
     // Expert outputs y in FP32: the combine then rounds only once, to the
     // block's bf16 output.  The single-CTA FP32 down GEMM takes one weight
     // block per item.
-    p.y_f32 = !h->dense && !h->fp4 && h->y_mode != 0;
+    p.y_f32 = !h->dense && h->y_mode != 0;
     if (p.y_f32 && !p.cta_pairs) p.down_paired = 0;
     // Interleaved gate|up tiles on CTA pairs (on request only): one
     // accumulator of N columns instead of two, so two fit TMEM and one
@@ -352,13 +352,14 @@ ForwardPlan plan_forward(const beam_moe *h, int T)
     p.gu_interleaved = h->gu_layout == 1 && p.cta_pairs && h->I % 128 == 0;
     if (h->fp4) {
         // NVFP4 weights: the single-CTA kernel with token tiles of up to 128
-        // rows from the sorted copy, one weight block per down item, bf16 y
+        // rows from the sorted copy, one weight block per down item, FP32 y
+        // as for bf16 weights
         if (p.tile_rows > 128) p.tile_rows = 128;
         p.cta_pairs = 0;
         p.grid = h->gemm_ctas > 0 ? h->gemm_ctas : h->num_sms;
         p.down_paired = 0;
         p.gather = 0;
-        p.y_f32 = 0;
+        p.y_f32 = h->y_mode != 0;
         p.gu_interleaved = 0;
     }
     if (h->dense) {
@@ -591,7 +592,8 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
         dk = use_pair ? (plan.down_paired ? GemmKind::kDownPairedY32 : GemmKind::kDownY32)
                       : GemmKind::kDownF32;
     if (h->fp4)
-        e = launch_grouped_gemm_fp4(GemmKind::kDown, BN, h->fp4_down, h->tm_h, g, grid, s);
+        e = launch_grouped_gemm_fp4(plan.y_f32 ? GemmKind::kDownF32 : GemmKind::kDown, BN, h->fp4_down,
+                                    h->tm_h, g, grid, s);
     else
         e = use_pair ? launch_grouped_gemm_pair(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s)
                      : launch_grouped_gemm(dk, BN, h->tm_down, h->tm_down, h->tm_h, g, grid, s);

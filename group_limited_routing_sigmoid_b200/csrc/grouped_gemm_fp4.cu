@@ -90,8 +90,10 @@ struct Fp4Cfg {
     static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory");
     static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "token tiles of 16..128 rows");
-    static_assert(EPI == kStoreBF16 || NUM_A == 2, "SwiGLU needs the gate and up tiles");
-    static_assert(EPI == kSwiGLU || EPI == kStoreBF16, "bf16 epilogues only");
+    static_assert(EPI != kSwiGLU || NUM_A == 2, "SwiGLU needs the gate and up tiles");
+    static_assert(EPI == kSwiGLU || NUM_A == 1, "one matrix for the store epilogues");
+    static_assert(EPI == kSwiGLU || EPI == kStoreBF16 || EPI == kStoreF32, "fp4 epilogues");
+    static_assert(32 * kFp4Ch * 4 <= kStagingWarpBytes, "staging block (FP32)");
     static_assert((2 * kFp4MaxRaw + 2 * kFp4AStages + 6) * 8 + 4 <= kFp4BarrierBytes, "barriers");
     static_assert(32 * kFp4Ch * 2 <= kStagingWarpBytes, "staging block");
     static_assert(kFp4ConvWarps == 4 * (kFp4TileK / 16), "a converter warp per quadrant and block");
@@ -198,6 +200,33 @@ __device__ __forceinline__ void fp4_epilogue_block(uint32_t taddr, int nrows, in
             if (c0 + j < nrows) {
                 const uint4 val = *reinterpret_cast<const uint4 *>(stg + v * 16);
                 *reinterpret_cast<uint4 *>(out + (size_t)(row0 + c0 + j) * ldo + part * 8) = val;
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// FP32 outputs: the chains' sum times sa, 16 token rows at a time through
+// the warp's staging block, each row's 32 columns (this warp's output
+// columns) stored as 16-byte vectors.
+template <int CH, int CHAINS, int CHAIN_STRIDE>
+__device__ __forceinline__ void fp4_epilogue_f32(uint32_t taddr, int nrows, int row0, int lane,
+                                                 uint8_t *stg, float *out, int ldo, float sa)
+{
+    float *sh = reinterpret_cast<float *>(stg);   // [CH token rows][32 columns]
+#pragma unroll 1
+    for (int c0 = 0; c0 < nrows; c0 += CH) {
+        float g[CH];
+        load_chains<CH, CHAINS>(taddr + c0, CHAIN_STRIDE, g);
+#pragma unroll
+        for (int j = 0; j < CH; ++j) sh[j * 32 + lane] = g[j] * sa;
+        __syncwarp();
+#pragma unroll
+        for (int w = lane; w < CH * 8; w += 32) {
+            const int j = w >> 3, part = w & 7;
+            if (c0 + j < nrows) {
+                const float4 val = *reinterpret_cast<const float4 *>(sh + j * 32 + part * 4);
+                *reinterpret_cast<float4 *>(out + (size_t)(row0 + c0 + j) * ldo + part * 4) = val;
             }
         }
         __syncwarp();
@@ -551,6 +580,10 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                 fp4_epilogue_block<EPI, kFp4Ch, BN, C::CHAINS, NUM_A * BN>(
                     taddr, it.nrows, it.row0, lane, stg, p.out + col0, p.R,
                     w.a[0].global * kFp4TokenUnscale, w.a[1].global * kFp4TokenUnscale);
+            else if constexpr (EPI == kStoreF32)
+                fp4_epilogue_f32<kFp4Ch, C::CHAINS, NUM_A * BN>(
+                    taddr, it.nrows, it.row0, lane, stg, p.out_f32 + col0, p.R,
+                    w.a[0].global * kFp4TokenUnscale);
             else
                 fp4_epilogue_block<EPI, kFp4Ch, 0, C::CHAINS, NUM_A * BN>(
                     taddr, it.nrows, it.row0, lane, stg, p.out + col0, p.R,
@@ -628,6 +661,9 @@ cudaError_t launch_fp4_kind(GemmKind kind, const Fp4Operands &w, const BoxMaps &
     if (kind == GemmKind::kDown)
         return launch_pdl(grouped_gemm_fp4_kernel<BN, 1, kStoreBF16>, dim3(grid), dim3(kFp4Threads),
                           Fp4Cfg<BN, 1, kStoreBF16>::SMEM_BYTES, stream, b, w, args);
+    if (kind == GemmKind::kDownF32 && args.out_f32 != nullptr)
+        return launch_pdl(grouped_gemm_fp4_kernel<BN, 1, kStoreF32>, dim3(grid), dim3(kFp4Threads),
+                          Fp4Cfg<BN, 1, kStoreF32>::SMEM_BYTES, stream, b, w, args);
     return cudaErrorInvalidValue;
 }
 }  // namespace
@@ -635,9 +671,10 @@ cudaError_t launch_fp4_kind(GemmKind kind, const Fp4Operands &w, const BoxMaps &
 cudaError_t prepare_grouped_gemm_fp4()
 {
     cudaError_t err;
-#define BEAM_PREP_FP4(BN)                                                  \
-    if ((err = set_smem_fp4<BN, 2, kSwiGLU>()) != cudaSuccess) return err; \
-    if ((err = set_smem_fp4<BN, 1, kStoreBF16>()) != cudaSuccess) return err;
+#define BEAM_PREP_FP4(BN)                                                    \
+    if ((err = set_smem_fp4<BN, 2, kSwiGLU>()) != cudaSuccess) return err;   \
+    if ((err = set_smem_fp4<BN, 1, kStoreBF16>()) != cudaSuccess) return err; \
+    if ((err = set_smem_fp4<BN, 1, kStoreF32>()) != cudaSuccess) return err;
     BEAM_PREP_FP4(16)
     BEAM_PREP_FP4(32)
     BEAM_PREP_FP4(64)
