@@ -154,10 +154,100 @@ __global__ void __launch_bounds__(256) dispatch_rows_kernel(
     row_pair[row] = p;
 }
 
+// All of the above in one block, for at most kDispatchBlock pairs when no
+// sorted copy is made (the decode path): the count kernel's ranks, the scan
+// kernel's counts, offsets and tile prefix, and the row maps.  Thread p
+// takes pair p; threads e < E also take expert e in the scans.
+__global__ void __launch_bounds__(kDispatchBlock) dispatch_small_kernel(
+    const int *status, const int32_t *__restrict__ idx, int P, int E, int BN,
+    int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ tile_off,
+    int32_t *__restrict__ pair_row, int32_t *__restrict__ row_pair)
+{
+    pdl_launch_dependents();
+    pdl_wait();
+    if (status_is_set(status)) return;   // a check failed earlier in this pass
+    extern __shared__ int32_t wcnt[];   // [32 warps][E], then the experts' offsets [E]
+    int32_t *off_s = wcnt + 32 * E;
+    __shared__ int32_t wsum_c[32], wsum_t[32];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    const int e = tid < P ? idx[tid] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rk = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rk == 0) wcnt[warp * E + e] = __popc(peers);
+    __syncthreads();
+    int run = 0;   // thread tid < E: expert tid's pairs before each warp, and in all
+    if (tid < E) {
+        for (int w = 0; w < 32; ++w) {
+            const int c = wcnt[w * E + tid];
+            wcnt[w * E + tid] = run;
+            run += c;
+        }
+    }
+    const int nt = (run + BN - 1) / BN;
+    int ic = run, it = nt;   // inclusive warp scans over the experts
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int vc = __shfl_up_sync(0xffffffffu, ic, off);
+        const int vt = __shfl_up_sync(0xffffffffu, it, off);
+        if (lane >= off) {
+            ic += vc;
+            it += vt;
+        }
+    }
+    if (lane == 31) {
+        wsum_c[warp] = ic;
+        wsum_t[warp] = it;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        int vc = lane < nw ? wsum_c[lane] : 0;
+        int vt = lane < nw ? wsum_t[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int uc = __shfl_up_sync(0xffffffffu, vc, off);
+            const int ut = __shfl_up_sync(0xffffffffu, vt, off);
+            if (lane >= off) {
+                vc += uc;
+                vt += ut;
+            }
+        }
+        if (lane < nw) {
+            wsum_c[lane] = vc;
+            wsum_t[lane] = vt;
+        }
+    }
+    __syncthreads();
+    if (tid < E) {
+        const int bc = warp > 0 ? wsum_c[warp - 1] : 0;
+        const int bt = warp > 0 ? wsum_t[warp - 1] : 0;
+        const int o = bc + ic - run;
+        counts[tid] = run;
+        offsets[tid] = o;
+        off_s[tid] = o;
+        tile_off[tid] = bt + it - nt;
+        if (tid == E - 1) {
+            offsets[E] = bc + ic;
+            tile_off[E] = bt + it;
+        }
+    }
+    __syncthreads();
+    if (e >= 0) {
+        const int row = off_s[e] + wcnt[warp * E + e] + rk;
+        pair_row[tid] = row;
+        row_pair[row] = tid;
+    }
+}
+
 cudaError_t prepare_dispatch(int E)
 {
-    return cudaFuncSetAttribute(dispatch_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)(sizeof(int32_t) * 32 * (size_t)E));
+    cudaError_t err = cudaFuncSetAttribute(dispatch_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)(sizeof(int32_t) * 32 * (size_t)E));
+    if (err != cudaSuccess) return err;
+    return cudaFuncSetAttribute(dispatch_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(sizeof(int32_t) * 33 * (size_t)E));
 }
 
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t stream)
@@ -165,6 +255,10 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t stream)
     const int P = a.T * a.top_k;
     const int nblk = (P + kDispatchBlock - 1) / kDispatchBlock;
     const size_t smem = sizeof(int32_t) * 32 * (size_t)a.E;
+    if (nblk <= 1 && !a.copy_rows && a.E <= kDispatchBlock)
+        return launch_pdl(dispatch_small_kernel, dim3(1), dim3(kDispatchBlock), smem + sizeof(int32_t) * a.E,
+                          stream, a.status, a.idx, P, a.E, a.tile_rows, a.counts, a.offsets, a.tile_off,
+                          a.pair_row, a.row_pair);
     cudaError_t err = launch_pdl(dispatch_count_kernel, dim3(nblk), dim3(kDispatchBlock), smem,
                                  stream, a.status, a.idx, P, a.E, a.block_cnt, a.rank);
     if (err != cudaSuccess) return err;

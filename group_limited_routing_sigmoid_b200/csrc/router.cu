@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(
         for (int m = 0; m < EPL; ++m) {
             const int e = e_base + m;
             if (logits_out) logits_out[(size_t)t * E + e] = l[m];
-            s[m] = 1.0f / (1.0f + expf(-l[m]));
+            s[m] = __frcp_rn(1.0f + expf(-l[m]));   // the correctly rounded 1 / (1 + e^-l)
             b[m] = s[m] + bias_r[m];
         }
 
