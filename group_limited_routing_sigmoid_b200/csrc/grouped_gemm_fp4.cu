@@ -528,8 +528,11 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
             tc_fence_after();
             const uint32_t d0 = tmem_base + (uint32_t)(C::A_COLS + acc * C::ACC_COLS);
             for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(smem_u32(&cfull[cs]), cp, p.ctl) ||
-                    !mbar_wait(smem_u32(&rfull[rs]), rp, p.ctl)) {
+                // the converters' arrival implies the stage's raw data landed
+                // (they waited for it) and its token rows are converted: no
+                // wait on the raw ring here (one wait less per stage measured
+                // 8% off the step: the issuing thread sets the pace)
+                if (!mbar_wait(smem_u32(&cfull[cs]), cp, p.ctl)) {
                     ok = false;
                     break;
                 }
