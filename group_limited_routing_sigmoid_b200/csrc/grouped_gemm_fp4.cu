@@ -30,7 +30,14 @@
 //   warps 2..5    epilogue, one per quadrant: as the bf16 kernel, with the
 //                 FP32 accumulators first multiplied by the per-tensor scales.
 //
-// Accumulator chains: small tiles spread the four K sub-steps of a stage over
+// Stages: a pipeline stage holds two 64-wide K steps (the codes and scales
+// of two consecutive tiles of the layout, the token rows of both steps), so
+// every per-stage cost of the issuing threads and the converters (barrier
+// waits, fences, commits) is paid once per 128 of K.  At 16-row tiles those
+// costs, not the tensor core, set the pace: one wait less per stage took 8%
+// off the decode step, two steps per stage 20% more.
+//
+// Accumulator chains: small tiles spread the four K sub-steps of a step over
 // CHAINS independent accumulators per matrix, so consecutive MMAs never add
 // into the same accumulator; the epilogue adds the chains in chain order in
 // FP32.
@@ -58,7 +65,8 @@ constexpr int kFp4ConvWarps = 16;                          // four per quadrant,
 constexpr int kFp4ConvFirst = 2 + kFp4EpiWarps;            // first converter warp
 constexpr int kFp4Issuer2 = kFp4ConvFirst + kFp4ConvWarps;  // warp of the second MMA issuer
 constexpr int kFp4Threads = 32 * (kFp4Issuer2 + 1);          // 736
-constexpr int kFp4AStages = 4;                             // decoded A tiles in TMEM
+constexpr int kFp4AStagesMax = 4;                          // decoded A stages in TMEM, at most
+constexpr int kFp4KS = 2;                                  // 64-wide K steps per pipeline stage
 constexpr int kFp4Ch = 16;                                 // epilogue columns per chunk
 constexpr int kFp4MaxRaw = 24;
 constexpr int kFp4BarrierBytes = 1024;
@@ -69,16 +77,21 @@ constexpr int kAColsPerTile = kBK / 2;                     // 64 bf16 of a row: 
 
 template <int BN, int NUM_A, int EPI>
 struct Fp4Cfg {
-    static constexpr int B_BYTES = BN * kBK * 2;
-    static constexpr int RAW_USED = B_BYTES + NUM_A * (kFp4CodeTile + kFp4ScaleTile);
+    static constexpr int B_BYTES = BN * kBK * 2;                 // token rows of one K step
+    static constexpr int CODES = kFp4KS * kFp4CodeTile;           // one matrix's codes per stage
+    static constexpr int SCALES = kFp4KS * kFp4ScaleTile;
+    static constexpr int RAW_USED = kFp4KS * B_BYTES + NUM_A * (CODES + SCALES);
     static constexpr int RAW_STAGE = (RAW_USED + 1023) / 1024 * 1024;   // keeps B 1024-aligned
     static constexpr int STAGING = kFp4EpiWarps * kStagingWarpBytes;
     static constexpr int FIXED = 1024 + STAGING + kFp4BarrierBytes + kFp4LutBytes + kTableBytes;
     static constexpr int RAW_FIT = (kMaxDynSmem - FIXED) / RAW_STAGE;
     static constexpr int RAW_STAGES = RAW_FIT > kFp4MaxRaw ? kFp4MaxRaw : RAW_FIT;
-    static constexpr int A_COLS = kFp4AStages * NUM_A * kAColsPerTile;
     static constexpr int CHAINS = BN >= 64 ? 1 : 64 / BN;        // 4 for 16 rows, 2 for 32
     static constexpr int ACC_COLS = CHAINS * NUM_A * BN;         // [chain][matrix][BN]
+    static constexpr int A_STAGE_COLS = NUM_A * kFp4KS * kAColsPerTile;
+    static constexpr int A_STAGES =
+        kFp4AStagesMax * A_STAGE_COLS + 2 * ACC_COLS <= 512 ? kFp4AStagesMax : 2;
+    static constexpr int A_COLS = A_STAGES * A_STAGE_COLS;
     // MMA issuers: gate and up each from their own thread (measured: the
     // gate|up GEMM 10% faster at 16-row tiles); down keeps one (splitting
     // its chains between two threads measured 15% slower)
@@ -94,7 +107,8 @@ struct Fp4Cfg {
     static_assert(EPI == kSwiGLU || NUM_A == 1, "one matrix for the store epilogues");
     static_assert(EPI == kSwiGLU || EPI == kStoreBF16 || EPI == kStoreF32, "fp4 epilogues");
     static_assert(32 * kFp4Ch * 4 <= kStagingWarpBytes, "staging block (FP32)");
-    static_assert((2 * kFp4MaxRaw + 2 * kFp4AStages + 6) * 8 + 4 <= kFp4BarrierBytes, "barriers");
+    static_assert((2 * kFp4MaxRaw + 2 * kFp4AStagesMax + 6) * 8 + 4 <= kFp4BarrierBytes, "barriers");
+    static_assert(kFp4KS * B_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "token tiles 1024-aligned");
     static_assert(32 * kFp4Ch * 2 <= kStagingWarpBytes, "staging block");
     static_assert(kFp4ConvWarps == 4 * (kFp4TileK / 16), "a converter warp per quadrant and block");
     static_assert(CHAINS <= kBK / 16, "a chain per K sub-step at most");
@@ -344,8 +358,8 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
     uint64_t *rfull = reinterpret_cast<uint64_t *>(staging + C::STAGING);
     uint64_t *rempty = rfull + kFp4MaxRaw;
     uint64_t *cfull = rempty + kFp4MaxRaw;
-    uint64_t *cempty = cfull + kFp4AStages;
-    uint64_t *tfull = cempty + kFp4AStages;
+    uint64_t *cempty = cfull + kFp4AStagesMax;
+    uint64_t *tfull = cempty + kFp4AStagesMax;
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;                                          // one per issuer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 2);
@@ -363,7 +377,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
             mbar_init(smem_u32(&rfull[s]), 1);
             mbar_init(smem_u32(&rempty[s]), C::ISSUERS);   // a commit from each issuer
         }
-        for (int s = 0; s < kFp4AStages; ++s) {
+        for (int s = 0; s < C::A_STAGES; ++s) {
             mbar_init(smem_u32(&cfull[s]), kFp4ConvWarps);   // one elected lane per warp
             mbar_init(smem_u32(&cempty[s]), C::ISSUERS);
         }
@@ -394,7 +408,8 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
     const int WT = p.R / kBM;
     // no work while the status word is set (a failed check or wait)
     const int total = status_is_set(p.ctl.status) ? 0 : WT * s_tile[p.E];
-    const int KB = p.K / kBK;
+    // stages of kFp4KS K steps (hidden and inter are multiples of 128)
+    const int KB = p.K / (kBK * kFp4KS);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -409,8 +424,8 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                 const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
                 const size_t rt = (size_t)it.e * w.row_tiles + it.wt;
                 const int n_load = (it.nrows + 15) & ~15;
-                const uint32_t bytes =
-                    NUM_A * (kFp4CodeTile + kFp4ScaleTile) + (uint32_t)n_load * (kBK * 2);
+                const uint32_t bytes = NUM_A * (C::CODES + C::SCALES) +
+                                       (uint32_t)(kFp4KS * n_load * (kBK * 2));
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(smem_u32(&rempty[rs]), rp ^ 1u, p.ctl)) {
                         ok = false;
@@ -419,23 +434,27 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                     const uint32_t dst = base + (uint32_t)(rs * C::RAW_STAGE);
                     const uint32_t fb = smem_u32(&rfull[rs]);
                     mbar_arrive_expect_tx(fb, bytes);
-                    int off = 0;
 #pragma unroll
-                    for (int bi = 4; bi >= 1; --bi) {   // token rows: boxes of 128, 64, 32, 16 rows
-                        const int hgt = 8 << bi;
-                        if (hgt <= BN && n_load - off >= hgt) {
-                            tma_load_2d(dst + off * (kBK * 2), &tmB.m[bi], kb * kBK, it.row0 + off,
-                                        fb, pol_x);
-                            off += hgt;
+                    for (int ks = 0; ks < kFp4KS; ++ks) {
+                        int off = 0;
+#pragma unroll
+                        for (int bi = 4; bi >= 1; --bi) {   // token rows: boxes of 128, 64, 32, 16 rows
+                            const int hgt = 8 << bi;
+                            if (hgt <= BN && n_load - off >= hgt) {
+                                tma_load_2d(dst + ks * C::B_BYTES + off * (kBK * 2), &tmB.m[bi],
+                                            (kb * kFp4KS + ks) * kBK, it.row0 + off, fb, pol_x);
+                                off += hgt;
+                            }
                         }
                     }
-                    const size_t tile = rt * (size_t)w.k_steps + kb;
+                    // the stage's K steps are consecutive tiles of the layout
+                    const size_t tile = rt * (size_t)w.k_steps + (size_t)kb * kFp4KS;
 #pragma unroll
                     for (int a = 0; a < NUM_A; ++a) {
-                        bulk_load(dst + C::B_BYTES + a * kFp4CodeTile,
-                                  w.a[a].codes + tile * kFp4CodeTile, kFp4CodeTile, fb, pol_w);
-                        bulk_load(dst + C::B_BYTES + NUM_A * kFp4CodeTile + a * kFp4ScaleTile,
-                                  w.a[a].scales + tile * kFp4ScaleTile, kFp4ScaleTile, fb, pol_w);
+                        bulk_load(dst + kFp4KS * C::B_BYTES + a * C::CODES,
+                                  w.a[a].codes + tile * kFp4CodeTile, C::CODES, fb, pol_w);
+                        bulk_load(dst + kFp4KS * C::B_BYTES + NUM_A * C::CODES + a * C::SCALES,
+                                  w.a[a].scales + tile * kFp4ScaleTile, C::SCALES, fb, pol_w);
                     }
                     ++issued;
                     ring_step(rs, rp, C::RAW_STAGES);
@@ -476,23 +495,29 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                 ok = __all_sync(0xffffffffu, got);
                 if (!ok) break;
                 tc_fence_after();
-                if (!fp4_tokens_to_f16(reinterpret_cast<uint32_t *>(base_ptr + rs * C::RAW_STAGE),
-                                       n_load * (kBK / 2), it.nrows, cidx, 32 * kFp4ConvWarps))
-                    record_status(p.ctl.status, kStatusRange);
-                const uint8_t *raw = base_ptr + rs * C::RAW_STAGE + C::B_BYTES;
+                bool fits = true;
 #pragma unroll
-                for (int a = 0; a < NUM_A; ++a) {
-                    // this block of row r: 8 code bytes and one scale byte
-                    const uint2 c = *reinterpret_cast<const uint2 *>(
-                        raw + a * kFp4CodeTile + blk * (kFp4TileRows * 8) + r * 8);
-                    const uint32_t sb =
-                        lut_s[raw[NUM_A * kFp4CodeTile + a * kFp4ScaleTile + blk * kFp4TileRows + r]];
-                    uint32_t lo[4], hi[4];
-                    fp4_decode4_f16(c.x, sb | (sb << 16), lo);
-                    fp4_decode4_f16(c.y, sb | (sb << 16), hi);
-                    const uint32_t v[8] = {lo[0], lo[1], lo[2], lo[3], hi[0], hi[1], hi[2], hi[3]};
-                    tmem_st8(lane_base + (uint32_t)((cs * NUM_A + a) * kAColsPerTile), v);
-                }
+                for (int ks = 0; ks < kFp4KS; ++ks)
+                    fits &= fp4_tokens_to_f16(
+                        reinterpret_cast<uint32_t *>(base_ptr + rs * C::RAW_STAGE + ks * C::B_BYTES),
+                        n_load * (kBK / 2), it.nrows, cidx, 32 * kFp4ConvWarps);
+                if (!fits) record_status(p.ctl.status, kStatusRange);
+                const uint8_t *raw = base_ptr + rs * C::RAW_STAGE + kFp4KS * C::B_BYTES;
+#pragma unroll
+                for (int a = 0; a < NUM_A; ++a)
+#pragma unroll
+                    for (int ks = 0; ks < kFp4KS; ++ks) {
+                        // this block of row r in K step ks: 8 code bytes and one scale byte
+                        const uint2 c = *reinterpret_cast<const uint2 *>(
+                            raw + a * C::CODES + ks * kFp4CodeTile + blk * (kFp4TileRows * 8) + r * 8);
+                        const uint32_t sb = lut_s[raw[NUM_A * C::CODES + a * C::SCALES +
+                                                      ks * kFp4ScaleTile + blk * kFp4TileRows + r]];
+                        uint32_t lo[4], hi[4];
+                        fp4_decode4_f16(c.x, sb | (sb << 16), lo);
+                        fp4_decode4_f16(c.y, sb | (sb << 16), hi);
+                        const uint32_t v[8] = {lo[0], lo[1], lo[2], lo[3], hi[0], hi[1], hi[2], hi[3]};
+                        tmem_st8(lane_base + (uint32_t)(cs * C::A_STAGE_COLS + (a * kFp4KS + ks) * kAColsPerTile), v);
+                    }
                 // every lane's stores complete (the token rows' generic
                 // writes made visible to the MMA's reads too), then one
                 // arrival for the warp (512 same-address arrivals a stage
@@ -503,7 +528,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&cfull[cs]));
                 ring_step(rs, rp, C::RAW_STAGES);
-                ring_step(cs, cp, kFp4AStages);
+                ring_step(cs, cp, C::A_STAGES);
             }
         }
     } else if ((warp == 1 || (warp == kFp4Issuer2 && C::ISSUERS == 2)) && lane == 0) {
@@ -537,24 +562,28 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a0 = tmem_base + (uint32_t)(cs * NUM_A * kAColsPerTile);
+                const uint32_t a0 = tmem_base + (uint32_t)(cs * C::A_STAGE_COLS);
                 const uint32_t b_addr = base + (uint32_t)(rs * C::RAW_STAGE);
 #pragma unroll
-                for (int k = 0; k < kBK / 16; ++k) {
-                    // K sub-step k adds into chain k % CHAINS, first written at kb 0
-                    const int chain = k % C::CHAINS;
-                    if (NUM_A == 1 && C::ISSUERS == 2 && (chain & 1) != mi) continue;
-                    const int a = NUM_A == 2 ? mi : 0;
-                    const uint32_t d = d0 + (uint32_t)((chain * NUM_A + a) * BN);
-                    const uint64_t bdesc = umma_desc_sw128(b_addr + k * 32);
-                    const uint32_t accum = (kb > 0 || k >= C::CHAINS) ? 1u : 0u;
-                    umma_bf16_tmem_a(d, a0 + a * kAColsPerTile + k * 8, bdesc, idesc, accum);
-                    issued_any = true;
-                }
+                for (int ks = 0; ks < kFp4KS; ++ks)
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        // K sub-step k of step ks adds into chain k % CHAINS, first
+                        // written in the first stage's first step
+                        const int chain = k % C::CHAINS;
+                        if (NUM_A == 1 && C::ISSUERS == 2 && (chain & 1) != mi) continue;
+                        const int a = NUM_A == 2 ? mi : 0;
+                        const uint32_t d = d0 + (uint32_t)((chain * NUM_A + a) * BN);
+                        const uint64_t bdesc = umma_desc_sw128(b_addr + ks * C::B_BYTES + k * 32);
+                        const uint32_t accum = (kb > 0 || ks > 0 || k >= C::CHAINS) ? 1u : 0u;
+                        umma_bf16_tmem_a(d, a0 + (a * kFp4KS + ks) * kAColsPerTile + k * 8, bdesc, idesc,
+                                         accum);
+                        issued_any = true;
+                    }
                 umma_commit(smem_u32(&rempty[rs]));
                 umma_commit(smem_u32(&cempty[cs]));
                 ring_step(rs, rp, C::RAW_STAGES);
-                ring_step(cs, cp, kFp4AStages);
+                ring_step(cs, cp, C::A_STAGES);
             }
             if (!ok) break;
             umma_commit(smem_u32(&tfull[acc]));
