@@ -66,7 +66,8 @@ constexpr int kFp4ConvFirst = 2 + kFp4EpiWarps;            // first converter wa
 constexpr int kFp4Issuer2 = kFp4ConvFirst + kFp4ConvWarps;  // warp of the second MMA issuer
 constexpr int kFp4Threads = 32 * (kFp4Issuer2 + 1);          // 736
 constexpr int kFp4AStagesMax = 4;                          // decoded A stages in TMEM, at most
-constexpr int kFp4KS = 2;                                  // 64-wide K steps per pipeline stage
+// 64-wide K steps per pipeline stage: 2 for gate|up (what TMEM holds with two
+// accumulator buffers), 4 for down when K allows
 constexpr int kFp4Ch = 16;                                 // epilogue columns per chunk
 constexpr int kFp4MaxRaw = 24;
 constexpr int kFp4BarrierBytes = 1024;
@@ -75,12 +76,12 @@ constexpr float kFp4TokenScale = 0.00390625f;              // 2^-8: token rows a
 constexpr float kFp4TokenUnscale = 256.0f;
 constexpr int kAColsPerTile = kBK / 2;                     // 64 bf16 of a row: 32 TMEM columns
 
-template <int BN, int NUM_A, int EPI>
+template <int BN, int NUM_A, int EPI, int KS>
 struct Fp4Cfg {
     static constexpr int B_BYTES = BN * kBK * 2;                 // token rows of one K step
-    static constexpr int CODES = kFp4KS * kFp4CodeTile;           // one matrix's codes per stage
-    static constexpr int SCALES = kFp4KS * kFp4ScaleTile;
-    static constexpr int RAW_USED = kFp4KS * B_BYTES + NUM_A * (CODES + SCALES);
+    static constexpr int CODES = KS * kFp4CodeTile;           // one matrix's codes per stage
+    static constexpr int SCALES = KS * kFp4ScaleTile;
+    static constexpr int RAW_USED = KS * B_BYTES + NUM_A * (CODES + SCALES);
     static constexpr int RAW_STAGE = (RAW_USED + 1023) / 1024 * 1024;   // keeps B 1024-aligned
     static constexpr int STAGING = kFp4EpiWarps * kStagingWarpBytes;
     static constexpr int FIXED = 1024 + STAGING + kFp4BarrierBytes + kFp4LutBytes + kTableBytes;
@@ -88,7 +89,7 @@ struct Fp4Cfg {
     static constexpr int RAW_STAGES = RAW_FIT > kFp4MaxRaw ? kFp4MaxRaw : RAW_FIT;
     static constexpr int CHAINS = BN >= 64 ? 1 : 64 / BN;        // 4 for 16 rows, 2 for 32
     static constexpr int ACC_COLS = CHAINS * NUM_A * BN;         // [chain][matrix][BN]
-    static constexpr int A_STAGE_COLS = NUM_A * kFp4KS * kAColsPerTile;
+    static constexpr int A_STAGE_COLS = NUM_A * KS * kAColsPerTile;
     static constexpr int A_STAGES =
         kFp4AStagesMax * A_STAGE_COLS + 2 * ACC_COLS <= 512 ? kFp4AStagesMax : 2;
     static constexpr int A_COLS = A_STAGES * A_STAGE_COLS;
@@ -108,7 +109,7 @@ struct Fp4Cfg {
     static_assert(EPI == kSwiGLU || EPI == kStoreBF16 || EPI == kStoreF32, "fp4 epilogues");
     static_assert(32 * kFp4Ch * 4 <= kStagingWarpBytes, "staging block (FP32)");
     static_assert((2 * kFp4MaxRaw + 2 * kFp4AStagesMax + 6) * 8 + 4 <= kFp4BarrierBytes, "barriers");
-    static_assert(kFp4KS * B_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "token tiles 1024-aligned");
+    static_assert(KS * B_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "token tiles 1024-aligned");
     static_assert(32 * kFp4Ch * 2 <= kStagingWarpBytes, "staging block");
     static_assert(kFp4ConvWarps == 4 * (kFp4TileK / 16), "a converter warp per quadrant and block");
     static_assert(CHAINS <= kBK / 16, "a chain per K sub-step at most");
@@ -345,11 +346,11 @@ __device__ __forceinline__ bool fp4_tokens_to_f16(uint32_t *bw, int words, int v
 
 }  // namespace
 
-template <int BN, int NUM_A, int EPI>
+template <int BN, int NUM_A, int EPI, int KS>
 __global__ void __launch_bounds__(kFp4Threads, 1)
     grouped_gemm_fp4_kernel(const __grid_constant__ BoxMaps tmB, const Fp4Operands w, GemmArgs p)
 {
-    using C = Fp4Cfg<BN, NUM_A, EPI>;
+    using C = Fp4Cfg<BN, NUM_A, EPI, KS>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -408,8 +409,8 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
     const int WT = p.R / kBM;
     // no work while the status word is set (a failed check or wait)
     const int total = status_is_set(p.ctl.status) ? 0 : WT * s_tile[p.E];
-    // stages of kFp4KS K steps (hidden and inter are multiples of 128)
-    const int KB = p.K / (kBK * kFp4KS);
+    // stages of KS K steps (hidden and inter are multiples of 128)
+    const int KB = p.K / (kBK * KS);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -425,7 +426,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                 const size_t rt = (size_t)it.e * w.row_tiles + it.wt;
                 const int n_load = (it.nrows + 15) & ~15;
                 const uint32_t bytes = NUM_A * (C::CODES + C::SCALES) +
-                                       (uint32_t)(kFp4KS * n_load * (kBK * 2));
+                                       (uint32_t)(KS * n_load * (kBK * 2));
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(smem_u32(&rempty[rs]), rp ^ 1u, p.ctl)) {
                         ok = false;
@@ -435,25 +436,25 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                     const uint32_t fb = smem_u32(&rfull[rs]);
                     mbar_arrive_expect_tx(fb, bytes);
 #pragma unroll
-                    for (int ks = 0; ks < kFp4KS; ++ks) {
+                    for (int ks = 0; ks < KS; ++ks) {
                         int off = 0;
 #pragma unroll
                         for (int bi = 4; bi >= 1; --bi) {   // token rows: boxes of 128, 64, 32, 16 rows
                             const int hgt = 8 << bi;
                             if (hgt <= BN && n_load - off >= hgt) {
                                 tma_load_2d(dst + ks * C::B_BYTES + off * (kBK * 2), &tmB.m[bi],
-                                            (kb * kFp4KS + ks) * kBK, it.row0 + off, fb, pol_x);
+                                            (kb * KS + ks) * kBK, it.row0 + off, fb, pol_x);
                                 off += hgt;
                             }
                         }
                     }
                     // the stage's K steps are consecutive tiles of the layout
-                    const size_t tile = rt * (size_t)w.k_steps + (size_t)kb * kFp4KS;
+                    const size_t tile = rt * (size_t)w.k_steps + (size_t)kb * KS;
 #pragma unroll
                     for (int a = 0; a < NUM_A; ++a) {
-                        bulk_load(dst + kFp4KS * C::B_BYTES + a * C::CODES,
+                        bulk_load(dst + KS * C::B_BYTES + a * C::CODES,
                                   w.a[a].codes + tile * kFp4CodeTile, C::CODES, fb, pol_w);
-                        bulk_load(dst + kFp4KS * C::B_BYTES + NUM_A * C::CODES + a * C::SCALES,
+                        bulk_load(dst + KS * C::B_BYTES + NUM_A * C::CODES + a * C::SCALES,
                                   w.a[a].scales + tile * kFp4ScaleTile, C::SCALES, fb, pol_w);
                     }
                     ++issued;
@@ -497,16 +498,16 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                 tc_fence_after();
                 bool fits = true;
 #pragma unroll
-                for (int ks = 0; ks < kFp4KS; ++ks)
+                for (int ks = 0; ks < KS; ++ks)
                     fits &= fp4_tokens_to_f16(
                         reinterpret_cast<uint32_t *>(base_ptr + rs * C::RAW_STAGE + ks * C::B_BYTES),
                         n_load * (kBK / 2), it.nrows, cidx, 32 * kFp4ConvWarps);
                 if (!fits) record_status(p.ctl.status, kStatusRange);
-                const uint8_t *raw = base_ptr + rs * C::RAW_STAGE + kFp4KS * C::B_BYTES;
+                const uint8_t *raw = base_ptr + rs * C::RAW_STAGE + KS * C::B_BYTES;
 #pragma unroll
                 for (int a = 0; a < NUM_A; ++a)
 #pragma unroll
-                    for (int ks = 0; ks < kFp4KS; ++ks) {
+                    for (int ks = 0; ks < KS; ++ks) {
                         // this block of row r in K step ks: 8 code bytes and one scale byte
                         const uint2 c = *reinterpret_cast<const uint2 *>(
                             raw + a * C::CODES + ks * kFp4CodeTile + blk * (kFp4TileRows * 8) + r * 8);
@@ -516,7 +517,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                         fp4_decode4_f16(c.x, sb | (sb << 16), lo);
                         fp4_decode4_f16(c.y, sb | (sb << 16), hi);
                         const uint32_t v[8] = {lo[0], lo[1], lo[2], lo[3], hi[0], hi[1], hi[2], hi[3]};
-                        tmem_st8(lane_base + (uint32_t)(cs * C::A_STAGE_COLS + (a * kFp4KS + ks) * kAColsPerTile), v);
+                        tmem_st8(lane_base + (uint32_t)(cs * C::A_STAGE_COLS + (a * KS + ks) * kAColsPerTile), v);
                     }
                 // every lane's stores complete (the token rows' generic
                 // writes made visible to the MMA's reads too), then one
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                 const uint32_t a0 = tmem_base + (uint32_t)(cs * C::A_STAGE_COLS);
                 const uint32_t b_addr = base + (uint32_t)(rs * C::RAW_STAGE);
 #pragma unroll
-                for (int ks = 0; ks < kFp4KS; ++ks)
+                for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k) {
                         // K sub-step k of step ks adds into chain k % CHAINS, first
@@ -576,7 +577,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                         const uint32_t d = d0 + (uint32_t)((chain * NUM_A + a) * BN);
                         const uint64_t bdesc = umma_desc_sw128(b_addr + ks * C::B_BYTES + k * 32);
                         const uint32_t accum = (kb > 0 || ks > 0 || k >= C::CHAINS) ? 1u : 0u;
-                        umma_bf16_tmem_a(d, a0 + (a * kFp4KS + ks) * kAColsPerTile + k * 8, bdesc, idesc,
+                        umma_bf16_tmem_a(d, a0 + (a * KS + ks) * kAColsPerTile + k * 8, bdesc, idesc,
                                          accum);
                         issued_any = true;
                     }
@@ -675,12 +676,20 @@ __global__ void __launch_bounds__(256) fp4_dequant_kernel(const uint8_t *__restr
 }
 
 namespace {
-template <int BN, int NUM_A, int EPI>
+template <int BN, int NUM_A, int EPI, int KS>
 cudaError_t set_smem_fp4()
 {
-    return cudaFuncSetAttribute(grouped_gemm_fp4_kernel<BN, NUM_A, EPI>,
+    return cudaFuncSetAttribute(grouped_gemm_fp4_kernel<BN, NUM_A, EPI, KS>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Fp4Cfg<BN, NUM_A, EPI>::SMEM_BYTES);
+                                Fp4Cfg<BN, NUM_A, EPI, KS>::SMEM_BYTES);
+}
+
+template <int BN, int EPI, int KS>
+cudaError_t launch_fp4_down(const Fp4Operands &w, const BoxMaps &b, const GemmArgs &args, int grid,
+                            cudaStream_t stream)
+{
+    return launch_pdl(grouped_gemm_fp4_kernel<BN, 1, EPI, KS>, dim3(grid), dim3(kFp4Threads),
+                      Fp4Cfg<BN, 1, EPI, KS>::SMEM_BYTES, stream, b, w, args);
 }
 
 template <int BN>
@@ -688,14 +697,16 @@ cudaError_t launch_fp4_kind(GemmKind kind, const Fp4Operands &w, const BoxMaps &
                             const GemmArgs &args, int grid, cudaStream_t stream)
 {
     if (kind == GemmKind::kGateUp)
-        return launch_pdl(grouped_gemm_fp4_kernel<BN, 2, kSwiGLU>, dim3(grid), dim3(kFp4Threads),
-                          Fp4Cfg<BN, 2, kSwiGLU>::SMEM_BYTES, stream, b, w, args);
+        return launch_pdl(grouped_gemm_fp4_kernel<BN, 2, kSwiGLU, 2>, dim3(grid), dim3(kFp4Threads),
+                          Fp4Cfg<BN, 2, kSwiGLU, 2>::SMEM_BYTES, stream, b, w, args);
+    // down: four K steps per stage when K is a multiple of 256
+    const bool ks4 = args.K % (4 * kBK) == 0;
     if (kind == GemmKind::kDown)
-        return launch_pdl(grouped_gemm_fp4_kernel<BN, 1, kStoreBF16>, dim3(grid), dim3(kFp4Threads),
-                          Fp4Cfg<BN, 1, kStoreBF16>::SMEM_BYTES, stream, b, w, args);
+        return ks4 ? launch_fp4_down<BN, kStoreBF16, 4>(w, b, args, grid, stream)
+                   : launch_fp4_down<BN, kStoreBF16, 2>(w, b, args, grid, stream);
     if (kind == GemmKind::kDownF32 && args.out_f32 != nullptr)
-        return launch_pdl(grouped_gemm_fp4_kernel<BN, 1, kStoreF32>, dim3(grid), dim3(kFp4Threads),
-                          Fp4Cfg<BN, 1, kStoreF32>::SMEM_BYTES, stream, b, w, args);
+        return ks4 ? launch_fp4_down<BN, kStoreF32, 4>(w, b, args, grid, stream)
+                   : launch_fp4_down<BN, kStoreF32, 2>(w, b, args, grid, stream);
     return cudaErrorInvalidValue;
 }
 }  // namespace
@@ -703,10 +714,12 @@ cudaError_t launch_fp4_kind(GemmKind kind, const Fp4Operands &w, const BoxMaps &
 cudaError_t prepare_grouped_gemm_fp4()
 {
     cudaError_t err;
-#define BEAM_PREP_FP4(BN)                                                    \
-    if ((err = set_smem_fp4<BN, 2, kSwiGLU>()) != cudaSuccess) return err;   \
-    if ((err = set_smem_fp4<BN, 1, kStoreBF16>()) != cudaSuccess) return err; \
-    if ((err = set_smem_fp4<BN, 1, kStoreF32>()) != cudaSuccess) return err;
+#define BEAM_PREP_FP4(BN)                                                       \
+    if ((err = set_smem_fp4<BN, 2, kSwiGLU, 2>()) != cudaSuccess) return err;   \
+    if ((err = set_smem_fp4<BN, 1, kStoreBF16, 2>()) != cudaSuccess) return err; \
+    if ((err = set_smem_fp4<BN, 1, kStoreF32, 2>()) != cudaSuccess) return err;  \
+    if ((err = set_smem_fp4<BN, 1, kStoreBF16, 4>()) != cudaSuccess) return err; \
+    if ((err = set_smem_fp4<BN, 1, kStoreF32, 4>()) != cudaSuccess) return err;
     BEAM_PREP_FP4(16)
     BEAM_PREP_FP4(32)
     BEAM_PREP_FP4(64)
