@@ -83,6 +83,24 @@ def test_nvfp4_block(T, ctas, tile, resid):
     moe.close()
 
 
+# inter 256: the down GEMM takes four K steps per stage (K/64 a multiple of
+# four), at every token tile size
+@pytest.mark.parametrize("T,tile", [(300, 16), (300, 32), (1000, 64), (1000, 128)])
+def test_nvfp4_block_four_k_steps_per_stage(T, tile):
+    wl = dataclasses.replace(W.WORKLOADS["tiny_nvfp4"], inter=256)
+    g = W.generator(wl, "cuda")
+    d = W.make_nvfp4_weights(wl, "cuda", g)
+    d.update(W.make_tokens(wl, "cuda", g, T=T))
+    moe = BeamMoE.from_workload(wl, d, max_tokens=T)
+    moe.set_gemm_tuning(0, tile, -1, 1)
+    plan = moe.launch_plan(T)
+    assert plan["tile_rows"] == tile
+    rep = check_block(wl, d, moe)
+    _log(f"nvfp4_inter256_T{T}_tile{tile}", rep, plan)
+    assert rep.ok(), rep
+    moe.close()
+
+
 def test_nvfp4_beam_decode():
     wl = W.WORKLOADS["decode_nvfp4"]
     g = W.generator(wl, "cuda")
