@@ -90,8 +90,11 @@ struct Fp4Cfg {
     static constexpr int CHAINS = BN >= 64 ? 1 : 64 / BN;        // 4 for 16 rows, 2 for 32
     static constexpr int ACC_COLS = CHAINS * NUM_A * BN;         // [chain][matrix][BN]
     static constexpr int A_STAGE_COLS = NUM_A * KS * kAColsPerTile;
+    // as many A stages as tensor memory holds beside two accumulator
+    // buffers, up to four (two at least: then one accumulator buffer)
+    static constexpr int A_STAGES_FIT = (512 - 2 * ACC_COLS) / A_STAGE_COLS;
     static constexpr int A_STAGES =
-        kFp4AStagesMax * A_STAGE_COLS + 2 * ACC_COLS <= 512 ? kFp4AStagesMax : 2;
+        A_STAGES_FIT > kFp4AStagesMax ? kFp4AStagesMax : (A_STAGES_FIT < 2 ? 2 : A_STAGES_FIT);
     static constexpr int A_COLS = A_STAGES * A_STAGE_COLS;
     // MMA issuers: gate and up each from their own thread (measured: the
     // gate|up GEMM 10% faster at 16-row tiles); down keeps one (splitting
