@@ -173,15 +173,17 @@ def workload_config(name: str, wl) -> dict:
             "post_norm": wl.post_norm, "expert_weights": wl.weight_format}
 
 
-def kernels_per_forward(plan: dict, dense: bool, residual: bool) -> int:
+def kernels_per_forward(plan: dict, dense: bool, residual: bool, pairs: int, n_experts: int) -> int:
     """Kernels of this library one forward pass launches, from its launch plan."""
     if dense:
         # table set-up, gate|up, down, combine (only for the residual update)
         return 1 + 1 + 1 + int(residual)
     # router: logits + selection (CUDA cores) or tensor-core logits, selection,
     # exact re-derivation, selection of the re-derived tokens; dispatch:
-    # count, scan, permute or row maps; the two GEMMs; combine
-    return (4 if plan["router_tensor_cores"] else 2) + 3 + 2 + 1
+    # count, scan, permute or row maps, or one block for at most 1024 pairs
+    # when the GEMM gathers its token rows; the two GEMMs; combine
+    one_block = plan["gather_rows"] == 1 and pairs <= 1024 and n_experts <= 1024
+    return (4 if plan["router_tensor_cores"] else 2) + (1 if one_block else 3) + 2 + 1
 
 
 def expert_weight_bytes(wl) -> float:
@@ -424,8 +426,8 @@ def run_ours(args):
                 "windows": len(e2e_win), "steps_per_window": e2e_steps,
                 "h2d_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0),
                 "d2h_bytes_per_step": T * H * 2 + (T * H * 4 if wl.residual_k else 0)},
-        "gpu_launches": kernels_per_forward(plan, dense, bool(wl.residual_k)) * steps_done * n_win,
-        "gpu_launches_per_step": kernels_per_forward(plan, dense, bool(wl.residual_k)),
+        "gpu_launches": kernels_per_forward(plan, dense, bool(wl.residual_k), wl.T * wl.top_k, wl.n_experts) * steps_done * n_win,
+        "gpu_launches_per_step": kernels_per_forward(plan, dense, bool(wl.residual_k), wl.T * wl.top_k, wl.n_experts),
         "roofline": roof,
         "launch_plan": plan,
     }
