@@ -124,10 +124,11 @@ def test_tiny_residual(norm):
     moe.close()
 
 
-@pytest.mark.parametrize("gather", [-1, 1, 0])
-def test_tiny_dispatch_is_a_stable_counting_sort(gather):
+# T=1000 takes the three-kernel dispatch; T of at most 128 (top-8: 1024
+# pairs) with gathered token rows takes the one-block dispatch
+@pytest.mark.parametrize("gather,T", [(-1, 1000), (1, 1000), (0, 1000), (1, 100), (1, 1), (0, 100)])
+def test_tiny_dispatch_is_a_stable_counting_sort(gather, T):
     wl = W.WORKLOADS["tiny"]
-    T = 1000
     d = _inputs(wl, T)
     moe = BeamMoE.from_workload(wl, d, max_tokens=T)
     moe.set_gemm_tuning(gather_rows=gather)
