@@ -3,13 +3,13 @@
 // epilogue as the single-CTA bf16 kernel (grouped_gemm.cu); what differs is
 // the path of a weight tile to the tensor cores:
 //
-//   warp 0        producer: per K step, bulk copies of the tile's 4096 bytes
-//                 of codes and 512 bytes of block scales (per matrix) and the
-//                 TMA boxes of the token rows, into a deep ring in shared
-//                 memory;
+//   warp 0        producer: per stage of KS K steps, bulk copies of KS tiles'
+//                 4096 bytes of codes and 512 bytes of block scales each (per
+//                 matrix, consecutive in the layout) and the TMA boxes of the
+//                 token rows of each step, into a ring in shared memory;
 //   warps 6..21   converters, four per TMEM lane quadrant: thread r of the
 //                 g-th warp of a quadrant decodes the g-th 16-element block
-//                 of weight row r of a stage to f16 (hardware E2M1 -> f16
+//                 of weight row r of each K step to f16 (hardware E2M1 -> f16
 //                 conversion and one f16 multiply by the block scale: every
 //                 product has at most 6 significant bits and lies between
 //                 2^-10 and 2688 in magnitude, so it is exact) and writes it
@@ -20,22 +20,25 @@
 //                 that, and a larger value sets the status word
 //                 (BEAM_ERR_RANGE); the epilogue multiplies by 2^8 again;
 //   warps 1, 22   MMA issuers (lane 0): A (the decoded weights) from TMEM,
-//                 four stages deep, B (the token rows) from the shared-memory
-//                 stage.  gate|up: warp 1 issues the gate MMAs and warp 22
-//                 the up MMAs; down: warp 1 alone.  At 16-row token tiles
-//                 the issuing thread, not the tensor pipe, sets the pace (an
-//                 issued MMA of this shape is ~100 cycles of issue for a few
-//                 cycles of tensor work), so two issuers cut the gate|up time
-//                 by about a tenth; splitting down the same way was slower;
+//                 two to four stages deep, B (the token rows) from the
+//                 shared-memory stage.  gate|up: warp 1 issues the gate MMAs
+//                 and warp 22 the up MMAs; down: warp 1 alone.  At 16-row
+//                 token tiles the issuing thread, not the tensor pipe, sets
+//                 the pace (an issued MMA of this shape is ~100 cycles of
+//                 issue for a few cycles of tensor work), so two issuers cut
+//                 the gate|up time by about a tenth; splitting down the same
+//                 way was slower.  An issuer waits only for the converters'
+//                 arrival: they waited for the raw stage before converting;
 //   warps 2..5    epilogue, one per quadrant: as the bf16 kernel, with the
 //                 FP32 accumulators first multiplied by the per-tensor scales.
 //
-// Stages: a pipeline stage holds two 64-wide K steps (the codes and scales
-// of two consecutive tiles of the layout, the token rows of both steps), so
-// every per-stage cost of the issuing threads and the converters (barrier
-// waits, fences, commits) is paid once per 128 of K.  At 16-row tiles those
-// costs, not the tensor core, set the pace: one wait less per stage took 8%
-// off the decode step, two steps per stage 20% more.
+// Stages: a pipeline stage holds KS 64-wide K steps (the codes and scales
+// of KS consecutive tiles of the layout, the token rows of each step): 2 for
+// gate|up, 4 for down when K/64 allows.  Every per-stage cost of the issuing
+// threads and the converters (barrier waits, fences, commits) is then paid
+// once per 64 KS of K.  At 16-row tiles those costs, not the tensor core,
+// set the pace: one wait less per stage took 8% off the decode step, two
+// steps per stage 20% more, four for down another 7%.
 //
 // Accumulator chains: small tiles spread the four K sub-steps of a step over
 // CHAINS independent accumulators per matrix, so consecutive MMAs never add
