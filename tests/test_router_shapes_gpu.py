@@ -76,3 +76,32 @@ def test_largest_supported_shapes():
     rep = check_block(wl, d, moe)
     assert rep.ok(), rep
     moe.close()
+
+
+@pytest.mark.parametrize("hidden,T", [(384, 64), (384, 1), (128, 37), (1024, 64), (5120, 64),
+                                      (5120, 1)])
+def test_small_batch_router(hidden, T):
+    """Batches of at most 64 tokens take the small-batch logits kernel with
+    its cost-chosen K slices: 2 and 6 slices of 64 (hidden 128, 384), 8 of
+    128 (hidden 1024), 8 of 640 (hidden 5120). Checked here: the logits
+    against their exact value, the routing against the oracle, and a second
+    call equal to the first bit for bit."""
+    import torch
+    wl = dataclasses.replace(W.WORKLOADS["decode"], name=f"small_router_{hidden}", T=T,
+                             hidden=hidden, inter=128)
+    g = W.generator(wl, "cuda")
+    d = W.make_weights(wl, "cuda", g)
+    d.update(W.make_tokens(wl, "cuda", g))
+    moe = BeamMoE.from_workload(wl, d, max_tokens=64)
+    got = moe.router_logits(d["x"]).cpu().double().numpy()
+    ref = oracle.bf16_to_f64(W.bf16_bits(d["x"])) @ d["router_w"].cpu().double().numpy().T
+    assert np.abs(got - ref).max() < 2e-6 * max(1.0, np.abs(ref).max())
+    idx, w = moe.route(d["x"])
+    idx2, w2 = moe.route(d["x"])
+    assert torch.equal(idx, idx2) and torch.equal(w, w2)
+    r = oracle.route(W.bf16_bits(d["x"]), d["router_w"].cpu().numpy(), d["bias"].cpu().numpy(),
+                     wl.n_group, wl.topk_group, wl.top_k)
+    keep = (r.gap_expert >= NEAR_TIE) & (r.gap_group >= NEAR_TIE) & (r.gap_order >= NEAR_TIE)
+    np.testing.assert_array_equal(idx.cpu().numpy()[keep], r.idx[keep])
+    assert np.abs(w.cpu().numpy()[keep] - r.w[keep]).max() <= W_ABS
+    moe.close()
