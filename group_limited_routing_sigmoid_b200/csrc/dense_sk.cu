@@ -311,42 +311,82 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!s_last) continue;
             __threadfence();
             // the last arriver: every segment's sums in K order, then the
-            // epilogue.  Thread et takes weight row r = et % 128 of tokens
-            // et / 128, + 2, + 4, ...: per segment all its loads are issued
-            // before any is added, so a segment costs one memory round trip.
+            // epilogue.  Thread et takes weight rows r4 .. r4 + 3 (r4 =
+            // 4 * (et % 32)) of tokens et / 32, + 8, + 16, ...; in passes of
+            // IP tokens it issues the 16-byte loads of SG segments at once
+            // before adding them, so a pass costs ceil(segments / SG) memory
+            // round trips.
             const int b0 = unit_owner((long long)sg.t * KB, U, G);
             const int b1 = unit_owner((long long)(sg.t + 1) * KB - 1, U, G);
-            const int r = et & (kBM - 1);
-            constexpr int NPT = BN / 2;                      // tokens per thread
-            float v[NPT][C::NUM_A];
+            const int r4 = (et & 31) * 4;
+            const int ng = et >> 5;
+            constexpr int TPT = BN / 8;                      // tokens per thread
+            constexpr int IP = TPT < 4 ? TPT : 4;            // tokens per pass
+            constexpr int SG = GATEUP ? 2 : 5;               // segments per batch of loads
+            constexpr int LDN = C::NUM_A * kBM;              // floats per token row of a slot
+#pragma unroll 1
+            for (int i0 = 0; i0 < TPT; i0 += IP) {
+                float4 v[IP][C::NUM_A];
 #pragma unroll
-            for (int i = 0; i < NPT; ++i)
+                for (int i = 0; i < IP; ++i)
 #pragma unroll
-                for (int a = 0; a < C::NUM_A; ++a) v[i][a] = 0.f;
-            for (int cb = b0; cb <= b1; ++cb) {
-                const int ft = (int)(unit_start(cb, U, G) / KB);   // cb's first tile
-                const float *src = part + (size_t)(2 * cb + (sg.t == ft ? 0 : 1)) * C::PART + r;
-                float ld[NPT][C::NUM_A];
+                    for (int a = 0; a < C::NUM_A; ++a) v[i][a] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+                for (int c0 = b0; c0 <= b1; c0 += SG) {
+                    float4 ld[SG][IP][C::NUM_A];
 #pragma unroll
-                for (int i = 0; i < NPT; ++i) {
-                    const int n = (et >> 7) + 2 * i;
+                    for (int q = 0; q < SG; ++q) {
+                        const int cb = c0 + q;
+                        const float *src = part + r4;
+                        if (cb <= b1) {
+                            const int ft = (int)(unit_start(cb, U, G) / KB);   // cb's first tile
+                            src += (size_t)(2 * cb + (sg.t == ft ? 0 : 1)) * C::PART;
+                        }
 #pragma unroll
-                    for (int a = 0; a < C::NUM_A; ++a)
-                        ld[i][a] = n < nrows ? __ldcg(src + (size_t)n * C::NUM_A * kBM + a * kBM) : 0.f;
+                        for (int i = 0; i < IP; ++i) {
+                            const int n = ng + 8 * (i0 + i);
+#pragma unroll
+                            for (int a = 0; a < C::NUM_A; ++a)
+                                ld[q][i][a] = (cb <= b1 && n < nrows)
+                                                  ? __ldcg(reinterpret_cast<const float4 *>(src + (size_t)n * LDN + a * kBM))
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < SG; ++q) {
+                        if (c0 + q > b1) break;
+#pragma unroll
+                        for (int i = 0; i < IP; ++i)
+#pragma unroll
+                            for (int a = 0; a < C::NUM_A; ++a) {
+                                v[i][a].x += ld[q][i][a].x;
+                                v[i][a].y += ld[q][i][a].y;
+                                v[i][a].z += ld[q][i][a].z;
+                                v[i][a].w += ld[q][i][a].w;
+                            }
+                    }
                 }
 #pragma unroll
-                for (int i = 0; i < NPT; ++i)
+                for (int i = 0; i < IP; ++i) {
+                    const int n = ng + 8 * (i0 + i);
+                    if (n >= nrows) continue;
+                    float o[4];
+                    const float *g = &v[i][0].x;
+                    if constexpr (GATEUP) {
+                        const float *u = &v[i][C::NUM_A - 1].x;
 #pragma unroll
-                    for (int a = 0; a < C::NUM_A; ++a) v[i][a] += ld[i][a];
-            }
+                        for (int c = 0; c < 4; ++c) o[c] = silu_f32(g[c]) * u[c];
+                    } else {
 #pragma unroll
-            for (int i = 0; i < NPT; ++i) {
-                const int n = (et >> 7) + 2 * i;
-                if (n >= nrows) continue;
-                float o;
-                if constexpr (GATEUP) o = silu_f32(v[i][0]) * v[i][1];
-                else o = v[i][0];
-                p.out[(size_t)(row0 + n) * p.R + wt * kBM + r] = __float2bfloat16_rn(o);
+                        for (int c = 0; c < 4; ++c) o[c] = g[c];
+                    }
+                    __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
+                    __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
+                    uint2 pk;
+                    pk.x = *reinterpret_cast<uint32_t *>(&lo);
+                    pk.y = *reinterpret_cast<uint32_t *>(&hi);
+                    *reinterpret_cast<uint2 *>(p.out + (size_t)(row0 + n) * p.R + wt * kBM + r4) = pk;
+                }
             }
             if (et == 0) cnt[sg.t] = 0;   // ready for the next pass
         }
