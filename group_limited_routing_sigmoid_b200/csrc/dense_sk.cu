@@ -138,6 +138,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_barrier_init();
         tma_prefetch_desc(&tmA0);
         if (GATEUP) tma_prefetch_desc(&tmA1);
+        // the first 8 weight tiles of this CTA's range into L2 while the
+        // preceding kernel finishes; a prefetch only warms the coherent L2,
+        // so issuing it before the wait for that kernel is safe
+        {
+            const int NT0 = (T + BN - 1) / BN, KB0 = p.K / kBK;
+            const long long U0 = (long long)(p.R / kBM) * NT0 * KB0;
+            Seg s0;
+            if (U0 > 0 && segment(blockIdx.x, 0, U0, gridDim.x, KB0, s0)) {
+                const int wt0 = s0.t / NT0;
+                const int kend = s0.k0 + 8 < s0.k1 ? s0.k0 + 8 : s0.k1;
+                for (int kb = s0.k0; kb < kend; ++kb) {
+                    tma_prefetch_l2_2d(&tmA0, kb * kBK, wt0 * kBM);
+                    if (GATEUP) tma_prefetch_l2_2d(&tmA1, kb * kBK, wt0 * kBM);
+                }
+            }
+        }
     }
     if (warp == 1) {
         __syncwarp();
