@@ -122,9 +122,14 @@ class ClockSampler:
 # helpers
 # ---------------------------------------------------------------------------
 
-def kernel_hash() -> str:
+# the sources of the bf16 grouped GEMMs: the default for a traffic entry
+# that names no sources of its own
+GEMM_SOURCES = ("grouped_gemm.cu", "grouped_gemm_pair.cu", "gemm_common.cuh", "common.cuh", "kernels.cuh")
+
+
+def kernel_hash(files=GEMM_SOURCES) -> str:
     h = hashlib.sha256()
-    for fn in ("grouped_gemm.cu", "grouped_gemm_pair.cu", "gemm_common.cuh", "common.cuh", "kernels.cuh"):
+    for fn in files:
         with open(os.path.join(ROOT, "group_limited_routing_sigmoid_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -139,7 +144,7 @@ def ncu_traffic(workload: str):
     with open(path) as f:
         t = json.load(f)
     entry = t.get(workload)
-    if not entry or entry.get("kernel_hash") != kernel_hash():
+    if not entry or entry.get("kernel_hash") != kernel_hash(tuple(entry.get("sources", GEMM_SOURCES))):
         return None
     return entry.get("dram_bytes_per_launch")
 

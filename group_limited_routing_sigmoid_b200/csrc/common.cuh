@@ -142,16 +142,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// Prefetch of one tile of a 2-D tensor into L2 (no shared memory, no
-// completion to wait for).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int32_t x, int32_t y)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y)
-                 : "memory");
-}
-
 // Four rows of a 2-D tensor, at row coordinates r0..r3 and columns
 // x..x+63 (the map's box is 64 columns by one row), into four consecutive
 // 128-byte rows of shared memory, with the map's swizzle; completes on the

@@ -52,6 +52,16 @@ struct SkCfg {
     static_assert(SMEM_BYTES <= kMaxDynSmem, "shared memory");
 };
 
+// Prefetch of one tile of a 2-D tensor into L2 (no shared memory, no
+// completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int32_t x, int32_t y)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
 struct Seg {
     int t;        // tile
     int k0, k1;   // K steps [k0, k1)
