@@ -10,13 +10,15 @@
 // cuts it into segments, each a K range of one tile:
 //   - a segment that covers its whole tile finishes it in the epilogue
 //     (SwiGLU to bf16 h for gate|up; bf16 out for down);
-//   - a partial segment writes its FP32 sums to the CTA's slot (slot 0 for
-//     the CTA's first segment, 1 for its last), then counts itself in the
-//     tile's arrival counter.  The CTA that brings the count to the tile's
-//     segment number adds every segment's sums in K order (the CTAs in
-//     increasing order), so the result does not depend on which CTA arrives
-//     last, and applies the epilogue.  Nobody waits: the last arriver finds
-//     the others' sums complete.
+//   - a tile cut between CTAs b0 < ... < b1 is finished by b0, the owner of
+//     its first K steps.  That piece is the last segment of b0's range, so b0
+//     reaches it last.  Every other piece writes its FP32 sums to its CTA's
+//     slot (slot 0 for the CTA's first segment, 1 for its last) and counts
+//     itself in the tile's counter.  b0 waits (bounded) for the count, then
+//     adds the pieces in K order to its own sums, read straight from TMEM, and
+//     applies the epilogue.  A CTA waits only on higher-numbered CTAs, which
+//     publish their pieces of the tile before any wait of their own, and all
+//     CTAs are resident (one per SM, the grid no larger than the SM count).
 // The counters are zeroed by the layer's set-up kernel before each pass.
 //
 // Roles as the single-CTA grouped GEMM (grouped_gemm.cu): warp 0 TMA
@@ -104,6 +106,28 @@ __device__ __forceinline__ bool epi_sync(uint64_t *bar, uint32_t &phase, const W
     const bool ok = mbar_wait(smem_u32(bar), phase, ctl);
     phase ^= 1u;
     return ok;
+}
+
+// Wait (bounded) until *count reaches target: the other pieces of a tile are
+// published.  Their CTAs are resident (one CTA per SM, the grid no larger
+// than the SM count) and never wait for this one, since a CTA waits only on
+// pieces of higher-numbered CTAs.  Gives up as mbar_wait does.
+__device__ __forceinline__ bool wait_count(const int *count, int target, const WaitCtl &ctl)
+{
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
+        if (v >= target) return true;
+        __nanosleep(64);
+        if ((it & 15u) == 15u) {
+            if (status_is_set(ctl.status)) return false;
+            if ((long long)(global_timer_ns() - t0) > ctl.limit_ns) {
+                record_status(ctl.status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
 }
 
 }  // namespace
@@ -318,102 +342,89 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(smem_u32(&tempty[acc]));
                 continue;
             }
-            // a partial K range: FP32 sums to this CTA's slot, [token][matrix][128]
-            float *slot = part + (size_t)(2 * b + (sg.first ? 0 : 1)) * C::PART;
-#pragma unroll 1
-            for (int a = 0; a < C::NUM_A; ++a)
-                epilogue_f32_staged(taddr + a * BN, nrows, 0, half, lane, stg, slot + a * kBM + quad * 32,
-                                    C::NUM_A * kBM);
-            tc_fence_before();
-            mbar_arrive(smem_u32(&tempty[acc]));   // TMEM is free again; the rest reads memory
-            __threadfence();
-            if (!__all_sync(0xffffffffu, epi_sync(epi_bar, ephase, p.ctl))) break;
-            if (et == 0) {
-                const int b0 = unit_owner((long long)sg.t * KB, U, G);
-                const int b1 = unit_owner((long long)(sg.t + 1) * KB - 1, U, G);
-                s_last = atomicAdd(&cnt[sg.t], 1) == b1 - b0;
-            }
-            if (!__all_sync(0xffffffffu, epi_sync(epi_bar, ephase, p.ctl))) break;
-            if (!s_last) continue;
-            __threadfence();
-            // the last arriver: every segment's sums in K order, then the
-            // epilogue.  Thread et takes weight rows r4 .. r4 + 3 (r4 =
-            // 4 * (et % 32)) of tokens et / 32, + 8, + 16, ...; in passes of
-            // IP tokens it issues the 16-byte loads of SG segments at once
-            // before adding them, so a pass costs ceil(segments / SG) memory
-            // round trips.
+            // a partial K range of tile sg.t, whose pieces belong to CTAs
+            // b0 .. b1 in K order.  b0's piece (the tile's first K steps) is
+            // the last segment of b0's range, so b0 reaches it last: b0 adds
+            // the others' published pieces to its own, still in TMEM.
             const int b0 = unit_owner((long long)sg.t * KB, U, G);
             const int b1 = unit_owner((long long)(sg.t + 1) * KB - 1, U, G);
-            const int r4 = (et & 31) * 4;
-            const int ng = et >> 5;
-            constexpr int TPT = BN / 8;                      // tokens per thread
-            constexpr int IP = TPT < 4 ? TPT : 4;            // tokens per pass
-            constexpr int SG = GATEUP ? 2 : 5;               // segments per batch of loads
-            constexpr int LDN = C::NUM_A * kBM;              // floats per token row of a slot
+            if (b != b0) {
+                // FP32 sums to this CTA's slot, [token][matrix][128], then publish
+                float *slot = part + (size_t)(2 * b + (sg.first ? 0 : 1)) * C::PART;
 #pragma unroll 1
-            for (int i0 = 0; i0 < TPT; i0 += IP) {
-                float4 v[IP][C::NUM_A];
-#pragma unroll
-                for (int i = 0; i < IP; ++i)
-#pragma unroll
-                    for (int a = 0; a < C::NUM_A; ++a) v[i][a] = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int a = 0; a < C::NUM_A; ++a)
+                    epilogue_f32_staged(taddr + a * BN, nrows, 0, half, lane, stg, slot + a * kBM + quad * 32,
+                                        C::NUM_A * kBM);
+                tc_fence_before();
+                mbar_arrive(smem_u32(&tempty[acc]));   // TMEM is free again
+                __threadfence();
+                if (!__all_sync(0xffffffffu, epi_sync(epi_bar, ephase, p.ctl))) break;
+                if (et == 0) atomicAdd(&cnt[sg.t], 1);
+                continue;
+            }
+            // b0: wait (bounded) until the b1 - b0 other pieces are published
+            if (et == 0) s_last = wait_count(&cnt[sg.t], b1 - b0, p.ctl) ? 1 : 0;
+            if (!__all_sync(0xffffffffu, epi_sync(epi_bar, ephase, p.ctl))) break;
+            if (!s_last) break;
+            __threadfence();
+            // Thread (quad, lane) holds weight row r = quad * 32 + lane of its
+            // token chunks (CH columns, alternating between the quadrant's two
+            // warps): its own sums from TMEM, then the pieces of b0 + 1 ..
+            // b1 in order, SG pieces' loads at once.
+            const int r = quad * 32 + lane;
+            constexpr int CH = C::CH;
+            constexpr int SG = GATEUP ? 1 : 2;          // pieces per batch of loads
+            constexpr int LDN = C::NUM_A * kBM;         // floats per token row of a slot
 #pragma unroll 1
-                for (int c0 = b0; c0 <= b1; c0 += SG) {
-                    float4 ld[SG][IP][C::NUM_A];
+            for (int c0 = half * CH; c0 < nrows; c0 += 2 * CH) {
+                float v[C::NUM_A][CH];
+#pragma unroll
+                for (int a = 0; a < C::NUM_A; ++a) {
+                    uint32_t u[CH];
+                    tmem_ld<CH>(taddr + a * BN + c0, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) v[a][j] = 0.f + __uint_as_float(u[j]);
+                }
+#pragma unroll 1
+                for (int q0 = b0 + 1; q0 <= b1; q0 += SG) {
+                    float ld[SG][C::NUM_A][CH];
 #pragma unroll
                     for (int q = 0; q < SG; ++q) {
-                        const int cb = c0 + q;
-                        const float *src = part + r4;
+                        const int cb = q0 + q;
+                        const float *src = part + r;
                         if (cb <= b1) {
                             const int ft = (int)(unit_start(cb, U, G) / KB);   // cb's first tile
                             src += (size_t)(2 * cb + (sg.t == ft ? 0 : 1)) * C::PART;
                         }
 #pragma unroll
-                        for (int i = 0; i < IP; ++i) {
-                            const int n = ng + 8 * (i0 + i);
+                        for (int a = 0; a < C::NUM_A; ++a)
 #pragma unroll
-                            for (int a = 0; a < C::NUM_A; ++a)
-                                ld[q][i][a] = (cb <= b1 && n < nrows)
-                                                  ? __ldcg(reinterpret_cast<const float4 *>(src + (size_t)n * LDN + a * kBM))
-                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-                        }
+                            for (int j = 0; j < CH; ++j)
+                                ld[q][a][j] = (cb <= b1 && c0 + j < nrows)
+                                                  ? __ldcg(src + (size_t)(c0 + j) * LDN + a * kBM)
+                                                  : 0.f;
                     }
 #pragma unroll
                     for (int q = 0; q < SG; ++q) {
-                        if (c0 + q > b1) break;
+                        if (q0 + q > b1) break;
 #pragma unroll
-                        for (int i = 0; i < IP; ++i)
+                        for (int a = 0; a < C::NUM_A; ++a)
 #pragma unroll
-                            for (int a = 0; a < C::NUM_A; ++a) {
-                                v[i][a].x += ld[q][i][a].x;
-                                v[i][a].y += ld[q][i][a].y;
-                                v[i][a].z += ld[q][i][a].z;
-                                v[i][a].w += ld[q][i][a].w;
-                            }
+                            for (int j = 0; j < CH; ++j) v[a][j] += ld[q][a][j];
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < IP; ++i) {
-                    const int n = ng + 8 * (i0 + i);
-                    if (n >= nrows) continue;
-                    float o[4];
-                    const float *g = &v[i][0].x;
-                    if constexpr (GATEUP) {
-                        const float *u = &v[i][C::NUM_A - 1].x;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) o[c] = silu_f32(g[c]) * u[c];
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) o[c] = g[c];
-                    }
-                    __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
-                    __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
-                    uint2 pk;
-                    pk.x = *reinterpret_cast<uint32_t *>(&lo);
-                    pk.y = *reinterpret_cast<uint32_t *>(&hi);
-                    *reinterpret_cast<uint2 *>(p.out + (size_t)(row0 + n) * p.R + wt * kBM + r4) = pk;
+                for (int j = 0; j < CH; ++j) {
+                    if (c0 + j >= nrows) break;
+                    float o;
+                    if constexpr (GATEUP) o = silu_f32(v[0][j]) * v[C::NUM_A - 1][j];
+                    else o = v[0][j];
+                    p.out[(size_t)(row0 + c0 + j) * p.R + wt * kBM + r] = __float2bfloat16_rn(o);
                 }
             }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty[acc]));
             if (et == 0) cnt[sg.t] = 0;   // ready for the next pass
         }
     }
