@@ -12,6 +12,12 @@
 #include "fp4.cuh"
 #include "kernels.cuh"
 
+namespace beam {
+// The dense stream-K GEMMs' wait on a global counter, checked the same way
+// (defined in dense_sk.cu beside the wait).
+cudaError_t launch_count_wait_check(WaitCtl ctl, cudaStream_t stream);
+}  // namespace beam
+
 using namespace beam;
 
 struct beam_moe {
@@ -1380,7 +1386,11 @@ int beam_moe_check_wait_timeout(beam_moe_t h, void *stream)
     ctl.limit_ns = h->wait_limit_ns;
     cudaError_t e = launch_wait_timeout_check(ctl, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(h, e, "self-check launch");
-    return beam_moe_get_status(h, stream);
+    const int first = beam_moe_get_status(h, stream);   // read and cleared
+    e = launch_count_wait_check(ctl, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(h, e, "self-check launch");
+    const int second = beam_moe_get_status(h, stream);
+    return first != BEAM_ERR_TIMEOUT ? first : second;
 }
 
 const char *beam_moe_last_error(beam_moe_t h) { return h ? h->err : g_create_err; }

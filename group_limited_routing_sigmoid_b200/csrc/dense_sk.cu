@@ -494,4 +494,22 @@ cudaError_t launch_dense_sk(bool gate_up, int BN, const CUtensorMap &a0, const C
     }
 }
 
+// Failure-detection check of wait_count: one thread polls a counter that
+// nothing increments, with the caller's limit; it must give up and record
+// kStatusTimeout.
+namespace {
+__device__ int g_unset_count;   // zero, never written
+}
+
+__global__ void count_wait_check_kernel(WaitCtl ctl)
+{
+    if (threadIdx.x == 0) wait_count(&g_unset_count, 1, ctl);
+}
+
+cudaError_t launch_count_wait_check(WaitCtl ctl, cudaStream_t stream)
+{
+    count_wait_check_kernel<<<1, 32, 0, stream>>>(ctl);
+    return cudaGetLastError();
+}
+
 }  // namespace beam

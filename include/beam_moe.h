@@ -465,10 +465,13 @@ int beam_moe_profile_begin(beam_moe_t h, int max_calls);
 int beam_moe_profile_end(beam_moe_t h, float *stage_ms, int *calls);
 
 /*
- * Failure-detection check: launch one kernel that waits, with the handle's
- * wait limit, on a barrier that nothing completes; it must give up, record
- * BEAM_ERR_TIMEOUT in the status word and return.  Returns the status word
- * as beam_moe_get_status does.  Synchronous.
+ * Failure-detection check of the two kinds of in-kernel wait, each with the
+ * handle's wait limit: one kernel waits on a shared-memory barrier that
+ * nothing completes, a second polls a global counter that nothing
+ * increments (the wait of the dense stream-K GEMMs).  Each must give up,
+ * record BEAM_ERR_TIMEOUT in the status word and return; the status word is
+ * read and cleared after each.  Returns BEAM_ERR_TIMEOUT if both did, else
+ * the first other status.  Synchronous.
  */
 int beam_moe_check_wait_timeout(beam_moe_t h, void *stream);
 

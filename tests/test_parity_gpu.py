@@ -273,8 +273,9 @@ def test_launch_plan_follows_tokens_per_expert_and_tuning():
 
 
 def test_bounded_wait_reports_timeout_and_context_survives():
-    """A wait on a barrier that nothing completes gives up after the limit,
-    records BEAM_ERR_TIMEOUT and returns; the context stays usable."""
+    """A wait on a barrier that nothing completes, and a wait on a global
+    counter that nothing increments, each give up after the limit, record
+    BEAM_ERR_TIMEOUT and return; the context stays usable."""
     wl = W.WORKLOADS["tiny"]
     d = _inputs(wl)
     moe = BeamMoE.from_workload(wl, d)
