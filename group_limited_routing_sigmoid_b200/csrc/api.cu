@@ -541,6 +541,7 @@ int run_forward(beam_moe *h, cudaStream_t s, const void *x, int T, void *out, fl
     d.row_pair = h->row_pair;
     d.xp = h->xp;
     d.copy_rows = !plan.gather;
+    d.xp_f16 = h->fp4 ? 1 : 0;
     cudaError_t e = launch_dispatch(d, s);
     if (e == cudaSuccess && h->checks)
         e = launch_check_dispatch(h->idx, h->counts, h->offsets, h->tile_off, h->pair_row,

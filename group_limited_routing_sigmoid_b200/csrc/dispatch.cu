@@ -111,12 +111,16 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
 }
 
 // One warp per pair: its row in the sorted buffer, the maps both ways, and
-// the copy of the token's hidden vector (16-byte vectors).
+// the copy of the token's hidden vector (16-byte vectors).  With to_f16 the
+// copy holds f16 values of x x 2^-8, the operand type of the NVFP4 GEMMs
+// (the MMA takes A and B of one type); a value beyond the f16 range sets
+// BEAM_ERR_RANGE in the status word.
 __global__ void __launch_bounds__(256) dispatch_permute_kernel(
     const int *status, const int32_t *__restrict__ idx, const int32_t *__restrict__ rank,
     const int32_t *__restrict__ block_base, const int32_t *__restrict__ offsets,
     const __nv_bfloat16 *__restrict__ x, int P, int H, int E, int top_k,
-    int32_t *__restrict__ pair_row, int32_t *__restrict__ row_pair, __nv_bfloat16 *__restrict__ xp)
+    int32_t *__restrict__ pair_row, int32_t *__restrict__ row_pair, __nv_bfloat16 *__restrict__ xp,
+    int to_f16)
 {
     pdl_launch_dependents();
     pdl_wait();
@@ -133,7 +137,26 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
     const int t = p / top_k;
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
     uint4 *dst = reinterpret_cast<uint4 *>(xp + (size_t)row * H);
-    for (int i = lane; i < H / 8; i += 32) dst[i] = src[i];
+    if (!to_f16) {
+        for (int i = lane; i < H / 8; i += 32) dst[i] = src[i];
+        return;
+    }
+    bool fits = true;
+    for (int i = lane; i < H / 8; i += 32) {
+        const uint4 v = src[i];
+        uint4 o;
+        const uint32_t *vw = &v.x;
+        uint32_t *ow = &o.x;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float lo = __uint_as_float(vw[q] << 16) * 0.00390625f;
+            const float hi = __uint_as_float(vw[q] & 0xffff0000u) * 0.00390625f;
+            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(ow[q]) : "f"(hi), "f"(lo));
+            if (fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f) fits = false;
+        }
+        dst[i] = o;
+    }
+    if (!fits) record_status(const_cast<int *>(status), kStatusRange);
 }
 
 // The maps only, a thread per pair: used when the gate|up GEMM gathers its
@@ -269,7 +292,7 @@ cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t stream)
     if (a.copy_rows)
         return launch_pdl(dispatch_permute_kernel, dim3((P + 7) / 8), dim3(256), 0, stream, a.status, a.idx,
                           a.rank, a.block_base, a.offsets, a.x, P, a.H, a.E, a.top_k, a.pair_row,
-                          a.row_pair, a.xp);
+                          a.row_pair, a.xp, a.xp_f16);
     return launch_pdl(dispatch_rows_kernel, dim3((P + 255) / 256), dim3(256), 0, stream, a.status, a.idx,
                       a.rank, a.block_base, a.offsets, P, a.E, a.pair_row, a.row_pair);
 }

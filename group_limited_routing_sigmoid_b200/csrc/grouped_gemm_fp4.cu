@@ -13,12 +13,14 @@
 //                 conversion and one f16 multiply by the block scale: every
 //                 product has at most 6 significant bits and lies between
 //                 2^-10 and 2688 in magnitude, so it is exact) and writes it
-//                 to TMEM lane r with tcgen05.st.  The converters also turn
-//                 the stage's token rows from bf16 into f16 times 2^-8 in
-//                 place (the MMA takes A and B of one type): exact for
-//                 every |x| from 2^-9 up to 65504 x 2^8, within 2^-17 below
-//                 that, and a larger value sets the status word
-//                 (BEAM_ERR_RANGE); the epilogue multiplies by 2^8 again;
+//                 to TMEM lane r with tcgen05.st.  The token rows arrive as
+//                 f16 times 2^-8 (the MMA takes A and B of one type): the
+//                 dispatch writes x's sorted rows that way, and the gate|up
+//                 epilogue writes h that way (the bf16 rounding of h first,
+//                 as for bf16 weights).  That is exact for every |x| from
+//                 2^-9 up to 65504 x 2^8 and within 2^-17 below that; a
+//                 larger value sets the status word (BEAM_ERR_RANGE).  The
+//                 epilogue multiplies by 2^8 again;
 //   warps 1, 22   MMA issuers (lane 0): A (the decoded weights) from TMEM,
 //                 two to four stages deep, B (the token rows) from the
 //                 shared-memory stage.  gate|up: warp 1 issues the gate MMAs
@@ -193,11 +195,14 @@ __device__ __forceinline__ void load_chains(uint32_t taddr, int stride, float (&
 // accumulators: SwiGLU of (gate x sa, up x sb), or the value x sa; one warp
 // per lane quadrant takes every chunk of CH columns.  The up accumulator is
 // UP_OFFSET columns after the gate's; chain c of either CHAIN_STRIDE x c.
+// SwiGLU writes h as the down GEMM's operand: f16 of bf16(h) x 2^-8, and
+// BEAM_ERR_RANGE in the status word if a stored value is beyond f16 range.
 template <int EPI, int CH, int UP_OFFSET, int CHAINS, int CHAIN_STRIDE>
 __device__ __forceinline__ void fp4_epilogue_block(uint32_t taddr, int nrows, int row0, int lane,
                                                    uint8_t *stg, __nv_bfloat16 *out, int ldo,
-                                                   float sa, float sb)
+                                                   float sa, float sb, int *status)
 {
+    bool fits = true;
     constexpr int VPR = 4;   // 16-byte vectors per 32 bf16
 #pragma unroll 1
     for (int c0 = 0; c0 < nrows; c0 += CH) {
@@ -207,9 +212,13 @@ __device__ __forceinline__ void fp4_epilogue_block(uint32_t taddr, int nrows, in
         if constexpr (EPI == kSwiGLU) {
             float u[CH];
             load_chains<CH, CHAINS>(taddr + UP_OFFSET + c0, CHAIN_STRIDE, u);
+            unsigned short *shu = reinterpret_cast<unsigned short *>(sh);
 #pragma unroll
-            for (int j = 0; j < CH; ++j)
-                sh[j * 32 + lane] = __float2bfloat16_rn(silu_f32(g[j] * sa) * (u[j] * sb));
+            for (int j = 0; j < CH; ++j) {
+                const float hv = __bfloat162float(__float2bfloat16_rn(silu_f32(g[j] * sa) * (u[j] * sb))) * kFp4TokenScale;
+                if (c0 + j < nrows && fabsf(hv) > 65504.0f) fits = false;
+                shu[j * 32 + lane] = __half_as_ushort(__float2half_rn(hv));
+            }
         } else {
 #pragma unroll
             for (int j = 0; j < CH; ++j) sh[j * 32 + lane] = __float2bfloat16_rn(g[j] * sa);
@@ -225,6 +234,7 @@ __device__ __forceinline__ void fp4_epilogue_block(uint32_t taddr, int nrows, in
         }
         __syncwarp();
     }
+    if (!fits) record_status(status, kStatusRange);
 }
 
 // FP32 outputs: the chains' sum times sa, 16 token rows at a time through
@@ -328,26 +338,6 @@ __device__ __forceinline__ void fp4_decode4_f16(uint32_t codes, uint32_t scale2,
         : "r"(codes));
 #pragma unroll
     for (int i = 0; i < 4; ++i) asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o[i]) : "r"(h[i]), "r"(scale2));
-}
-
-// Token rows of a stage, bf16 -> f16 x 2^-8 in place: 32-bit words i of
-// `words` (two elements each; a row is 32 words), this thread taking every
-// `step`-th from `first`.  Returns false if a word of the first `valid_rows`
-// rows exceeds the f16 range.
-__device__ __forceinline__ bool fp4_tokens_to_f16(uint32_t *bw, int words, int valid_rows, int first,
-                                                  int step)
-{
-    bool fits = true;
-    for (int i = first; i < words; i += step) {
-        const uint32_t v = bw[i];
-        const float lo = __uint_as_float(v << 16) * kFp4TokenScale;
-        const float hi = __uint_as_float(v & 0xffff0000u) * kFp4TokenScale;
-        uint32_t f;
-        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(f) : "f"(hi), "f"(lo));
-        if ((i >> 5) < valid_rows && (fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f)) fits = false;
-        bw[i] = f;
-    }
-    return fits;
 }
 
 }  // namespace
@@ -492,23 +482,13 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         int rs = 0, cs = 0;
         uint32_t rp = 0, cp = 0;
         bool ok = true;
-        const int cidx = threadIdx.x - 32 * kFp4ConvFirst;   // 0 .. 32 * kFp4ConvWarps - 1
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const Item it = decode_item(item, WT, p.E, s_counts, s_offsets, s_tile);
-            const int n_load = (it.nrows + 15) & ~15;
             for (int kb = 0; kb < KB; ++kb) {
                 const bool got = mbar_wait(smem_u32(&rfull[rs]), rp, p.ctl) &&
                                  mbar_wait(smem_u32(&cempty[cs]), cp ^ 1u, p.ctl);
                 ok = __all_sync(0xffffffffu, got);
                 if (!ok) break;
                 tc_fence_after();
-                bool fits = true;
-#pragma unroll
-                for (int ks = 0; ks < KS; ++ks)
-                    fits &= fp4_tokens_to_f16(
-                        reinterpret_cast<uint32_t *>(base_ptr + rs * C::RAW_STAGE + ks * C::B_BYTES),
-                        n_load * (kBK / 2), it.nrows, cidx, 32 * kFp4ConvWarps);
-                if (!fits) record_status(p.ctl.status, kStatusRange);
                 const uint8_t *raw = base_ptr + rs * C::RAW_STAGE + KS * C::B_BYTES;
 #pragma unroll
                 for (int a = 0; a < NUM_A; ++a)
@@ -525,12 +505,9 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                         const uint32_t v[8] = {lo[0], lo[1], lo[2], lo[3], hi[0], hi[1], hi[2], hi[3]};
                         tmem_st8(lane_base + (uint32_t)(cs * C::A_STAGE_COLS + (a * KS + ks) * kAColsPerTile), v);
                     }
-                // every lane's stores complete (the token rows' generic
-                // writes made visible to the MMA's reads too), then one
-                // arrival for the warp (512 same-address arrivals a stage
-                // would serialise)
+                // every lane's stores complete, then one arrival for the
+                // warp (512 same-address arrivals a stage would serialise)
                 tmem_st_wait();
-                fence_view_async_shared();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&cfull[cs]));
@@ -618,7 +595,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
             if constexpr (EPI == kSwiGLU)
                 fp4_epilogue_block<EPI, kFp4Ch, BN, C::CHAINS, NUM_A * BN>(
                     taddr, it.nrows, it.row0, lane, stg, p.out + col0, p.R,
-                    w.a[0].global * kFp4TokenUnscale, w.a[1].global * kFp4TokenUnscale);
+                    w.a[0].global * kFp4TokenUnscale, w.a[1].global * kFp4TokenUnscale, p.ctl.status);
             else if constexpr (EPI == kStoreF32)
                 fp4_epilogue_f32<kFp4Ch, C::CHAINS, NUM_A * BN>(
                     taddr, it.nrows, it.row0, lane, stg, p.out_f32 + col0, p.R,
@@ -626,7 +603,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
             else
                 fp4_epilogue_block<EPI, kFp4Ch, 0, C::CHAINS, NUM_A * BN>(
                     taddr, it.nrows, it.row0, lane, stg, p.out + col0, p.R,
-                    w.a[0].global * kFp4TokenUnscale, 1.0f);
+                    w.a[0].global * kFp4TokenUnscale, 1.0f, p.ctl.status);
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
         }

@@ -97,6 +97,7 @@ struct DispatchArgs {
     int32_t *row_pair;           // [P]
     __nv_bfloat16 *xp;           // [P, H] expert-sorted activations
     int copy_rows;               // 0: maps only (the gate|up GEMM gathers from x)
+    int xp_f16 = 0;              // 1: sorted rows as f16 x 2^-8 (NVFP4 GEMM operands)
 };
 cudaError_t launch_dispatch(const DispatchArgs &a, cudaStream_t stream);
 cudaError_t prepare_dispatch(int E);   // shared-memory limit of the counting kernel
