@@ -36,7 +36,8 @@
 //
 // Stages: a pipeline stage holds KS 64-wide K steps (the codes and scales
 // of KS consecutive tiles of the layout, the token rows of each step): 2 for
-// gate|up, 4 for down when K/64 allows.  Every per-stage cost of the issuing
+// gate|up; for down 5 when K/64 allows it and the token tile has at most 32
+// rows, else 4 when K/64 allows.  Every per-stage cost of the issuing
 // threads and the converters (barrier waits, fences, commits) is then paid
 // once per 64 KS of K.  At 16-row tiles those costs, not the tensor core,
 // set the pace: one wait less per stage took 8% off the decode step, two
@@ -682,7 +683,16 @@ cudaError_t launch_fp4_kind(GemmKind kind, const Fp4Operands &w, const BoxMaps &
     if (kind == GemmKind::kGateUp)
         return launch_pdl(grouped_gemm_fp4_kernel<BN, 2, kSwiGLU, 2>, dim3(grid), dim3(kFp4Threads),
                           Fp4Cfg<BN, 2, kSwiGLU, 2>::SMEM_BYTES, stream, b, w, args);
-    // down: four K steps per stage when K is a multiple of 256
+    // down: five K steps per stage when K is a multiple of 320 and the token
+    // tile has at most 32 rows (two raw stages of five steps then fit in
+    // shared memory), else four when K is a multiple of 256
+    if constexpr (BN <= 32) {
+        if (args.K % (5 * kBK) == 0) {
+            if (kind == GemmKind::kDown) return launch_fp4_down<BN, kStoreBF16, 5>(w, b, args, grid, stream);
+            if (kind == GemmKind::kDownF32 && args.out_f32 != nullptr)
+                return launch_fp4_down<BN, kStoreF32, 5>(w, b, args, grid, stream);
+        }
+    }
     const bool ks4 = args.K % (4 * kBK) == 0;
     if (kind == GemmKind::kDown)
         return ks4 ? launch_fp4_down<BN, kStoreBF16, 4>(w, b, args, grid, stream)
@@ -703,6 +713,10 @@ cudaError_t prepare_grouped_gemm_fp4()
     if ((err = set_smem_fp4<BN, 1, kStoreF32, 2>()) != cudaSuccess) return err;  \
     if ((err = set_smem_fp4<BN, 1, kStoreBF16, 4>()) != cudaSuccess) return err; \
     if ((err = set_smem_fp4<BN, 1, kStoreF32, 4>()) != cudaSuccess) return err;
+    if ((err = set_smem_fp4<16, 1, kStoreBF16, 5>()) != cudaSuccess) return err;
+    if ((err = set_smem_fp4<16, 1, kStoreF32, 5>()) != cudaSuccess) return err;
+    if ((err = set_smem_fp4<32, 1, kStoreBF16, 5>()) != cudaSuccess) return err;
+    if ((err = set_smem_fp4<32, 1, kStoreF32, 5>()) != cudaSuccess) return err;
     BEAM_PREP_FP4(16)
     BEAM_PREP_FP4(32)
     BEAM_PREP_FP4(64)

@@ -84,10 +84,13 @@ def test_nvfp4_block(T, ctas, tile, resid):
 
 
 # inter 256: the down GEMM takes four K steps per stage (K/64 a multiple of
-# four), at every token tile size
-@pytest.mark.parametrize("T,tile", [(300, 16), (300, 32), (1000, 64), (1000, 128)])
-def test_nvfp4_block_four_k_steps_per_stage(T, tile):
-    wl = dataclasses.replace(W.WORKLOADS["tiny_nvfp4"], inter=256)
+# four), at every token tile size; inter 640: five K steps per stage for
+# tiles of 16 and 32 rows (K/64 a multiple of five), two for larger tiles
+@pytest.mark.parametrize("T,tile,inter", [(300, 16, 256), (300, 32, 256), (1000, 64, 256),
+                                          (1000, 128, 256), (300, 16, 640), (37, 32, 640),
+                                          (300, 64, 640)])
+def test_nvfp4_block_several_k_steps_per_stage(T, tile, inter):
+    wl = dataclasses.replace(W.WORKLOADS["tiny_nvfp4"], inter=inter)
     g = W.generator(wl, "cuda")
     d = W.make_nvfp4_weights(wl, "cuda", g)
     d.update(W.make_tokens(wl, "cuda", g, T=T))
@@ -96,7 +99,7 @@ def test_nvfp4_block_four_k_steps_per_stage(T, tile):
     plan = moe.launch_plan(T)
     assert plan["tile_rows"] == tile
     rep = check_block(wl, d, moe)
-    _log(f"nvfp4_inter256_T{T}_tile{tile}", rep, plan)
+    _log(f"nvfp4_inter{inter}_T{T}_tile{tile}", rep, plan)
     assert rep.ok(), rep
     moe.close()
 
