@@ -77,7 +77,6 @@ constexpr int kFp4AStagesMax = 4;                          // decoded A stages i
 constexpr int kFp4Ch = 16;                                 // epilogue columns per chunk
 constexpr int kFp4MaxRaw = 24;
 constexpr int kFp4BarrierBytes = 1024;
-constexpr int kFp4LutBytes = 256 * 2;                      // E4M3 byte -> f16 scale
 constexpr float kFp4TokenScale = 0.00390625f;              // 2^-8: token rows as f16
 constexpr float kFp4TokenUnscale = 256.0f;
 constexpr int kAColsPerTile = kBK / 2;                     // 64 bf16 of a row: 32 TMEM columns
@@ -90,7 +89,7 @@ struct Fp4Cfg {
     static constexpr int RAW_USED = KS * B_BYTES + NUM_A * (CODES + SCALES);
     static constexpr int RAW_STAGE = (RAW_USED + 1023) / 1024 * 1024;   // keeps B 1024-aligned
     static constexpr int STAGING = kFp4EpiWarps * kStagingWarpBytes;
-    static constexpr int FIXED = 1024 + STAGING + kFp4BarrierBytes + kFp4LutBytes + kTableBytes;
+    static constexpr int FIXED = 1024 + STAGING + kFp4BarrierBytes + kTableBytes;
     static constexpr int RAW_FIT = (kMaxDynSmem - FIXED) / RAW_STAGE;
     static constexpr int RAW_STAGES = RAW_FIT > kFp4MaxRaw ? kFp4MaxRaw : RAW_FIT;
     static constexpr int CHAINS = BN >= 64 ? 1 : 64 / BN;        // 4 for 16 rows, 2 for 32
@@ -315,12 +314,6 @@ __device__ __forceinline__ void fp4_decode4(uint32_t codes, uint32_t scale_bits,
     }
 }
 
-// The f16 encoding of an E4M3 value (exact: E4M3 values lie between 2^-9
-// and 448 in magnitude, all normal f16 numbers).
-__device__ __forceinline__ uint32_t fp4_scale_bits_f16(uint32_t byte)
-{
-    return __half_as_ushort(__float2half_rn(e4m3_float(byte)));
-}
 
 // Four code bytes (eight E2M1 elements, element 2j in the low nibble of byte
 // j) times one block scale, as four f16x2 words (element 2j in the low
@@ -361,8 +354,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;                                          // one per issuer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 2);
-    uint16_t *lut_s = reinterpret_cast<uint16_t *>(staging + C::STAGING + kFp4BarrierBytes);
-    int *s_counts = reinterpret_cast<int *>(lut_s + 256);
+    int *s_counts = reinterpret_cast<int *>(staging + C::STAGING + kFp4BarrierBytes);
     int *s_offsets = s_counts + p.E;
     int *s_tile = s_offsets + (p.E + 1);
 
@@ -392,9 +384,6 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (converter)
-        for (int i = threadIdx.x - 32 * kFp4ConvFirst; i < 256; i += 32 * kFp4ConvWarps)
-            lut_s[i] = (uint16_t)fp4_scale_bits_f16((uint32_t)i);
     pdl_launch_dependents();
     pdl_wait();   // set-up above overlaps the previous kernel; data from here on
     load_tables(p, s_counts, s_offsets, s_tile);
@@ -498,11 +487,16 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
                         // this block of row r in K step ks: 8 code bytes and one scale byte
                         const uint2 c = *reinterpret_cast<const uint2 *>(
                             raw + a * C::CODES + ks * kFp4CodeTile + blk * (kFp4TileRows * 8) + r * 8);
-                        const uint32_t sb = lut_s[raw[NUM_A * C::CODES + a * C::SCALES +
-                                                      ks * kFp4ScaleTile + blk * kFp4TileRows + r]];
+                        // the scale byte in both halves, widened to f16x2 by
+                        // the hardware (exact: every E4M3 value is a normal f16)
+                        const uint32_t sbyte = raw[NUM_A * C::CODES + a * C::SCALES +
+                                                   ks * kFp4ScaleTile + blk * kFp4TileRows + r];
+                        const unsigned short pair = (unsigned short)(sbyte | (sbyte << 8));
+                        uint32_t s2;
+                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(pair));
                         uint32_t lo[4], hi[4];
-                        fp4_decode4_f16(c.x, sb | (sb << 16), lo);
-                        fp4_decode4_f16(c.y, sb | (sb << 16), hi);
+                        fp4_decode4_f16(c.x, s2, lo);
+                        fp4_decode4_f16(c.y, s2, hi);
                         const uint32_t v[8] = {lo[0], lo[1], lo[2], lo[3], hi[0], hi[1], hi[2], hi[3]};
                         tmem_st8(lane_base + (uint32_t)(cs * C::A_STAGE_COLS + (a * KS + ks) * kAColsPerTile), v);
                     }
